@@ -1,0 +1,231 @@
+"""Float64 CPU oracle for the GDLA forward pass (test infrastructure).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline / reference
+legs of ``bench.py`` may import this package.  The product library never loads
+it, and it imports nothing from the product package: the two share no code.
+
+The arithmetic lives in ``gdla_oracle.c`` (plain C, double precision, OpenMP
+over rows and heads); this module only compiles it with gcc and marshals
+arrays.  Inputs may be CPU torch tensors (bfloat16, float32, float64) or numpy
+arrays (float32, float64, or uint16 holding bfloat16 bits); bfloat16 is handed
+to C as raw bit patterns and widened there exactly.  Results are float64 numpy
+arrays.
+
+Each function restates one step of the forward pass as the page
+"Motif 3: Technical Report" (paper.rainbus.top digest), step 2 "GDLA forward",
+writes it; ``gdla_oracle.c`` lists the readings taken where the page is silent.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SOURCE = os.path.join(_HERE, "gdla_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "_liboracle_gdla.so")
+
+BF16, F64, F32 = 0, 1, 2
+
+
+def compile_source(src: str, out: str) -> str:
+    """Compile one oracle C source into a shared library (gcc, OpenMP)."""
+    tmp = out + ".tmp%d" % os.getpid()
+    cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
+           "-ffp-contract=off", src, "-o", tmp, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, out)
+    return out
+
+
+def build(force: bool = False) -> str:
+    """Compile ``gdla_oracle.c`` into ``oracle/_liboracle_gdla.so`` if stale."""
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(SOURCE)):
+        return _LIB_PATH
+    return compile_source(SOURCE, _LIB_PATH)
+
+
+def _arr(x):
+    """Return (contiguous host array, pointer, dtype code) for one input."""
+    import torch
+    if isinstance(x, torch.Tensor):
+        x = x.detach()
+        if x.device.type != "cpu":
+            raise ValueError("oracle inputs must live on the CPU")
+        x = x.contiguous()
+        if x.dtype == torch.bfloat16:
+            a = x.view(torch.int16).numpy().view(np.uint16)
+            return a, a.ctypes.data, BF16
+        if x.dtype == torch.float32:
+            a = x.numpy()
+            return a, a.ctypes.data, F32
+        a = x.to(torch.float64).numpy()
+        return a, a.ctypes.data, F64
+    a = np.ascontiguousarray(x)
+    if a.dtype == np.float32:
+        return a, a.ctypes.data, F32
+    if a.dtype == np.uint16:  # raw bfloat16 bits
+        return a, a.ctypes.data, BF16
+    a = np.ascontiguousarray(a, dtype=np.float64)
+    return a, a.ctypes.data, F64
+
+
+def _rows(rows, total):
+    if rows is None:
+        return None, None, total
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1))
+    if r.size and (r.min() < 0 or r.max() >= total):
+        raise ValueError("row index out of range")
+    return r, r.ctypes.data, int(r.size)
+
+
+class Oracle:
+    """Bindings to one compiled copy of the C oracle."""
+
+    def __init__(self, lib_path: str):
+        lib = ctypes.CDLL(lib_path)
+        vp, i32, i64, f64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_double
+        lib.gdla_oracle_rmsnorm.argtypes = [vp, i32, vp, i32, f64, i64, i32, vp]
+        lib.gdla_oracle_rmsnorm.restype = None
+        lib.gdla_oracle_kv_expand.argtypes = [vp, vp, i32, i64, i32, i32, i32, i32, vp, vp]
+        lib.gdla_oracle_kv_expand.restype = None
+        lib.gdla_oracle_attention_path.argtypes = [vp, i32, vp, i32, vp, i32, i32, i64, i32, i32,
+                                                   i32, i64, i32, f64, vp, i64, vp]
+        lib.gdla_oracle_attention_path.restype = None
+        lib.gdla_oracle_differential_gate.argtypes = [vp, vp, vp, i32, vp, i32, i32, i32, i32,
+                                                      vp, i64, vp]
+        lib.gdla_oracle_differential_gate.restype = None
+        lib.gdla_oracle_attn.argtypes = [vp, i32, vp, i32, vp, i32, vp, i32, vp, i32, vp, i32,
+                                         i32, i64, i32, i32, i32, i32, i64, i32, f64, vp, i64, vp]
+        lib.gdla_oracle_attn.restype = ctypes.c_int
+        lib.gdla_oracle_version.restype = ctypes.c_int
+        self.lib = lib
+        self.path = lib_path
+
+    # a1: RMSNorm of the KV latent
+    def rmsnorm(self, c, w=None, eps: float = 1e-6) -> np.ndarray:
+        """c / sqrt(mean(c^2) + eps) * w, row by row; w=None means ones."""
+        ca, cp, cdt = _arr(c)
+        n, dl = ca.shape[0], ca.shape[-1]
+        out = np.empty((n, dl), dtype=np.float64)
+        wa, wp, wdt = (None, None, F64) if w is None else _arr(w)
+        self.lib.gdla_oracle_rmsnorm(cp, cdt, wp, wdt, float(eps), n, dl, out.ctypes.data)
+        return out
+
+    # a2: W^KV_b up-projection
+    def kv_expand(self, c_hat, w_kvb, n_kv_heads: int, dk: int, dv: int):
+        """Returns K [N,Hkv,dk], V [N,Hkv,dv] from the normalised latent."""
+        ch = np.ascontiguousarray(np.asarray(c_hat, dtype=np.float64))
+        wa, wp, wdt = _arr(w_kvb)
+        n, dl = ch.shape
+        if tuple(wa.shape) != (dl, n_kv_heads * (dk + dv)):
+            raise ValueError("W^KV_b must be [d_latent, Hkv*(dk+dv)]")
+        k = np.empty((n, n_kv_heads, dk), dtype=np.float64)
+        v = np.empty((n, n_kv_heads, dv), dtype=np.float64)
+        self.lib.gdla_oracle_kv_expand(ch.ctypes.data, wp, wdt, n, dl, n_kv_heads, dk, dv,
+                                       k.ctypes.data, v.ctypes.data)
+        return k, v
+
+    # a3/a4/a5: one attention path under the mask
+    def attention_path(self, q, k, v, window: int = 0, causal: bool = True, scale=None,
+                       rows=None) -> np.ndarray:
+        """q [B,T,H,d], k/v [B,T,Hkv,d]; head h reads KV head h // (H // Hkv).
+
+        Returns H[n_rows, H, d] for flat rows b*T+i (every row when None).
+        """
+        qa, qp, qdt = _arr(q)
+        ka, kp, kdt = _arr(k)
+        va, vp, vdt = _arr(v)
+        B, T, H, d = qa.shape
+        Hkv = ka.shape[2]
+        if scale is None:
+            scale = 1.0 / np.sqrt(d)
+        r, rp, n = _rows(rows, B * T)
+        out = np.empty((n, H, d), dtype=np.float64)
+        self.lib.gdla_oracle_attention_path(qp, qdt, kp, kdt, vp, vdt, B, T, H, Hkv, d,
+                                            int(window), int(bool(causal)), float(scale), rp, n,
+                                            out.ctypes.data)
+        return out
+
+    # a6/a7/a8: Repeat_g, differential combine, gate
+    def differential_gate(self, hs, hn, lam, gate, rows=None) -> np.ndarray:
+        """D = H_S - lambda * Repeat_g(H_N); O = G * D.  Returns O[n_rows, Hs*d].
+
+        hs [n,Hs,d] and hn [n,Hn,d] are per evaluated row; lam [..,Hs] and
+        gate [..,Hs*d] are addressed by the flat row index (rows, or 0..n-1).
+        """
+        hs = np.ascontiguousarray(np.asarray(hs, dtype=np.float64))
+        hn = np.ascontiguousarray(np.asarray(hn, dtype=np.float64))
+        la, lp, ldt = _arr(lam)
+        ga, gp, gdt = _arr(gate)
+        n, Hs, d = hs.shape
+        Hn = hn.shape[1]
+        r, rp, nr = _rows(rows, la.size // Hs)
+        if rows is not None and nr != n:
+            raise ValueError("rows must list one flat index per evaluated row")
+        out = np.empty((n, Hs * d), dtype=np.float64)
+        self.lib.gdla_oracle_differential_gate(hs.ctypes.data, hn.ctypes.data, lp, ldt, gp, gdt,
+                                               Hs, Hn, d, rp, n, out.ctypes.data)
+        return out
+
+    # whole attention forward
+    def gdla_attn(self, q_sig, q_noise, k, v, lam, gate, window: int = 0, causal: bool = True,
+                  scale=None, rows=None) -> np.ndarray:
+        """O[n_rows, Hs*d] in float64 for flat rows b*T+i (all when None).
+
+        q_sig [B,T,Hs,d], q_noise [B,T,Hn,d], k/v [B,T,Hkv,d], lam [B,T,Hs],
+        gate [B,T,Hs*d].
+        """
+        qs, qsp, qsdt = _arr(q_sig)
+        qn, qnp, qndt = _arr(q_noise)
+        ka, kp, kdt = _arr(k)
+        va, vp, vdt = _arr(v)
+        la, lp, ldt = _arr(lam)
+        ga, gp, gdt = _arr(gate)
+        B, T, Hs, d = qs.shape
+        Hn = qn.shape[2]
+        Hkv = ka.shape[2]
+        if scale is None:
+            scale = 1.0 / np.sqrt(d)
+        r, rp, n = _rows(rows, B * T)
+        out = np.empty((n, Hs * d), dtype=np.float64)
+        rc = self.lib.gdla_oracle_attn(qsp, qsdt, qnp, qndt, kp, kdt, vp, vdt, lp, ldt, gp, gdt,
+                                       B, T, Hs, Hn, Hkv, d, int(window), int(bool(causal)),
+                                       float(scale), rp, n, out.ctypes.data)
+        if rc != 0:
+            raise ValueError("oracle rejected the head counts (need Hs % Hn == 0, Hn == Hkv)")
+        return out
+
+
+_default = None
+
+
+def default() -> Oracle:
+    """The oracle built from ``gdla_oracle.c`` (compiled on first use)."""
+    global _default
+    if _default is None:
+        _default = Oracle(build())
+    return _default
+
+
+def rmsnorm(*a, **k):
+    return default().rmsnorm(*a, **k)
+
+
+def kv_expand(*a, **k):
+    return default().kv_expand(*a, **k)
+
+
+def attention_path(*a, **k):
+    return default().attention_path(*a, **k)
+
+
+def differential_gate(*a, **k):
+    return default().differential_gate(*a, **k)
+
+
+def gdla_attn(*a, **k):
+    return default().gdla_attn(*a, **k)

@@ -1,0 +1,241 @@
+/*
+ * Float64 CPU oracle for the GDLA (Grouped Differential Latent Attention)
+ * forward pass.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or
+ * call this file: it exists so that tests, the smoke check and the benchmark's
+ * CPU-baseline leg can compare the CUDA kernels against a plain, slow,
+ * obviously correct restatement of the method.  It shares no code, header or
+ * constant with the CUDA library.
+ *
+ * Sources (web pages; "step 2" is the page's own numbering):
+ *   [R]  "Motif 3: Technical Report" digest at paper.rainbus.top, step 2
+ *        ("GDLA forward"): x_t -> query latent c^Q_t (1024) and KV latent
+ *        c_KV,t (512) -> RMSNorm -> W^KV_b expands 16 KV heads -> signal and
+ *        noise query paths each attend over the shared KV heads -> noise output
+ *        repeated g times per group -> D_t = H_S,t - lambda_t (.) Repeat_g(H_N,t)
+ *        -> sigmoid gate G_t from the query latent multiplies D_t elementwise
+ *        -> W^O.  Same page, "technical novelty" paragraph: both query paths
+ *        share one up-projected KV; lambda is per token and sigmoid-bounded.
+ *   [P]  "Вышла новая модель Motif 3" (pikabu.ru): 16 shared KV heads for
+ *        64 signal / 16 noise query heads; window 128 with full attention in
+ *        every 4th layer.
+ *
+ * Readings taken where the pages are silent (each is listed in the design doc):
+ *   - signal head h uses KV head floor(h/g) and noise head floor(h/g)
+ *     (interleaved repeat: "repeat per group" in [R]);
+ *   - noise head n uses KV head n (Hn == Hkv);
+ *   - lambda is one scalar per (token, signal head); lambda and the gate arrive
+ *     already passed through their sigmoids;
+ *   - sliding window W keeps keys j with i-W < j <= i; W = 0 means full causal;
+ *   - RMSNorm is c / sqrt(mean(c^2) + eps) * w;
+ *   - the W^KV_b columns of KV head h are [K_h (dk) | V_h (dv)].
+ *
+ * Every function computes in double, in the order the definition is written:
+ * no tiling, no online softmax, no reassociation.  Inputs may be given as
+ * bfloat16 bit patterns, float32 or float64 (dtype codes below); bfloat16 and
+ * float32 widen to double exactly.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_BF16 0
+#define ORACLE_F64 1
+#define ORACLE_F32 2
+
+static double load_elem(const void *p, int dtype, int64_t i) {
+  if (dtype == ORACLE_F64) return ((const double *)p)[i];
+  if (dtype == ORACLE_F32) return (double)((const float *)p)[i];
+  /* bfloat16: the upper 16 bits of an IEEE binary32 */
+  uint32_t bits = ((uint32_t)((const uint16_t *)p)[i]) << 16;
+  float f;
+  memcpy(&f, &bits, sizeof f);
+  return (double)f;
+}
+
+int gdla_oracle_version(void) { return 1; }
+
+/*
+ * RMSNorm of the KV latent ([R] step 2: "c_KV,t ... -> RMSNorm").
+ *   out[t, k] = c[t, k] / sqrt(mean_k c[t, k]^2 + eps) * w[k]
+ * w == NULL means a weight of ones.
+ */
+void gdla_oracle_rmsnorm(const void *c, int c_dt, const void *w, int w_dt,
+                         double eps, int64_t n_tokens, int d_latent,
+                         double *out) {
+  int64_t t;
+#pragma omp parallel for schedule(static)
+  for (t = 0; t < n_tokens; ++t) {
+    double ss = 0.0;
+    for (int k = 0; k < d_latent; ++k) {
+      double x = load_elem(c, c_dt, t * d_latent + k);
+      ss += x * x;
+    }
+    double r = sqrt(ss / (double)d_latent + eps);
+    for (int k = 0; k < d_latent; ++k) {
+      double wk = w ? load_elem(w, w_dt, k) : 1.0;
+      out[t * d_latent + k] = load_elem(c, c_dt, t * d_latent + k) / r * wk;
+    }
+  }
+}
+
+/*
+ * Up-projection W^KV_b ([R] step 2: "W^KV_b expands 16 KV heads").
+ *   KV[t, col] = sum_k c_hat[t, k] * W[k, col],  W is [d_latent, Hkv*(dk+dv)]
+ *   K[t, h, x] = KV[t, h*(dk+dv) + x]          for x <  dk
+ *   V[t, h, x] = KV[t, h*(dk+dv) + dk + x]     for x <  dv
+ */
+void gdla_oracle_kv_expand(const double *c_hat, const void *w, int w_dt,
+                           int64_t n_tokens, int d_latent, int n_kv_heads,
+                           int dk, int dv, double *k_out, double *v_out) {
+  const int64_t ncol = (int64_t)n_kv_heads * (dk + dv);
+  int64_t t;
+#pragma omp parallel for schedule(static)
+  for (t = 0; t < n_tokens; ++t) {
+    for (int64_t col = 0; col < ncol; ++col) {
+      double acc = 0.0;
+      for (int k = 0; k < d_latent; ++k)
+        acc += c_hat[t * d_latent + k] * load_elem(w, w_dt, (int64_t)k * ncol + col);
+      int64_t h = col / (dk + dv), x = col % (dk + dv);
+      if (x < dk)
+        k_out[(t * n_kv_heads + h) * dk + x] = acc;
+      else
+        v_out[(t * n_kv_heads + h) * dv + (x - dk)] = acc;
+    }
+  }
+}
+
+/* Key range kept by the mask for query i ([P]: window 128, full attention
+ * every 4th layer).  causal == 0: all keys.  causal, window == 0: j <= i.
+ * causal, window W > 0: i - W < j <= i. */
+static void key_range(int64_t i, int64_t T, int64_t window, int causal,
+                      int64_t *lo, int64_t *hi) {
+  if (!causal) {
+    *lo = 0;
+    *hi = T - 1;
+    return;
+  }
+  *hi = i;
+  *lo = 0;
+  if (window > 0 && i - window + 1 > 0) *lo = i - window + 1;
+}
+
+/*
+ * One attention path (signal or noise), [R] step 2: each query path attends
+ * over the shared KV heads.  For every requested row r = b*T + i and head h:
+ *   s_j = scale * sum_c Q[b,i,h,c] K[b,j,kv(h),c]         j in J(i)
+ *   p_j = exp(s_j - max_j s_j)
+ *   H[row, h, :] = sum_j p_j V[b,j,kv(h),:] / sum_j p_j
+ * kv(h) = h / (H / Hkv).  Q is [B,T,H,d], K and V are [B,T,Hkv,d].
+ * rows == NULL means every row (n_rows must then be B*T).
+ */
+void gdla_oracle_attention_path(const void *q, int q_dt, const void *k,
+                                int k_dt, const void *v, int v_dt, int B,
+                                int64_t T, int H, int Hkv, int d,
+                                int64_t window, int causal, double scale,
+                                const int64_t *rows, int64_t n_rows,
+                                double *out) {
+  const int group = H / Hkv;
+  (void)B;
+  int64_t task;
+#pragma omp parallel
+  {
+    double *s = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+    double *acc = (double *)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(dynamic, 1)
+    for (task = 0; task < n_rows * H; ++task) {
+      int64_t ri = task / H;
+      int h = (int)(task % H);
+      int64_t row = rows ? rows[ri] : ri;
+      int64_t b = row / T, i = row % T;
+      int kvh = h / group;
+      int64_t lo, hi;
+      key_range(i, T, window, causal, &lo, &hi);
+      const int64_t qoff = (row * H + h) * d;
+      double m = -INFINITY;
+      for (int64_t j = lo; j <= hi; ++j) {
+        const int64_t koff = ((b * T + j) * Hkv + kvh) * d;
+        double dot = 0.0;
+        for (int c = 0; c < d; ++c)
+          dot += load_elem(q, q_dt, qoff + c) * load_elem(k, k_dt, koff + c);
+        s[j - lo] = scale * dot;
+        if (s[j - lo] > m) m = s[j - lo];
+      }
+      double denom = 0.0;
+      for (int c = 0; c < d; ++c) acc[c] = 0.0;
+      for (int64_t j = lo; j <= hi; ++j) {
+        const double p = exp(s[j - lo] - m);
+        const int64_t voff = ((b * T + j) * Hkv + kvh) * d;
+        denom += p;
+        for (int c = 0; c < d; ++c) acc[c] += p * load_elem(v, v_dt, voff + c);
+      }
+      double *o = out + (ri * H + h) * d;
+      for (int c = 0; c < d; ++c) o[c] = acc[c] / denom;
+    }
+    free(s);
+    free(acc);
+  }
+}
+
+/*
+ * Differential combine and output gate, [R] step 2:
+ *   D[h]  = H_S[h] - lambda[h] * H_N[h / g]          (Repeat_g, interleaved)
+ *   O[h]  = G[h*d : (h+1)*d] (.) D[h]
+ * hs: [n_rows, Hs, d], hn: [n_rows, Hn, d] (already gathered per row).
+ * lambda: [B*T, Hs], gate: [B*T, Hs*d], both addressed by the flat row index
+ * rows[ri] (rows == NULL: ri itself).  out: [n_rows, Hs*d].
+ */
+void gdla_oracle_differential_gate(const double *hs, const double *hn,
+                                   const void *lam, int lam_dt,
+                                   const void *gate, int gate_dt, int Hs,
+                                   int Hn, int d, const int64_t *rows,
+                                   int64_t n_rows, double *out) {
+  const int g = Hs / Hn;
+  int64_t ri;
+#pragma omp parallel for schedule(static)
+  for (ri = 0; ri < n_rows; ++ri) {
+    const int64_t row = rows ? rows[ri] : ri;
+    for (int h = 0; h < Hs; ++h) {
+      const double l = load_elem(lam, lam_dt, row * Hs + h);
+      const int n = h / g;
+      for (int c = 0; c < d; ++c) {
+        const double diff = hs[(ri * Hs + h) * d + c] - l * hn[(ri * Hn + n) * d + c];
+        const double gv = load_elem(gate, gate_dt, row * (int64_t)Hs * d + (int64_t)h * d + c);
+        out[ri * (int64_t)Hs * d + (int64_t)h * d + c] = gv * diff;
+      }
+    }
+  }
+}
+
+/*
+ * Whole GDLA attention forward for a subset of rows: the signal path over
+ * Q_sig (Hs heads, KV head h/g), the noise path over Q_noise (Hn heads, KV
+ * head n), then the differential combine and the gate.
+ * Returns 0, or -1 when the head counts do not divide (Hs % Hn, Hn != Hkv).
+ */
+int gdla_oracle_attn(const void *q_sig, int qs_dt, const void *q_noise,
+                     int qn_dt, const void *k, int k_dt, const void *v,
+                     int v_dt, const void *lam, int lam_dt, const void *gate,
+                     int gate_dt, int B, int64_t T, int Hs, int Hn, int Hkv,
+                     int d, int64_t window, int causal, double scale,
+                     const int64_t *rows, int64_t n_rows, double *out) {
+  if (Hn <= 0 || Hkv <= 0 || Hs % Hn != 0 || Hn != Hkv) return -1;
+  double *hs = (double *)malloc(sizeof(double) * (size_t)(n_rows * Hs * d));
+  double *hn = (double *)malloc(sizeof(double) * (size_t)(n_rows * Hn * d));
+  if (!hs || !hn) {
+    free(hs);
+    free(hn);
+    return -2;
+  }
+  gdla_oracle_attention_path(q_sig, qs_dt, k, k_dt, v, v_dt, B, T, Hs, Hkv, d,
+                             window, causal, scale, rows, n_rows, hs);
+  gdla_oracle_attention_path(q_noise, qn_dt, k, k_dt, v, v_dt, B, T, Hn, Hkv,
+                             d, window, causal, scale, rows, n_rows, hn);
+  gdla_oracle_differential_gate(hs, hn, lam, lam_dt, gate, gate_dt, Hs, Hn, d,
+                                rows, n_rows, out);
+  free(hs);
+  free(hn);
+  return 0;
+}

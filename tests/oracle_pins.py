@@ -1,0 +1,309 @@
+"""Pins that tie the float64 oracle to facts fixed outside the oracle.
+
+Each ``pin_*`` takes an ``oracle.Oracle`` and raises AssertionError when the
+oracle disagrees with a value derived by hand, a closed form, a library
+routine (torch SDPA / rms_norm / matmul in float64) or an invariant that the
+GDLA forward must satisfy.  The operation is the one on the page
+"Motif 3: Technical Report" (paper.rainbus.top digest), step 2 "GDLA forward";
+head counts, window and lambda bounds come from the same page and from
+"Вышла новая модель Motif 3" (pikabu.ru).
+
+The pins are plain functions so that tests/test_oracle_mutants.py can run them
+against deliberately broken copies of the oracle.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import torch
+import torch.nn.functional as F
+
+from grouped_differential_attention_gdla_b200.inputs import custom, make_inputs
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _f64(t):
+    return t.to(torch.float64) if isinstance(t, torch.Tensor) else torch.as_tensor(t, dtype=torch.float64)
+
+
+def _small(B=2, T=19, Hs=8, Hn=2, Hkv=2, d=16, seed=3, window=0, causal=True):
+    wl = custom(B, T, Hs, Hn, Hkv, d, window=window, causal=causal)
+    return wl, make_inputs(wl, seed=seed)
+
+
+def _close(a, b, rtol=1e-11, atol=1e-12, what=""):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    assert a.shape == b.shape, f"{what}: shape {a.shape} vs {b.shape}"
+    err = np.abs(a - b).max() if a.size else 0.0
+    tol = atol + rtol * (np.abs(b).max() if b.size else 0.0)
+    assert err <= tol, f"{what}: max abs err {err:.3e} > {tol:.3e}"
+
+
+def _sdpa(q, k, v, group, window, causal, scale):
+    """torch SDPA in float64 on CPU with KV heads repeated per group."""
+    q = _f64(q).permute(0, 2, 1, 3)
+    k = _f64(k).repeat_interleave(group, dim=2).permute(0, 2, 1, 3)
+    v = _f64(v).repeat_interleave(group, dim=2).permute(0, 2, 1, 3)
+    T = q.shape[2]
+    i = torch.arange(T).view(T, 1)
+    j = torch.arange(T).view(1, T)
+    if causal:
+        keep = j <= i
+        if window > 0:
+            keep = keep & (j > i - window)
+    else:
+        keep = torch.ones(T, T, dtype=torch.bool)
+    out = F.scaled_dot_product_attention(q, k, v, attn_mask=keep, scale=scale)
+    return out.permute(0, 2, 1, 3)  # [B,T,H,d]
+
+
+# ---------------------------------------------------------------- golden values
+
+def pin_hand_example(o):
+    """Two-token case derived by hand (tests/golden/hand_example.json)."""
+    with open(os.path.join(GOLDEN, "hand_example.json")) as f:
+        g = json.load(f)
+    ln3 = math.log(3.0)
+    k = [[[[ln3 if x == "LN3" else x for x in hd] for hd in tok] for tok in b] for b in g["k"]]
+    args = dict(q_sig=np.array(g["q_sig"]), q_noise=np.array(g["q_noise"]), k=np.array(k),
+                v=np.array(g["v"]), lam=np.array(g["lam"]), gate=np.array(g["gate"]),
+                scale=g["shape"]["scale"])
+    _close(o.gdla_attn(**args, window=0, causal=True), g["expected"]["causal"], what="causal")
+    _close(o.gdla_attn(**args, window=1, causal=True), g["expected"]["window1"], what="W=1")
+    _close(o.gdla_attn(**args, window=0, causal=False), g["expected"]["noncausal"],
+           what="non-causal")
+    hs = o.attention_path(args["q_sig"], args["k"], args["v"], scale=1.0, rows=[1])
+    hn = o.attention_path(args["q_noise"], args["k"], args["v"], scale=1.0, rows=[1])
+    _close(hs[0], g["expected_paths_row1_causal"]["H_S"], what="H_S row 1")
+    _close(hn[0], g["expected_paths_row1_causal"]["H_N"], what="H_N row 1")
+
+
+# ---------------------------------------------------------------- closed forms
+
+def pin_first_row_closed_form(o):
+    """Row i=0 sees one key: O = G * (1 - lambda) * V[b, 0, h//g]."""
+    wl, x = _small()
+    out = o.gdla_attn(x["q_sig"], x["q_noise"], x["k"], x["v"], x["lam"], x["gate"])
+    out = out.reshape(wl.B, wl.T, wl.Hs, wl.d)
+    v0 = _f64(x["v"])[:, 0].repeat_interleave(wl.g, dim=1)           # [B,Hs,d]
+    lam = _f64(x["lam"])[:, 0].unsqueeze(-1)                           # [B,Hs,1]
+    gate = _f64(x["gate"])[:, 0].reshape(wl.B, wl.Hs, wl.d)
+    _close(out[:, 0], (gate * (1 - lam) * v0).numpy(), what="row 0")
+
+
+def pin_window_one_closed_form(o):
+    """W=1 keeps only the diagonal: O[i] = G * (1 - lambda) * V[i, h//g]."""
+    wl, x = _small(window=1)
+    out = o.gdla_attn(x["q_sig"], x["q_noise"], x["k"], x["v"], x["lam"], x["gate"], window=1)
+    out = out.reshape(wl.B, wl.T, wl.Hs, wl.d)
+    v = _f64(x["v"]).repeat_interleave(wl.g, dim=2)
+    lam = _f64(x["lam"]).unsqueeze(-1)
+    gate = _f64(x["gate"]).reshape(wl.B, wl.T, wl.Hs, wl.d)
+    _close(out, (gate * (1 - lam) * v).numpy(), what="W=1")
+
+
+def pin_equal_keys_mean(o):
+    """Equal key rows give uniform weights: H = mean of V over the kept keys."""
+    for window, causal in ((0, True), (4, True), (0, False)):
+        wl, x = _small(T=13, window=window, causal=causal)
+        k = x["k"].clone()
+        k[:] = k[:, :1]                                   # every key row = key 0
+        T = wl.T
+        v = _f64(x["v"])                                  # [B,T,Hkv,d]
+        mean = torch.empty_like(v)
+        for i in range(T):
+            lo = 0 if not causal else (max(0, i - window + 1) if window > 0 else 0)
+            hi = T - 1 if not causal else i
+            mean[:, i] = v[:, lo:hi + 1].mean(dim=1)
+        mean_s = mean.repeat_interleave(wl.g, dim=2)
+        lam = _f64(x["lam"]).unsqueeze(-1)
+        gate = _f64(x["gate"]).reshape(wl.B, T, wl.Hs, wl.d)
+        want = gate * (1 - lam) * mean_s
+        got = o.gdla_attn(x["q_sig"], x["q_noise"], k, x["v"], x["lam"], x["gate"],
+                          window=window, causal=causal).reshape(wl.B, T, wl.Hs, wl.d)
+        _close(got, want.numpy(), rtol=1e-10, what=f"equal keys W={window} causal={causal}")
+
+
+# ---------------------------------------------------------------- library routines
+
+def pin_lambda0_gate1_is_gqa_sdpa(o):
+    """lambda=0, G=1 reduces GDLA to grouped-query attention (torch SDPA)."""
+    for window, causal in ((0, True), (5, True), (0, False)):
+        wl, x = _small(window=window, causal=causal)
+        lam0 = torch.zeros_like(x["lam"])
+        gate1 = torch.ones_like(x["gate"])
+        got = o.gdla_attn(x["q_sig"], x["q_noise"], x["k"], x["v"], lam0, gate1,
+                          window=window, causal=causal)
+        want = _sdpa(x["q_sig"], x["k"], x["v"], wl.g, window, causal, 1 / math.sqrt(wl.d))
+        _close(got, want.reshape(wl.B * wl.T, -1).numpy(), rtol=1e-10,
+               what=f"GQA W={window} causal={causal}")
+
+
+def pin_differential_matches_sdpa_paths(o):
+    """Full combine against two SDPA calls: O = G*(SDPA_S - lambda*Repeat_g(SDPA_N))."""
+    for window, causal in ((0, True), (7, True), (0, False)):
+        wl, x = _small(T=23, window=window, causal=causal, seed=11)
+        sc = 1 / math.sqrt(wl.d)
+        hs = _sdpa(x["q_sig"], x["k"], x["v"], wl.g, window, causal, sc)
+        hn = _sdpa(x["q_noise"], x["k"], x["v"], 1, window, causal, sc)
+        lam = _f64(x["lam"]).unsqueeze(-1)
+        gate = _f64(x["gate"]).reshape(wl.B, wl.T, wl.Hs, wl.d)
+        want = gate * (hs - lam * hn.repeat_interleave(wl.g, dim=2))
+        got = o.gdla_attn(x["q_sig"], x["q_noise"], x["k"], x["v"], x["lam"], x["gate"],
+                          window=window, causal=causal)
+        _close(got, want.reshape(wl.B * wl.T, -1).numpy(), rtol=1e-10,
+               what=f"GDLA W={window} causal={causal}")
+        got_n = o.attention_path(x["q_noise"], x["k"], x["v"], window=window, causal=causal)
+        _close(got_n, hn.reshape(wl.B * wl.T, wl.Hn, wl.d).numpy(), rtol=1e-10, what="H_N")
+
+
+def pin_rmsnorm_matches_torch(o):
+    """RMSNorm against torch.nn.functional.rms_norm (float64) and a constant row."""
+    g = torch.Generator().manual_seed(5)
+    c = torch.randn(37, 512, generator=g, dtype=torch.float32).to(torch.bfloat16)
+    w = (torch.rand(512, generator=g) + 0.5).to(torch.bfloat16)
+    want = F.rms_norm(_f64(c), (512,), weight=_f64(w), eps=1e-6)
+    _close(o.rmsnorm(c, w, 1e-6), want.numpy(), rtol=1e-12, what="rms_norm")
+    want1 = F.rms_norm(_f64(c), (512,), weight=None, eps=1e-6)
+    _close(o.rmsnorm(c, None, 1e-6), want1.numpy(), rtol=1e-12, what="rms_norm w=1")
+    # a constant row a gives a / sqrt(a^2 + eps) in every position
+    a = 0.0078125
+    const = np.full((2, 512), a)
+    const[1] = -a
+    got = o.rmsnorm(const, None, 1e-6)
+    _close(got[0], np.full(512, a / math.sqrt(a * a + 1e-6)), rtol=1e-13, what="const row")
+    _close(got[1], np.full(512, -a / math.sqrt(a * a + 1e-6)), rtol=1e-13, what="neg row")
+
+
+def pin_expand_matches_matmul(o):
+    """W^KV_b expand against a float64 matmul and the [K_h | V_h] column split."""
+    g = torch.Generator().manual_seed(9)
+    n, dl, hkv, dk = 21, 64, 3, 8
+    c_hat = torch.randn(n, dl, generator=g, dtype=torch.float64)
+    w = torch.randn(dl, hkv * 2 * dk, generator=g, dtype=torch.float32).to(torch.bfloat16)
+    kv = (c_hat @ _f64(w)).reshape(n, hkv, 2 * dk)
+    k, v = o.kv_expand(c_hat.numpy(), w, hkv, dk, dk)
+    _close(k, kv[:, :, :dk].numpy(), rtol=1e-12, what="K")
+    _close(v, kv[:, :, dk:].numpy(), rtol=1e-12, what="V")
+    # one-hot W: latent coordinate l lands in head l // 16, slot l % 16
+    eye = np.zeros((dl, hkv * 2 * dk))
+    for l in range(min(dl, hkv * 2 * dk)):
+        eye[l, l] = 1.0
+    k1, v1 = o.kv_expand(c_hat.numpy(), eye, hkv, dk, dk)
+    for l in range(hkv * 2 * dk):
+        h, x = divmod(l, 2 * dk)
+        val = (k1[:, h, x] if x < dk else v1[:, h, x - dk])
+        _close(val, c_hat[:, l].numpy(), rtol=0, atol=0, what=f"one-hot col {l}")
+
+
+# ---------------------------------------------------------------- identities
+
+def pin_noise_equal_signal_cancels(o):
+    """Q_noise[n] copied into every signal head of group n, lambda=1, G=1: O == 0."""
+    for window, causal in ((0, True), (3, True), (0, False)):
+        wl, x = _small(window=window, causal=causal)
+        qs = x["q_noise"].repeat_interleave(wl.g, dim=2).contiguous()
+        got = o.gdla_attn(qs, x["q_noise"], x["k"], x["v"], torch.ones_like(x["lam"]),
+                          torch.ones_like(x["gate"]), window=window, causal=causal)
+        assert np.all(got == 0.0), f"D=0 identity broken: max |O| = {np.abs(got).max()}"
+
+
+def pin_window_covering_T_is_full(o):
+    """A window of T or more keeps every causal key: identical to full causal."""
+    wl, x = _small(T=17)
+    full = o.gdla_attn(x["q_sig"], x["q_noise"], x["k"], x["v"], x["lam"], x["gate"])
+    for w in (wl.T, wl.T + 5):
+        win = o.gdla_attn(x["q_sig"], x["q_noise"], x["k"], x["v"], x["lam"], x["gate"], window=w)
+        assert np.array_equal(full, win), f"window {w} differs from full causal"
+    short = o.gdla_attn(x["q_sig"], x["q_noise"], x["k"], x["v"], x["lam"], x["gate"],
+                        window=wl.T - 1)
+    assert not np.array_equal(full, short), "window T-1 must drop key 0 of the last row"
+
+
+def pin_gate_is_elementwise(o):
+    """gate=1 gives D itself; any gate G gives exactly G * D."""
+    wl, x = _small()
+    d_only = o.gdla_attn(x["q_sig"], x["q_noise"], x["k"], x["v"], x["lam"],
+                         torch.ones_like(x["gate"]))
+    gated = o.gdla_attn(x["q_sig"], x["q_noise"], x["k"], x["v"], x["lam"], x["gate"])
+    g = _f64(x["gate"]).reshape(wl.B * wl.T, -1).numpy()
+    assert np.array_equal(gated, g * d_only), "O != G * D"
+    assert not np.array_equal(gated, d_only)
+
+
+def pin_linear_in_v(o):
+    """O is linear in V for fixed Q, K, lambda, G."""
+    wl, x = _small(seed=21)
+    g = torch.Generator().manual_seed(22)
+    v2 = torch.randn(x["v"].shape, generator=g, dtype=torch.float64)
+    v1 = _f64(x["v"])
+    args = (x["q_sig"], x["q_noise"], x["k"])
+    o1 = o.gdla_attn(*args, v1, x["lam"], x["gate"])
+    o2 = o.gdla_attn(*args, v2, x["lam"], x["gate"])
+    o12 = o.gdla_attn(*args, v1 + 2.5 * v2, x["lam"], x["gate"])
+    _close(o12, o1 + 2.5 * o2, rtol=1e-12, what="linearity in V")
+
+
+def pin_key_shift_invariance(o):
+    """Adding one vector to every key row of a KV head leaves softmax unchanged."""
+    wl, x = _small(seed=31)
+    g = torch.Generator().manual_seed(32)
+    shift = torch.randn(1, 1, wl.Hkv, wl.d, generator=g, dtype=torch.float64)
+    base = o.gdla_attn(x["q_sig"], x["q_noise"], x["k"], x["v"], x["lam"], x["gate"])
+    moved = o.gdla_attn(x["q_sig"], x["q_noise"], _f64(x["k"]) + shift, x["v"], x["lam"],
+                        x["gate"])
+    _close(moved, base, rtol=1e-10, what="key shift")
+
+
+def pin_causality(o):
+    """Changing keys/values after position i0 leaves rows <= i0 untouched."""
+    wl, x = _small(seed=41)
+    i0 = 9
+    k2, v2 = x["k"].clone(), x["v"].clone()
+    k2[:, i0 + 1:] = -k2[:, i0 + 1:] * 3
+    v2[:, i0 + 1:] = v2[:, i0 + 1:] + 1
+    a = o.gdla_attn(x["q_sig"], x["q_noise"], x["k"], x["v"], x["lam"], x["gate"])
+    b = o.gdla_attn(x["q_sig"], x["q_noise"], k2, v2, x["lam"], x["gate"])
+    a = a.reshape(wl.B, wl.T, -1)
+    b = b.reshape(wl.B, wl.T, -1)
+    assert np.array_equal(a[:, :i0 + 1], b[:, :i0 + 1]), "future keys leaked into the past"
+    assert not np.array_equal(a[:, i0 + 1:], b[:, i0 + 1:])
+
+
+def pin_batch_permutation(o):
+    """Permuting the batch permutes the output rows."""
+    wl, x = _small(B=3, seed=51)
+    perm = torch.tensor([2, 0, 1])
+    a = o.gdla_attn(x["q_sig"], x["q_noise"], x["k"], x["v"], x["lam"], x["gate"])
+    xp = {k: v[perm] for k, v in x.items()}
+    b = o.gdla_attn(xp["q_sig"], xp["q_noise"], xp["k"], xp["v"], xp["lam"], xp["gate"])
+    assert np.array_equal(a.reshape(wl.B, wl.T, -1)[perm.numpy()], b.reshape(wl.B, wl.T, -1))
+
+
+def pin_row_subset(o):
+    """Evaluating a subset of rows gives exactly those rows of the full result."""
+    wl, x = _small(seed=61)
+    full = o.gdla_attn(x["q_sig"], x["q_noise"], x["k"], x["v"], x["lam"], x["gate"])
+    rows = [0, 5, wl.T - 1, wl.T, 2 * wl.T - 1]
+    sub = o.gdla_attn(x["q_sig"], x["q_noise"], x["k"], x["v"], x["lam"], x["gate"], rows=rows)
+    assert np.array_equal(full[rows], sub)
+
+
+def pin_scale_placement(o):
+    """The scale multiplies q.k: doubling q and halving the scale changes nothing."""
+    wl, x = _small(seed=71)
+    sc = 1 / math.sqrt(wl.d)
+    a = o.gdla_attn(x["q_sig"], x["q_noise"], x["k"], x["v"], x["lam"], x["gate"], scale=sc)
+    b = o.gdla_attn(_f64(x["q_sig"]) * 2, _f64(x["q_noise"]) * 2, x["k"], x["v"], x["lam"],
+                    x["gate"], scale=sc / 2)
+    assert np.array_equal(a, b)
+    c = o.gdla_attn(x["q_sig"], x["q_noise"], x["k"], x["v"], x["lam"], x["gate"])
+    assert np.array_equal(a, c), "default scale must be 1/sqrt(d)"
+
+
+ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -1,0 +1,63 @@
+"""Every plausible slip in the oracle must be caught by at least one pin.
+
+Each mutant is a copy of oracle/gdla_oracle.c with one planted mistake (a
+dropped term, a wrong sign, a wrong or transposed index, an off-by-one mask),
+compiled on the CPU into a scratch directory.  The test runs the pins of
+tests/oracle_pins.py against it and requires at least one of them to fail.
+Every mutant keeps all memory accesses in bounds.
+"""
+import os
+
+import pytest
+
+import oracle
+from oracle_pins import ALL_PINS
+
+MUTANTS = {
+    "sign_of_noise_term": ("- l * hn[", "+ l * hn["),
+    "dropped_lambda": ("- l * hn[", "- hn["),
+    "repeat_tiled_not_interleaved": ("const int n = h / g;", "const int n = h % Hn;"),
+    "kv_head_tiled": ("int kvh = h / group;", "int kvh = h % Hkv;"),
+    "window_off_by_one": ("if (window > 0 && i - window + 1 > 0) *lo = i - window + 1;",
+                          "if (window > 0 && i - window > 0) *lo = i - window;"),
+    "causal_excludes_diagonal": ("*hi = i;", "*hi = i > 0 ? i - 1 : 0;"),
+    "dropped_gate": ("= gv * diff;", "= diff;"),
+    "dropped_scale": ("s[j - lo] = scale * dot;", "s[j - lo] = dot;"),
+    "dropped_normaliser": ("o[c] = acc[c] / denom;", "o[c] = acc[c];"),
+    "values_read_from_keys": ("acc[c] += p * load_elem(v, v_dt, voff + c);",
+                              "acc[c] += p * load_elem(k, k_dt, voff + c);"),
+    "gate_index_transposed": ("(int64_t)h * d + c);", "(int64_t)c * Hs + h);"),
+    "lambda_head_reversed": ("load_elem(lam, lam_dt, row * Hs + h);",
+                             "load_elem(lam, lam_dt, row * Hs + (Hs - 1 - h));"),
+    "rms_dropped_eps": ("sqrt(ss / (double)d_latent + eps)", "sqrt(ss / (double)d_latent)"),
+    "rms_sum_not_mean": ("sqrt(ss / (double)d_latent + eps)", "sqrt(ss + eps)"),
+    "expand_w_transposed": ("(int64_t)k * ncol + col)", "col * d_latent + k)"),
+    "expand_k_v_swapped": ("if (x < dk)\n        k_out", "if (x >= dk)\n        k_out"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path):
+    src = open(oracle.SOURCE).read()
+    old, new = MUTANTS[name]
+    assert src.count(old) >= 1, f"mutation anchor for {name} not found"
+    mutated = src.replace(old, new, 1)
+    if name == "expand_k_v_swapped":
+        # keep the store indices in range after swapping the branches
+        mutated = mutated.replace("k_out[(t * n_kv_heads + h) * dk + x] = acc;",
+                                  "k_out[(t * n_kv_heads + h) * dk + (x - dk)] = acc;", 1)
+        mutated = mutated.replace("v_out[(t * n_kv_heads + h) * dv + (x - dk)] = acc;",
+                                  "v_out[(t * n_kv_heads + h) * dv + x] = acc;", 1)
+    path = os.path.join(str(tmp_path), "mutant.c")
+    with open(path, "w") as f:
+        f.write(mutated)
+    lib = oracle.compile_source(path, os.path.join(str(tmp_path), "libmutant.so"))
+    o = oracle.Oracle(lib)
+    caught = []
+    for pin in ALL_PINS:
+        try:
+            pin(o)
+        except AssertionError:
+            caught.append(pin.__name__)
+            break
+    assert caught, f"no pin catches the planted mistake '{name}'"
