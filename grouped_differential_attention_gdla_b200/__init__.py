@@ -1,0 +1,14 @@
+"""B200-native (sm_100a) forward pass of Grouped Differential Latent Attention.
+
+The compute lives in libgdla.so (hand-written tcgen05/TMA CUDA kernels behind a
+C ABI, include/gdla.h); this package is its Python binding.  PyTorch supplies
+device memory and streams only.
+
+    gdla_kv_expand(c_kv, w_kvb, rms_w=None, eps=1e-6) -> (K, V)
+    gdla_attn_fwd(q_sig, q_noise, k, v, lam, gate, window=0, causal=True) -> out
+"""
+from ._binding import (GDLAError, EXPORTED, LIB_PATH, gdla_attn_fwd, gdla_kv_expand,
+                       gdla_status_string, gdla_version, load_library)
+
+__all__ = ["GDLAError", "EXPORTED", "LIB_PATH", "gdla_attn_fwd", "gdla_kv_expand",
+           "gdla_status_string", "gdla_version", "load_library"]

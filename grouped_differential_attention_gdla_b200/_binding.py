@@ -1,0 +1,150 @@
+"""ctypes binding of libgdla.so: argument marshalling only.
+
+Every step of the forward pass runs in the library's CUDA kernels; this module
+checks tensor dtypes, shapes and contiguity, passes raw device pointers, sizes
+and the current CUDA stream, and turns status codes into exceptions.  There is
+no fallback: without the compiled library every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgdla.so")
+
+GDLA_OK = 0
+GDLA_ERR_INVALID_ARG = -1
+GDLA_ERR_UNSUPPORTED = -2
+GDLA_ERR_ALIGNMENT = -3
+GDLA_ERR_CUDA = -4
+GDLA_ERR_TIMEOUT = -5
+
+# every symbol include/gdla.h declares
+EXPORTED = ("gdla_version", "gdla_status_string", "gdla_kv_expand", "gdla_attn_fwd")
+
+_lib = None
+
+
+class GDLAError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {gdla_status_string(code)} (status {code})")
+
+
+def load_library(path: Optional[str] = None) -> ctypes.CDLL:
+    """Load libgdla.so (raises when it has not been built)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError(
+            f"libgdla.so not found at {p}; build it with "
+            "`python -m grouped_differential_attention_gdla_b200.build`")
+    lib = ctypes.CDLL(p)
+    vp, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
+    lib.gdla_version.argtypes = []
+    lib.gdla_version.restype = i32
+    lib.gdla_status_string.argtypes = [i32]
+    lib.gdla_status_string.restype = ctypes.c_char_p
+    lib.gdla_kv_expand.argtypes = [vp, vp, vp, f32, vp, vp, i64, i32, i32, i32, vp, vp]
+    lib.gdla_kv_expand.restype = i32
+    lib.gdla_attn_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32, i64,
+                                  i32, f32, vp, vp]
+    lib.gdla_attn_fwd.restype = i32
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def gdla_version() -> int:
+    return load_library().gdla_version()
+
+
+def gdla_status_string(code: int) -> str:
+    return load_library().gdla_status_string(int(code)).decode()
+
+
+def _check(t: torch.Tensor, name: str, shape=None) -> int:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != torch.bfloat16:
+        raise ValueError(f"{name} must be bfloat16, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    return t.data_ptr()
+
+
+def _stream_ptr(device: torch.device, stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def gdla_kv_expand(c_kv: torch.Tensor, w_kvb: torch.Tensor, rms_w: Optional[torch.Tensor] = None,
+                   eps: float = 1e-6, d_head: int = 128, k_out: Optional[torch.Tensor] = None,
+                   v_out: Optional[torch.Tensor] = None, d_status: Optional[torch.Tensor] = None,
+                   stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """RMSNorm(c_kv) @ W^KV_b split into K, V [N, Hkv, d_head] (bf16, CUDA)."""
+    if c_kv.dim() != 2 or w_kvb.dim() != 2:
+        raise ValueError("c_kv must be [N, d_latent] and w_kvb [d_latent, Hkv*2*d_head]")
+    n, dl = c_kv.shape
+    if w_kvb.shape[0] != dl or w_kvb.shape[1] % (2 * d_head) != 0:
+        raise ValueError("w_kvb must be [d_latent, Hkv*2*d_head]")
+    hkv = w_kvb.shape[1] // (2 * d_head)
+    if k_out is None:
+        k_out = torch.empty((n, hkv, d_head), dtype=torch.bfloat16, device=c_kv.device)
+    if v_out is None:
+        v_out = torch.empty((n, hkv, d_head), dtype=torch.bfloat16, device=c_kv.device)
+    pc = _check(c_kv, "c_kv")
+    pw = _check(w_kvb, "w_kvb")
+    pr = _check(rms_w, "rms_w", (dl,)) if rms_w is not None else None
+    pk = _check(k_out, "k_out", (n, hkv, d_head))
+    pv = _check(v_out, "v_out", (n, hkv, d_head))
+    ps = d_status.data_ptr() if d_status is not None else None
+    rc = load_library().gdla_kv_expand(pc, pr, pw, float(eps), pk, pv, n, dl, hkv, d_head, ps,
+                                       _stream_ptr(c_kv.device, stream))
+    if rc != GDLA_OK:
+        raise GDLAError(rc, "gdla_kv_expand")
+    return k_out, v_out
+
+
+def gdla_attn_fwd(q_sig: torch.Tensor, q_noise: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                  lam: torch.Tensor, gate: torch.Tensor, window: int = 0, causal: bool = True,
+                  scale: float = 0.0, out: Optional[torch.Tensor] = None,
+                  d_status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Fused GDLA attention forward; returns out [B, T, Hs*d] (bf16, CUDA).
+
+    q_sig [B,T,Hs,d], q_noise [B,T,Hn,d], k/v [B,T,Hkv,d], lam [B,T,Hs],
+    gate [B,T,Hs*d].  window 0 = full causal; scale <= 0 means 1/sqrt(d).
+    """
+    if q_sig.dim() != 4:
+        raise ValueError("q_sig must be [B, T, Hs, d]")
+    B, T, Hs, d = q_sig.shape
+    Hn = q_noise.shape[2] if q_noise.dim() == 4 else -1
+    Hkv = k.shape[2] if k.dim() == 4 else -1
+    if out is None:
+        out = torch.empty((B, T, Hs * d), dtype=torch.bfloat16, device=q_sig.device)
+    ptrs = [
+        _check(q_sig, "q_sig"),
+        _check(q_noise, "q_noise", (B, T, Hn, d)),
+        _check(k, "k", (B, T, Hkv, d)),
+        _check(v, "v", (B, T, Hkv, d)),
+        _check(lam, "lam", (B, T, Hs)),
+        _check(gate, "gate", (B, T, Hs * d)),
+        _check(out, "out", (B, T, Hs * d)),
+    ]
+    ps = d_status.data_ptr() if d_status is not None else None
+    rc = load_library().gdla_attn_fwd(*ptrs, B, T, Hs, Hn, Hkv, d, int(window), int(bool(causal)),
+                                      float(scale), ps, _stream_ptr(q_sig.device, stream))
+    if rc != GDLA_OK:
+        raise GDLAError(rc, "gdla_attn_fwd")
+    return out

@@ -1,0 +1,197 @@
+// gdla_api.cu - the C ABI of libgdla.so (declared in include/gdla.h).
+//
+// Host side only: argument validation, TMA tensor-map encoding (driver entry
+// point fetched through the runtime, so the library links no libcuda), and
+// kernel launches on the caller's stream.  The library never allocates,
+// frees or synchronises.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "gdla.h"
+#include "attn_fwd.cuh"
+#include "kv_expand.cuh"
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// Resolved once; immutable afterwards (C++11 guarantees thread-safe init).
+EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Row-major bf16 tensor of `rank` dims given innermost-first; box innermost-first.
+bool make_map(CUtensorMap *map, const void *base, int rank, const uint64_t *dims,
+              const uint32_t *box) {
+  EncodeTiledFn fn = encode_tiled_fn();
+  if (!fn) return false;
+  cuuint64_t gdim[5];
+  cuuint64_t gstride[4];
+  cuuint32_t bdim[5];
+  cuuint32_t estride[5];
+  uint64_t stride = 2;  // bytes
+  for (int i = 0; i < rank; ++i) {
+    gdim[i] = dims[i];
+    bdim[i] = box[i];
+    estride[i] = 1;
+    if (i > 0) gstride[i - 1] = stride;
+    stride *= dims[i];
+  }
+  const CUresult r =
+      fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank),
+         const_cast<void *>(base), gdim, gstride, bdim, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D>
+int launch_attn(const void *q_sig, const void *q_noise, const void *k, const void *v,
+                const gdla::AttnParams &prm, int Hs, int Hn, cudaStream_t stream) {
+  using L = gdla::AttnSmemLayout<D>;
+  CUtensorMap tm_qs, tm_qn, tm_k, tm_v;
+  const uint64_t T = static_cast<uint64_t>(prm.T), B = static_cast<uint64_t>(prm.B);
+  const uint64_t dqs[3] = {static_cast<uint64_t>(Hs) * D, T, B};
+  const uint64_t dqn[3] = {static_cast<uint64_t>(Hn) * D, T, B};
+  const uint32_t qbox[3] = {64, gdla::kBM, 1};
+  const uint32_t kvbox[3] = {64, gdla::kBN, 1};
+  if (!make_map(&tm_qs, q_sig, 3, dqs, qbox) || !make_map(&tm_qn, q_noise, 3, dqn, qbox) ||
+      !make_map(&tm_k, k, 3, dqn, kvbox) || !make_map(&tm_v, v, 3, dqn, kvbox))
+    return GDLA_ERR_CUDA;
+  // at least 116 KB so that one CTA (and one 512-column TMEM allocation) sits on an SM
+  const uint32_t smem = L::kAlloc > 118784u ? L::kAlloc : 118784u;
+  auto kern = gdla::gdla_attn_fwd_kernel<D>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return GDLA_ERR_CUDA;
+  const uint64_t blocks = static_cast<uint64_t>(prm.n_qblk) * B * static_cast<uint64_t>(Hn);
+  if (blocks > 0x7fffffffull) return GDLA_ERR_UNSUPPORTED;
+  kern<<<static_cast<unsigned>(blocks), gdla::kAttnThreads, smem, stream>>>(tm_qs, tm_qn, tm_k,
+                                                                            tm_v, prm);
+  return cudaGetLastError() == cudaSuccess ? GDLA_OK : GDLA_ERR_CUDA;
+}
+
+template <int DH>
+int launch_expand(const void *c_kv, const void *w_kvb, const gdla::ExpandParams &prm,
+                  cudaStream_t stream) {
+  using L = gdla::ExpandSmemLayout<DH>;
+  CUtensorMap tm_c, tm_w;
+  const uint64_t dc[2] = {static_cast<uint64_t>(prm.d_latent), static_cast<uint64_t>(prm.n_tokens)};
+  const uint32_t cbox[2] = {64, gdla::kExpBM};
+  const uint64_t dw[2] = {static_cast<uint64_t>(prm.n_kv_heads) * 2 * DH,
+                          static_cast<uint64_t>(prm.d_latent)};
+  const uint32_t wbox[2] = {64, gdla::kExpKC};
+  if (!make_map(&tm_c, c_kv, 2, dc, cbox) || !make_map(&tm_w, w_kvb, 2, dw, wbox))
+    return GDLA_ERR_CUDA;
+  auto kern = gdla::gdla_kv_expand_kernel<DH>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(L::kAlloc)) != cudaSuccess)
+    return GDLA_ERR_CUDA;
+  const uint64_t blocks = (static_cast<uint64_t>(prm.n_tokens) + gdla::kExpBM - 1) / gdla::kExpBM;
+  if (blocks > 0x7fffffffull) return GDLA_ERR_UNSUPPORTED;
+  kern<<<static_cast<unsigned>(blocks), gdla::kExpThreads, L::kAlloc, stream>>>(tm_c, tm_w, prm);
+  return cudaGetLastError() == cudaSuccess ? GDLA_OK : GDLA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int gdla_version(void) { return 100; /* 0.1.0 */ }
+
+const char *gdla_status_string(int code) {
+  switch (code) {
+    case GDLA_OK: return "ok";
+    case GDLA_ERR_INVALID_ARG: return "invalid argument (null pointer, negative size or bad flag)";
+    case GDLA_ERR_UNSUPPORTED: return "unsupported shape for the sm_100a kernels";
+    case GDLA_ERR_ALIGNMENT: return "a tensor pointer is not 16-byte aligned";
+    case GDLA_ERR_CUDA: return "a CUDA runtime or driver call failed";
+    case GDLA_ERR_TIMEOUT: return "a device-side pipeline wait timed out";
+    default: return "unknown status code";
+  }
+}
+
+int gdla_kv_expand(const void *c_kv, const void *rms_w, const void *w_kvb, float eps,
+                   void *k_out, void *v_out, int64_t n_tokens, int d_latent, int n_kv_heads,
+                   int d_head, int *d_status, void *stream) {
+  if (n_tokens < 0 || d_latent <= 0 || n_kv_heads <= 0 || d_head <= 0) return GDLA_ERR_INVALID_ARG;
+  if (!std::isfinite(eps) || eps < 0.f) return GDLA_ERR_INVALID_ARG;
+  if (n_tokens == 0) return GDLA_OK;
+  if (!c_kv || !w_kvb || !k_out || !v_out) return GDLA_ERR_INVALID_ARG;
+  if (d_latent % 64 != 0 || d_latent > 512) return GDLA_ERR_UNSUPPORTED;
+  if (d_head != 64 && d_head != 128) return GDLA_ERR_UNSUPPORTED;
+  if (n_tokens > 0x7fffffffll) return GDLA_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(n_kv_heads) * 2 * d_head > 0x7fffffffll) return GDLA_ERR_UNSUPPORTED;
+  if (!aligned16(c_kv) || !aligned16(w_kvb) || !aligned16(k_out) || !aligned16(v_out) ||
+      (rms_w && !aligned16(rms_w)))
+    return GDLA_ERR_ALIGNMENT;
+  gdla::ExpandParams prm;
+  prm.rms_w = static_cast<const __nv_bfloat16 *>(rms_w);
+  prm.k_out = static_cast<__nv_bfloat16 *>(k_out);
+  prm.v_out = static_cast<__nv_bfloat16 *>(v_out);
+  prm.status = d_status;
+  prm.n_tokens = n_tokens;
+  prm.d_latent = d_latent;
+  prm.n_kv_heads = n_kv_heads;
+  prm.eps = eps;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return d_head == 128 ? launch_expand<128>(c_kv, w_kvb, prm, s)
+                       : launch_expand<64>(c_kv, w_kvb, prm, s);
+}
+
+int gdla_attn_fwd(const void *q_sig, const void *q_noise, const void *k, const void *v,
+                  const void *lambda, const void *gate, void *out, int B, int64_t T, int Hs,
+                  int Hn, int Hkv, int d, int64_t window, int causal, float scale,
+                  int *d_status, void *stream) {
+  if (B < 0 || T < 0 || Hs <= 0 || Hn <= 0 || Hkv <= 0 || d <= 0) return GDLA_ERR_INVALID_ARG;
+  if (window < 0 || (causal != 0 && causal != 1) || (causal == 0 && window > 0))
+    return GDLA_ERR_INVALID_ARG;
+  if (std::isnan(scale) || std::isinf(scale)) return GDLA_ERR_INVALID_ARG;
+  if (B == 0 || T == 0) return GDLA_OK;
+  if (!q_sig || !q_noise || !k || !v || !lambda || !gate || !out) return GDLA_ERR_INVALID_ARG;
+  if (Hn != Hkv || Hs % Hn != 0) return GDLA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return GDLA_ERR_UNSUPPORTED;
+  if (T > 0x7fffffffll - gdla::kBM) return GDLA_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(Hs) * d > 0x7fffffffll) return GDLA_ERR_UNSUPPORTED;
+  if (!aligned16(q_sig) || !aligned16(q_noise) || !aligned16(k) || !aligned16(v) ||
+      !aligned16(lambda) || !aligned16(gate) || !aligned16(out))
+    return GDLA_ERR_ALIGNMENT;
+  gdla::AttnParams prm;
+  prm.lam = static_cast<const __nv_bfloat16 *>(lambda);
+  prm.gate = static_cast<const __nv_bfloat16 *>(gate);
+  prm.out = static_cast<__nv_bfloat16 *>(out);
+  prm.status = d_status;
+  prm.B = B;
+  prm.T = static_cast<int>(T);
+  prm.Hs = Hs;
+  prm.Hn = Hn;
+  prm.g = Hs / Hn;
+  prm.n_qblk = static_cast<int>((T + gdla::kBM - 1) / gdla::kBM);
+  prm.window = (window >= T) ? 0 : window;  // a window covering every key is full causal
+  prm.causal = causal;
+  const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(d));
+  prm.scale_log2 = sc * 1.4426950408889634f;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return d == 128 ? launch_attn<128>(q_sig, q_noise, k, v, prm, Hs, Hn, s)
+                  : launch_attn<64>(q_sig, q_noise, k, v, prm, Hs, Hn, s);
+}
+
+}  // extern "C"

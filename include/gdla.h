@@ -1,0 +1,123 @@
+/*
+ * gdla.h - C ABI of libgdla.so, the B200 (sm_100a) forward pass of Grouped
+ * Differential Latent Attention (GDLA).
+ *
+ * The operation is the one the page "Motif 3: Technical Report"
+ * (paper.rainbus.top digest), step 2 "GDLA forward", writes out:
+ *
+ *   c_KV,t --RMSNorm--> --W^KV_b--> K_t, V_t           (16 shared KV heads)
+ *   H_S = softmax(Q_sig K^T * scale + mask) V           (signal query heads)
+ *   H_N = softmax(Q_noise K^T * scale + mask) V         (noise query heads)
+ *   D_t = H_S,t - lambda_t (.) Repeat_g(H_N,t)           (g = Hs / Hn)
+ *   O_t = G_t (.) D_t                                    (sigmoid gate, given)
+ *
+ * Head counts 64 signal / 16 noise / 16 shared KV heads and the 1-full : 3
+ * sliding (window 128) schedule come from the same page and from
+ * "Вышла новая модель Motif 3" (pikabu.ru).  Readings of what the pages leave
+ * open, fixed by this ABI:
+ *   - signal head h pairs with noise head h / g and reads KV head h / g;
+ *     noise head n reads KV head n (so Hn must equal Hkv);
+ *   - lambda holds one value per (token, signal head) and, like the gate, is
+ *     passed in after its sigmoid; the library only multiplies;
+ *   - a window W > 0 keeps keys j with i - W < j <= i; W = 0 is full causal;
+ *   - W^KV_b stores the columns of KV head h as [K_h (d_head) | V_h (d_head)].
+ *
+ * Conventions for every entry point:
+ *   - Tensors are dense, row-major and contiguous, bfloat16 unless stated.
+ *     Every pointer must be 16-byte aligned (the kernels move data with TMA
+ *     and 16-byte vector accesses); otherwise GDLA_ERR_ALIGNMENT.
+ *   - Device pointers only (cudaMalloc'd, or memory the GPU can address).
+ *     The caller owns all memory.  The library never allocates, frees or
+ *     synchronises: a call validates its arguments, enqueues its kernel on
+ *     `stream` (a cudaStream_t; NULL is the legacy default stream) and
+ *     returns.  Results are ready when that stream reaches the call.
+ *   - Argument errors are reported before anything is enqueued; in that case
+ *     the call has no effect.
+ *   - d_status (optional, may be NULL): a device int that a kernel sets to
+ *     GDLA_ERR_TIMEOUT if one of its internal pipeline waits gives up (after
+ *     about two seconds); the kernel then stops early and its output is
+ *     undefined.  The library never clears it; the caller zeroes it.
+ *   - The library keeps no mutable global state; calls from several host
+ *     threads are safe.
+ */
+#ifndef GDLA_H_
+#define GDLA_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by every entry point (and written to d_status). */
+#define GDLA_OK 0
+#define GDLA_ERR_INVALID_ARG (-1) /* null pointer, negative size, bad flag  */
+#define GDLA_ERR_UNSUPPORTED (-2) /* valid but not a shape the kernels take */
+#define GDLA_ERR_ALIGNMENT (-3)   /* a pointer is not 16-byte aligned        */
+#define GDLA_ERR_CUDA (-4)        /* a CUDA runtime/driver call failed       */
+#define GDLA_ERR_TIMEOUT (-5)     /* a device-side wait gave up (d_status)   */
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int gdla_version(void);
+
+/* Static, human-readable text for a status code (never NULL). */
+const char *gdla_status_string(int code);
+
+/*
+ * gdla_kv_expand - RMSNorm of the KV latent followed by the W^KV_b
+ * up-projection ("Motif 3: Technical Report", paper.rainbus.top, step 2:
+ * "RMSNorm, then W^KV_b expands 16 KV heads").
+ *
+ *   r_t        = sqrt(mean_k c_kv[t, k]^2 + eps)
+ *   chat[t, k] = c_kv[t, k] / r_t * rms_w[k]          (fp32, rounded to bf16)
+ *   KV[t, :]   = chat[t, :] @ w_kvb                   (fp32 accumulate)
+ *   k_out[t, h, :] = KV[t, h*2*d_head + 0      : h*2*d_head + d_head]
+ *   v_out[t, h, :] = KV[t, h*2*d_head + d_head : (h+1)*2*d_head]
+ *
+ * c_kv   [n_tokens, d_latent]                        bf16, read
+ * rms_w  [d_latent] or NULL (weight of ones)         bf16, read
+ * w_kvb  [d_latent, n_kv_heads * 2 * d_head]         bf16, read
+ * k_out  [n_tokens, n_kv_heads, d_head]              bf16, written
+ * v_out  [n_tokens, n_kv_heads, d_head]              bf16, written
+ * eps    finite, >= 0
+ * Supported: d_latent a multiple of 64 in [64, 512]; d_head 64 or 128;
+ * n_kv_heads >= 1.  n_tokens == 0 is a no-op returning GDLA_OK.
+ * k_out/v_out may not overlap any input.
+ */
+int gdla_kv_expand(const void *c_kv, const void *rms_w, const void *w_kvb,
+                   float eps, void *k_out, void *v_out, int64_t n_tokens,
+                   int d_latent, int n_kv_heads, int d_head, int *d_status,
+                   void *stream);
+
+/*
+ * gdla_attn_fwd - fused GDLA attention forward ("Motif 3: Technical Report",
+ * paper.rainbus.top, step 2): both query paths attend over the shared KV
+ * heads, the noise output is repeated per group, subtracted with the
+ * per-token lambda, and the result is multiplied by the gate.  H_S and H_N
+ * stay on chip.
+ *
+ * q_sig   [B, T, Hs, d]      bf16, read
+ * q_noise [B, T, Hn, d]      bf16, read
+ * k, v    [B, T, Hkv, d]     bf16, read
+ * lambda  [B, T, Hs]         bf16, read (values in [0, 1] expected)
+ * gate    [B, T, Hs * d]     bf16, read
+ * out     [B, T, Hs * d]     bf16, written; must not overlap any input
+ * window  0 = full causal; W > 0 = sliding window (keys i-W < j <= i)
+ * causal  1 = causal mask; 0 = no mask at all (window must then be 0)
+ * scale   softmax scale on q.k; <= 0 selects 1/sqrt(d)
+ *
+ * Supported: Hn == Hkv, Hs % Hn == 0, d in {64, 128}, T < 2^31.
+ * B == 0 or T == 0 is a no-op returning GDLA_OK.
+ * Output rows are computed in fp32 and rounded to bf16 once.
+ */
+int gdla_attn_fwd(const void *q_sig, const void *q_noise, const void *k,
+                  const void *v, const void *lambda, const void *gate,
+                  void *out, int B, int64_t T, int Hs, int Hn, int Hkv, int d,
+                  int64_t window, int causal, float scale, int *d_status,
+                  void *stream);
+
+#ifdef __cplusplus
+} /* extern "C" */
+#endif
+
+#endif /* GDLA_H_ */

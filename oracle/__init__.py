@@ -101,6 +101,10 @@ class Oracle:
         lib.gdla_oracle_attn.argtypes = [vp, i32, vp, i32, vp, i32, vp, i32, vp, i32, vp, i32,
                                          i32, i64, i32, i32, i32, i32, i64, i32, f64, vp, i64, vp]
         lib.gdla_oracle_attn.restype = ctypes.c_int
+        lib.gdla_oracle_attn_compact.argtypes = [vp, i32, vp, i32, vp, i32, vp, i32, vp, i32, vp,
+                                                 i32, i64, i32, i32, i32, i32, i64, i32, f64, vp,
+                                                 i64, vp]
+        lib.gdla_oracle_attn_compact.restype = ctypes.c_int
         lib.gdla_oracle_version.restype = ctypes.c_int
         self.lib = lib
         self.path = lib_path
@@ -200,6 +204,38 @@ class Oracle:
         return out
 
 
+    def gdla_attn_rows(self, q_sig_rows, q_noise_rows, k, v, lam_rows, gate_rows, rows,
+                       window: int = 0, causal: bool = True, scale=None) -> np.ndarray:
+        """Same as gdla_attn, with the query-side inputs gathered per row.
+
+        q_sig_rows [n,Hs,d], q_noise_rows [n,Hn,d], lam_rows [n,Hs] and
+        gate_rows [n,Hs*d] hold only the evaluated rows (flat indices b*T+i in
+        ``rows``, same order); k and v stay full [B,T,Hkv,d].
+        """
+        qs, qsp, qsdt = _arr(q_sig_rows)
+        qn, qnp, qndt = _arr(q_noise_rows)
+        ka, kp, kdt = _arr(k)
+        va, vp, vdt = _arr(v)
+        la, lp, ldt = _arr(lam_rows)
+        ga, gp, gdt = _arr(gate_rows)
+        B, T, Hkv, d = ka.shape
+        n, Hs = qs.shape[0], qs.shape[1]
+        Hn = qn.shape[1]
+        if scale is None:
+            scale = 1.0 / np.sqrt(d)
+        r, rp, nr = _rows(rows, B * T)
+        if nr != n or la.shape[0] != n or ga.shape[0] != n:
+            raise ValueError("row-gathered inputs must have one entry per row")
+        out = np.empty((n, Hs * d), dtype=np.float64)
+        rc = self.lib.gdla_oracle_attn_compact(qsp, qsdt, qnp, qndt, kp, kdt, vp, vdt, lp, ldt, gp,
+                                               gdt, T, Hs, Hn, Hkv, d, int(window),
+                                               int(bool(causal)), float(scale), rp, n,
+                                               out.ctypes.data)
+        if rc != 0:
+            raise ValueError("oracle rejected the head counts (need Hs % Hn == 0, Hn == Hkv)")
+        return out
+
+
 _default = None
 
 
@@ -229,3 +265,7 @@ def differential_gate(*a, **k):
 
 def gdla_attn(*a, **k):
     return default().gdla_attn(*a, **k)
+
+
+def gdla_attn_rows(*a, **k):
+    return default().gdla_attn_rows(*a, **k)

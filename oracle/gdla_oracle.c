@@ -131,14 +131,13 @@ static void key_range(int64_t i, int64_t T, int64_t window, int causal,
  * kv(h) = h / (H / Hkv).  Q is [B,T,H,d], K and V are [B,T,Hkv,d].
  * rows == NULL means every row (n_rows must then be B*T).
  */
-void gdla_oracle_attention_path(const void *q, int q_dt, const void *k,
-                                int k_dt, const void *v, int v_dt, int B,
-                                int64_t T, int H, int Hkv, int d,
+static void attention_path_impl(const void *q, int q_dt, int q_compact,
+                                const void *k, int k_dt, const void *v,
+                                int v_dt, int64_t T, int H, int Hkv, int d,
                                 int64_t window, int causal, double scale,
                                 const int64_t *rows, int64_t n_rows,
                                 double *out) {
   const int group = H / Hkv;
-  (void)B;
   int64_t task;
 #pragma omp parallel
   {
@@ -153,7 +152,7 @@ void gdla_oracle_attention_path(const void *q, int q_dt, const void *k,
       int kvh = h / group;
       int64_t lo, hi;
       key_range(i, T, window, causal, &lo, &hi);
-      const int64_t qoff = (row * H + h) * d;
+      const int64_t qoff = ((q_compact ? ri : row) * H + h) * d;
       double m = -INFINITY;
       for (int64_t j = lo; j <= hi; ++j) {
         const int64_t koff = ((b * T + j) * Hkv + kvh) * d;
@@ -179,6 +178,17 @@ void gdla_oracle_attention_path(const void *q, int q_dt, const void *k,
   }
 }
 
+void gdla_oracle_attention_path(const void *q, int q_dt, const void *k,
+                                int k_dt, const void *v, int v_dt, int B,
+                                int64_t T, int H, int Hkv, int d,
+                                int64_t window, int causal, double scale,
+                                const int64_t *rows, int64_t n_rows,
+                                double *out) {
+  (void)B;
+  attention_path_impl(q, q_dt, 0, k, k_dt, v, v_dt, T, H, Hkv, d, window,
+                      causal, scale, rows, n_rows, out);
+}
+
 /*
  * Differential combine and output gate, [R] step 2:
  *   D[h]  = H_S[h] - lambda[h] * H_N[h / g]          (Repeat_g, interleaved)
@@ -187,16 +197,17 @@ void gdla_oracle_attention_path(const void *q, int q_dt, const void *k,
  * lambda: [B*T, Hs], gate: [B*T, Hs*d], both addressed by the flat row index
  * rows[ri] (rows == NULL: ri itself).  out: [n_rows, Hs*d].
  */
-void gdla_oracle_differential_gate(const double *hs, const double *hn,
+static void differential_gate_impl(const double *hs, const double *hn,
                                    const void *lam, int lam_dt,
-                                   const void *gate, int gate_dt, int Hs,
-                                   int Hn, int d, const int64_t *rows,
-                                   int64_t n_rows, double *out) {
+                                   const void *gate, int gate_dt,
+                                   int lg_compact, int Hs, int Hn, int d,
+                                   const int64_t *rows, int64_t n_rows,
+                                   double *out) {
   const int g = Hs / Hn;
   int64_t ri;
 #pragma omp parallel for schedule(static)
   for (ri = 0; ri < n_rows; ++ri) {
-    const int64_t row = rows ? rows[ri] : ri;
+    const int64_t row = (rows && !lg_compact) ? rows[ri] : ri;
     for (int h = 0; h < Hs; ++h) {
       const double l = load_elem(lam, lam_dt, row * Hs + h);
       const int n = h / g;
@@ -209,17 +220,29 @@ void gdla_oracle_differential_gate(const double *hs, const double *hn,
   }
 }
 
+void gdla_oracle_differential_gate(const double *hs, const double *hn,
+                                   const void *lam, int lam_dt,
+                                   const void *gate, int gate_dt, int Hs,
+                                   int Hn, int d, const int64_t *rows,
+                                   int64_t n_rows, double *out) {
+  differential_gate_impl(hs, hn, lam, lam_dt, gate, gate_dt, 0, Hs, Hn, d,
+                         rows, n_rows, out);
+}
+
 /*
  * Whole GDLA attention forward for a subset of rows: the signal path over
  * Q_sig (Hs heads, KV head h/g), the noise path over Q_noise (Hn heads, KV
  * head n), then the differential combine and the gate.
- * Returns 0, or -1 when the head counts do not divide (Hs % Hn, Hn != Hkv).
+ * compact == 0: q_sig, q_noise, lambda and gate are full [B,T,...] tensors.
+ * compact == 1: they hold only the evaluated rows, in the order of rows[]
+ * (K and V stay full).  Returns 0, or -1 when the head counts do not divide
+ * (Hs % Hn, Hn != Hkv).
  */
-int gdla_oracle_attn(const void *q_sig, int qs_dt, const void *q_noise,
+static int attn_impl(const void *q_sig, int qs_dt, const void *q_noise,
                      int qn_dt, const void *k, int k_dt, const void *v,
                      int v_dt, const void *lam, int lam_dt, const void *gate,
-                     int gate_dt, int B, int64_t T, int Hs, int Hn, int Hkv,
-                     int d, int64_t window, int causal, double scale,
+                     int gate_dt, int compact, int64_t T, int Hs, int Hn,
+                     int Hkv, int d, int64_t window, int causal, double scale,
                      const int64_t *rows, int64_t n_rows, double *out) {
   if (Hn <= 0 || Hkv <= 0 || Hs % Hn != 0 || Hn != Hkv) return -1;
   double *hs = (double *)malloc(sizeof(double) * (size_t)(n_rows * Hs * d));
@@ -229,13 +252,37 @@ int gdla_oracle_attn(const void *q_sig, int qs_dt, const void *q_noise,
     free(hn);
     return -2;
   }
-  gdla_oracle_attention_path(q_sig, qs_dt, k, k_dt, v, v_dt, B, T, Hs, Hkv, d,
-                             window, causal, scale, rows, n_rows, hs);
-  gdla_oracle_attention_path(q_noise, qn_dt, k, k_dt, v, v_dt, B, T, Hn, Hkv,
-                             d, window, causal, scale, rows, n_rows, hn);
-  gdla_oracle_differential_gate(hs, hn, lam, lam_dt, gate, gate_dt, Hs, Hn, d,
-                                rows, n_rows, out);
+  attention_path_impl(q_sig, qs_dt, compact, k, k_dt, v, v_dt, T, Hs, Hkv, d,
+                      window, causal, scale, rows, n_rows, hs);
+  attention_path_impl(q_noise, qn_dt, compact, k, k_dt, v, v_dt, T, Hn, Hkv,
+                      d, window, causal, scale, rows, n_rows, hn);
+  differential_gate_impl(hs, hn, lam, lam_dt, gate, gate_dt, compact, Hs, Hn,
+                         d, rows, n_rows, out);
   free(hs);
   free(hn);
   return 0;
+}
+
+int gdla_oracle_attn(const void *q_sig, int qs_dt, const void *q_noise,
+                     int qn_dt, const void *k, int k_dt, const void *v,
+                     int v_dt, const void *lam, int lam_dt, const void *gate,
+                     int gate_dt, int B, int64_t T, int Hs, int Hn, int Hkv,
+                     int d, int64_t window, int causal, double scale,
+                     const int64_t *rows, int64_t n_rows, double *out) {
+  (void)B;
+  return attn_impl(q_sig, qs_dt, q_noise, qn_dt, k, k_dt, v, v_dt, lam, lam_dt,
+                   gate, gate_dt, 0, T, Hs, Hn, Hkv, d, window, causal, scale,
+                   rows, n_rows, out);
+}
+
+int gdla_oracle_attn_compact(const void *q_sig, int qs_dt, const void *q_noise,
+                             int qn_dt, const void *k, int k_dt, const void *v,
+                             int v_dt, const void *lam, int lam_dt,
+                             const void *gate, int gate_dt, int64_t T, int Hs,
+                             int Hn, int Hkv, int d, int64_t window,
+                             int causal, double scale, const int64_t *rows,
+                             int64_t n_rows, double *out) {
+  return attn_impl(q_sig, qs_dt, q_noise, qn_dt, k, k_dt, v, v_dt, lam, lam_dt,
+                   gate, gate_dt, 1, T, Hs, Hn, Hkv, d, window, causal, scale,
+                   rows, n_rows, out);
 }

@@ -294,6 +294,17 @@ def pin_row_subset(o):
     assert np.array_equal(full[rows], sub)
 
 
+def pin_row_gathered_inputs(o):
+    """The row-gathered form equals the full form at those rows."""
+    wl, x = _small(B=2, T=21, seed=65, window=6)
+    rows = np.array([3, 0, 20, 21, 40, 33])
+    full = o.gdla_attn(x["q_sig"], x["q_noise"], x["k"], x["v"], x["lam"], x["gate"], window=6)
+    flat = lambda t: t.reshape(wl.B * wl.T, *t.shape[2:])[torch.as_tensor(rows)]
+    got = o.gdla_attn_rows(flat(x["q_sig"]), flat(x["q_noise"]), x["k"], x["v"], flat(x["lam"]),
+                           flat(x["gate"]), rows, window=6)
+    assert np.array_equal(full[rows], got)
+
+
 def pin_scale_placement(o):
     """The scale multiplies q.k: doubling q and halving the scale changes nothing."""
     wl, x = _small(seed=71)

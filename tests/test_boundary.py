@@ -1,0 +1,105 @@
+"""The C-ABI library on the host: it loads, exports every entry point that
+include/gdla.h declares, and rejects bad arguments with the documented status
+before touching CUDA (no GPU is needed for any call made here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import grouped_differential_attention_gdla_b200 as gdla
+from grouped_differential_attention_gdla_b200 import _binding
+from grouped_differential_attention_gdla_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdla.h")
+
+OK, INVALID, UNSUPPORTED, ALIGN = 0, -1, -2, -3
+A = 0x100000  # a 16-byte aligned fake device address; never dereferenced here
+M = 0x100008  # misaligned fake address
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return gdla.load_library()
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdla_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = _declared_functions()
+    assert set(declared) == {"gdla_version", "gdla_status_string", "gdla_kv_expand",
+                             "gdla_attn_fwd"}
+    for name in declared:
+        assert hasattr(lib, name), f"{name} missing from libgdla.so"
+    assert set(declared) == set(_binding.EXPORTED)
+
+
+def test_version_and_status_strings(lib):
+    assert gdla.gdla_version() >= 100
+    for code in (0, -1, -2, -3, -4, -5):
+        s = gdla.gdla_status_string(code)
+        assert s and s != "unknown status code"
+    assert gdla.gdla_status_string(7) == "unknown status code"
+
+
+def _attn(lib, q=A, qn=A, k=A, v=A, lam=A, gate=A, out=A, B=1, T=256, Hs=8, Hn=2, Hkv=2, d=64,
+          window=0, causal=1, scale=0.0):
+    return lib.gdla_attn_fwd(q, qn, k, v, lam, gate, out, B, T, Hs, Hn, Hkv, d, window, causal,
+                             ctypes.c_float(scale), None, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), INVALID), (dict(qn=None), INVALID), (dict(k=None), INVALID),
+    (dict(v=None), INVALID), (dict(lam=None), INVALID), (dict(gate=None), INVALID),
+    (dict(out=None), INVALID), (dict(B=-1), INVALID), (dict(T=-5), INVALID),
+    (dict(Hs=0), INVALID), (dict(Hn=0), INVALID), (dict(d=0), INVALID),
+    (dict(window=-1), INVALID), (dict(causal=2), INVALID),
+    (dict(causal=0, window=4), INVALID), (dict(scale=float("nan")), INVALID),
+    (dict(scale=float("inf")), INVALID),
+    (dict(Hs=6, Hn=4, Hkv=4), UNSUPPORTED), (dict(Hn=2, Hkv=4), UNSUPPORTED),
+    (dict(d=32), UNSUPPORTED), (dict(d=96), UNSUPPORTED), (dict(T=2 ** 31), UNSUPPORTED),
+    (dict(q=M), ALIGN), (dict(qn=M), ALIGN), (dict(k=M), ALIGN), (dict(v=M), ALIGN),
+    (dict(lam=M), ALIGN), (dict(gate=M), ALIGN), (dict(out=M), ALIGN),
+    (dict(T=0), OK), (dict(B=0), OK), (dict(T=0, q=None, out=None), OK),
+])
+def test_attn_argument_errors(lib, kw, code):
+    assert _attn(lib, **kw) == code
+
+
+def _expand(lib, c=A, w=None, wk=A, eps=1e-6, k=A, v=A, n=300, dl=512, hkv=16, dh=128):
+    return lib.gdla_kv_expand(c, w, wk, ctypes.c_float(eps), k, v, n, dl, hkv, dh, None, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(c=None), INVALID), (dict(wk=None), INVALID), (dict(k=None), INVALID),
+    (dict(v=None), INVALID), (dict(n=-1), INVALID), (dict(dl=0), INVALID),
+    (dict(hkv=0), INVALID), (dict(dh=0), INVALID), (dict(eps=-1e-6), INVALID),
+    (dict(eps=float("nan")), INVALID), (dict(eps=float("inf")), INVALID),
+    (dict(dl=100), UNSUPPORTED), (dict(dl=576), UNSUPPORTED), (dict(dh=96), UNSUPPORTED),
+    (dict(n=2 ** 31), UNSUPPORTED),
+    (dict(c=M), ALIGN), (dict(wk=M), ALIGN), (dict(k=M), ALIGN), (dict(v=M), ALIGN),
+    (dict(w=M), ALIGN),
+    (dict(n=0), OK), (dict(n=0, c=None), OK),
+])
+def test_expand_argument_errors(lib, kw, code):
+    assert _expand(lib, **kw) == code
+
+
+def test_binding_rejects_host_tensors():
+    import torch
+    x = torch.zeros(1, 4, 2, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        gdla.gdla_attn_fwd(x, x[:, :, :1], x[:, :, :1], x[:, :, :1],
+                           torch.zeros(1, 4, 2, dtype=torch.bfloat16),
+                           torch.zeros(1, 4, 128, dtype=torch.bfloat16))
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(RuntimeError, match="libgdla.so not found"):
+        gdla.load_library(str(tmp_path / "libgdla.so"))
