@@ -214,6 +214,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else if (warp == 9) {
     // =============================== MMA issuer
+    // Per slot X the issue order is S_X(j) .. PV_X(j), S_X(j+1), so that slot
+    // B's MMAs run while slot A's softmax works and vice versa.  S_X(j+1)
+    // overwrites the TMEM columns PV_X(j) reads P from; tcgen05.mma
+    // instructions from one thread execute in issue order, so the read of P
+    // precedes the overwrite.
     if (lane == 0) {
       constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBN, false, false);
       constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, D, false, true);
@@ -221,8 +226,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       uint32_t o_commits[2] = {0, 0};
       uint32_t p_waits[2] = {0, 0};
       uint32_t ofree_waits[2] = {0, 0};
-      uint32_t c = 0;
+      uint32_t c = 0;  // ring position of the next K/V tile to consume
       bool ok = true;
+      auto issue_s = [&](int x, uint32_t k_base) {
+        const uint32_t q_base = sbase + L::kQOff + x * L::kQBytes;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t qoff = (k >> 2) * (kBM * 128) + (k & 3) * 32;
+          const uint32_t koff = (k >> 2) * (kBN * 128) + (k & 3) * 32;
+          umma_ss(t_s(x), sdesc_sw128(q_base + qoff, 16, 1024),
+                  sdesc_sw128(k_base + koff, 16, 1024), kIdescS, k > 0 ? 1u : 0u);
+        }
+        umma_commit(s_full(x));
+      };
       for (int ph = 0; ph < n_phases && ok; ++ph) {
         const int nslot = min(2, n_heads - 2 * ph);
 #pragma unroll
@@ -232,8 +248,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             ++q_uses[x];
           }
         }
-        for (int j = j_lo; j <= j_hi && ok; ++j) {
-          // ---- S_X = Q_X K_j^T
+        if (!ok) break;
+        // prologue: S_X(j_lo)
+        {
           const int sk = static_cast<int>(c % kKvStages);
           ok = mbar_wait(kv_full(sk), (c / kKvStages) & 1u, abort_flag);
           if (!ok) break;
@@ -241,33 +258,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const uint32_t k_base = sbase + L::kKvOff + sk * L::kKvBytes;
 #pragma unroll
           for (int x = 0; x < 2; ++x) {
-            if (x >= nslot || !ok) break;
-            // the previous PV of this slot reads P from the S columns: let it finish
-            if (o_commits[x] > 0) {
-              ok = mbar_wait(o_done(x), (o_commits[x] - 1) & 1u, abort_flag);
-              if (!ok) break;
-              tc_fence_after();
+            if (x < nslot) {
+              issue_s(x, k_base);
+              if (j_lo == j_hi) umma_commit(q_empty(x));
             }
-            const uint32_t q_base = sbase + L::kQOff + x * L::kQBytes;
-#pragma unroll
-            for (int k = 0; k < D / 16; ++k) {
-              const uint32_t koff = (k >> 2) * (kBM * 128) + (k & 3) * 32;
-              const uint32_t kkoff = (k >> 2) * (kBN * 128) + (k & 3) * 32;
-              umma_ss(t_s(x), sdesc_sw128(q_base + koff, 16, 1024),
-                      sdesc_sw128(k_base + kkoff, 16, 1024), kIdescS, k > 0 ? 1u : 0u);
-            }
-            umma_commit(s_full(x));
-            if (j == j_hi) umma_commit(q_empty(x));
           }
-          if (!ok) break;
           umma_commit(kv_empty(sk));
           ++c;
-          // ---- O_X += P_X V_j
+        }
+        for (int j = j_lo; j <= j_hi && ok; ++j) {
           const int sv = static_cast<int>(c % kKvStages);
           ok = mbar_wait(kv_full(sv), (c / kKvStages) & 1u, abort_flag);
           if (!ok) break;
           tc_fence_after();
+          ++c;
           const uint32_t v_base = sbase + L::kKvOff + sv * L::kKvBytes;
+          int sk = 0;
+          uint32_t k_base = 0;
 #pragma unroll
           for (int x = 0; x < 2; ++x) {
             if (x >= nslot || !ok) break;
@@ -289,10 +296,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
             umma_commit(o_done(x));
             ++o_commits[x];
+            if (j < j_hi) {
+              if (x == 0) {
+                sk = static_cast<int>(c % kKvStages);
+                ok = mbar_wait(kv_full(sk), (c / kKvStages) & 1u, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                k_base = sbase + L::kKvOff + sk * L::kKvBytes;
+              }
+              issue_s(x, k_base);
+              if (j + 1 == j_hi) umma_commit(q_empty(x));
+            }
           }
           if (!ok) break;
           umma_commit(kv_empty(sv));
-          ++c;
+          if (j < j_hi) {
+            umma_commit(kv_empty(sk));
+            ++c;
+          }
         }
       }
       // drain: every MMA issued above must finish before TMEM is released
@@ -333,17 +354,40 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           c_hi = p.T - 1 - kbase;
           c_lo = -1;
         }
-        // pass 1: masked row max over the tile (32 columns live at a time)
-        float mt = -INFINITY;
+        // CTA-uniform: does any row of the block lose a key of this tile?
+        bool masked;
+        if (p.causal) {
+          masked = (kbase + kBN - 1 > q0) ||
+                   (p.window > 0 && static_cast<int64_t>(kbase) <= q0 + kBM - 1 - p.window);
+        } else {
+          masked = kbase + kBN > p.T;
+        }
+        // pass 1: row max of the tile (32 columns live at a time)
+        float mt;
+        if (!masked) {
+          float ma = -INFINITY, mb = -INFINITY;
 #pragma unroll
-        for (int cc = 0; cc < kBN / 32; ++cc) {
-          uint32_t raw[32];
-          tmem_ld32(t_s(x) + lane_off + cc * 32, raw);
-          tmem_wait_ld();
+          for (int cc = 0; cc < kBN / 32; cc += 2) {
+            uint32_t r0[32], r1[32];
+            tmem_ld32x2_sync(t_s(x) + lane_off + cc * 32, t_s(x) + lane_off + cc * 32 + 32, r0, r1);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int c = cc * 32 + e;
-            if (c >= c_lo && c <= c_hi) mt = fmaxf(mt, __uint_as_float(raw[e]));
+            for (int e = 0; e < 32; e += 2) {
+              ma = fmax3(ma, __uint_as_float(r0[e]), __uint_as_float(r0[e + 1]));
+              mb = fmax3(mb, __uint_as_float(r1[e]), __uint_as_float(r1[e + 1]));
+            }
+          }
+          mt = fmaxf(ma, mb);
+        } else {
+          mt = -INFINITY;
+#pragma unroll
+          for (int cc = 0; cc < kBN / 32; ++cc) {
+            uint32_t raw[32];
+            tmem_ld32_sync(t_s(x) + lane_off + cc * 32, raw);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int c = cc * 32 + e;
+              if (c >= c_lo && c <= c_hi) mt = fmaxf(mt, __uint_as_float(raw[e]));
+            }
           }
         }
         mt = mt * sl2;  // scale > 0 keeps the arg max
@@ -357,26 +401,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const float m_safe = (m_use == -INFINITY) ? 0.f : m_use;
         // pass 2: P = exp2(S*c - m) as bf16 pairs.  The P columns of chunk cc
         // ([16cc, 16cc+16)) lie below the S columns still to be read.
-        float rs = 0.f;
+        const uint64_t sl2x2 = f2_make(sl2, sl2);
+        const uint64_t negm2 = f2_make(-m_safe, -m_safe);
+        uint64_t rs2 = f2_make(0.f, 0.f);
 #pragma unroll
         for (int cc = 0; cc < kBN / 32; ++cc) {
           uint32_t raw[32];
-          tmem_ld32(t_s(x) + lane_off + cc * 32, raw);
-          tmem_wait_ld();
+          tmem_ld32_sync(t_s(x) + lane_off + cc * 32, raw);
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const int c0 = cc * 32 + 2 * e;
-            const float s0 = (c0 >= c_lo && c0 <= c_hi) ? __uint_as_float(raw[2 * e]) * sl2 : -INFINITY;
-            const float s1 =
-                (c0 + 1 >= c_lo && c0 + 1 <= c_hi) ? __uint_as_float(raw[2 * e + 1]) * sl2 : -INFINITY;
-            const float p0 = ex2_approx(s0 - m_safe);
-            const float p1 = ex2_approx(s1 - m_safe);
-            rs += p0 + p1;
+            float t0, t1;
+            f2_split(f2_fma(f2_from_bits(raw[2 * e], raw[2 * e + 1]), sl2x2, negm2), t0, t1);
+            if (masked) {
+              const int c0 = cc * 32 + 2 * e;
+              if (!(c0 >= c_lo && c0 <= c_hi)) t0 = -INFINITY;
+              if (!(c0 + 1 >= c_lo && c0 + 1 <= c_hi)) t1 = -INFINITY;
+            }
+            const float p0 = ex2_approx(t0);
+            const float p1 = ex2_approx(t1);
+            rs2 = f2_add(rs2, f2_make(p0, p1));
             pk[e] = pack_bf16x2(p0, p1);
           }
           tmem_st16(t_s(x) + lane_off + cc * 16, pk);
         }
+        float rs0, rs1;
+        f2_split(rs2, rs0, rs1);
+        const float rs = rs0 + rs1;
         l_run = l_run * alpha + rs;
         m_run = m_use;
         // O holds the sum over earlier tiles; rescale it when the max moved
@@ -390,8 +441,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
           for (int cc = 0; cc < D / 32; ++cc) {
             uint32_t o[32];
-            tmem_ld32(t_o(x) + lane_off + cc * 32, o);
-            tmem_wait_ld();
+            tmem_ld32_sync(t_o(x) + lane_off + cc * 32, o);
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
             tmem_st32(t_o(x) + lane_off + cc * 32, o);
@@ -415,8 +465,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32];
-          tmem_ld32(t_o(x) + lane_off + cc * 32, o);
-          tmem_wait_ld();
+          tmem_ld32_sync(t_o(x) + lane_off + cc * 32, o);
 #pragma unroll
           for (int e = 0; e < 32; ++e) hn_smem[(cc * 32 + e) * kBM + r] = __uint_as_float(o[e]) * inv_l;
         }
@@ -441,8 +490,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32];
-          tmem_ld32(t_o(x) + lane_off + cc * 32, o);
-          tmem_wait_ld();
+          tmem_ld32_sync(t_o(x) + lane_off + cc * 32, o);
           if (row_ok) {
             const uint4 *gp = reinterpret_cast<const uint4 *>(p.gate + goff + cc * 32);
             uint4 *op = reinterpret_cast<uint4 *>(p.out + goff + cc * 32);

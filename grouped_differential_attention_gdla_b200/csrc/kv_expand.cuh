@@ -235,8 +235,7 @@ __global__ void __launch_bounds__(kExpThreads, 1)
 #pragma unroll
         for (int cc = 0; cc < NT / 32; ++cc) {
           uint32_t a[32];
-          tmem_ld32(acc + cc * 32, a);
-          tmem_wait_ld();
+          tmem_ld32_sync(acc + cc * 32, a);
           if (t < p.n_tokens) {
             const bool is_v = cc * 32 >= DH;
             const int col = cc * 32 - (is_v ? DH : 0);
