@@ -5,18 +5,22 @@
 // h = g*k .. g*k+g-1 attend over the shared KV head k;
 //   D[h] = H_S[h] - lambda[h] * H_N[h / g],   O[h] = G[h] * D[h].
 //
-// One CTA owns one (batch b, KV group k, block of 128 query tokens).  It runs
-// the g+1 heads of the group in phases of two "slots" (A, B): phase 0 is
-// (noise, signal 0), then (signal 1, signal 2), ...  Both slots of a phase
-// share the same query rows and therefore every K/V tile the TMA warp brings
-// into shared memory.  Per KV tile of 128 keys:
+// One CTA owns one (batch b, KV group k, block of 128 query tokens) and runs
+// the group's g+1 heads (noise first) in phases of two "slots" A and B.  In a
+// normal phase the slots hold two heads over the same query rows, so every
+// K/V tile the TMA warp stages in shared memory serves both.  When the head
+// count is odd the last head runs as a split phase: both slots take the same
+// head, slot A the even and slot B the odd K/V tiles, and the two partial
+// softmax states (m, l, O) are merged in the epilogue.  Per K/V tile:
 //   S_X  = Q_X K^T          tcgen05.mma, A = Q (smem), B = K (smem), D = TMEM
-//   P_X  = exp2(S_X*c - m)  softmax warpgroup X: tcgen05.ld, online max/sum,
-//                           bf16 P written back over S_X with tcgen05.st
+//   P_X  = exp2(S_X*c - m)  softmax warpgroup X (one thread per row):
+//                           tcgen05.ld, row max, bf16 P written over S_X
 //   O_X += P_X V            tcgen05.mma, A = P (TMEM), B = V (smem)
-// The noise head's normalised output H_N goes to shared memory (fp32) and is
+// The running max m is kept integral (log2 units), so P's bf16 rounding does
+// not depend on which tiles a slot has seen and the split merge is exact.
+// The noise head's normalised output H_N stays in shared memory (fp32) and is
 // subtracted in the epilogue of every signal head of the group; neither H_S
-// nor H_N is written to global memory.
+// nor H_N reaches global memory.
 //
 // Warp roles (320 threads):
 //   warps 0-3  softmax + epilogue for slot A (TMEM lanes 0..127)
@@ -24,7 +28,7 @@
 //   warp  8    TMA producer (Q tiles, K/V ring)
 //   warp  9    TMEM allocator and single-thread MMA issuer
 //
-// TMEM (512 columns): S_A [0,128) S_B [128,256) O_A [256,256+d) O_B [256+d, 256+2d).
+// TMEM (512 columns): S_A [0,128) S_B [128,256) O_A [256,256+d) O_B [256+d,256+2d).
 // P_X occupies the first 64 columns of S_X as packed bf16 pairs.
 #pragma once
 
@@ -32,11 +36,18 @@
 
 namespace gdla {
 
-constexpr int kBM = 128;          // query rows per slot
-constexpr int kBN = 128;          // keys per K/V tile
-constexpr int kKvStages = 3;      // K/V ring depth (tiles)
-constexpr int kAttnThreads = 320;
+constexpr int kBM = 128;      // query rows per slot
+constexpr int kBN = 128;      // keys per K/V tile
+constexpr int kKvStages = 3;  // K/V ring depth (tiles)
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kAttnThreads = 10 * 32;
+constexpr int kSlotThreads = 128;          // one warpgroup per slot
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: O is rescaled only if the max grows by > 2^8
+// Of every 16 score pairs in a 32-column chunk of an unmasked tile, this many
+// take 2^x from the FMA-pipe polynomial instead of the MUFU ex2 unit, which
+// would otherwise cap the softmax at one exponential per MMA-consumed score.
+constexpr int kPolyPairs = 0;
 
 struct AttnParams {
   const __nv_bfloat16 *lam;   // [B, T, Hs]
@@ -63,18 +74,42 @@ struct AttnSmemLayout {
   static constexpr uint32_t kKvOff = kQOff + 2 * kQBytes;
   static constexpr uint32_t kHnOff = kKvOff + kKvStages * kKvBytes;
   static constexpr uint32_t kBarOff = kHnOff + kHnBytes;
-  // barriers: q_full[2] q_empty[2] kv_full[S] kv_empty[S] s_full[2] p_full[2]
-  //           o_done[2] o_free[2] hn_ready
-  static constexpr uint32_t kNumBars = 2 + 2 + 2 * kKvStages + 2 + 2 + 2 + 2 + 1;
+  // q_full[2] q_empty[2] kv_full[S] kv_empty[S] s_full[2] p_full[2] o_done[2]
+  // o_free[2] hn_ready split_ready
+  static constexpr uint32_t kNumBars = 2 + 2 + 2 * kKvStages + 2 + 2 + 2 + 2 + 2;
   static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;
   static constexpr uint32_t kBytes = kMiscOff + 16;
-  static constexpr uint32_t kAlloc = kBytes + 1024;  // slack to align the base to 1024
 };
 
-// Key window of query row i inside tile j: columns [c_lo, c_hi] are kept.
-struct RowMask {
-  int c_lo, c_hi;
+// Which heads the two slots run in phase `ph` (head index 0 = noise,
+// i >= 1 = signal head i-1 of the group).
+struct PhasePlan {
+  int nslot;   // active slots
+  bool split;  // both slots run head0 on alternating K/V tiles
+  int head0, head1;
 };
+
+__device__ __forceinline__ PhasePlan phase_plan(int ph, int n_heads, int n_tiles) {
+  PhasePlan pl;
+  const int first = 2 * ph;
+  if (first + 1 < n_heads) {
+    pl.nslot = 2;
+    pl.split = false;
+    pl.head0 = first;
+    pl.head1 = first + 1;
+  } else if (n_tiles >= 2) {
+    pl.nslot = 2;
+    pl.split = true;
+    pl.head0 = first;
+    pl.head1 = first;
+  } else {
+    pl.nslot = 1;
+    pl.split = false;
+    pl.head0 = first;
+    pl.head1 = -1;
+  }
+  return pl;
+}
 
 __device__ __forceinline__ void write_status(int *status, int code) {
   if (status) atomicExch(status, code);
@@ -87,9 +122,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                          const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   using L = AttnSmemLayout<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                              ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t smem[];
+  // swizzled TMA/UMMA tiles need a 1024-byte aligned base; refuse to run otherwise
+  if ((smem_u32(smem) & 1023u) != 0) {
+    if (threadIdx.x == 0) write_status(p.status, -4 /* GDLA_ERR_CUDA */);
+    return;
+  }
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + L::kBarOff;
   auto q_full = [&](int x) { return bar0 + 8u * (0 + x); };
@@ -101,6 +139,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   auto o_done = [&](int x) { return bar0 + 8u * (8 + 2 * kKvStages + x); };
   auto o_free = [&](int x) { return bar0 + 8u * (10 + 2 * kKvStages + x); };
   const uint32_t hn_ready = bar0 + 8u * (12 + 2 * kKvStages);
+  const uint32_t split_ready = bar0 + 8u * (13 + 2 * kKvStages);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
   float *hn_smem = reinterpret_cast<float *>(smem + L::kHnOff);  // [D][kBM]
@@ -129,27 +168,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     j_hi = (p.T - 1) / kBN;
   }
   const int n_tiles = j_hi - j_lo + 1;
-  const int n_heads = p.g + 1;               // noise head + g signal heads
+  const int n_heads = p.g + 1;  // noise head + g signal heads
   const int n_phases = (n_heads + 1) / 2;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(q_full(i), 1);
-      mbar_init(q_empty(i), 1);
-      mbar_init(s_full(i), 1);
-      mbar_init(p_full(i), kBM);
-      mbar_init(o_done(i), 1);
-      mbar_init(o_free(i), kBM);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(q_full(s), 1);
+      mbar_init(q_empty(s), 1);
+      mbar_init(s_full(s), 1);
+      mbar_init(p_full(s), kSlotThreads);
+      mbar_init(o_done(s), 1);
+      mbar_init(o_free(s), kSlotThreads);
     }
     for (int s = 0; s < kKvStages; ++s) {
       mbar_init(kv_full(s), 1);
       mbar_init(kv_empty(s), 1);
     }
-    mbar_init(hn_ready, kBM);
+    mbar_init(hn_ready, kSlotThreads);
+    mbar_init(split_ready, kSlotThreads);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
@@ -159,9 +199,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t tmem = *tmem_slot;
   auto t_s = [&](int x) { return tmem + 128u * static_cast<uint32_t>(x); };
   auto t_o = [&](int x) { return tmem + 256u + static_cast<uint32_t>(D * x); };
+  // TMEM column (relative to S_X) of the packed P for keys 16k .. 16k+15
+  auto p_col = [](int k) -> uint32_t { return 8u * k; };
 
-  if (warp == 8) {
+  if (warp == kProducerWarp) {
     // =============================== TMA producer
+    // Ring order per phase: K_0 .. K_{A-1}, then V_t, K_{t+A} for t = 0..n-1,
+    // where A = 1 (normal phase) or 2 (split phase) is how far ahead of the
+    // values the MMA warp consumes keys.
     if (lane == 0) {
       tma_prefetch_desc(&tm_qs);
       tma_prefetch_desc(&tm_qn);
@@ -170,36 +215,43 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       uint32_t q_uses[2] = {0, 0};
       uint32_t c = 0;  // K/V ring position
       bool ok = true;
+      auto load_kv = [&](int t, bool is_v) {
+        const int s = static_cast<int>(c % kKvStages);
+        ok = mbar_wait(kv_empty(s), ((c / kKvStages) & 1u) ^ 1u, abort_flag);
+        if (!ok) return;
+        const uint32_t dst = sbase + L::kKvOff + s * L::kKvBytes;
+        mbar_arrive_expect_tx(kv_full(s), L::kKvBytes);
+        const CUtensorMap *map = is_v ? &tm_v : &tm_k;
+#pragma unroll
+        for (int kb = 0; kb < D / 64; ++kb)
+          tma_load_3d(dst + kb * (kBN * 128), map, kv_full(s), kvh * D + kb * 64,
+                      (j_lo + t) * kBN, b);
+        ++c;
+      };
       for (int ph = 0; ph < n_phases && ok; ++ph) {
+        const PhasePlan pl = phase_plan(ph, n_heads, n_tiles);
+        const int nq = pl.split ? 1 : pl.nslot;
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
-          const int hi = 2 * ph + x;
-          if (hi >= n_heads || !ok) break;
+          if (x >= nq || !ok) break;
           ok = mbar_wait(q_empty(x), (q_uses[x] & 1u) ^ 1u, abort_flag);
           if (!ok) break;
           ++q_uses[x];
+          const int hi = x == 0 ? pl.head0 : pl.head1;
           const uint32_t dst = sbase + L::kQOff + x * L::kQBytes;
           mbar_arrive_expect_tx(q_full(x), L::kQBytes);
-          const bool noise = (hi == 0);
+          const bool noise = hi == 0;
           const int head = noise ? kvh : p.g * kvh + (hi - 1);
           const CUtensorMap *map = noise ? &tm_qn : &tm_qs;
 #pragma unroll
           for (int kb = 0; kb < D / 64; ++kb)
             tma_load_3d(dst + kb * (kBM * 128), map, q_full(x), head * D + kb * 64, q0, b);
         }
-        for (int j = j_lo; j <= j_hi && ok; ++j) {
-          for (int kv = 0; kv < 2 && ok; ++kv) {
-            const int s = static_cast<int>(c % kKvStages);
-            ok = mbar_wait(kv_empty(s), ((c / kKvStages) & 1u) ^ 1u, abort_flag);
-            if (!ok) break;
-            const uint32_t dst = sbase + L::kKvOff + s * L::kKvBytes;
-            mbar_arrive_expect_tx(kv_full(s), L::kKvBytes);
-            const CUtensorMap *map = kv == 0 ? &tm_k : &tm_v;
-#pragma unroll
-            for (int kb = 0; kb < D / 64; ++kb)
-              tma_load_3d(dst + kb * (kBN * 128), map, kv_full(s), kvh * D + kb * 64, j * kBN, b);
-            ++c;
-          }
+        const int ahead = pl.split ? 2 : 1;
+        for (int t = 0; t < ahead && t < n_tiles && ok; ++t) load_kv(t, false);
+        for (int t = 0; t < n_tiles && ok; ++t) {
+          load_kv(t, true);
+          if (ok && t + ahead < n_tiles) load_kv(t + ahead, false);
         }
       }
       if (!ok) {
@@ -212,24 +264,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (q_uses[x]) mbar_wait_for(q_full(x), (q_uses[x] - 1) & 1u, 100000000ull);
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == kMmaWarp) {
     // =============================== MMA issuer
-    // Per slot X the issue order is S_X(j) .. PV_X(j), S_X(j+1), so that slot
-    // B's MMAs run while slot A's softmax works and vice versa.  S_X(j+1)
-    // overwrites the TMEM columns PV_X(j) reads P from; tcgen05.mma
-    // instructions from one thread execute in issue order, so the read of P
+    // Per slot X the issue order is S_X(t) .. PV_X(t), S_X(t+A): slot B's
+    // MMAs run while slot A's softmax works and vice versa.  S_X(t+A)
+    // overwrites the TMEM columns PV_X(t) reads P from; tcgen05.mma
+    // instructions of one thread execute in issue order, so the read of P
     // precedes the overwrite.
     if (lane == 0) {
       constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBN, false, false);
       constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, D, false, true);
       uint32_t q_uses[2] = {0, 0};
-      uint32_t o_commits[2] = {0, 0};
       uint32_t p_waits[2] = {0, 0};
       uint32_t ofree_waits[2] = {0, 0};
+      uint32_t o_commits[2] = {0, 0};
       uint32_t c = 0;  // ring position of the next K/V tile to consume
       bool ok = true;
-      auto issue_s = [&](int x, uint32_t k_base) {
-        const uint32_t q_base = sbase + L::kQOff + x * L::kQBytes;
+      auto issue_s = [&](int x, int qbuf, uint32_t k_base) {
+        const uint32_t q_base = sbase + L::kQOff + qbuf * L::kQBytes;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t qoff = (k >> 2) * (kBM * 128) + (k & 3) * 32;
@@ -239,49 +291,68 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         umma_commit(s_full(x));
       };
+      // waits for the next ring entry; returns its stage and smem address
+      auto next_stage = [&](uint32_t &base) -> int {
+        const int s = static_cast<int>(c % kKvStages);
+        ok = mbar_wait(kv_full(s), (c / kKvStages) & 1u, abort_flag);
+        tc_fence_after();
+        base = sbase + L::kKvOff + s * L::kKvBytes;
+        ++c;
+        return s;
+      };
       for (int ph = 0; ph < n_phases && ok; ++ph) {
-        const int nslot = min(2, n_heads - 2 * ph);
+        const PhasePlan pl = phase_plan(ph, n_heads, n_tiles);
+        const int nq = pl.split ? 1 : pl.nslot;
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
-          if (x < nslot && ok) {
+          if (x < nq && ok) {
             ok = mbar_wait(q_full(x), q_uses[x] & 1u, abort_flag);
             ++q_uses[x];
           }
         }
         if (!ok) break;
-        // prologue: S_X(j_lo)
-        {
-          const int sk = static_cast<int>(c % kKvStages);
-          ok = mbar_wait(kv_full(sk), (c / kKvStages) & 1u, abort_flag);
+        const int ahead = pl.split ? 2 : 1;
+        // prologue: the first S of every slot
+        if (!pl.split) {
+          uint32_t kb;
+          const int s = next_stage(kb);
           if (!ok) break;
-          tc_fence_after();
-          const uint32_t k_base = sbase + L::kKvOff + sk * L::kKvBytes;
 #pragma unroll
           for (int x = 0; x < 2; ++x) {
-            if (x < nslot) {
-              issue_s(x, k_base);
-              if (j_lo == j_hi) umma_commit(q_empty(x));
+            if (x < pl.nslot) {
+              issue_s(x, x, kb);
+              if (n_tiles == 1) umma_commit(q_empty(x));
             }
           }
-          umma_commit(kv_empty(sk));
-          ++c;
-        }
-        for (int j = j_lo; j <= j_hi && ok; ++j) {
-          const int sv = static_cast<int>(c % kKvStages);
-          ok = mbar_wait(kv_full(sv), (c / kKvStages) & 1u, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-          ++c;
-          const uint32_t v_base = sbase + L::kKvOff + sv * L::kKvBytes;
-          int sk = 0;
-          uint32_t k_base = 0;
+          umma_commit(kv_empty(s));
+        } else {
 #pragma unroll
           for (int x = 0; x < 2; ++x) {
-            if (x >= nslot || !ok) break;
+            uint32_t kb;
+            const int s = next_stage(kb);
+            if (!ok) break;
+            issue_s(x, 0, kb);
+            if (x == 1 && n_tiles == 2) umma_commit(q_empty(0));
+            umma_commit(kv_empty(s));
+          }
+          if (!ok) break;
+        }
+        for (int t = 0; t < n_tiles && ok; ++t) {
+          uint32_t vb;
+          const int sv = next_stage(vb);
+          if (!ok) break;
+          int sk = -1;
+          uint32_t kb = 0;
+#pragma unroll
+          for (int xx = 0; xx < 2; ++xx) {
+            if (pl.split && xx == 1) break;
+            const int x = pl.split ? (t & 1) : xx;
+            if (x >= pl.nslot || !ok) break;
             ok = mbar_wait(p_full(x), p_waits[x] & 1u, abort_flag);
             if (!ok) break;
             ++p_waits[x];
-            if (j == j_lo && ph > 0) {
+            const bool first_pv = pl.split ? (t == x) : (t == 0);
+            if (first_pv && ph > 0) {
               // the previous phase's epilogue must have read O_X
               ok = mbar_wait(o_free(x), ofree_waits[x] & 1u, abort_flag);
               if (!ok) break;
@@ -290,30 +361,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tc_fence_after();
 #pragma unroll
             for (int k = 0; k < kBN / 16; ++k) {
-              umma_ts(t_o(x), t_s(x) + 8u * k,
-                      sdesc_sw128(v_base + k * (16 * 128), kBN * 128, 1024), kIdescPV,
-                      (j > j_lo || k > 0) ? 1u : 0u);
+              umma_ts(t_o(x), t_s(x) + p_col(k),
+                      sdesc_sw128(vb + k * (16 * 128), kBN * 128, 1024), kIdescPV,
+                      (!first_pv || k > 0) ? 1u : 0u);
             }
             umma_commit(o_done(x));
             ++o_commits[x];
-            if (j < j_hi) {
-              if (x == 0) {
-                sk = static_cast<int>(c % kKvStages);
-                ok = mbar_wait(kv_full(sk), (c / kKvStages) & 1u, abort_flag);
+            const int tn = t + ahead;
+            if (tn < n_tiles) {
+              if (sk < 0) {
+                sk = next_stage(kb);
                 if (!ok) break;
-                tc_fence_after();
-                k_base = sbase + L::kKvOff + sk * L::kKvBytes;
               }
-              issue_s(x, k_base);
-              if (j + 1 == j_hi) umma_commit(q_empty(x));
+              issue_s(x, pl.split ? 0 : x, kb);
+              if (tn == n_tiles - 1) umma_commit(q_empty(pl.split ? 0 : x));
             }
           }
           if (!ok) break;
           umma_commit(kv_empty(sv));
-          if (j < j_hi) {
-            umma_commit(kv_empty(sk));
-            ++c;
-          }
+          if (sk >= 0) umma_commit(kv_empty(sk));
         }
       }
       // drain: every MMA issued above must finish before TMEM is released
@@ -322,11 +388,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (o_commits[x]) mbar_wait_for(o_done(x), (o_commits[x] - 1) & 1u, 100000000ull);
     }
   } else {
-    // =============================== softmax + epilogue (slot = warpgroup)
-    const int x = warp >> 2;        // slot
-    const int wq = warp & 3;        // TMEM lane quarter
+    // =============================== softmax + epilogue (one warpgroup per slot)
+    const int x = warp >> 2;          // slot
+    const int wq = warp & 3;          // TMEM lane quarter
     const int r = threadIdx.x & 127;  // row in the block = TMEM lane
-    const int i = q0 + r;           // query token
+    const int i = q0 + r;             // query token
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const float sl2 = p.scale_log2;
     uint32_t s_waits = 0;
@@ -334,17 +400,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     bool hn_waited = false;
     bool ok = true;
     for (int ph = 0; ph < n_phases && ok; ++ph) {
-      const int hi = 2 * ph + x;
-      if (hi >= n_heads) break;
+      const PhasePlan pl = phase_plan(ph, n_heads, n_tiles);
+      if (x >= pl.nslot) break;
+      const int hi = x == 0 ? pl.head0 : pl.head1;
+      const int t0 = pl.split ? x : 0;
+      const int step = pl.split ? 2 : 1;
+      const int my_tiles = pl.split ? (n_tiles - x + 1) / 2 : n_tiles;
       float m_run = -INFINITY, l_run = 0.f;
-      for (int j = j_lo; j <= j_hi; ++j) {
+      int k_idx = 0;
+      for (int t = t0; t < n_tiles; t += step, ++k_idx) {
         ok = mbar_wait(s_full(x), s_waits & 1u, abort_flag);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         ++s_waits;
         tc_fence_after();
-        // kept columns of this row in tile j
-        const int kbase = j * kBN;
+        const int kbase = (j_lo + t) * kBN;
+        // kept key columns of this row in the tile
         int c_lo, c_hi;
         if (p.causal) {
           c_hi = i - kbase;
@@ -362,7 +433,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         } else {
           masked = kbase + kBN > p.T;
         }
-        // pass 1: row max of the tile (32 columns live at a time)
+        // pass 1: row max of the tile (64 columns live at a time)
         float mt;
         if (!masked) {
           float ma = -INFINITY, mb = -INFINITY;
@@ -395,12 +466,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         float alpha = 1.f;
         float m_use = m_run;
         if (m_new > m_run + kRescaleThreshold || m_run == -INFINITY) {
-          m_use = m_new;
-          alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m_new);
+          m_use = ceilf(m_new);  // integral reference; -inf stays -inf
+          alpha = (m_run == -INFINITY) ? 0.f : exp2_int(m_run - m_use);
         }
         const float m_safe = (m_use == -INFINITY) ? 0.f : m_use;
-        // pass 2: P = exp2(S*c - m) as bf16 pairs.  The P columns of chunk cc
-        // ([16cc, 16cc+16)) lie below the S columns still to be read.
+        // pass 2: P = exp2(S*c - m) as bf16 pairs; chunk cc ([16cc, 16cc+16))
+        // lies below the S columns still to be read.
         const uint64_t sl2x2 = f2_make(sl2, sl2);
         const uint64_t negm2 = f2_make(-m_safe, -m_safe);
         uint64_t rs2 = f2_make(0.f, 0.f);
@@ -411,15 +482,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            float t0, t1;
-            f2_split(f2_fma(f2_from_bits(raw[2 * e], raw[2 * e + 1]), sl2x2, negm2), t0, t1);
+            float t0v, t1v;
+            f2_split(f2_fma(f2_from_bits(raw[2 * e], raw[2 * e + 1]), sl2x2, negm2), t0v, t1v);
+            float p0, p1;
             if (masked) {
               const int c0 = cc * 32 + 2 * e;
-              if (!(c0 >= c_lo && c0 <= c_hi)) t0 = -INFINITY;
-              if (!(c0 + 1 >= c_lo && c0 + 1 <= c_hi)) t1 = -INFINITY;
+              if (!(c0 >= c_lo && c0 <= c_hi)) t0v = -INFINITY;
+              if (!(c0 + 1 >= c_lo && c0 + 1 <= c_hi)) t1v = -INFINITY;
+              p0 = ex2_approx(t0v);
+              p1 = ex2_approx(t1v);
+            } else if (e >= 16 - kPolyPairs) {
+              exp2_poly_x2(t0v, t1v, p0, p1);
+            } else {
+              p0 = ex2_approx(t0v);
+              p1 = ex2_approx(t1v);
             }
-            const float p0 = ex2_approx(t0);
-            const float p1 = ex2_approx(t1);
             rs2 = f2_add(rs2, f2_make(p0, p1));
             pk[e] = pack_bf16x2(p0, p1);
           }
@@ -427,13 +504,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         float rs0, rs1;
         f2_split(rs2, rs0, rs1);
-        const float rs = rs0 + rs1;
-        l_run = l_run * alpha + rs;
+        l_run = l_run * alpha + (rs0 + rs1);
         m_run = m_use;
         // O holds the sum over earlier tiles; rescale it when the max moved
-        const bool need = (alpha != 1.f) && (j > j_lo);
+        const bool need = (alpha != 1.f) && (k_idx > 0);
         if (__any_sync(0xffffffffu, need)) {
-          const uint32_t prev = o_seen + static_cast<uint32_t>(j - 1 - j_lo);
+          const uint32_t prev = o_seen + static_cast<uint32_t>(k_idx - 1);
           ok = mbar_wait(o_done(x), prev & 1u, abort_flag);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
@@ -452,20 +528,49 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mbar_arrive(p_full(x));
       }
       if (!ok) break;
-      // ---- epilogue: wait for the last PV of this phase
-      const uint32_t last = o_seen + static_cast<uint32_t>(n_tiles - 1);
-      o_seen += static_cast<uint32_t>(n_tiles);
+      // ---- epilogue: wait for the last PV of this slot in this phase
+      const uint32_t last = o_seen + static_cast<uint32_t>(my_tiles - 1);
+      o_seen += static_cast<uint32_t>(my_tiles);
       ok = mbar_wait(o_done(x), last & 1u, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+      float l_tot = l_run;
+      // split phase: slot B hands (m, l) to slot A, which merges O_A and O_B;
+      // both maxima are integral, so the merge factors are exact powers of two
+      float fa = 1.f, fb = 0.f;
+      if (pl.split) {
+        float *pub = reinterpret_cast<float *>(smem + L::kQOff + L::kQBytes);  // Q_B is idle
+        if (x == 1) {
+          pub[r] = m_run;
+          pub[kBM + r] = l_run;
+          mbar_arrive(split_ready);
+          break;  // slot B is done; slot A writes the output
+        }
+        ok = mbar_wait(split_ready, 0, abort_flag);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        const float m_b = pub[r], l_b = pub[kBM + r];
+        const float m = fmaxf(m_run, m_b);
+        fa = (m_run == -INFINITY) ? 0.f : exp2_int(m_run - m);
+        fb = (m_b == -INFINITY) ? 0.f : exp2_int(m_b - m);
+        l_tot = l_run * fa + l_b * fb;
+      }
+      const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
       if (hi == 0) {
         // noise head: keep H_N = O / l on chip for the group's signal heads
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32];
           tmem_ld32_sync(t_o(x) + lane_off + cc * 32, o);
+          if (pl.split) {
+            uint32_t ob[32];
+            tmem_ld32_sync(t_o(1) + lane_off + cc * 32, ob);
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              o[e] = __float_as_uint(__uint_as_float(o[e]) * fa + __uint_as_float(ob[e]) * fb);
+          }
 #pragma unroll
           for (int e = 0; e < 32; ++e) hn_smem[(cc * 32 + e) * kBM + r] = __uint_as_float(o[e]) * inv_l;
         }
@@ -491,13 +596,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32];
           tmem_ld32_sync(t_o(x) + lane_off + cc * 32, o);
+          if (pl.split) {
+            uint32_t ob[32];
+            tmem_ld32_sync(t_o(1) + lane_off + cc * 32, ob);
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              o[e] = __float_as_uint(__uint_as_float(o[e]) * fa + __uint_as_float(ob[e]) * fb);
+          }
           if (row_ok) {
             const uint4 *gp = reinterpret_cast<const uint4 *>(p.gate + goff + cc * 32);
             uint4 *op = reinterpret_cast<uint4 *>(p.out + goff + cc * 32);
+            uint4 gv[4];
+#pragma unroll
+            for (int v = 0; v < 4; ++v) gv[v] = __ldg(gp + v);
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
-              const uint4 gv = __ldg(gp + v);
-              const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+              const uint32_t gw[4] = {gv[v].x, gv[v].y, gv[v].z, gv[v].w};
               uint32_t ow[4];
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
@@ -521,7 +635,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (*abort_flag && threadIdx.x == 0) write_status(p.status, -5 /* GDLA_ERR_TIMEOUT */);
-  if (warp == 9) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

@@ -77,7 +77,7 @@ int launch_attn(const void *q_sig, const void *q_noise, const void *k, const voi
       !make_map(&tm_k, k, 3, dqn, kvbox) || !make_map(&tm_v, v, 3, dqn, kvbox))
     return GDLA_ERR_CUDA;
   // at least 116 KB so that one CTA (and one 512-column TMEM allocation) sits on an SM
-  const uint32_t smem = L::kAlloc > 118784u ? L::kAlloc : 118784u;
+  const uint32_t smem = L::kBytes > 118784u ? L::kBytes : 118784u;
   auto kern = gdla::gdla_attn_fwd_kernel<D>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
