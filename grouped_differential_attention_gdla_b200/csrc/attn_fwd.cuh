@@ -204,188 +204,205 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (warp == kProducerWarp) {
     // =============================== TMA producer
-    // Ring order per phase: K_0 .. K_{A-1}, then V_t, K_{t+A} for t = 0..n-1,
-    // where A = 1 (normal phase) or 2 (split phase) is how far ahead of the
-    // values the MMA warp consumes keys.
-    if (lane == 0) {
+    // The whole warp runs the loop (warp-uniform control and addresses); one
+    // elected lane issues the copies.  Ring order per phase: K_0 .. K_{A-1},
+    // then V_t, K_{t+A} for t = 0..n-1, where A = 1 (normal phase) or 2
+    // (split phase) is how far ahead of the values the MMA warp needs keys.
+    const bool leader = elect_one();
+    if (leader) {
       tma_prefetch_desc(&tm_qs);
       tma_prefetch_desc(&tm_qn);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      uint32_t q_uses[2] = {0, 0};
-      uint32_t c = 0;  // K/V ring position
-      bool ok = true;
-      auto load_kv = [&](int t, bool is_v) {
-        const int s = static_cast<int>(c % kKvStages);
-        ok = mbar_wait(kv_empty(s), ((c / kKvStages) & 1u) ^ 1u, abort_flag);
-        if (!ok) return;
-        const uint32_t dst = sbase + L::kKvOff + s * L::kKvBytes;
+    }
+    uint32_t q_uses[2] = {0, 0};
+    uint32_t c = 0;  // K/V ring position
+    bool ok = true;
+    auto load_kv = [&](int t, bool is_v) {
+      const int s = static_cast<int>(c % kKvStages);
+      ok = __all_sync(0xffffffffu, mbar_wait(kv_empty(s), ((c / kKvStages) & 1u) ^ 1u, abort_flag));
+      if (!ok) return;
+      const uint32_t dst = sbase + L::kKvOff + s * L::kKvBytes;
+      if (leader) {
         mbar_arrive_expect_tx(kv_full(s), L::kKvBytes);
         const CUtensorMap *map = is_v ? &tm_v : &tm_k;
 #pragma unroll
         for (int kb = 0; kb < D / 64; ++kb)
           tma_load_3d(dst + kb * (kBN * 128), map, kv_full(s), kvh * D + kb * 64,
                       (j_lo + t) * kBN, b);
-        ++c;
-      };
-      for (int ph = 0; ph < n_phases && ok; ++ph) {
-        const PhasePlan pl = phase_plan(ph, n_heads, n_tiles);
-        const int nq = pl.split ? 1 : pl.nslot;
+      }
+      ++c;
+    };
+    for (int ph = 0; ph < n_phases && ok; ++ph) {
+      const PhasePlan pl = phase_plan(ph, n_heads, n_tiles);
+      const int nq = pl.split ? 1 : pl.nslot;
 #pragma unroll
-        for (int x = 0; x < 2; ++x) {
-          if (x >= nq || !ok) break;
-          ok = mbar_wait(q_empty(x), (q_uses[x] & 1u) ^ 1u, abort_flag);
-          if (!ok) break;
-          ++q_uses[x];
-          const int hi = x == 0 ? pl.head0 : pl.head1;
-          const uint32_t dst = sbase + L::kQOff + x * L::kQBytes;
+      for (int x = 0; x < 2; ++x) {
+        if (x >= nq || !ok) break;
+        ok = __all_sync(0xffffffffu, mbar_wait(q_empty(x), (q_uses[x] & 1u) ^ 1u, abort_flag));
+        if (!ok) break;
+        ++q_uses[x];
+        const int hi = x == 0 ? pl.head0 : pl.head1;
+        const uint32_t dst = sbase + L::kQOff + x * L::kQBytes;
+        const bool noise = hi == 0;
+        const int head = noise ? kvh : p.g * kvh + (hi - 1);
+        if (leader) {
           mbar_arrive_expect_tx(q_full(x), L::kQBytes);
-          const bool noise = hi == 0;
-          const int head = noise ? kvh : p.g * kvh + (hi - 1);
           const CUtensorMap *map = noise ? &tm_qn : &tm_qs;
 #pragma unroll
           for (int kb = 0; kb < D / 64; ++kb)
             tma_load_3d(dst + kb * (kBM * 128), map, q_full(x), head * D + kb * 64, q0, b);
         }
-        const int ahead = pl.split ? 2 : 1;
-        for (int t = 0; t < ahead && t < n_tiles && ok; ++t) load_kv(t, false);
-        for (int t = 0; t < n_tiles && ok; ++t) {
-          load_kv(t, true);
-          if (ok && t + ahead < n_tiles) load_kv(t + ahead, false);
-        }
       }
-      if (!ok) {
-        // unwinding: let the copies already issued land before the CTA exits
-        for (int s = 0; s < kKvStages; ++s) {
-          const uint32_t issued = c > static_cast<uint32_t>(s) ? (c - 1 - s) / kKvStages + 1 : 0;
-          if (issued) mbar_wait_for(kv_full(s), (issued - 1) & 1u, 100000000ull);
-        }
-        for (int x = 0; x < 2; ++x)
-          if (q_uses[x]) mbar_wait_for(q_full(x), (q_uses[x] - 1) & 1u, 100000000ull);
+      const int ahead = pl.split ? 2 : 1;
+      for (int t = 0; t < ahead && t < n_tiles && ok; ++t) load_kv(t, false);
+      for (int t = 0; t < n_tiles && ok; ++t) {
+        load_kv(t, true);
+        if (ok && t + ahead < n_tiles) load_kv(t + ahead, false);
       }
+    }
+    if (!ok && leader) {
+      // unwinding: let the copies already issued land before the CTA exits
+      for (int s = 0; s < kKvStages; ++s) {
+        const uint32_t issued = c > static_cast<uint32_t>(s) ? (c - 1 - s) / kKvStages + 1 : 0;
+        if (issued) mbar_wait_for(kv_full(s), (issued - 1) & 1u, 100000000ull);
+      }
+      for (int x = 0; x < 2; ++x)
+        if (q_uses[x]) mbar_wait_for(q_full(x), (q_uses[x] - 1) & 1u, 100000000ull);
     }
   } else if (warp == kMmaWarp) {
     // =============================== MMA issuer
-    // Per slot X the issue order is S_X(t) .. PV_X(t), S_X(t+A): slot B's
-    // MMAs run while slot A's softmax works and vice versa.  S_X(t+A)
-    // overwrites the TMEM columns PV_X(t) reads P from; tcgen05.mma
-    // instructions of one thread execute in issue order, so the read of P
-    // precedes the overwrite.
-    if (lane == 0) {
-      constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBN, false, false);
-      constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, D, false, true);
-      uint32_t q_uses[2] = {0, 0};
-      uint32_t p_waits[2] = {0, 0};
-      uint32_t ofree_waits[2] = {0, 0};
-      uint32_t o_commits[2] = {0, 0};
-      uint32_t c = 0;  // ring position of the next K/V tile to consume
-      bool ok = true;
-      auto issue_s = [&](int x, int qbuf, uint32_t k_base) {
-        const uint32_t q_base = sbase + L::kQOff + qbuf * L::kQBytes;
+    // The whole warp runs the loop so descriptors stay warp-uniform; one
+    // elected lane issues every tcgen05.mma and commit.  Per slot X the issue
+    // order is S_X(t) .. PV_X(t), S_X(t+A): slot B's MMAs run while slot A's
+    // softmax works and vice versa.  S_X(t+A) overwrites the TMEM columns
+    // PV_X(t) reads P from; tcgen05.mma instructions of one thread execute in
+    // issue order, so the read of P precedes the overwrite.
+    const bool leader = elect_one();
+    constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBN, false, false);
+    constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, D, false, true);
+    uint32_t q_uses[2] = {0, 0};
+    uint32_t p_waits[2] = {0, 0};
+    uint32_t ofree_waits[2] = {0, 0};
+    uint32_t o_commits[2] = {0, 0};
+    uint32_t c = 0;  // ring position of the next K/V tile to consume
+    bool ok = true;
+    // descriptor of a K-major tile at `base`; k-step k adds a constant offset
+    auto issue_s = [&](int x, int qbuf, uint32_t k_base) {
+      const uint64_t qd = sdesc_sw128(sbase + L::kQOff + qbuf * L::kQBytes, 16, 1024);
+      const uint64_t kd = sdesc_sw128(k_base, 16, 1024);
+      if (leader) {
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t qoff = (k >> 2) * (kBM * 128) + (k & 3) * 32;
           const uint32_t koff = (k >> 2) * (kBN * 128) + (k & 3) * 32;
-          umma_ss(t_s(x), sdesc_sw128(q_base + qoff, 16, 1024),
-                  sdesc_sw128(k_base + koff, 16, 1024), kIdescS, k > 0 ? 1u : 0u);
+          umma_ss(t_s(x), qd + (qoff >> 4), kd + (koff >> 4), kIdescS, k > 0 ? 1u : 0u);
         }
         umma_commit(s_full(x));
-      };
-      // waits for the next ring entry; returns its stage and smem address
-      auto next_stage = [&](uint32_t &base) -> int {
-        const int s = static_cast<int>(c % kKvStages);
-        ok = mbar_wait(kv_full(s), (c / kKvStages) & 1u, abort_flag);
-        tc_fence_after();
-        base = sbase + L::kKvOff + s * L::kKvBytes;
-        ++c;
-        return s;
-      };
-      for (int ph = 0; ph < n_phases && ok; ++ph) {
-        const PhasePlan pl = phase_plan(ph, n_heads, n_tiles);
-        const int nq = pl.split ? 1 : pl.nslot;
+      }
+    };
+    // waits for the next ring entry; returns its stage and smem address
+    auto next_stage = [&](uint32_t &base) -> int {
+      const int s = static_cast<int>(c % kKvStages);
+      ok = __all_sync(0xffffffffu, mbar_wait(kv_full(s), (c / kKvStages) & 1u, abort_flag));
+      tc_fence_after();
+      base = sbase + L::kKvOff + s * L::kKvBytes;
+      ++c;
+      return s;
+    };
+    for (int ph = 0; ph < n_phases && ok; ++ph) {
+      const PhasePlan pl = phase_plan(ph, n_heads, n_tiles);
+      const int nq = pl.split ? 1 : pl.nslot;
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        if (x < nq && ok) {
+          ok = __all_sync(0xffffffffu, mbar_wait(q_full(x), q_uses[x] & 1u, abort_flag));
+          ++q_uses[x];
+        }
+      }
+      if (!ok) break;
+      const int ahead = pl.split ? 2 : 1;
+      // prologue: the first S of every slot
+      if (!pl.split) {
+        uint32_t kb;
+        const int s = next_stage(kb);
+        if (!ok) break;
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
-          if (x < nq && ok) {
-            ok = mbar_wait(q_full(x), q_uses[x] & 1u, abort_flag);
-            ++q_uses[x];
+          if (x < pl.nslot) {
+            issue_s(x, x, kb);
+            if (n_tiles == 1 && leader) umma_commit(q_empty(x));
           }
         }
-        if (!ok) break;
-        const int ahead = pl.split ? 2 : 1;
-        // prologue: the first S of every slot
-        if (!pl.split) {
+        if (leader) umma_commit(kv_empty(s));
+      } else {
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
           uint32_t kb;
           const int s = next_stage(kb);
           if (!ok) break;
-#pragma unroll
-          for (int x = 0; x < 2; ++x) {
-            if (x < pl.nslot) {
-              issue_s(x, x, kb);
-              if (n_tiles == 1) umma_commit(q_empty(x));
-            }
-          }
-          umma_commit(kv_empty(s));
-        } else {
-#pragma unroll
-          for (int x = 0; x < 2; ++x) {
-            uint32_t kb;
-            const int s = next_stage(kb);
-            if (!ok) break;
-            issue_s(x, 0, kb);
+          issue_s(x, 0, kb);
+          if (leader) {
             if (x == 1 && n_tiles == 2) umma_commit(q_empty(0));
             umma_commit(kv_empty(s));
           }
-          if (!ok) break;
         }
-        for (int t = 0; t < n_tiles && ok; ++t) {
-          uint32_t vb;
-          const int sv = next_stage(vb);
-          if (!ok) break;
-          int sk = -1;
-          uint32_t kb = 0;
+        if (!ok) break;
+      }
+      for (int t = 0; t < n_tiles && ok; ++t) {
+        uint32_t vb;
+        const int sv = next_stage(vb);
+        if (!ok) break;
+        const uint64_t vd = sdesc_sw128(vb, kBN * 128, 1024);
+        int sk = -1;
+        uint32_t kb = 0;
 #pragma unroll
-          for (int xx = 0; xx < 2; ++xx) {
-            if (pl.split && xx == 1) break;
-            const int x = pl.split ? (t & 1) : xx;
-            if (x >= pl.nslot || !ok) break;
-            ok = mbar_wait(p_full(x), p_waits[x] & 1u, abort_flag);
+        for (int xx = 0; xx < 2; ++xx) {
+          if (pl.split && xx == 1) break;
+          const int x = pl.split ? (t & 1) : xx;
+          if (x >= pl.nslot || !ok) break;
+          const uint32_t pw = x == 0 ? p_waits[0] : p_waits[1];
+          ok = __all_sync(0xffffffffu, mbar_wait(p_full(x), pw & 1u, abort_flag));
+          if (!ok) break;
+          if (x == 0) ++p_waits[0]; else ++p_waits[1];
+          const bool first_pv = pl.split ? (t == x) : (t == 0);
+          if (first_pv && ph > 0) {
+            // the previous phase's epilogue must have read O_X
+            const uint32_t fw = x == 0 ? ofree_waits[0] : ofree_waits[1];
+            ok = __all_sync(0xffffffffu, mbar_wait(o_free(x), fw & 1u, abort_flag));
             if (!ok) break;
-            ++p_waits[x];
-            const bool first_pv = pl.split ? (t == x) : (t == 0);
-            if (first_pv && ph > 0) {
-              // the previous phase's epilogue must have read O_X
-              ok = mbar_wait(o_free(x), ofree_waits[x] & 1u, abort_flag);
-              if (!ok) break;
-              ++ofree_waits[x];
-            }
-            tc_fence_after();
-#pragma unroll
-            for (int k = 0; k < kBN / 16; ++k) {
-              umma_ts(t_o(x), t_s(x) + p_col(k),
-                      sdesc_sw128(vb + k * (16 * 128), kBN * 128, 1024), kIdescPV,
-                      (!first_pv || k > 0) ? 1u : 0u);
-            }
-            umma_commit(o_done(x));
-            ++o_commits[x];
-            const int tn = t + ahead;
-            if (tn < n_tiles) {
-              if (sk < 0) {
-                sk = next_stage(kb);
-                if (!ok) break;
-              }
-              issue_s(x, pl.split ? 0 : x, kb);
-              if (tn == n_tiles - 1) umma_commit(q_empty(pl.split ? 0 : x));
-            }
+            if (x == 0) ++ofree_waits[0]; else ++ofree_waits[1];
           }
-          if (!ok) break;
+          tc_fence_after();
+          if (leader) {
+#pragma unroll
+            for (int k = 0; k < kBN / 16; ++k)
+              umma_ts(t_o(x), t_s(x) + p_col(k), vd + ((k * (16 * 128)) >> 4), kIdescPV,
+                      (!first_pv || k > 0) ? 1u : 0u);
+            umma_commit(o_done(x));
+          }
+          if (x == 0) ++o_commits[0]; else ++o_commits[1];
+          const int tn = t + ahead;
+          if (tn < n_tiles) {
+            if (sk < 0) {
+              sk = next_stage(kb);
+              if (!ok) break;
+            }
+            issue_s(x, pl.split ? 0 : x, kb);
+            if (tn == n_tiles - 1 && leader) umma_commit(q_empty(pl.split ? 0 : x));
+          }
+        }
+        if (!ok) break;
+        if (leader) {
           umma_commit(kv_empty(sv));
           if (sk >= 0) umma_commit(kv_empty(sk));
         }
       }
-      // drain: every MMA issued above must finish before TMEM is released
-#pragma unroll
-      for (int x = 0; x < 2; ++x)
-        if (o_commits[x]) mbar_wait_for(o_done(x), (o_commits[x] - 1) & 1u, 100000000ull);
+    }
+    // drain: every MMA issued above must finish before TMEM is released
+    if (leader) {
+      if (o_commits[0]) mbar_wait_for(o_done(0), (o_commits[0] - 1) & 1u, 100000000ull);
+      if (o_commits[1]) mbar_wait_for(o_done(1), (o_commits[1] - 1) & 1u, 100000000ull);
     }
   } else {
     // =============================== softmax + epilogue (one warpgroup per slot)

@@ -103,76 +103,81 @@ __global__ void __launch_bounds__(kExpThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 4) {
-    // =============================== TMA producer
-    if (lane == 0) {
+    // =============================== TMA producer (warp-uniform loop, one lane issues)
+    const bool leader = elect_one();
+    if (leader) {
       tma_prefetch_desc(&tm_c);
       tma_prefetch_desc(&tm_w);
       mbar_arrive_expect_tx(a_full, static_cast<uint32_t>(kExpBM * DL * 2));
       for (int kb = 0; kb < n_kb; ++kb)
         tma_load_2d(sbase + L::kAOff + kb * (kExpBM * 128), &tm_c, a_full, kb * 64,
                     static_cast<int32_t>(m0));
-      uint32_t c = 0;
-      bool ok = true;
-      for (int h = 0; h < H && ok; ++h) {
-        for (int kc = 0; kc < n_chunks; ++kc) {
-          const int s = static_cast<int>(c % kExpStages);
-          ok = mbar_wait(w_empty(s), ((c / kExpStages) & 1u) ^ 1u, abort_flag);
-          if (!ok) break;
+    }
+    uint32_t c = 0;
+    bool ok = true;
+    for (int h = 0; h < H && ok; ++h) {
+      for (int kc = 0; kc < n_chunks; ++kc) {
+        const int s = static_cast<int>(c % kExpStages);
+        ok = __all_sync(0xffffffffu, mbar_wait(w_empty(s), ((c / kExpStages) & 1u) ^ 1u, abort_flag));
+        if (!ok) break;
+        const uint32_t dst = sbase + L::kWOff + s * L::kStageBytes;
+        if (leader) {
           mbar_arrive_expect_tx(w_full(s), L::kStageBytes);
-          const uint32_t dst = sbase + L::kWOff + s * L::kStageBytes;
 #pragma unroll
           for (int nb = 0; nb < NT / 64; ++nb)
             tma_load_2d(dst + nb * (kExpKC * 128), &tm_w, w_full(s), h * NT + nb * 64,
                         kc * kExpKC);
-          ++c;
         }
-      }
-      if (!ok) {
-        for (int s = 0; s < kExpStages; ++s) {
-          const uint32_t issued = c > static_cast<uint32_t>(s) ? (c - 1 - s) / kExpStages + 1 : 0;
-          if (issued) mbar_wait_for(w_full(s), (issued - 1) & 1u, 100000000ull);
-        }
-        mbar_wait_for(a_full, 0, 100000000ull);
+        ++c;
       }
     }
+    if (!ok && leader) {
+      for (int s = 0; s < kExpStages; ++s) {
+        const uint32_t issued = c > static_cast<uint32_t>(s) ? (c - 1 - s) / kExpStages + 1 : 0;
+        if (issued) mbar_wait_for(w_full(s), (issued - 1) & 1u, 100000000ull);
+      }
+      mbar_wait_for(a_full, 0, 100000000ull);
+    }
   } else if (warp == 5) {
-    // =============================== MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t kIdesc = idesc_bf16_f32(kExpBM, NT, false, true);
-      bool ok = mbar_wait(a_ready, 0, abort_flag);
+    // =============================== MMA issuer (warp-uniform loop, one lane issues)
+    const bool leader = elect_one();
+    constexpr uint32_t kIdesc = idesc_bf16_f32(kExpBM, NT, false, true);
+    bool ok = __all_sync(0xffffffffu, mbar_wait(a_ready, 0, abort_flag));
+    tc_fence_after();
+    const uint64_t ad = sdesc_sw128(sbase + L::kAOff, 16, 1024);
+    uint32_t c = 0;
+    uint32_t commits = 0;
+    for (int h = 0; h < H && ok; ++h) {
+      const int buf = h & 1;
+      const uint32_t use = static_cast<uint32_t>(h >> 1);
+      ok = __all_sync(0xffffffffu, mbar_wait(acc_empty(buf), (use & 1u) ^ 1u, abort_flag));
+      if (!ok) break;
       tc_fence_after();
-      uint32_t c = 0;
-      uint32_t commits = 0;
-      for (int h = 0; h < H && ok; ++h) {
-        const int buf = h & 1;
-        const uint32_t use = static_cast<uint32_t>(h >> 1);
-        ok = mbar_wait(acc_empty(buf), (use & 1u) ^ 1u, abort_flag);
+      const uint32_t d_tmem = tmem + static_cast<uint32_t>(buf * NT);
+      for (int kc = 0; kc < n_chunks && ok; ++kc) {
+        const int s = static_cast<int>(c % kExpStages);
+        ok = __all_sync(0xffffffffu, mbar_wait(w_full(s), (c / kExpStages) & 1u, abort_flag));
         if (!ok) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem + static_cast<uint32_t>(buf * NT);
-        for (int kc = 0; kc < n_chunks && ok; ++kc) {
-          const int s = static_cast<int>(c % kExpStages);
-          ok = mbar_wait(w_full(s), (c / kExpStages) & 1u, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t w_base = sbase + L::kWOff + s * L::kStageBytes;
+        const uint64_t wd = sdesc_sw128(sbase + L::kWOff + s * L::kStageBytes, kExpKC * 128, 1024);
+        if (leader) {
 #pragma unroll
           for (int kk = 0; kk < kExpKC / 16; ++kk) {
             const int ks = kc * (kExpKC / 16) + kk;  // 16-wide k step over the latent
-            const uint32_t a_addr = sbase + L::kAOff + (ks >> 2) * (kExpBM * 128) + (ks & 3) * 32;
-            const uint32_t b_addr = w_base + kk * (16 * 128);
-            umma_ss(d_tmem, sdesc_sw128(a_addr, 16, 1024),
-                    sdesc_sw128(b_addr, kExpKC * 128, 1024), kIdesc, (kc > 0 || kk > 0) ? 1u : 0u);
+            const uint32_t a_off = (ks >> 2) * (kExpBM * 128) + (ks & 3) * 32;
+            umma_ss(d_tmem, ad + (a_off >> 4), wd + ((kk * (16 * 128)) >> 4), kIdesc,
+                    (kc > 0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(w_empty(s));
-          ++c;
         }
-        if (!ok) break;
-        umma_commit(acc_full(buf));
-        ++commits;
+        ++c;
       }
-      if (commits) mbar_wait_for(acc_full((commits - 1) & 1), ((commits - 1) >> 1) & 1u, 100000000ull);
+      if (!ok) break;
+      if (leader) umma_commit(acc_full(buf));
+      ++commits;
     }
+    if (commits && leader)
+      mbar_wait_for(acc_full((commits - 1) & 1), ((commits - 1) >> 1) & 1u, 100000000ull);
   } else {
     // =============================== norm + epilogue (warps 0-3, one row per thread)
     const int r = threadIdx.x;  // row = TMEM lane
