@@ -280,14 +280,31 @@ def run_ours(args):
         print(json.dumps(result), flush=True)
 
 
+def _csrc_hash():
+    """Hash of the CUDA sources, to tell whether profiled counters still apply."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "grouped_differential_attention_gdla_b200",
+                                           "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 def _traffic_from_profiles(name):
-    """DRAM bytes per attention launch from the committed ncu summary, if any."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
-    try:
+    """DRAM bytes (read + write) per attention launch from a committed ncu
+    summary under profiles/ (a line "traffic: workload=<w> csrc=<hash>
+    bytes=<n>"), or None when none matches this workload and these sources."""
+    import glob
+    import re
+    want = _csrc_hash()
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
         with open(path) as f:
-            return json.load(f).get(name)
-    except (OSError, ValueError):
-        return None
+            for m in re.finditer(r"traffic: workload=(\S+) csrc=(\S+) bytes=(\d+)", f.read()):
+                if m.group(1) == name and m.group(2) == want:
+                    return int(m.group(3))
+    return None
 
 
 def _oracle_sample(wl, x, seconds):

@@ -8,7 +8,8 @@ device memory and streams only.
     gdla_attn_fwd(q_sig, q_noise, k, v, lam, gate, window=0, causal=True) -> out
 """
 from ._binding import (GDLAError, EXPORTED, LIB_PATH, gdla_attn_fwd, gdla_kv_expand,
-                       gdla_status_string, gdla_version, load_library)
+                       gdla_selftest_wait_timeout, gdla_status_string, gdla_version,
+                       load_library)
 
 __all__ = ["GDLAError", "EXPORTED", "LIB_PATH", "gdla_attn_fwd", "gdla_kv_expand",
-           "gdla_status_string", "gdla_version", "load_library"]
+           "gdla_selftest_wait_timeout", "gdla_status_string", "gdla_version", "load_library"]

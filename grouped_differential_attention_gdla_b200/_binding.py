@@ -24,7 +24,8 @@ GDLA_ERR_CUDA = -4
 GDLA_ERR_TIMEOUT = -5
 
 # every symbol include/gdla.h declares
-EXPORTED = ("gdla_version", "gdla_status_string", "gdla_kv_expand", "gdla_attn_fwd")
+EXPORTED = ("gdla_version", "gdla_status_string", "gdla_kv_expand", "gdla_attn_fwd",
+            "gdla_selftest_wait_timeout")
 
 _lib = None
 
@@ -56,6 +57,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.gdla_attn_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32, i64,
                                   i32, f32, vp, vp]
     lib.gdla_attn_fwd.restype = i32
+    lib.gdla_selftest_wait_timeout.argtypes = [vp, i64, vp]
+    lib.gdla_selftest_wait_timeout.restype = i32
     if path is None:
         _lib = lib
     return lib
@@ -148,3 +151,13 @@ def gdla_attn_fwd(q_sig: torch.Tensor, q_noise: torch.Tensor, k: torch.Tensor, v
     if rc != GDLA_OK:
         raise GDLAError(rc, "gdla_attn_fwd")
     return out
+
+
+def gdla_selftest_wait_timeout(d_status: torch.Tensor, limit_ns: int, stream=None) -> None:
+    """Run the bounded-wait self test; d_status (int32 CUDA tensor) gets -5."""
+    if d_status.device.type != "cuda" or d_status.dtype != torch.int32:
+        raise ValueError("d_status must be an int32 CUDA tensor")
+    rc = load_library().gdla_selftest_wait_timeout(d_status.data_ptr(), int(limit_ns),
+                                                   _stream_ptr(d_status.device, stream))
+    if rc != GDLA_OK:
+        raise GDLAError(rc, "gdla_selftest_wait_timeout")

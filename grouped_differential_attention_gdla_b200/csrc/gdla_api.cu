@@ -14,6 +14,7 @@
 #include "gdla.h"
 #include "attn_fwd.cuh"
 #include "kv_expand.cuh"
+#include "selftest.cuh"
 
 namespace {
 
@@ -192,6 +193,14 @@ int gdla_attn_fwd(const void *q_sig, const void *q_noise, const void *k, const v
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return d == 128 ? launch_attn<128>(q_sig, q_noise, k, v, prm, Hs, Hn, s)
                   : launch_attn<64>(q_sig, q_noise, k, v, prm, Hs, Hn, s);
+}
+
+int gdla_selftest_wait_timeout(int *d_status, int64_t limit_ns, void *stream) {
+  if (!d_status || limit_ns <= 0 || limit_ns > 1000000000ll) return GDLA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(d_status) & 3u) != 0) return GDLA_ERR_ALIGNMENT;
+  gdla::gdla_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      d_status, static_cast<uint64_t>(limit_ns));
+  return cudaGetLastError() == cudaSuccess ? GDLA_OK : GDLA_ERR_CUDA;
 }
 
 }  // extern "C"

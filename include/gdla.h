@@ -116,6 +116,24 @@ int gdla_attn_fwd(const void *q_sig, const void *q_noise, const void *k,
                   int64_t window, int causal, float scale, int *d_status,
                   void *stream);
 
+/*
+ * gdla_selftest_wait_timeout - device-side check of the failure path.
+ *
+ * Every pipeline wait inside the kernels above polls an mbarrier with a time
+ * limit; when it passes, the kernel writes GDLA_ERR_TIMEOUT to d_status,
+ * stops early and releases what it holds, instead of hanging the GPU.  This
+ * entry point runs that same wait, in one warp, on a barrier that nothing
+ * ever completes, and gives up after limit_ns nanoseconds.
+ *
+ * d_status  device int, required; receives GDLA_ERR_TIMEOUT when the kernel
+ *           has run (the caller zeroes it beforehand)
+ * limit_ns  1 .. 1e9
+ * Returns GDLA_OK once the kernel is enqueued on `stream`; GDLA_ERR_INVALID_ARG
+ * for a null status pointer or a limit out of range.  Nothing traps or
+ * faults: the CUDA context stays usable afterwards.
+ */
+int gdla_selftest_wait_timeout(int *d_status, int64_t limit_ns, void *stream);
+
 #ifdef __cplusplus
 } /* extern "C" */
 #endif

@@ -34,7 +34,7 @@ def _declared_functions():
 def test_exports_every_declared_symbol(lib):
     declared = _declared_functions()
     assert set(declared) == {"gdla_version", "gdla_status_string", "gdla_kv_expand",
-                             "gdla_attn_fwd"}
+                             "gdla_attn_fwd", "gdla_selftest_wait_timeout"}
     for name in declared:
         assert hasattr(lib, name), f"{name} missing from libgdla.so"
     assert set(declared) == set(_binding.EXPORTED)
@@ -103,3 +103,11 @@ def test_binding_rejects_host_tensors():
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(RuntimeError, match="libgdla.so not found"):
         gdla.load_library(str(tmp_path / "libgdla.so"))
+
+
+@pytest.mark.parametrize("status,limit,code", [
+    (None, 1000, INVALID), (A, 0, INVALID), (A, -5, INVALID), (A, 2 * 10 ** 9, INVALID),
+    (0x100002, 1000, ALIGN),
+])
+def test_selftest_argument_errors(lib, status, limit, code):
+    assert lib.gdla_selftest_wait_timeout(status, limit, None) == code
