@@ -147,10 +147,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work item: heaviest query blocks first (causal), KV groups interleaved
-  const int groups = p.B * p.Hn;
-  const int qblk = p.n_qblk - 1 - static_cast<int>(blockIdx.x / groups);
-  const int grp = static_cast<int>(blockIdx.x % groups);
+  // ---- work item, heaviest query blocks first.  Full attention: KV groups
+  // one after another, so CTAs running at the same time stream the same
+  // group's K/V tiles and those stay in L2.  Sliding window: all groups of a
+  // query block together, so the block's query/gate/output rows are read and
+  // written as whole contiguous token rows.
+  int grp, qblk;
+  if (p.window == 0) {
+    grp = static_cast<int>(blockIdx.x / p.n_qblk);
+    qblk = p.n_qblk - 1 - static_cast<int>(blockIdx.x % p.n_qblk);
+  } else {
+    const int groups = p.B * p.Hn;
+    grp = static_cast<int>(blockIdx.x % groups);
+    qblk = p.n_qblk - 1 - static_cast<int>(blockIdx.x / groups);
+  }
   const int b = grp / p.Hn;
   const int kvh = grp % p.Hn;
   const int q0 = qblk * kBM;
