@@ -22,11 +22,16 @@
 // subtracted in the epilogue of every signal head of the group; neither H_S
 // nor H_N reaches global memory.
 //
-// Warp roles (320 threads):
-//   warps 0-3  softmax + epilogue for slot A (TMEM lanes 0..127)
-//   warps 4-7  softmax + epilogue for slot B
-//   warp  8    TMA producer (Q tiles, K/V ring)
-//   warp  9    TMEM allocator and single-thread MMA issuer
+// Warp roles (512 threads, registers re-split with setmaxnreg):
+//   warps  0-3   softmax for slot A (TMEM lanes 0..127)             176 regs
+//   warps  4-7   softmax for slot B                                  176 regs
+//   warps  8-11  epilogue for both slots: O / l, H_N, gate, output   96 regs
+//   warp  12     TMA producer (Q tiles, K/V ring)                    } 56 regs
+//   warp  13     TMEM allocator and MMA issuer                       }
+//   warps 14-15  idle (complete the fourth warpgroup)                }
+// A softmax warpgroup hands each finished head to the epilogue warpgroup
+// (row sums and maxima through shared memory) and goes straight on to the
+// next phase; the next PV into the same O columns waits for the epilogue.
 //
 // TMEM (512 columns): S_A [0,128) S_B [128,256) O_A [256,256+d) O_B [256+d,256+2d).
 // P_X occupies the first 64 columns of S_X as packed bf16 pairs.
@@ -39,9 +44,21 @@ namespace gdla {
 constexpr int kBM = 128;      // query rows per slot
 constexpr int kBN = 128;      // keys per K/V tile
 constexpr int kKvStages = 3;  // K/V ring depth (tiles)
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kAttnThreads = 10 * 32;
+constexpr int kProducerWarp = 12;
+constexpr int kMmaWarp = 13;
+constexpr int kAttnThreads = 16 * 32;
+// Register split.  The block launches with kLaunchRegs per thread (the
+// compiler's cap for 16 warps, four per SM sub-partition); the control and
+// epilogue warpgroups give registers back and the softmax warpgroups take
+// them, within the launch pool.  The host refuses to launch a build whose
+// per-thread register count differs from kLaunchRegs.
+constexpr uint32_t kLaunchRegs = 128;
+constexpr uint32_t kSoftmaxRegs = 152;
+constexpr uint32_t kEpilogueRegs = 96;
+constexpr uint32_t kControlRegs = 112;
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kEpilogueRegs + 128 * kControlRegs <=
+                  kAttnThreads * kLaunchRegs,
+              "register split must fit in the launch pool");
 constexpr int kSlotThreads = 128;          // one warpgroup per slot
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: O is rescaled only if the max grows by > 2^8
 // Of every 16 score pairs in a 32-column chunk of an unmasked tile, this many
@@ -73,10 +90,12 @@ struct AttnSmemLayout {
   static constexpr uint32_t kQOff = 0;
   static constexpr uint32_t kKvOff = kQOff + 2 * kQBytes;
   static constexpr uint32_t kHnOff = kKvOff + kKvStages * kKvBytes;
-  static constexpr uint32_t kBarOff = kHnOff + kHnBytes;
+  static constexpr uint32_t kStatOff = kHnOff + kHnBytes;  // float stat[slot][l, m][row]
+  static constexpr uint32_t kStatBytes = 2 * 2 * kBM * 4;
+  static constexpr uint32_t kBarOff = kStatOff + kStatBytes;
   // q_full[2] q_empty[2] kv_full[S] kv_empty[S] s_full[2] p_full[2] o_done[2]
-  // o_free[2] hn_ready split_ready
-  static constexpr uint32_t kNumBars = 2 + 2 + 2 * kKvStages + 2 + 2 + 2 + 2 + 2;
+  // o_free[2] epi_go[2] stat_free[2]
+  static constexpr uint32_t kNumBars = 2 + 2 + 2 * kKvStages + 2 + 2 + 2 + 2 + 2 + 2;
   static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;
   static constexpr uint32_t kBytes = kMiscOff + 16;
 };
@@ -111,6 +130,19 @@ __device__ __forceinline__ PhasePlan phase_plan(int ph, int n_heads, int n_tiles
   return pl;
 }
 
+// How a 32-column chunk of a masked score tile (a sliding-window edge or the
+// causal diagonal) looks to the 32 rows of one warp, warp-uniformly: every
+// column kept, none kept, or mixed.  Per warp at most one chunk is mixed, so
+// only it pays for per-column tests, and chunks no row keeps cost neither
+// TMEM loads nor exponentials.
+constexpr int kChunkFull = 0, kChunkEmpty = 1, kChunkMixed = 2;
+__device__ __forceinline__ int chunk_class(int cc, int c_lo, int c_hi) {
+  const int col0 = cc * 32, col1 = col0 + 31;
+  if (__all_sync(0xffffffffu, c_lo <= col0 && col1 <= c_hi)) return kChunkFull;
+  if (__all_sync(0xffffffffu, col1 < c_lo || col0 > c_hi)) return kChunkEmpty;
+  return kChunkMixed;
+}
+
 __device__ __forceinline__ void write_status(int *status, int code) {
   if (status) atomicExch(status, code);
 }
@@ -138,11 +170,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   auto p_full = [&](int x) { return bar0 + 8u * (6 + 2 * kKvStages + x); };
   auto o_done = [&](int x) { return bar0 + 8u * (8 + 2 * kKvStages + x); };
   auto o_free = [&](int x) { return bar0 + 8u * (10 + 2 * kKvStages + x); };
-  const uint32_t hn_ready = bar0 + 8u * (12 + 2 * kKvStages);
-  const uint32_t split_ready = bar0 + 8u * (13 + 2 * kKvStages);
+  auto epi_go = [&](int x) { return bar0 + 8u * (12 + 2 * kKvStages + x); };
+  auto stat_free = [&](int x) { return bar0 + 8u * (14 + 2 * kKvStages + x); };
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
   float *hn_smem = reinterpret_cast<float *>(smem + L::kHnOff);  // [D][kBM]
+  float *stat = reinterpret_cast<float *>(smem + L::kStatOff);   // [2][2][kBM]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -194,8 +227,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(kv_full(s), 1);
       mbar_init(kv_empty(s), 1);
     }
-    mbar_init(hn_ready, kSlotThreads);
-    mbar_init(split_ready, kSlotThreads);
+    mbar_init(epi_go(0), kSlotThreads);
+    mbar_init(epi_go(1), kSlotThreads);
+    mbar_init(stat_free(0), kSlotThreads);
+    mbar_init(stat_free(1), kSlotThreads);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -212,6 +247,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   // TMEM column (relative to S_X) of the packed P for keys 16k .. 16k+15
   auto p_col = [](int k) -> uint32_t { return 8u * k; };
 
+  if (warp >= 12) {
+  // =============================== control warpgroup (warps 12-15)
+  regs_decrease<kControlRegs>();
   if (warp == kProducerWarp) {
     // =============================== TMA producer
     // The whole warp runs the loop (warp-uniform control and addresses); one
@@ -414,8 +452,126 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (o_commits[0]) mbar_wait_for(o_done(0), (o_commits[0] - 1) & 1u, 100000000ull);
       if (o_commits[1]) mbar_wait_for(o_done(1), (o_commits[1] - 1) & 1u, 100000000ull);
     }
+  }
+  } else if (warp >= 8) {
+    // =============================== epilogue warpgroup (warps 8-11)
+    regs_decrease<kEpilogueRegs>();
+    const int wq = warp & 3;          // TMEM lane quarter
+    const int r = threadIdx.x & 127;  // row in the block = TMEM lane
+    const int i = q0 + r;             // query token
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const bool row_ok = i < p.T;
+    const int64_t row = static_cast<int64_t>(b) * p.T + i;
+    uint32_t go_waits[2] = {0, 0};
+    uint32_t pv_seen[2] = {0, 0};  // PV commits per slot in finished phases
+    bool ok = true;
+    // waits until slot x has handed over the head it ran in this phase and
+    // its last PV (number `last` of the slot) has completed
+    auto wait_slot = [&](int x, uint32_t last) -> bool {
+      const uint32_t gw = x == 0 ? go_waits[0] : go_waits[1];
+      bool w = mbar_wait(epi_go(x), gw & 1u, abort_flag);
+      if (x == 0) ++go_waits[0]; else ++go_waits[1];
+      if (w) w = mbar_wait(o_done(x), last & 1u, abort_flag);
+      w = __all_sync(0xffffffffu, w);
+      tc_fence_after();
+      return w;
+    };
+    for (int ph = 0; ph < n_phases && ok; ++ph) {
+      const PhasePlan pl = phase_plan(ph, n_heads, n_tiles);
+      const int tiles0 = pl.split ? (n_tiles + 1) / 2 : n_tiles;
+      const int tiles1 = pl.split ? n_tiles / 2 : n_tiles;
+      // one epilogue per slot, or one merged epilogue for a split head
+      const int n_epi = pl.split ? 1 : pl.nslot;
+      for (int e_i = 0; e_i < n_epi && ok; ++e_i) {
+        const int x = e_i;
+        const int hi = x == 0 ? pl.head0 : pl.head1;
+        float fa = 1.f, fb = 0.f, l_tot;
+        if (pl.split) {
+          ok = wait_slot(0, pv_seen[0] + tiles0 - 1);
+          if (ok) ok = wait_slot(1, pv_seen[1] + tiles1 - 1);
+          if (!ok) break;
+          // both maxima are integral, so the merge factors are exact powers of two
+          const float l_a = stat[0 * 2 * kBM + r], m_a = stat[0 * 2 * kBM + kBM + r];
+          const float l_b = stat[1 * 2 * kBM + r], m_b = stat[1 * 2 * kBM + kBM + r];
+          const float m = fmaxf(m_a, m_b);
+          fa = (m_a == -INFINITY) ? 0.f : exp2_int(m_a - m);
+          fb = (m_b == -INFINITY) ? 0.f : exp2_int(m_b - m);
+          l_tot = l_a * fa + l_b * fb;
+          mbar_arrive(stat_free(0));
+          mbar_arrive(stat_free(1));
+        } else {
+          ok = wait_slot(x, pv_seen[x == 0 ? 0 : 1] + (x == 0 ? tiles0 : tiles1) - 1);
+          if (!ok) break;
+          l_tot = stat[x * 2 * kBM + r];
+          mbar_arrive(stat_free(x));
+        }
+        const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
+        if (hi == 0) {
+          // noise head (never split: it runs in phase 0 next to signal head 0):
+          // H_N = O / l stays in shared memory for the group's signal heads;
+          // this warpgroup is also the only reader, row by row
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            tmem_ld32_sync(t_o(x) + lane_off + cc * 32, o);
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              hn_smem[(cc * 32 + e) * kBM + r] = __uint_as_float(o[e]) * inv_l;
+          }
+        } else {
+          const int h = p.g * kvh + (hi - 1);
+          const int64_t goff = (row * p.Hs + h) * static_cast<int64_t>(D);
+          float lam = 0.f;
+          if (row_ok) lam = __bfloat162float(p.lam[row * p.Hs + h]);
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            tmem_ld32_sync(t_o(x) + lane_off + cc * 32, o);
+            if (pl.split) {
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh) {
+                uint32_t ob[16];
+                tmem_ld16_sync(t_o(1) + lane_off + cc * 32 + hh * 16, ob);
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                  o[hh * 16 + e] = __float_as_uint(__uint_as_float(o[hh * 16 + e]) * fa +
+                                                   __uint_as_float(ob[e]) * fb);
+              }
+            }
+            if (row_ok) {
+              const uint4 *gp = reinterpret_cast<const uint4 *>(p.gate + goff + cc * 32);
+              uint4 *op = reinterpret_cast<uint4 *>(p.out + goff + cc * 32);
+              uint4 gv[4];
+#pragma unroll
+              for (int v = 0; v < 4; ++v) gv[v] = __ldg(gp + v);
+#pragma unroll
+              for (int v = 0; v < 4; ++v) {
+                const uint32_t gw[4] = {gv[v].x, gv[v].y, gv[v].z, gv[v].w};
+                uint32_t ow[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const int c0 = cc * 32 + v * 8 + 2 * e;
+                  const float d0 = __uint_as_float(o[v * 8 + 2 * e]) * inv_l -
+                                   lam * hn_smem[c0 * kBM + r];
+                  const float d1 = __uint_as_float(o[v * 8 + 2 * e + 1]) * inv_l -
+                                   lam * hn_smem[(c0 + 1) * kBM + r];
+                  ow[e] = pack_bf16x2(bf16lo_to_f32(gw[e]) * d0, bf16hi_to_f32(gw[e]) * d1);
+                }
+                op[v] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(o_free(x));
+        if (pl.split) mbar_arrive(o_free(1));
+      }
+      pv_seen[0] += static_cast<uint32_t>(tiles0);
+      if (pl.nslot == 2) pv_seen[1] += static_cast<uint32_t>(tiles1);
+    }
   } else {
-    // =============================== softmax + epilogue (one warpgroup per slot)
+    // =============================== softmax (one warpgroup per slot)
+    regs_increase<kSoftmaxRegs>();
     const int x = warp >> 2;          // slot
     const int wq = warp & 3;          // TMEM lane quarter
     const int r = threadIdx.x & 127;  // row in the block = TMEM lane
@@ -424,7 +580,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const float sl2 = p.scale_log2;
     uint32_t s_waits = 0;
     uint32_t o_seen = 0;  // PV commits of this slot in finished phases
-    bool hn_waited = false;
+    uint32_t handoffs = 0;  // heads handed to the epilogue warpgroup
     bool ok = true;
     for (int ph = 0; ph < n_phases && ok; ++ph) {
       const PhasePlan pl = phase_plan(ph, n_heads, n_tiles);
@@ -477,14 +633,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           mt = fmaxf(ma, mb);
         } else {
           mt = -INFINITY;
-#pragma unroll
+#pragma unroll 1
           for (int cc = 0; cc < kBN / 32; ++cc) {
+            const int cls = chunk_class(cc, c_lo, c_hi);
+            if (cls == kChunkEmpty) continue;
             uint32_t raw[32];
             tmem_ld32_sync(t_s(x) + lane_off + cc * 32, raw);
+            if (cls == kChunkFull) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int c = cc * 32 + e;
-              if (c >= c_lo && c <= c_hi) mt = fmaxf(mt, __uint_as_float(raw[e]));
+              for (int e = 0; e < 32; e += 2)
+                mt = fmax3(mt, __uint_as_float(raw[e]), __uint_as_float(raw[e + 1]));
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e) {
+                const int c = cc * 32 + e;
+                if (c >= c_lo && c <= c_hi) mt = fmaxf(mt, __uint_as_float(raw[e]));
+              }
             }
           }
         }
@@ -502,32 +666,56 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint64_t sl2x2 = f2_make(sl2, sl2);
         const uint64_t negm2 = f2_make(-m_safe, -m_safe);
         uint64_t rs2 = f2_make(0.f, 0.f);
+        if (!masked) {
 #pragma unroll
-        for (int cc = 0; cc < kBN / 32; ++cc) {
-          uint32_t raw[32];
-          tmem_ld32_sync(t_s(x) + lane_off + cc * 32, raw);
-          uint32_t pk[16];
+          for (int cc = 0; cc < kBN / 32; ++cc) {
+            uint32_t raw[32];
+            tmem_ld32_sync(t_s(x) + lane_off + cc * 32, raw);
+            uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            float t0v, t1v;
-            f2_split(f2_fma(f2_from_bits(raw[2 * e], raw[2 * e + 1]), sl2x2, negm2), t0v, t1v);
-            float p0, p1;
-            if (masked) {
-              const int c0 = cc * 32 + 2 * e;
-              if (!(c0 >= c_lo && c0 <= c_hi)) t0v = -INFINITY;
-              if (!(c0 + 1 >= c_lo && c0 + 1 <= c_hi)) t1v = -INFINITY;
-              p0 = ex2_approx(t0v);
-              p1 = ex2_approx(t1v);
-            } else if (e >= 16 - kPolyPairs) {
-              exp2_poly_x2(t0v, t1v, p0, p1);
-            } else {
-              p0 = ex2_approx(t0v);
-              p1 = ex2_approx(t1v);
+            for (int e = 0; e < 16; ++e) {
+              float t0v, t1v;
+              f2_split(f2_fma(f2_from_bits(raw[2 * e], raw[2 * e + 1]), sl2x2, negm2), t0v, t1v);
+              float p0, p1;
+              if (e >= 16 - kPolyPairs) {
+                exp2_poly_x2(t0v, t1v, p0, p1);
+              } else {
+                p0 = ex2_approx(t0v);
+                p1 = ex2_approx(t1v);
+              }
+              rs2 = f2_add(rs2, f2_make(p0, p1));
+              pk[e] = pack_bf16x2(p0, p1);
             }
-            rs2 = f2_add(rs2, f2_make(p0, p1));
-            pk[e] = pack_bf16x2(p0, p1);
+            tmem_st16(t_s(x) + lane_off + cc * 16, pk);
           }
-          tmem_st16(t_s(x) + lane_off + cc * 16, pk);
+        } else {
+#pragma unroll 1
+          for (int cc = 0; cc < kBN / 32; ++cc) {
+            const int cls = chunk_class(cc, c_lo, c_hi);
+            uint32_t pk[16];
+            if (cls == kChunkEmpty) {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) pk[e] = 0u;
+            } else {
+              uint32_t raw[32];
+              tmem_ld32_sync(t_s(x) + lane_off + cc * 32, raw);
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                float t0v, t1v;
+                f2_split(f2_fma(f2_from_bits(raw[2 * e], raw[2 * e + 1]), sl2x2, negm2), t0v, t1v);
+                if (cls == kChunkMixed) {
+                  const int c0 = cc * 32 + 2 * e;
+                  if (!(c0 >= c_lo && c0 <= c_hi)) t0v = -INFINITY;
+                  if (!(c0 + 1 >= c_lo && c0 + 1 <= c_hi)) t1v = -INFINITY;
+                }
+                const float p0 = ex2_approx(t0v);
+                const float p1 = ex2_approx(t1v);
+                rs2 = f2_add(rs2, f2_make(p0, p1));
+                pk[e] = pack_bf16x2(p0, p1);
+              }
+            }
+            tmem_st16(t_s(x) + lane_off + cc * 16, pk);
+          }
         }
         float rs0, rs1;
         f2_split(rs2, rs0, rs1);
@@ -555,107 +743,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mbar_arrive(p_full(x));
       }
       if (!ok) break;
-      // ---- epilogue: wait for the last PV of this slot in this phase
-      const uint32_t last = o_seen + static_cast<uint32_t>(my_tiles - 1);
-      o_seen += static_cast<uint32_t>(my_tiles);
-      ok = mbar_wait(o_done(x), last & 1u, abort_flag);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      float l_tot = l_run;
-      // split phase: slot B hands (m, l) to slot A, which merges O_A and O_B;
-      // both maxima are integral, so the merge factors are exact powers of two
-      float fa = 1.f, fb = 0.f;
-      if (pl.split) {
-        float *pub = reinterpret_cast<float *>(smem + L::kQOff + L::kQBytes);  // Q_B is idle
-        if (x == 1) {
-          pub[r] = m_run;
-          pub[kBM + r] = l_run;
-          mbar_arrive(split_ready);
-          break;  // slot B is done; slot A writes the output
-        }
-        ok = mbar_wait(split_ready, 0, abort_flag);
+      // ---- hand the head to the epilogue warpgroup: row sum and reference
+      // max.  The epilogue must have read the previous hand-off first (a
+      // phase with one tile per slot waits on nothing else from it).
+      if (handoffs > 0) {
+        ok = mbar_wait(stat_free(x), (handoffs - 1) & 1u, abort_flag);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
-        tc_fence_after();
-        const float m_b = pub[r], l_b = pub[kBM + r];
-        const float m = fmaxf(m_run, m_b);
-        fa = (m_run == -INFINITY) ? 0.f : exp2_int(m_run - m);
-        fb = (m_b == -INFINITY) ? 0.f : exp2_int(m_b - m);
-        l_tot = l_run * fa + l_b * fb;
       }
-      const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
-      if (hi == 0) {
-        // noise head: keep H_N = O / l on chip for the group's signal heads
-#pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t o[32];
-          tmem_ld32_sync(t_o(x) + lane_off + cc * 32, o);
-          if (pl.split) {
-            uint32_t ob[32];
-            tmem_ld32_sync(t_o(1) + lane_off + cc * 32, ob);
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-              o[e] = __float_as_uint(__uint_as_float(o[e]) * fa + __uint_as_float(ob[e]) * fb);
-          }
-#pragma unroll
-          for (int e = 0; e < 32; ++e) hn_smem[(cc * 32 + e) * kBM + r] = __uint_as_float(o[e]) * inv_l;
-        }
-        tc_fence_before();
-        mbar_arrive(o_free(x));
-        mbar_arrive(hn_ready);
-      } else {
-        if (!hn_waited) {
-          if (x != 0) {
-            ok = mbar_wait(hn_ready, 0, abort_flag);
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok) break;
-          }
-          hn_waited = true;
-        }
-        const int h = p.g * kvh + (hi - 1);
-        const bool row_ok = i < p.T;
-        const int64_t row = static_cast<int64_t>(b) * p.T + i;
-        float lam = 0.f;
-        if (row_ok) lam = __bfloat162float(p.lam[row * p.Hs + h]);
-        const int64_t goff = (row * p.Hs + h) * static_cast<int64_t>(D);
-#pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t o[32];
-          tmem_ld32_sync(t_o(x) + lane_off + cc * 32, o);
-          if (pl.split) {
-            uint32_t ob[32];
-            tmem_ld32_sync(t_o(1) + lane_off + cc * 32, ob);
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-              o[e] = __float_as_uint(__uint_as_float(o[e]) * fa + __uint_as_float(ob[e]) * fb);
-          }
-          if (row_ok) {
-            const uint4 *gp = reinterpret_cast<const uint4 *>(p.gate + goff + cc * 32);
-            uint4 *op = reinterpret_cast<uint4 *>(p.out + goff + cc * 32);
-            uint4 gv[4];
-#pragma unroll
-            for (int v = 0; v < 4; ++v) gv[v] = __ldg(gp + v);
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              const uint32_t gw[4] = {gv[v].x, gv[v].y, gv[v].z, gv[v].w};
-              uint32_t ow[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int c0 = cc * 32 + v * 8 + 2 * e;
-                const float d0 = __uint_as_float(o[v * 8 + 2 * e]) * inv_l -
-                                 lam * hn_smem[c0 * kBM + r];
-                const float d1 = __uint_as_float(o[v * 8 + 2 * e + 1]) * inv_l -
-                                 lam * hn_smem[(c0 + 1) * kBM + r];
-                ow[e] = pack_bf16x2(bf16lo_to_f32(gw[e]) * d0, bf16hi_to_f32(gw[e]) * d1);
-              }
-              op[v] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
-            }
-          }
-        }
-        tc_fence_before();
-        mbar_arrive(o_free(x));
-      }
+      ++handoffs;
+      stat[x * 2 * kBM + r] = l_run;
+      stat[x * 2 * kBM + kBM + r] = m_run;
+      o_seen += static_cast<uint32_t>(my_tiles);
+      mbar_arrive(epi_go(x));
     }
   }
 

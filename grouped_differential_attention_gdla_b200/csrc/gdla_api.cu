@@ -83,6 +83,12 @@ int launch_attn(const void *q_sig, const void *q_noise, const void *k, const voi
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return GDLA_ERR_CUDA;
+  // The kernel re-splits its register pool between warpgroups (setmaxnreg);
+  // that is only sound for the per-thread count it was written for, so any
+  // other build is refused rather than launched.
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return GDLA_ERR_CUDA;
+  if (fa.numRegs != static_cast<int>(gdla::kLaunchRegs)) return GDLA_ERR_UNSUPPORTED;
   const uint64_t blocks = static_cast<uint64_t>(prm.n_qblk) * B * static_cast<uint64_t>(Hn);
   if (blocks > 0x7fffffffull) return GDLA_ERR_UNSUPPORTED;
   kern<<<static_cast<unsigned>(blocks), gdla::kAttnThreads, smem, stream>>>(tm_qs, tm_qn, tm_k,
