@@ -485,6 +485,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int e_i = 0; e_i < n_epi && ok; ++e_i) {
         const int x = e_i;
         const int hi = x == 0 ? pl.head0 : pl.head1;
+        if (hi != 0 && row_ok) {
+          // the gate row and lambda of this head head for L2 while the slot
+          // still computes, so the loads below do not wait on HBM
+          const int h = p.g * kvh + (hi - 1);
+          const __nv_bfloat16 *gr = p.gate + (row * p.Hs + h) * static_cast<int64_t>(D);
+#pragma unroll
+          for (int ln = 0; ln < D * 2 / 128; ++ln) prefetch_l2(gr + ln * 64);
+          prefetch_l2(p.lam + row * p.Hs + h);
+        }
         float fa = 1.f, fb = 0.f, l_tot;
         if (pl.split) {
           ok = wait_slot(0, pv_seen[0] + tiles0 - 1);
