@@ -89,10 +89,24 @@ int launch_attn(const void *q_sig, const void *q_noise, const void *k, const voi
   cudaFuncAttributes fa;
   if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return GDLA_ERR_CUDA;
   if (fa.numRegs != static_cast<int>(gdla::kLaunchRegs)) return GDLA_ERR_UNSUPPORTED;
-  const uint64_t blocks = static_cast<uint64_t>(prm.n_qblk) * B * static_cast<uint64_t>(Hn);
-  if (blocks > 0x7fffffffull) return GDLA_ERR_UNSUPPORTED;
-  kern<<<static_cast<unsigned>(blocks), gdla::kAttnThreads, smem, stream>>>(tm_qs, tm_qn, tm_k,
-                                                                            tm_v, prm);
+  const uint64_t items = static_cast<uint64_t>(prm.n_qblk) * B * static_cast<uint64_t>(Hn);
+  if (items > 0x7fffffffull) return GDLA_ERR_UNSUPPORTED;
+  gdla::AttnParams run = prm;
+  run.n_items = static_cast<int>(items);
+  // Sliding-window items are short and alike: one resident CTA per SM walks
+  // them, so each CTA's next item loads while its current one finishes.  Full
+  // attention items differ in length; one CTA each lets the hardware balance.
+  uint64_t grid = items;
+  if (prm.window > 0) {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        sms <= 0)
+      return GDLA_ERR_CUDA;
+    if (grid > static_cast<uint64_t>(sms)) grid = static_cast<uint64_t>(sms);
+  }
+  kern<<<static_cast<unsigned>(grid), gdla::kAttnThreads, smem, stream>>>(tm_qs, tm_qn, tm_k,
+                                                                          tm_v, run);
   return cudaGetLastError() == cudaSuccess ? GDLA_OK : GDLA_ERR_CUDA;
 }
 

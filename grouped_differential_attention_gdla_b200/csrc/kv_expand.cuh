@@ -72,7 +72,6 @@ __global__ void __launch_bounds__(kExpThreads, 1)
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
 
   const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
   const int64_t m0 = static_cast<int64_t>(blockIdx.x) * kExpBM;
   const int DL = p.d_latent;
   const int n_kb = DL / 64;         // 64-wide column blocks of the latent tile
