@@ -54,13 +54,19 @@ constexpr int kAttnThreads = 16 * 32;
 // epilogue warpgroups give registers back and the softmax warpgroups take
 // them, within the launch pool.  The host refuses to launch a build whose
 // per-thread register count differs from kLaunchRegs.
+// The sliding-window kernel's softmax has no unmasked-tile path and its
+// epilogue stages tiles through shared memory, so it moves registers from
+// the softmax to the epilogue.
 constexpr uint32_t kLaunchRegs = 128;
-constexpr uint32_t kSoftmaxRegs = 152;
-constexpr uint32_t kEpilogueRegs = 96;
-constexpr uint32_t kControlRegs = 112;
-static_assert(2 * 128 * kSoftmaxRegs + 128 * kEpilogueRegs + 128 * kControlRegs <=
-                  kAttnThreads * kLaunchRegs,
-              "register split must fit in the launch pool");
+template <bool kWin>
+struct RegSplit {
+  static constexpr uint32_t kSoftmax = kWin ? 144 : 152;
+  static constexpr uint32_t kEpilogue = kWin ? 112 : 96;
+  static constexpr uint32_t kControl = 112;
+  static_assert(2 * 128 * kSoftmax + 128 * kEpilogue + 128 * kControl <=
+                    kAttnThreads * kLaunchRegs,
+                "register split must fit in the launch pool");
+};
 constexpr int kSlotThreads = 128;          // one warpgroup per slot
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: O is rescaled only if the max grows by > 2^8
 // Of every 16 score pairs in a 32-column chunk of an unmasked tile, this many
@@ -89,7 +95,10 @@ template <int D>
 struct AttnSmemLayout {
   static constexpr uint32_t kQBytes = kBM * D * 2;
   static constexpr uint32_t kKvBytes = kBN * D * 2;
-  static constexpr uint32_t kHnBytes = kBM * D * 4;
+  static constexpr uint32_t kHnBytes = kBM * D * 4;  // H_N fp32
+  // Sliding window: the ring keeps two stages and the third holds the
+  // epilogue's gate/output tile, [D/64] 128B-swizzled halves of [kBM][64].
+  static constexpr uint32_t kStageHalf = kBM * 128;
   static constexpr uint32_t kQOff = 0;
   static constexpr uint32_t kKvOff = kQOff + 2 * kQBytes;
   static constexpr uint32_t kHnOff = kKvOff + kKvStages * kKvBytes;
@@ -97,8 +106,8 @@ struct AttnSmemLayout {
   static constexpr uint32_t kStatBytes = 2 * 2 * kBM * 4;
   static constexpr uint32_t kBarOff = kStatOff + kStatBytes;
   // q_full[2] q_empty[2] kv_full[S] kv_empty[S] s_full[2] p_full[2] o_done[2]
-  // o_free[2] epi_go[2] stat_free[2]
-  static constexpr uint32_t kNumBars = 2 + 2 + 2 * kKvStages + 2 + 2 + 2 + 2 + 2 + 2;
+  // o_free[2] epi_go[2] stat_free[2] g_full g_done
+  static constexpr uint32_t kNumBars = 2 + 2 + 2 * kKvStages + 2 + 2 + 2 + 2 + 2 + 2 + 2;
   static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;
   static constexpr uint32_t kBytes = kMiscOff + 16;
 };
@@ -192,12 +201,16 @@ __device__ __forceinline__ void write_status(int *status, int code) {
   if (status) atomicExch(status, code);
 }
 
-template <int D>
+// kWin: sliding-window instantiation (p.window > 0); otherwise full
+// attention (causal or not).
+template <int D, bool kWin>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     gdla_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_qs,
                          const __grid_constant__ CUtensorMap tm_qn,
                          const __grid_constant__ CUtensorMap tm_k,
-                         const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+                         const __grid_constant__ CUtensorMap tm_v,
+                         const __grid_constant__ CUtensorMap tm_gate,
+                         const __grid_constant__ CUtensorMap tm_out, const AttnParams p) {
   using L = AttnSmemLayout<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   // swizzled TMA/UMMA tiles need a 1024-byte aligned base; refuse to run otherwise
@@ -217,6 +230,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   auto o_free = [&](int x) { return bar0 + 8u * (10 + 2 * kKvStages + x); };
   auto epi_go = [&](int x) { return bar0 + 8u * (12 + 2 * kKvStages + x); };
   auto stat_free = [&](int x) { return bar0 + 8u * (14 + 2 * kKvStages + x); };
+  const uint32_t g_full = bar0 + 8u * (16 + 2 * kKvStages);  // staged gate tile landed
+  const uint32_t g_done = bar0 + 8u * (17 + 2 * kKvStages);  // staged output tile written
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
   float *hn_smem = reinterpret_cast<float *>(smem + L::kHnOff);  // [D][kBM]
@@ -224,6 +239,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   const int warp = threadIdx.x >> 5;
 
+  // K/V ring depth: two stages in sliding-window mode, whose third stage is
+  // the epilogue's staging tile
+  constexpr uint32_t n_stages = kWin ? 2u : static_cast<uint32_t>(kKvStages);
   const int n_heads = p.g + 1;  // noise head + g signal heads
   const int n_phases = (n_heads + 1) / 2;
 
@@ -239,12 +257,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int s = 0; s < kKvStages; ++s) {
       mbar_init(kv_full(s), 1);
       // released once per entry by the lockstep issuer, or by both per-slot issuers
-      mbar_init(kv_empty(s), p.window > 0 ? 2 : 1);
+      mbar_init(kv_empty(s), kWin ? 2 : 1);
     }
     mbar_init(epi_go(0), kSlotThreads);
     mbar_init(epi_go(1), kSlotThreads);
     mbar_init(stat_free(0), kSlotThreads);
     mbar_init(stat_free(1), kSlotThreads);
+    mbar_init(g_full, 1);
+    mbar_init(g_done, kSlotThreads);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -263,7 +283,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (warp >= 12) {
   // =============================== control warpgroup (warps 12-15)
-  regs_decrease<kControlRegs>();
+  regs_decrease<RegSplit<kWin>::kControl>();
   if (warp == kProducerWarp) {
     // =============================== TMA producer
     // The whole warp runs the loop (warp-uniform control and addresses); one
@@ -285,9 +305,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
       const WorkItem w = work_item(p, item);
       auto load_kv = [&](int t, bool is_v) {
-        const int s = static_cast<int>(c % kKvStages);
+        const int s = static_cast<int>(c % n_stages);
         ok = __all_sync(0xffffffffu,
-                        mbar_wait(kv_empty(s), ((c / kKvStages) & 1u) ^ 1u, abort_flag));
+                        mbar_wait(kv_empty(s), ((c / n_stages) & 1u) ^ 1u, abort_flag));
         if (!ok) return;
         const uint32_t dst = sbase + L::kKvOff + s * L::kKvBytes;
         if (leader) {
@@ -332,14 +352,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     if (!ok && leader) {
       // unwinding: let the copies already issued land before the CTA exits
-      for (int s = 0; s < kKvStages; ++s) {
-        const uint32_t issued = c > static_cast<uint32_t>(s) ? (c - 1 - s) / kKvStages + 1 : 0;
+      for (uint32_t s = 0; s < n_stages; ++s) {
+        const uint32_t issued = c > s ? (c - 1 - s) / n_stages + 1 : 0;
         if (issued) mbar_wait_for(kv_full(s), (issued - 1) & 1u, 100000000ull);
       }
       for (int x = 0; x < 2; ++x)
         if (q_uses[x]) mbar_wait_for(q_full(x), (q_uses[x] - 1) & 1u, 100000000ull);
     }
-  } else if (warp == kMmaWarp && p.window == 0) {
+  } else if (!kWin && warp == kMmaWarp) {
     // =============================== MMA issuer for both slots, in lockstep
     // (full attention).  Per slot X the issue order is S_X(t) .. PV_X(t),
     // S_X(t+A), and slot A's pair goes first: slot B's MMAs run while slot
@@ -374,8 +394,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     };
     // waits for the next ring entry; returns its stage and smem address
     auto next_stage = [&](uint32_t &base) -> int {
-      const int s = static_cast<int>(c % kKvStages);
-      ok = __all_sync(0xffffffffu, mbar_wait(kv_full(s), (c / kKvStages) & 1u, abort_flag));
+      const int s = static_cast<int>(c % n_stages);
+      ok = __all_sync(0xffffffffu, mbar_wait(kv_full(s), (c / n_stages) & 1u, abort_flag));
       tc_fence_after();
       base = sbase + L::kKvOff + s * L::kKvBytes;
       ++c;
@@ -482,7 +502,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (o_commits[0]) mbar_wait_for(o_done(0), (o_commits[0] - 1) & 1u, 100000000ull);
       if (o_commits[1]) mbar_wait_for(o_done(1), (o_commits[1] - 1) & 1u, 100000000ull);
     }
-  } else if ((warp == kMmaWarp || warp == kMmaWarp + 1) && p.window > 0) {
+  } else if (kWin && (warp == kMmaWarp || warp == kMmaWarp + 1)) {
     // =============================== MMA issuers, one warp per slot
     // (sliding window, where a CTA's few tiles per head make the phase
     // boundaries, not the steady state, the critical path)
@@ -520,8 +540,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int last_t = pl.split ? x + 2 * ((w.n_tiles - 1 - x) / 2) : w.n_tiles - 1;
         bool first_pv = true;
         auto entry = [&](int t, bool is_v) {
-          const int s = static_cast<int>(c % kKvStages);
-          ok = __all_sync(0xffffffffu, mbar_wait(kv_full(s), (c / kKvStages) & 1u, abort_flag));
+          const int s = static_cast<int>(c % n_stages);
+          ok = __all_sync(0xffffffffu, mbar_wait(kv_full(s), (c / n_stages) & 1u, abort_flag));
           ++c;
           if (!ok) return;
           const bool mine = active && (!pl.split || (t & 1) == x);
@@ -580,12 +600,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
   } else if (warp >= 8) {
     // =============================== epilogue warpgroup (warps 8-11)
-    regs_decrease<kEpilogueRegs>();
+    // Sliding window (staged): a signal head's gate tile [128 rows][d]
+    // arrives by TMA in a 128B-swizzled staging buffer, each thread
+    // overwrites its row with the output in place, and TMA stores the tile:
+    // global traffic moves as whole tiles instead of 16-byte pieces of 128
+    // rows.  Full attention, where the epilogue is off the critical path,
+    // reads the gate and writes the output row by row.
+    regs_decrease<RegSplit<kWin>::kEpilogue>();
     const int wq = warp & 3;          // TMEM lane quarter
     const int r = threadIdx.x & 127;  // row in the block = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    constexpr bool staged = kWin;
+    const uint32_t gbuf = sbase + L::kKvOff + 2 * L::kKvBytes;  // staging (window mode)
+    const bool issuer = kWin && warp == 8 ? elect_one() : false;
+    // H_N: [d/4][kBM] float4 in the window kernel (one 16-byte load per 4
+    // columns), [d][kBM] floats in the full kernel (fewer live registers)
+    float4 *hn4 = reinterpret_cast<float4 *>(hn_smem);
     uint32_t go_waits[2] = {0, 0};
     uint32_t pv_seen[2] = {0, 0};  // PV commits per slot in finished phases
+    uint32_t g_issued = 0, g_seen = 0;  // staged gate tiles loaded / consumed
     bool ok = true;
     // waits until slot x has handed over the head it ran in this phase and
     // its last PV (number `last` of the slot) has completed
@@ -613,14 +646,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int e_i = 0; e_i < n_epi && ok; ++e_i) {
           const int x = e_i;
           const int hi = x == 0 ? pl.head0 : pl.head1;
-          if (hi != 0 && row_ok) {
-            // the gate row and lambda of this head head for L2 while the slot
-            // still computes, so the loads below do not wait on HBM
-            const int h = p.g * kvh + (hi - 1);
-            const __nv_bfloat16 *gr = p.gate + (row * p.Hs + h) * static_cast<int64_t>(D);
-  #pragma unroll
-            for (int ln = 0; ln < D * 2 / 128; ++ln) prefetch_l2(gr + ln * 64);
-            prefetch_l2(p.lam + row * p.Hs + h);
+          const int h = p.g * kvh + (hi - 1);  // signal head (hi >= 1)
+          if (hi != 0) {
+            if (staged) {
+              if (issuer) {
+                // the previous tile's stores must have read the buffer
+                bulk_wait_group_read0();
+                fence_proxy_async_smem();
+                mbar_arrive_expect_tx(g_full, (D / 64) * L::kStageHalf);
+#pragma unroll
+                for (int hf = 0; hf < D / 64; ++hf)
+                  tma_load_3d(gbuf + hf * L::kStageHalf, &tm_gate, g_full, h * D + hf * 64, w.q0,
+                              w.b);
+              }
+              ++g_issued;
+            } else if (row_ok) {
+              // the gate row heads for L2 while the slot still computes
+              const __nv_bfloat16 *gr = p.gate + (row * p.Hs + h) * static_cast<int64_t>(D);
+#pragma unroll
+              for (int ln = 0; ln < D * 2 / 128; ++ln) prefetch_l2(gr + ln * 64);
+            }
+            if (row_ok) prefetch_l2(p.lam + row * p.Hs + h);
           }
           float fa = 1.f, fb = 0.f, l_tot;
           if (pl.split) {
@@ -643,33 +689,111 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mbar_arrive(stat_free(x));
           }
           const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
+          // O of this head, chunk cc (32 columns), merged over a split head's slots
+          auto load_o = [&](int cc, uint32_t (&o)[32]) {
+            tmem_ld32_sync(t_o(x) + lane_off + cc * 32, o);
+            if (pl.split) {
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh) {
+                uint32_t ob[16];
+                tmem_ld16_sync(t_o(1) + lane_off + cc * 32 + hh * 16, ob);
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                  o[hh * 16 + e] = __float_as_uint(__uint_as_float(o[hh * 16 + e]) * fa +
+                                                   __uint_as_float(ob[e]) * fb);
+              }
+            }
+          };
+          // out = G (.) (O/l - lambda H_N) for 8 columns from column c
+          auto combine8 = [&](const uint32_t *o8, int c, uint4 gv, float lam) -> uint4 {
+            float hn[8];
+            if (kWin) {
+              const float4 n0 = hn4[(c >> 2) * kBM + r];
+              const float4 n1 = hn4[((c >> 2) + 1) * kBM + r];
+              hn[0] = n0.x; hn[1] = n0.y; hn[2] = n0.z; hn[3] = n0.w;
+              hn[4] = n1.x; hn[5] = n1.y; hn[6] = n1.z; hn[7] = n1.w;
+            }
+            const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+            uint32_t ow[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              if (!kWin) {
+                hn[2 * e] = hn_smem[(c + 2 * e) * kBM + r];
+                hn[2 * e + 1] = hn_smem[(c + 2 * e + 1) * kBM + r];
+              }
+              const float d0 = __uint_as_float(o8[2 * e]) * inv_l - lam * hn[2 * e];
+              const float d1 = __uint_as_float(o8[2 * e + 1]) * inv_l - lam * hn[2 * e + 1];
+              ow[e] = pack_bf16x2(bf16lo_to_f32(gw[e]) * d0, bf16hi_to_f32(gw[e]) * d1);
+            }
+            return make_uint4(ow[0], ow[1], ow[2], ow[3]);
+          };
           if (hi == 0) {
             // noise head (never split: it runs in phase 0 next to signal head 0):
             // H_N = O / l stays in shared memory for the group's signal heads;
             // this warpgroup is also the only reader, row by row
-  #pragma unroll
+#pragma unroll
             for (int cc = 0; cc < D / 32; ++cc) {
               uint32_t o[32];
               tmem_ld32_sync(t_o(x) + lane_off + cc * 32, o);
-  #pragma unroll
-              for (int e = 0; e < 32; ++e)
-                hn_smem[(cc * 32 + e) * kBM + r] = __uint_as_float(o[e]) * inv_l;
+              if (kWin) {
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                  hn4[(cc * 8 + q) * kBM + r] = make_float4(
+                      __uint_as_float(o[4 * q]) * inv_l, __uint_as_float(o[4 * q + 1]) * inv_l,
+                      __uint_as_float(o[4 * q + 2]) * inv_l, __uint_as_float(o[4 * q + 3]) * inv_l);
+              } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                  hn_smem[(cc * 32 + e) * kBM + r] = __uint_as_float(o[e]) * inv_l;
+              }
             }
+          } else if (staged) {
+            const float lam = row_ok ? __bfloat162float(p.lam[row * p.Hs + h]) : 0.f;
+            ok = __all_sync(0xffffffffu, mbar_wait(g_full, g_seen & 1u, abort_flag));
+            ++g_seen;
+            if (!ok) break;
+            // row r of a 128B-swizzled [128][64] half: 16-byte unit j sits at j ^ (r % 8)
+            const uint32_t rbase = gbuf + static_cast<uint32_t>(r) * 128u;
+#pragma unroll
+            for (int cc = 0; cc < D / 32; ++cc) {
+              uint32_t o[32];
+              load_o(cc, o);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const int j = (cc & 1) * 4 + q;
+                const uint32_t addr = rbase + static_cast<uint32_t>(cc >> 1) * L::kStageHalf +
+                                      (static_cast<uint32_t>(j ^ (r & 7)) << 4);
+                sts128(addr, combine8(o + q * 8, cc * 32 + q * 8, lds128(addr), lam));
+              }
+            }
+            // every row written (generic proxy) before the TMA store reads the tile
+            fence_proxy_async_smem();
+            mbar_arrive(g_done);
+            if (issuer) {
+              ok = mbar_wait(g_done, (g_seen - 1) & 1u, abort_flag);
+              if (ok) {
+#pragma unroll
+                for (int hf = 0; hf < D / 64; ++hf)
+                  tma_store_3d(&tm_out, gbuf + hf * L::kStageHalf, h * D + hf * 64, w.q0, w.b);
+                bulk_commit_group();
+              }
+            }
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
           } else {
-            const int h = p.g * kvh + (hi - 1);
             const int64_t goff = (row * p.Hs + h) * static_cast<int64_t>(D);
             float lam = 0.f;
             if (row_ok) lam = __bfloat162float(p.lam[row * p.Hs + h]);
-  #pragma unroll
+#pragma unroll
             for (int cc = 0; cc < D / 32; ++cc) {
               uint32_t o[32];
               tmem_ld32_sync(t_o(x) + lane_off + cc * 32, o);
               if (pl.split) {
-  #pragma unroll
+#pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                   uint32_t ob[16];
                   tmem_ld16_sync(t_o(1) + lane_off + cc * 32 + hh * 16, ob);
-  #pragma unroll
+#pragma unroll
                   for (int e = 0; e < 16; ++e)
                     o[hh * 16 + e] = __float_as_uint(__uint_as_float(o[hh * 16 + e]) * fa +
                                                      __uint_as_float(ob[e]) * fb);
@@ -679,13 +803,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 const uint4 *gp = reinterpret_cast<const uint4 *>(p.gate + goff + cc * 32);
                 uint4 *op = reinterpret_cast<uint4 *>(p.out + goff + cc * 32);
                 uint4 gv[4];
-  #pragma unroll
+#pragma unroll
                 for (int v = 0; v < 4; ++v) gv[v] = __ldg(gp + v);
-  #pragma unroll
+#pragma unroll
                 for (int v = 0; v < 4; ++v) {
                   const uint32_t gw[4] = {gv[v].x, gv[v].y, gv[v].z, gv[v].w};
                   uint32_t ow[4];
-  #pragma unroll
+#pragma unroll
                   for (int e = 0; e < 4; ++e) {
                     const int c0 = cc * 32 + v * 8 + 2 * e;
                     const float d0 = __uint_as_float(o[v * 8 + 2 * e]) * inv_l -
@@ -707,9 +831,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (pl.nslot == 2) pv_seen[1] += static_cast<uint32_t>(tiles1);
       }
     }
+    if (kWin && issuer) {
+      // a gate tile still in flight (after an abort) lands before the CTA exits;
+      // every output tile store completes
+      if (g_issued > g_seen) mbar_wait_for(g_full, (g_issued - 1) & 1u, 100000000ull);
+      bulk_wait_group0();
+    }
   } else {
     // =============================== softmax (one warpgroup per slot)
-    regs_increase<kSoftmaxRegs>();
+    regs_increase<RegSplit<kWin>::kSoftmax>();
     const int x = warp >> 2;          // slot
     const int wq = warp & 3;          // TMEM lane quarter
     const int r = threadIdx.x & 127;  // row in the block = TMEM lane
@@ -758,13 +888,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
           // pass 1: row max of the tile (64 columns live at a time)
           float mt;
-          if (!masked) {
+          if (!kWin && !masked) {
             float ma = -INFINITY, mb = -INFINITY;
-  #pragma unroll
+#pragma unroll
             for (int cc = 0; cc < kBN / 32; cc += 2) {
               uint32_t r0[32], r1[32];
               tmem_ld32x2_sync(t_s(x) + lane_off + cc * 32, t_s(x) + lane_off + cc * 32 + 32, r0, r1);
-  #pragma unroll
+#pragma unroll
               for (int e = 0; e < 32; e += 2) {
                 ma = fmax3(ma, __uint_as_float(r0[e]), __uint_as_float(r0[e + 1]));
                 mb = fmax3(mb, __uint_as_float(r1[e]), __uint_as_float(r1[e + 1]));
@@ -773,18 +903,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mt = fmaxf(ma, mb);
           } else {
             mt = -INFINITY;
-  #pragma unroll 1
+#pragma unroll 1
             for (int cc = 0; cc < kBN / 32; ++cc) {
-              const int cls = chunk_class(cc, c_lo, c_hi);
+              const int cls = kWin ? chunk_class(cc, c_lo, c_hi) : kChunkMixed;
               if (cls == kChunkEmpty) continue;
               uint32_t raw[32];
               tmem_ld32_sync(t_s(x) + lane_off + cc * 32, raw);
               if (cls == kChunkFull) {
-  #pragma unroll
+#pragma unroll
                 for (int e = 0; e < 32; e += 2)
                   mt = fmax3(mt, __uint_as_float(raw[e]), __uint_as_float(raw[e + 1]));
               } else {
-  #pragma unroll
+#pragma unroll
                 for (int e = 0; e < 32; ++e) {
                   const int c = cc * 32 + e;
                   if (c >= c_lo && c <= c_hi) mt = fmaxf(mt, __uint_as_float(raw[e]));
@@ -806,13 +936,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const uint64_t sl2x2 = f2_make(sl2, sl2);
           const uint64_t negm2 = f2_make(-m_safe, -m_safe);
           uint64_t rs2 = f2_make(0.f, 0.f);
-          if (!masked) {
-  #pragma unroll
+          if (!kWin && !masked) {
+#pragma unroll
             for (int cc = 0; cc < kBN / 32; ++cc) {
               uint32_t raw[32];
               tmem_ld32_sync(t_s(x) + lane_off + cc * 32, raw);
               uint32_t pk[16];
-  #pragma unroll
+#pragma unroll
               for (int e = 0; e < 16; ++e) {
                 float t0v, t1v;
                 f2_split(f2_fma(f2_from_bits(raw[2 * e], raw[2 * e + 1]), sl2x2, negm2), t0v, t1v);
@@ -829,17 +959,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               tmem_st16(t_s(x) + lane_off + cc * 16, pk);
             }
           } else {
-  #pragma unroll 1
+#pragma unroll 1
             for (int cc = 0; cc < kBN / 32; ++cc) {
-              const int cls = chunk_class(cc, c_lo, c_hi);
+              const int cls = kWin ? chunk_class(cc, c_lo, c_hi) : kChunkMixed;
               uint32_t pk[16];
               if (cls == kChunkEmpty) {
-  #pragma unroll
+#pragma unroll
                 for (int e = 0; e < 16; ++e) pk[e] = 0u;
               } else {
                 uint32_t raw[32];
                 tmem_ld32_sync(t_s(x) + lane_off + cc * 32, raw);
-  #pragma unroll
+#pragma unroll
                 for (int e = 0; e < 16; ++e) {
                   float t0v, t1v;
                   f2_split(f2_fma(f2_from_bits(raw[2 * e], raw[2 * e + 1]), sl2x2, negm2), t0v, t1v);
@@ -869,11 +999,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
-  #pragma unroll
+#pragma unroll
             for (int cc = 0; cc < D / 32; ++cc) {
               uint32_t o[32];
               tmem_ld32_sync(t_o(x) + lane_off + cc * 32, o);
-  #pragma unroll
+#pragma unroll
               for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
               tmem_st32(t_o(x) + lane_off + cc * 32, o);
             }

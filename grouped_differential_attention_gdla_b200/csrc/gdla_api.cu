@@ -68,18 +68,20 @@ template <int D>
 int launch_attn(const void *q_sig, const void *q_noise, const void *k, const void *v,
                 const gdla::AttnParams &prm, int Hs, int Hn, cudaStream_t stream) {
   using L = gdla::AttnSmemLayout<D>;
-  CUtensorMap tm_qs, tm_qn, tm_k, tm_v;
+  CUtensorMap tm_qs, tm_qn, tm_k, tm_v, tm_gate, tm_out;
   const uint64_t T = static_cast<uint64_t>(prm.T), B = static_cast<uint64_t>(prm.B);
   const uint64_t dqs[3] = {static_cast<uint64_t>(Hs) * D, T, B};
   const uint64_t dqn[3] = {static_cast<uint64_t>(Hn) * D, T, B};
   const uint32_t qbox[3] = {64, gdla::kBM, 1};
   const uint32_t kvbox[3] = {64, gdla::kBN, 1};
   if (!make_map(&tm_qs, q_sig, 3, dqs, qbox) || !make_map(&tm_qn, q_noise, 3, dqn, qbox) ||
-      !make_map(&tm_k, k, 3, dqn, kvbox) || !make_map(&tm_v, v, 3, dqn, kvbox))
+      !make_map(&tm_k, k, 3, dqn, kvbox) || !make_map(&tm_v, v, 3, dqn, kvbox) ||
+      !make_map(&tm_gate, prm.gate, 3, dqs, qbox) || !make_map(&tm_out, prm.out, 3, dqs, qbox))
     return GDLA_ERR_CUDA;
   // at least 116 KB so that one CTA (and one 512-column TMEM allocation) sits on an SM
   const uint32_t smem = L::kBytes > 118784u ? L::kBytes : 118784u;
-  auto kern = gdla::gdla_attn_fwd_kernel<D>;
+  auto kern = prm.window > 0 ? gdla::gdla_attn_fwd_kernel<D, true>
+                              : gdla::gdla_attn_fwd_kernel<D, false>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return GDLA_ERR_CUDA;
@@ -105,8 +107,8 @@ int launch_attn(const void *q_sig, const void *q_noise, const void *k, const voi
       return GDLA_ERR_CUDA;
     if (grid > static_cast<uint64_t>(sms)) grid = static_cast<uint64_t>(sms);
   }
-  kern<<<static_cast<unsigned>(grid), gdla::kAttnThreads, smem, stream>>>(tm_qs, tm_qn, tm_k,
-                                                                          tm_v, run);
+  kern<<<static_cast<unsigned>(grid), gdla::kAttnThreads, smem, stream>>>(
+      tm_qs, tm_qn, tm_k, tm_v, tm_gate, tm_out, run);
   return cudaGetLastError() == cudaSuccess ? GDLA_OK : GDLA_ERR_CUDA;
 }
 
