@@ -903,21 +903,39 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mt = fmaxf(ma, mb);
           } else {
             mt = -INFINITY;
+            if (kWin) {
+              // chunks no row of the warp keeps are not even read
 #pragma unroll 1
-            for (int cc = 0; cc < kBN / 32; ++cc) {
-              const int cls = kWin ? chunk_class(cc, c_lo, c_hi) : kChunkMixed;
-              if (cls == kChunkEmpty) continue;
-              uint32_t raw[32];
-              tmem_ld32_sync(t_s(x) + lane_off + cc * 32, raw);
-              if (cls == kChunkFull) {
+              for (int cc = 0; cc < kBN / 32; ++cc) {
+                const int cls = chunk_class(cc, c_lo, c_hi);
+                if (cls == kChunkEmpty) continue;
+                uint32_t raw[32];
+                tmem_ld32_sync(t_s(x) + lane_off + cc * 32, raw);
+                if (cls == kChunkFull) {
 #pragma unroll
-                for (int e = 0; e < 32; e += 2)
-                  mt = fmax3(mt, __uint_as_float(raw[e]), __uint_as_float(raw[e + 1]));
-              } else {
+                  for (int e = 0; e < 32; e += 2)
+                    mt = fmax3(mt, __uint_as_float(raw[e]), __uint_as_float(raw[e + 1]));
+                } else {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                  const int c = cc * 32 + e;
-                  if (c >= c_lo && c <= c_hi) mt = fmaxf(mt, __uint_as_float(raw[e]));
+                  for (int e = 0; e < 32; ++e) {
+                    const int c = cc * 32 + e;
+                    if (c >= c_lo && c <= c_hi) mt = fmaxf(mt, __uint_as_float(raw[e]));
+                  }
+                }
+              }
+            } else {
+#pragma unroll
+              for (int cp = 0; cp < kBN / 64; ++cp) {
+                uint32_t r2[2][32];
+                tmem_ld32x2_sync(t_s(x) + lane_off + cp * 64, t_s(x) + lane_off + cp * 64 + 32,
+                                 r2[0], r2[1]);
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+                  for (int e = 0; e < 32; ++e) {
+                    const int c = (cp * 2 + hh) * 32 + e;
+                    if (c >= c_lo && c <= c_hi) mt = fmaxf(mt, __uint_as_float(r2[hh][e]));
+                  }
                 }
               }
             }
@@ -936,32 +954,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const uint64_t sl2x2 = f2_make(sl2, sl2);
           const uint64_t negm2 = f2_make(-m_safe, -m_safe);
           uint64_t rs2 = f2_make(0.f, 0.f);
-          if (!kWin && !masked) {
-#pragma unroll
-            for (int cc = 0; cc < kBN / 32; ++cc) {
-              uint32_t raw[32];
-              tmem_ld32_sync(t_s(x) + lane_off + cc * 32, raw);
-              uint32_t pk[16];
-#pragma unroll
-              for (int e = 0; e < 16; ++e) {
-                float t0v, t1v;
-                f2_split(f2_fma(f2_from_bits(raw[2 * e], raw[2 * e + 1]), sl2x2, negm2), t0v, t1v);
-                float p0, p1;
-                if (e >= 16 - kPolyPairs) {
-                  exp2_poly_x2(t0v, t1v, p0, p1);
-                } else {
-                  p0 = ex2_approx(t0v);
-                  p1 = ex2_approx(t1v);
-                }
-                rs2 = f2_add(rs2, f2_make(p0, p1));
-                pk[e] = pack_bf16x2(p0, p1);
-              }
-              tmem_st16(t_s(x) + lane_off + cc * 16, pk);
-            }
-          } else {
+          if (kWin) {
+            // sliding window: chunks no row of the warp keeps are neither read
+            // nor exponentiated (their P is zero)
 #pragma unroll 1
             for (int cc = 0; cc < kBN / 32; ++cc) {
-              const int cls = kWin ? chunk_class(cc, c_lo, c_hi) : kChunkMixed;
+              const int cls = chunk_class(cc, c_lo, c_hi);
               uint32_t pk[16];
               if (cls == kChunkEmpty) {
 #pragma unroll
@@ -985,6 +983,60 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 }
               }
               tmem_st16(t_s(x) + lane_off + cc * 16, pk);
+            }
+          } else {
+            // full attention: the load of chunk cc+1 is in flight while chunk
+            // cc is exponentiated
+            uint32_t ra[32], rb[32];
+            tmem_ld32_sync(t_s(x) + lane_off, ra);
+            if (!masked) {
+#pragma unroll
+              for (int cc = 0; cc < kBN / 32; ++cc) {
+                uint32_t(&raw)[32] = (cc & 1) ? rb : ra;
+                uint32_t(&nxt)[32] = (cc & 1) ? ra : rb;
+                if (cc + 1 < kBN / 32) tmem_ld32(t_s(x) + lane_off + (cc + 1) * 32, nxt);
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                  float t0v, t1v;
+                  f2_split(f2_fma(f2_from_bits(raw[2 * e], raw[2 * e + 1]), sl2x2, negm2), t0v,
+                           t1v);
+                  float p0, p1;
+                  if (e >= 16 - kPolyPairs) {
+                    exp2_poly_x2(t0v, t1v, p0, p1);
+                  } else {
+                    p0 = ex2_approx(t0v);
+                    p1 = ex2_approx(t1v);
+                  }
+                  rs2 = f2_add(rs2, f2_make(p0, p1));
+                  pk[e] = pack_bf16x2(p0, p1);
+                }
+                tmem_st16(t_s(x) + lane_off + cc * 16, pk);
+                if (cc + 1 < kBN / 32) tmem_wait_ld_fence(nxt);
+              }
+            } else {
+#pragma unroll
+              for (int cc = 0; cc < kBN / 32; ++cc) {
+                uint32_t(&raw)[32] = (cc & 1) ? rb : ra;
+                uint32_t(&nxt)[32] = (cc & 1) ? ra : rb;
+                if (cc + 1 < kBN / 32) tmem_ld32(t_s(x) + lane_off + (cc + 1) * 32, nxt);
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                  float t0v, t1v;
+                  f2_split(f2_fma(f2_from_bits(raw[2 * e], raw[2 * e + 1]), sl2x2, negm2), t0v,
+                           t1v);
+                  const int c0 = cc * 32 + 2 * e;
+                  if (!(c0 >= c_lo && c0 <= c_hi)) t0v = -INFINITY;
+                  if (!(c0 + 1 >= c_lo && c0 + 1 <= c_hi)) t1v = -INFINITY;
+                  const float p0 = ex2_approx(t0v);
+                  const float p1 = ex2_approx(t1v);
+                  rs2 = f2_add(rs2, f2_make(p0, p1));
+                  pk[e] = pack_bf16x2(p0, p1);
+                }
+                tmem_st16(t_s(x) + lane_off + cc * 16, pk);
+                if (cc + 1 < kBN / 32) tmem_wait_ld_fence(nxt);
+              }
             }
           }
           float rs0, rs1;
