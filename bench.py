@@ -361,7 +361,8 @@ def _oracle_sample(wl, x, seconds):
 
     rng = np.random.default_rng(0)
     span = min(wl.T, 4096)
-    n_rows = 8
+    # rows per pass: a sliding-window row costs W pairs, a causal row up to span
+    n_rows = 256 if wl.window > 0 else 8
     total_flops, total_s, rows_done = 0, 0.0, 0
     cpu = {}
     for n in ("c_kv", "w_kvb", "k", "v"):
@@ -391,8 +392,6 @@ def _oracle_sample(wl, x, seconds):
         total_s += time.perf_counter() - t0
         total_flops += flops
         rows_done += n_rows
-        if not wl.latent and total_s > 0 and rows_done >= 4096:
-            break
     desc = ("%d query rows (all %d heads) drawn uniformly from the first %d tokens%s, float64 "
             "oracle" % (rows_done, wl.Hs + wl.Hn, span,
                         ", plus RMSNorm+W^KV_b expand of those %d tokens per pass" % span
