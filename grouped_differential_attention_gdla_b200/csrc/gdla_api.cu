@@ -13,6 +13,7 @@
 
 #include "gdla.h"
 #include "attn_fwd.cuh"
+#include "attn_win.cuh"
 #include "kv_expand.cuh"
 #include "selftest.cuh"
 
@@ -78,19 +79,6 @@ int launch_attn(const void *q_sig, const void *q_noise, const void *k, const voi
       !make_map(&tm_k, k, 3, dqn, kvbox) || !make_map(&tm_v, v, 3, dqn, kvbox) ||
       !make_map(&tm_gate, prm.gate, 3, dqs, qbox) || !make_map(&tm_out, prm.out, 3, dqs, qbox))
     return GDLA_ERR_CUDA;
-  // at least 116 KB so that one CTA (and one 512-column TMEM allocation) sits on an SM
-  const uint32_t smem = L::kBytes > 118784u ? L::kBytes : 118784u;
-  auto kern = prm.window > 0 ? gdla::gdla_attn_fwd_kernel<D, true>
-                              : gdla::gdla_attn_fwd_kernel<D, false>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
-    return GDLA_ERR_CUDA;
-  // The kernel re-splits its register pool between warpgroups (setmaxnreg);
-  // that is only sound for the per-thread count it was written for, so any
-  // other build is refused rather than launched.
-  cudaFuncAttributes fa;
-  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return GDLA_ERR_CUDA;
-  if (fa.numRegs != static_cast<int>(gdla::kLaunchRegs)) return GDLA_ERR_UNSUPPORTED;
   const uint64_t items = static_cast<uint64_t>(prm.n_qblk) * B * static_cast<uint64_t>(Hn);
   if (items > 0x7fffffffull) return GDLA_ERR_UNSUPPORTED;
   gdla::AttnParams run = prm;
@@ -107,6 +95,33 @@ int launch_attn(const void *q_sig, const void *q_noise, const void *k, const voi
       return GDLA_ERR_CUDA;
     if (grid > static_cast<uint64_t>(sms)) grid = static_cast<uint64_t>(sms);
   }
+  // every CTA allocates all 512 TMEM columns: at least 116 KB of shared
+  // memory keeps a second CTA off the SM
+  constexpr uint32_t kMinSmem = 118784u;
+  if (prm.window > 0 && prm.window <= gdla::kBN) {
+    // windows of at most one K/V tile: the union-row kernel
+    using LW = gdla::WinSmemLayout<D>;
+    const uint32_t smem = LW::kBytes > kMinSmem ? LW::kBytes : kMinSmem;
+    auto kern = gdla::gdla_attn_win_kernel<D>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return GDLA_ERR_CUDA;
+    kern<<<static_cast<unsigned>(grid), gdla::kWinThreads, smem, stream>>>(
+        tm_qs, tm_qn, tm_k, tm_v, tm_gate, tm_out, run);
+    return cudaGetLastError() == cudaSuccess ? GDLA_OK : GDLA_ERR_CUDA;
+  }
+  const uint32_t smem = L::kBytes > kMinSmem ? L::kBytes : kMinSmem;
+  auto kern = prm.window > 0 ? gdla::gdla_attn_fwd_kernel<D, true>
+                              : gdla::gdla_attn_fwd_kernel<D, false>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return GDLA_ERR_CUDA;
+  // The kernel re-splits its register pool between warpgroups (setmaxnreg);
+  // that is only sound for the per-thread count it was written for, so any
+  // other build is refused rather than launched.
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return GDLA_ERR_CUDA;
+  if (fa.numRegs != static_cast<int>(gdla::kLaunchRegs)) return GDLA_ERR_UNSUPPORTED;
   kern<<<static_cast<unsigned>(grid), gdla::kAttnThreads, smem, stream>>>(
       tm_qs, tm_qn, tm_k, tm_v, tm_gate, tm_out, run);
   return cudaGetLastError() == cudaSuccess ? GDLA_OK : GDLA_ERR_CUDA;

@@ -101,6 +101,15 @@ EDGE = [
     (2, 200, 8, 2, 64, 0, False),
     (1, 4097, 8, 2, 128, 0, True),
     (1, 4097, 8, 2, 128, 128, True),
+    # windows of at most one K/V tile (union-row kernel) and just above it
+    (1, 700, 8, 2, 128, 64, True),
+    (2, 333, 8, 2, 128, 127, True),
+    (1, 700, 8, 2, 128, 129, True),
+    (1, 300, 4, 4, 128, 128, True),   # g = 1
+    (1, 300, 4, 2, 128, 128, True),   # g = 2
+    (1, 300, 6, 2, 64, 128, True),    # g = 3, d = 64
+    (3, 257, 8, 2, 64, 100, True),
+    (1, 100, 8, 2, 128, 128, True),   # a single query block: no edge tile
 ]
 
 
