@@ -21,7 +21,7 @@
  *        64 signal / 16 noise query heads; window 128 with full attention in
  *        every 4th layer.
  *
- * Readings taken where the pages are silent (each is listed in the design doc):
+ * Readings taken where the pages are silent:
  *   - signal head h uses KV head floor(h/g) and noise head floor(h/g)
  *     (interleaved repeat: "repeat per group" in [R]);
  *   - noise head n uses KV head n (Hn == Hkv);
