@@ -24,6 +24,7 @@ from __future__ import annotations
 import argparse
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -320,15 +321,23 @@ def run_ours(args):
         print(json.dumps(result), flush=True)
 
 
+def _strip_comments(src):
+    """C/C++ source without its comments or blank-line differences."""
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
+
+
 def _csrc_hash():
-    """Hash of the CUDA sources, to tell whether profiled counters still apply."""
+    """Hash of the CUDA sources' code (comments excluded), to tell whether
+    profiled counters still apply to the kernels being timed."""
     import glob
     import hashlib
     h = hashlib.sha256()
     for f in sorted(glob.glob(os.path.join(ROOT, "grouped_differential_attention_gdla_b200",
                                            "csrc", "*"))):
-        with open(f, "rb") as fh:
-            h.update(fh.read())
+        with open(f, encoding="utf-8") as fh:
+            h.update(_strip_comments(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -218,7 +218,7 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
 }
 
 // 3-D tiled load of one box into shared memory; completion is signalled on
-// `bar` through its transaction count.  No cluster multicast.
+// `bar` through its transaction count; the tile lands in this CTA only.
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
                                             int32_t x, int32_t y, int32_t z) {
   asm volatile(
