@@ -4,17 +4,22 @@
                     [--impl ours|reference]
 
 A step is one pass of the whole hot path over one batch of synthetic input.
-The default workload is the latent-KV layer (B=1, T=32768, 64 signal / 16
-noise / 16 KV heads, d=128, full causal): RMSNorm + W^KV_b expand of the 512-d
-KV latent, then the fused GDLA attention.  Other workloads (--workload window,
-full, tiny, long_full, long_window) time the attention alone.
+The default step is the long-context pair of layers (64 signal / 16 noise /
+16 KV heads, d=128, B=1): one full-causal layer at T=131072 followed by one
+128-token sliding-window layer at T=262144, the 1 full : 3 sliding schedule's
+two kinds of attention layer.  --workload latent times the latent-KV layer
+(RMSNorm + W^KV_b expand of the 512-d KV latent, then full-causal attention,
+T=32768); window, full, tiny, long_full and long_window time one attention
+layer alone.
 
-Metric: TFLOP/s of algorithmic work (attention: 4*d FLOPs per kept (query,key)
-pair per query head; expand: 2*512*4096 per token), plus tokens/s.  Inputs are
-resident in HBM and larger than L2 (no flush needed); timing uses CUDA events
-on the launching stream with W untimed warm-up steps.  Multi-GPU runs are
-independent replicas (the forward pass has no cross-GPU exchange); the time is
-the maximum over ranks and the value is all ranks' work over that time.
+Metric: TFLOP/s of algorithmic work (attention: 4*d FLOPs per kept
+(query, key) pair per query head; expand: 2*512*4096 per token), plus
+tokens/s.  Inputs are resident in HBM and larger than L2 (no flush needed);
+timing uses CUDA events on the launching stream with W untimed warm-up steps,
+and every kernel launch is bracketed by its own events for the per-kernel
+roofline entries.  Multi-GPU runs are independent replicas (the forward pass
+has no cross-GPU exchange); the time is the maximum over ranks and the value
+is all ranks' work over that time.
 
 --impl reference times the float64 CPU oracle (the only other implementation of
 this method) on a bounded sample of the same workload.
@@ -37,6 +42,22 @@ if ROOT not in sys.path:
 METRIC = "GDLA attn fwd TFLOP/s and tokens/s on 1 B200; % of bf16 tensor or HBM roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
+# The layers one step runs, in order.
+STEPS = {
+    "long": ("long_full", "long_window"),
+    "latent": ("latent",),
+    "window": ("window",),
+    "full": ("full",),
+    "tiny": ("tiny",),
+    "long_full": ("long_full",),
+    "long_window": ("long_window",),
+}
+# A timed region at least this long runs tensor-bound kernels under the power
+# cap, so their fraction is taken against the sustained bf16 peak.
+SUSTAINED_AFTER_S = 2.0
+# Query rows the CPU sample draws from (the first tokens of batch element 0).
+SAMPLE_SPAN = 4096
+
 
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -53,6 +74,14 @@ def _dist():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return world, rank, local
+
+
+def attn_kernel_name(wl) -> str:
+    """The kernel gdla_attn_fwd dispatches this layer to (window >= T is full
+    causal; windows of 1..128 keys take the union-row kernel)."""
+    if wl.causal and 0 < wl.window < wl.T:
+        return "gdla_attn_win_kernel" if wl.window <= 128 else "gdla_attn_fwd_kernel<window>"
+    return "gdla_attn_fwd_kernel"
 
 
 class ClockSampler:
@@ -129,6 +158,82 @@ def _gpu_id(torch, dev):
         return str(dev.index or 0)
 
 
+class Layer:
+    """One layer of a step: its inputs, output buffer and launches."""
+
+    def __init__(self, wl, x, dev):
+        import torch
+        self.wl = wl
+        self.x = x
+        n_tok = wl.B * wl.T
+        self.kbuf = self.vbuf = None
+        if wl.latent:
+            self.kbuf = torch.empty((n_tok, wl.Hkv, wl.d), dtype=torch.bfloat16, device=dev)
+            self.vbuf = torch.empty_like(self.kbuf)
+        self.out = torch.empty((wl.B, wl.T, wl.Hs * wl.d), dtype=torch.bfloat16, device=dev)
+        # (label, kernel, flops, bytes) per launch, in launch order
+        self.launches = []
+        if wl.latent:
+            self.launches.append(("%s/expand" % wl.name, "gdla_kv_expand_kernel",
+                                  wl.expand_flops(), wl.expand_bytes()))
+        self.launches.append(("%s/attn" % wl.name, attn_kernel_name(wl), wl.attn_flops(),
+                              wl.attn_bytes()))
+
+    def run(self, gdla, status, stream, inp=None, out=None, events=None):
+        """Enqueue the layer; events[i] = (start, end) for launch i."""
+        wl = self.wl
+        inp = self.x if inp is None else inp
+        out = self.out if out is None else out
+        li = 0
+        if wl.latent:
+            if events is not None:
+                events[li][0].record(stream)
+            gdla.gdla_kv_expand(inp["c_kv"], inp["w_kvb"], None, eps=wl.eps, d_head=wl.d,
+                                k_out=self.kbuf, v_out=self.vbuf, d_status=status, stream=stream)
+            if events is not None:
+                events[li][1].record(stream)
+            li += 1
+            k = self.kbuf.view(wl.B, wl.T, wl.Hkv, wl.d)
+            v = self.vbuf.view(wl.B, wl.T, wl.Hkv, wl.d)
+        else:
+            k, v = inp["k"], inp["v"]
+        if events is not None:
+            events[li][0].record(stream)
+        gdla.gdla_attn_fwd(inp["q_sig"], inp["q_noise"], k, v, inp["lam"], inp["gate"],
+                           window=wl.window, causal=wl.causal, out=out, d_status=status,
+                           stream=stream)
+        if events is not None:
+            events[li][1].record(stream)
+
+
+def _roofline_entry(label, kernel, flops, nbytes, avg_ms, peaks, peak_src, sustained,
+                    traffic):
+    """Roofline figures of one kernel launch (algorithmic work / event time)."""
+    ridge = float(peaks["bf16_tflops"]) * 1e12 / (float(peaks["hbm_gbs"]) * 1e9)
+    tensor_bound = flops / max(1, nbytes) > ridge
+    tflops = flops / (avg_ms * 1e-3) / 1e12
+    gbs = nbytes / (avg_ms * 1e-3) / 1e9
+    e = {"kernel": kernel, "launch": label, "avg_launch_ms": round(avg_ms, 4),
+         "algorithmic_flop": flops, "algorithmic_bytes": nbytes,
+         "tflops": round(tflops, 2), "gbs": round(gbs, 1)}
+    if tensor_bound:
+        burst = float(peaks["bf16_tflops"])
+        sus = float(peaks["bf16_tflops_sustained"])
+        peak = sus if sustained else burst
+        e.update({"bound": "tensor", "achieved": round(tflops, 2), "peak": peak,
+                  "unit": "TFLOP/s", "frac": round(tflops / peak, 4),
+                  "frac_of_burst": round(tflops / burst, 4),
+                  "frac_of_sustained": round(tflops / sus, 4),
+                  "peak_source": "%s %s" % (peak_src, "bf16_tflops_sustained" if sustained
+                                            else "bf16_tflops")})
+    else:
+        peak = float(peaks["hbm_gbs"])
+        e.update({"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                  "frac": round(gbs / peak, 4), "peak_source": "%s hbm_gbs" % peak_src})
+    e["traffic"] = traffic
+    return e
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -150,42 +255,29 @@ def run_ours(args):
     gdla.load_library()
     dev = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
     torch.cuda.set_device(dev)
-    wl = WORKLOADS[args.workload]
-    x = make_inputs(wl, seed=replica_seed(rank), device=dev)
-    n_tok = wl.B * wl.T
+    layers = [Layer(WORKLOADS[n], make_inputs(WORKLOADS[n], seed=replica_seed(rank), device=dev),
+                    dev) for n in STEPS[args.workload]]
     stream = torch.cuda.current_stream(dev)
-    if wl.latent:
-        kbuf = torch.empty((n_tok, wl.Hkv, wl.d), dtype=torch.bfloat16, device=dev)
-        vbuf = torch.empty_like(kbuf)
-    out = torch.empty((wl.B, wl.T, wl.Hs * wl.d), dtype=torch.bfloat16, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
+    n_launch = sum(len(L.launches) for L in layers)
 
-    def step(ev=None, inp=x, strm=None):
+    def step(events=None, inputs=None, outs=None, strm=None):
         st = stream if strm is None else strm
-        if wl.latent:
-            gdla.gdla_kv_expand(inp["c_kv"], inp["w_kvb"], None, eps=wl.eps, d_head=wl.d,
-                                k_out=kbuf, v_out=vbuf, d_status=status, stream=st)
-            k = kbuf.view(wl.B, wl.T, wl.Hkv, wl.d)
-            v = vbuf.view(wl.B, wl.T, wl.Hkv, wl.d)
-        else:
-            k, v = inp["k"], inp["v"]
-        if ev is not None:
-            ev[0].record(st)
-        gdla.gdla_attn_fwd(inp["q_sig"], inp["q_noise"], k, v, inp["lam"], inp["gate"],
-                           window=wl.window, causal=wl.causal, out=out, d_status=status,
-                           stream=st)
-        if ev is not None:
-            ev[1].record(st)
+        li = 0
+        for j, L in enumerate(layers):
+            ev = None if events is None else events[li:li + len(L.launches)]
+            L.run(gdla, status, st, inp=None if inputs is None else inputs[j],
+                  out=None if outs is None else outs[j], events=ev)
+            li += len(L.launches)
 
-    launches_per_step = 2 if wl.latent else 1
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
     if int(status.item()) != 0:
         raise RuntimeError("kernel reported status %d during warm-up" % int(status.item()))
 
-    attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(args.steps)]
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n_launch)] for _ in range(args.steps)]
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(_gpu_id(torch, dev)) if rank == 0 else None
@@ -195,87 +287,42 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     t0.record(stream)
     for i in range(args.steps):
-        step(attn_ev[i])
+        step(events=ev[i])
     t1.record(stream)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     clocks = sampler.stop() if sampler else None
     ms = t0.elapsed_time(t1)
-    attn_ms = sum(a.elapsed_time(b) for a, b in attn_ev) / args.steps
+    launch_ms = [sum(ev[i][j][0].elapsed_time(ev[i][j][1]) for i in range(args.steps)) /
+                 args.steps for j in range(n_launch)]
     if int(status.item()) != 0:
         raise RuntimeError("kernel reported status %d" % int(status.item()))
     ms = max_over_ranks(ms, world, dev)
+    # the first tokens of each output, for the parity figures of the CPU sample
+    head_out = [L.out[:1, :min(L.wl.T, SAMPLE_SPAN)].float().cpu() for L in layers]
 
-    # ---- end to end through the public API from pinned host memory.  Every
-    # step copies its inputs host->device and its output device->host inside
-    # the timed region; steps are pipelined over three streams (upload of step
-    # i+1 and download of step i-1 overlap the kernels of step i), with two
-    # device buffers for inputs and outputs.
-    e2e_steps = max(2, min(args.steps, 6))
-    host = {n: t.to("cpu").pin_memory() for n, t in x.items()}
-    out_host = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = out.numel() * out.element_size()
-    dev_in = [{n: torch.empty_like(t) for n, t in x.items()} for _ in range(2)]
-    dev_out = [out, torch.empty_like(out)]
-    s_up, s_run, s_down = (torch.cuda.Stream(dev) for _ in range(3))
-    ev = {k: [torch.cuda.Event() for _ in range(2)] for k in ("up", "run", "down")}
-    for k in ev:
-        for e in ev[k]:
-            e.record(stream)
+    e2e_ms, e2e_steps, h2d, d2h = _e2e(args, layers, step, stream, dev, world)
 
-    def e2e_step(i):
-        nonlocal out
-        bsel = i % 2
-        s_up.wait_event(ev["run"][bsel])           # inputs of step i-2 consumed
-        with torch.cuda.stream(s_up):
-            for n, t in host.items():
-                dev_in[bsel][n].copy_(t, non_blocking=True)
-            ev["up"][bsel].record(s_up)
-        s_run.wait_event(ev["up"][bsel])
-        s_run.wait_event(ev["down"][bsel])         # output of step i-2 downloaded
-        with torch.cuda.stream(s_run):
-            out = dev_out[bsel]
-            step(inp=dev_in[bsel], strm=s_run)
-            ev["run"][bsel].record(s_run)
-        s_down.wait_event(ev["run"][bsel])
-        with torch.cuda.stream(s_down):
-            out_host[bsel].copy_(dev_out[bsel], non_blocking=True)
-            ev["down"][bsel].record(s_down)
-
-    e2e_step(0)
-    e2e_step(1)
-    torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(s_up)
-    for i in range(e2e_steps):
-        e2e_step(i)
-    s_down.wait_stream(s_run)
-    e1.record(s_down)
-    torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1)
-    e2e_ms = max_over_ranks(e2e_ms, world, dev)
-    if world > 1:
-        dist.barrier()
-    out = dev_out[0]
-
-    step_flops = wl.attn_flops() + (wl.expand_flops() if wl.latent else 0)
+    step_flops = sum(f for L in layers for (_, _, f, _) in L.launches)
+    n_tok = sum(L.wl.B * L.wl.T for L in layers)
     value = step_flops * args.steps * world / (ms * 1e-3) / 1e12
     e2e_value = step_flops * e2e_steps * world / (e2e_ms * 1e-3) / 1e12
     peaks, peak_src = _peaks()
-    if wl.window > 0:
-        bound, unit_r = "hbm", "GB/s"
-        achieved = wl.attn_bytes() / (attn_ms * 1e-3) / 1e9
-        peak = float(peaks["hbm_gbs"])
-    else:
-        bound, unit_r = "tensor", "TFLOP/s"
-        achieved = wl.attn_flops() / (attn_ms * 1e-3) / 1e12
-        peak = float(peaks["bf16_tflops_sustained"])
-    traffic = _traffic_from_profiles(wl.name)
+    sustained = ms * 1e-3 >= SUSTAINED_AFTER_S
+    entries = []
+    j = 0
+    for L in layers:
+        for (label, kernel, flops, nbytes) in L.launches:
+            traffic = _traffic_from_profiles(L.wl.name, kernel)
+            entries.append(_roofline_entry(label, kernel, flops, nbytes, launch_ms[j], peaks,
+                                           peak_src, sustained, traffic))
+            j += 1
+    kernel_ms = sum(launch_ms)
+    for e in entries:
+        e["share_of_step"] = round(e["avg_launch_ms"] / (ms / args.steps), 4)
+    top = max(entries, key=lambda e: e["avg_launch_ms"])
+    wl0 = layers[0].wl
     result = {
         "metric": METRIC,
         "value": round(value, 3),
@@ -291,34 +338,97 @@ def run_ours(args):
         "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16 inputs, sigmoid lambda/gate)",
         "config": {
-            "workload": wl.name, "B": wl.B, "T": wl.T, "Hs": wl.Hs, "Hn": wl.Hn, "Hkv": wl.Hkv,
-            "d": wl.d, "window": wl.window, "causal": wl.causal, "latent_kv": wl.latent,
+            "workload": args.workload,
+            "layers": [{"name": L.wl.name, "B": L.wl.B, "T": L.wl.T, "window": L.wl.window,
+                        "causal": L.wl.causal, "latent_kv": L.wl.latent} for L in layers],
+            "Hs": wl0.Hs, "Hn": wl0.Hn, "Hkv": wl0.Hkv, "d": wl0.d,
             "parallelism": "replicas" if world > 1 else "single GPU",
             "l2": "inputs larger than L2 (%.0f MB per step)" % (
-                (wl.attn_bytes() + (wl.expand_bytes() if wl.latent else 0)) / 1e6),
+                sum(nb for L in layers for (_, _, _, nb) in L.launches) / 1e6),
         },
-        "roofline": {
-            "kernel": "gdla_attn_fwd_kernel",
-            "bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit_r,
-            "frac": round(achieved / peak, 4),
-            "peak_source": "%s %s" % (peak_src, "hbm_gbs" if bound == "hbm" else
-                                      "bf16_tflops_sustained"),
-            "avg_launch_ms": round(attn_ms, 4),
-            "traffic": traffic,
-        },
+        "roofline": top,
+        "rooflines": entries,
+        "kernel_ms_per_step": round(kernel_ms, 4),
         "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "mode": "pinned host buffers, copies pipelined with compute over 3 streams"},
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": n_launch * args.steps,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(wl, x, seconds=args.cpu_seconds)
-    del host, out_host, dev_in, dev_out
+        result["cpu_baseline"], result["parity"] = cpu_baseline(layers, head_out,
+                                                                seconds=args.cpu_seconds)
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(result), flush=True)
+
+
+def _e2e(args, layers, step, stream, dev, world):
+    """End to end through the public API from pinned host memory: every step
+    copies all its inputs host->device and its outputs device->host inside
+    the timed region.  Steps are pipelined over three streams (upload of step
+    i+1 and download of step i-1 overlap the kernels of step i) with two
+    device buffer sets; the resident inputs and outputs are the first set."""
+    import torch
+    import torch.distributed as dist
+
+    e2e_steps = max(2, min(args.steps, 6 if len(layers) == 1 and layers[0].wl.T < 100000 else 3))
+    def pinned_copy(t):
+        h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        h.copy_(t)
+        return h
+
+    host = [{n: pinned_copy(t) for n, t in L.x.items()} for L in layers]
+    out_host = [torch.empty(L.out.shape, dtype=L.out.dtype, pin_memory=True) for L in layers]
+    h2d = sum(t.numel() * t.element_size() for hs in host for t in hs.values())
+    d2h = sum(L.out.numel() * L.out.element_size() for L in layers)
+    dev_in = [[L.x for L in layers], [{n: torch.empty_like(t) for n, t in L.x.items()}
+                                      for L in layers]]
+    dev_out = [[L.out for L in layers], [torch.empty_like(L.out) for L in layers]]
+    s_up, s_run, s_down = (torch.cuda.Stream(dev) for _ in range(3))
+    ev = {k: [torch.cuda.Event() for _ in range(2)] for k in ("up", "run", "down")}
+    for k in ev:
+        for e in ev[k]:
+            e.record(stream)
+
+    def e2e_step(i):
+        b = i % 2
+        s_up.wait_event(ev["run"][b])           # inputs of step i-2 consumed
+        with torch.cuda.stream(s_up):
+            for j in range(len(layers)):
+                for n, t in host[j].items():
+                    dev_in[b][j][n].copy_(t, non_blocking=True)
+            ev["up"][b].record(s_up)
+        s_run.wait_event(ev["up"][b])
+        s_run.wait_event(ev["down"][b])         # outputs of step i-2 downloaded
+        with torch.cuda.stream(s_run):
+            step(inputs=dev_in[b], outs=dev_out[b], strm=s_run)
+            ev["run"][b].record(s_run)
+        s_down.wait_event(ev["run"][b])
+        with torch.cuda.stream(s_down):
+            for j in range(len(layers)):
+                out_host[j].copy_(dev_out[b][j], non_blocking=True)
+            ev["down"][b].record(s_down)
+
+    e2e_step(0)
+    e2e_step(1)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(s_up)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    s_down.wait_stream(s_run)
+    e1.record(s_down)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    if world > 1:
+        dist.barrier()
+    del host, out_host, dev_in, dev_out
+    return e2e_ms, e2e_steps, h2d, d2h
 
 
 def _strip_comments(src):
@@ -341,44 +451,46 @@ def _csrc_hash():
     return h.hexdigest()[:16]
 
 
-def _traffic_from_profiles(name):
-    """DRAM bytes (read + write) per attention launch from a committed ncu
-    summary under profiles/ (a line "traffic: workload=<w> csrc=<hash>
-    bytes=<n>"), or None when none matches this workload and these sources."""
+def _traffic_from_profiles(name, kernel):
+    """DRAM bytes (read + write) per launch of `kernel` on workload `name`
+    from a committed ncu summary under profiles/ (a line "traffic:
+    workload=<w> kernel=<k> csrc=<hash> bytes=<n>"), or None when none
+    matches this workload, kernel and these sources."""
     import glob
-    import re
     want = _csrc_hash()
+    kname = kernel.split("<")[0]
+    pat = re.compile(r"traffic: workload=(\S+) kernel=(\S+) csrc=(\S+) bytes=(\d+)")
     for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
         with open(path) as f:
-            for m in re.finditer(r"traffic: workload=(\S+) csrc=(\S+) bytes=(\d+)", f.read()):
-                if m.group(1) == name and m.group(2) == want:
-                    return int(m.group(3))
+            for m in pat.finditer(f.read()):
+                if m.group(1) == name and m.group(2) == kname and m.group(3) == want:
+                    return int(m.group(4))
     return None
 
 
-def _oracle_sample(wl, x, seconds):
-    """Time the float64 oracle on a bounded sample of the workload.
+def _oracle_sample(wl, x, seconds, rng):
+    """Time the float64 oracle on a bounded sample of one layer.
 
-    Sample: query rows drawn uniformly from the first `span` tokens of batch 0
-    (all heads), plus, for the latent workload, the RMSNorm + expand of the
-    tokens those rows need.  Returns (flops, elapsed_s, description).
+    Sample: query rows drawn uniformly from the first SAMPLE_SPAN tokens of
+    batch element 0 (all heads), plus, for the latent layer, the RMSNorm +
+    expand of those tokens.  Returns (flops, elapsed_s, description, rows,
+    oracle outputs [n_rows, Hs*d]).
     """
     import numpy as np
     import torch
 
     import oracle
 
-    rng = np.random.default_rng(0)
-    span = min(wl.T, 4096)
+    span = min(wl.T, SAMPLE_SPAN)
     # rows per pass: a sliding-window row costs W pairs, a causal row up to span
     n_rows = 256 if wl.window > 0 else 8
-    total_flops, total_s, rows_done = 0, 0.0, 0
+    total_flops, total_s = 0, 0.0
     cpu = {}
     for n in ("c_kv", "w_kvb", "k", "v"):
         if n in x:
             t = x[n]
             cpu[n] = (t[:span] if n == "c_kv" else (t[:1, :span] if n in ("k", "v") else t)).cpu()
-    kv_cache = None
+    all_rows, all_ref = [], []
     while total_s < seconds:
         t0 = time.perf_counter()
         flops = 0
@@ -393,26 +505,53 @@ def _oracle_sample(wl, x, seconds):
         rows = np.sort(rng.integers(0, span, n_rows))
         idx = torch.as_tensor(rows, device=x["q_sig"].device)
         g = lambda t: t[0].index_select(0, idx).cpu()
-        oracle.gdla_attn_rows(g(x["q_sig"]), g(x["q_noise"]), k, v, g(x["lam"]), g(x["gate"]),
-                              rows, window=wl.window, causal=wl.causal)
+        ref = oracle.gdla_attn_rows(g(x["q_sig"]), g(x["q_noise"]), k, v, g(x["lam"]),
+                                    g(x["gate"]), rows, window=wl.window, causal=wl.causal)
         for i in rows:
             kept = min(int(i) + 1, wl.window) if wl.window > 0 else int(i) + 1
             flops += 4 * wl.d * (wl.Hs + wl.Hn) * kept
         total_s += time.perf_counter() - t0
         total_flops += flops
-        rows_done += n_rows
-    desc = ("%d query rows (all %d heads) drawn uniformly from the first %d tokens%s, float64 "
-            "oracle" % (rows_done, wl.Hs + wl.Hn, span,
-                        ", plus RMSNorm+W^KV_b expand of those %d tokens per pass" % span
-                        if wl.latent else ""))
-    return total_flops, total_s, desc
+        all_rows.append(rows)
+        all_ref.append(ref)
+    n_done = sum(len(r) for r in all_rows)
+    desc = ("%s: %d query rows (all %d heads) drawn uniformly from the first %d tokens%s" % (
+        wl.name, n_done, wl.Hs + wl.Hn, span,
+        ", plus RMSNorm+W^KV_b expand of those %d tokens per pass" % span if wl.latent else ""))
+    return total_flops, total_s, desc, np.concatenate(all_rows), np.concatenate(all_ref)
 
 
-def cpu_baseline(wl, x, seconds=15.0):
-    flops, s, desc = _oracle_sample(wl, x, seconds)
+def _parity(gpu_rows, ref):
+    """Error statistics of GPU output rows against the oracle's (per tensor
+    tolerance max|gpu - oracle| <= 1e-2 * max|oracle| + 1e-3)."""
+    import numpy as np
+    diff = np.abs(gpu_rows - ref)
+    idx = np.unravel_index(int(np.argmax(diff)), diff.shape)
+    max_ref = float(np.abs(ref).max())
+    tol = 1e-2 * max_ref + 1e-3
+    return {"rows": int(ref.shape[0]), "max_abs_err": float(diff.max()),
+            "mean_abs_err": float(diff.mean()), "rms_err": float(np.sqrt((diff ** 2).mean())),
+            "max_abs_oracle": max_ref, "tol": tol, "pass": bool(diff.max() <= tol),
+            "argmax_sample_col": [int(idx[0]), int(idx[1])]}
+
+
+def cpu_baseline(layers, head_out, seconds=15.0):
+    """The oracle timed on host cores over a bounded sample of every layer of
+    the step, and the parity figures of the GPU output on the same rows."""
+    import numpy as np
+    rng = np.random.default_rng(0)
+    flops, secs, descs, parity = 0, 0.0, [], {}
+    for L, ho in zip(layers, head_out):
+        f, s, d, rows, ref = _oracle_sample(L.wl, L.x, seconds / len(layers), rng)
+        flops += f
+        secs += s
+        descs.append(d)
+        gpu_rows = ho[0].numpy()[rows].astype(np.float64)
+        parity[L.wl.name] = _parity(gpu_rows, ref)
     threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    return {"value": round(flops / s / 1e12, 6), "unit": "TFLOP/s", "cores": threads,
-            "kind": "oracle", "sample": desc, "seconds": round(s, 2)}
+    return ({"value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s", "cores": threads,
+             "kind": "oracle", "sample": "; ".join(descs) + " (float64 oracle)",
+             "seconds": round(secs, 2)}, parity)
 
 
 def run_reference(args):
@@ -420,55 +559,61 @@ def run_reference(args):
     world, rank, local = _dist()
     if rank != 0:
         return
-    import torch
+    import numpy as np
 
     from grouped_differential_attention_gdla_b200.inputs import WORKLOADS, make_inputs
     import oracle
 
     oracle.build()
-    wl = WORKLOADS[args.workload]
+    wls = [WORKLOADS[n] for n in STEPS[args.workload]]
     # inputs drawn on the CPU in the same recipe; only the sampled slices are used
-    x = make_inputs(wl, seed=0, device="cpu", T=min(wl.T, 4096), B=1)
+    xs = [make_inputs(wl, seed=0, device="cpu", T=min(wl.T, SAMPLE_SPAN), B=1) for wl in wls]
     per_step = max(2.0, min(20.0, 60.0 / max(1, args.steps + args.warmup)))
+    rng = np.random.default_rng(0)
     for _ in range(args.warmup):
-        _oracle_sample(wl, x, per_step / 4)
+        for wl, x in zip(wls, xs):
+            _oracle_sample(wl, x, per_step / 4 / len(wls), rng)
     flops, secs = 0, 0.0
-    desc = ""
+    descs = []
     for _ in range(args.steps):
-        f, s, desc = _oracle_sample(wl, x, per_step)
-        flops += f
-        secs += s
+        descs = []
+        for wl, x in zip(wls, xs):
+            f, s, d, _, _ = _oracle_sample(wl, x, per_step / len(wls), rng)
+            flops += f
+            secs += s
+            descs.append(d)
     value = flops / secs / 1e12
     threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    n_tok = wl.B * wl.T
+    n_tok = sum(wl.B * wl.T for wl in wls)
+    step_flops = sum(wl.attn_flops() + (wl.expand_flops() if wl.latent else 0) for wl in wls)
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
         "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(secs * 1e3 / args.steps, 2), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (same recipe, CPU draw)",
-        "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "Hs": wl.Hs, "Hn": wl.Hn,
-                   "Hkv": wl.Hkv, "d": wl.d, "window": wl.window, "causal": wl.causal,
-                   "latent_kv": wl.latent},
+        "config": {"workload": args.workload,
+                   "layers": [{"name": wl.name, "B": wl.B, "T": wl.T, "window": wl.window,
+                               "causal": wl.causal, "latent_kv": wl.latent} for wl in wls],
+                   "Hs": wls[0].Hs, "Hn": wls[0].Hn, "Hkv": wls[0].Hkv, "d": wls[0].d},
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": threads,
-                         "kind": "oracle", "sample": desc + " (per step)"},
+                         "kind": "oracle", "sample": "; ".join(descs) + " (per step)"},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
         "note": "float64 CPU oracle on %d host threads; tokens/s of the full workload would be "
-                "%.3g" % (threads, n_tok * value * 1e12 / max(1, wl.attn_flops())),
+                "%.3g" % (threads, n_tok * value * 1e12 / max(1, step_flops)),
     }), flush=True)
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="latent",
-                    choices=["latent", "window", "full", "tiny", "long_full", "long_window"])
+    ap.add_argument("--workload", default="long", choices=sorted(STEPS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--cpu-seconds", type=float, default=16.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -1,9 +1,15 @@
 """ctypes binding of libgdla.so: argument marshalling only.
 
 Every step of the forward pass runs in the library's CUDA kernels; this module
-checks tensor dtypes, shapes and contiguity, passes raw device pointers, sizes
-and the current CUDA stream, and turns status codes into exceptions.  There is
-no fallback: without the compiled library every call raises.
+checks tensor dtypes, shapes, devices and contiguity, passes raw device
+pointers, sizes and the current CUDA stream, and turns status codes into
+exceptions.  There is no fallback: without the compiled library every call
+raises.
+
+Device-side failures (a pipeline wait that gave up) land in an int32 status
+word.  Calls that pass no ``d_status`` share one word per device; read it with
+``check_status()`` after the stream has passed the calls, or set
+``GDLA_SYNC_CHECK=1`` to synchronise and check after every call.
 """
 from __future__ import annotations
 
@@ -28,6 +34,8 @@ EXPORTED = ("gdla_version", "gdla_status_string", "gdla_kv_expand", "gdla_attn_f
             "gdla_selftest_wait_timeout")
 
 _lib = None
+# One status word per device, used when a caller passes none (see check_status).
+_default_status = {}
 
 
 class GDLAError(RuntimeError):
@@ -86,6 +94,52 @@ def _check(t: torch.Tensor, name: str, shape=None) -> int:
     return t.data_ptr()
 
 
+def _same_device(device: torch.device, tensors) -> None:
+    for name, t in tensors:
+        if t is not None and t.device != device:
+            raise ValueError(f"{name} is on {t.device}, expected {device} like the other inputs")
+
+
+def _status_ptr(d_status: Optional[torch.Tensor], device: torch.device) -> int:
+    """Device pointer of the int32 status word; the per-device default word
+    when the caller passes none."""
+    if d_status is None:
+        d_status = _default_status.get(device)
+        if d_status is None:
+            d_status = torch.zeros(1, dtype=torch.int32, device=device)
+            _default_status[device] = d_status
+    if not isinstance(d_status, torch.Tensor) or d_status.dtype != torch.int32:
+        raise ValueError("d_status must be an int32 tensor")
+    if d_status.device != device:
+        raise ValueError(f"d_status is on {d_status.device}, expected {device}")
+    if d_status.numel() < 1:
+        raise ValueError("d_status must hold at least one element")
+    return d_status.data_ptr()
+
+
+def check_status(device=None, d_status: Optional[torch.Tensor] = None) -> None:
+    """Synchronise `device` and raise GDLAError if a kernel reported a failure
+    in `d_status` (default: the word used by calls that passed none).  The
+    word is cleared afterwards, so a later check reports only later calls."""
+    if d_status is None:
+        dev = torch.device("cuda", torch.cuda.current_device()) if device is None \
+            else torch.device(device)
+        if dev.index is None:
+            dev = torch.device("cuda", torch.cuda.current_device())
+        d_status = _default_status.get(dev)
+        if d_status is None:
+            return
+    torch.cuda.synchronize(d_status.device)
+    code = int(d_status[0].item())
+    if code != GDLA_OK:
+        d_status.zero_()
+        raise GDLAError(code, "device-side status")
+
+
+def _sync_check_enabled() -> bool:
+    return os.environ.get("GDLA_SYNC_CHECK", "0") not in ("", "0")
+
+
 def _stream_ptr(device: torch.device, stream) -> int:
     if stream is None:
         stream = torch.cuda.current_stream(device)
@@ -112,11 +166,15 @@ def gdla_kv_expand(c_kv: torch.Tensor, w_kvb: torch.Tensor, rms_w: Optional[torc
     pr = _check(rms_w, "rms_w", (dl,)) if rms_w is not None else None
     pk = _check(k_out, "k_out", (n, hkv, d_head))
     pv = _check(v_out, "v_out", (n, hkv, d_head))
-    ps = d_status.data_ptr() if d_status is not None else None
+    _same_device(c_kv.device, [("w_kvb", w_kvb), ("rms_w", rms_w), ("k_out", k_out),
+                               ("v_out", v_out)])
+    ps = _status_ptr(d_status, c_kv.device)
     rc = load_library().gdla_kv_expand(pc, pr, pw, float(eps), pk, pv, n, dl, hkv, d_head, ps,
                                        _stream_ptr(c_kv.device, stream))
     if rc != GDLA_OK:
         raise GDLAError(rc, "gdla_kv_expand")
+    if _sync_check_enabled():
+        check_status(c_kv.device, d_status)
     return k_out, v_out
 
 
@@ -145,11 +203,15 @@ def gdla_attn_fwd(q_sig: torch.Tensor, q_noise: torch.Tensor, k: torch.Tensor, v
         _check(gate, "gate", (B, T, Hs * d)),
         _check(out, "out", (B, T, Hs * d)),
     ]
-    ps = d_status.data_ptr() if d_status is not None else None
+    _same_device(q_sig.device, [("q_noise", q_noise), ("k", k), ("v", v), ("lam", lam),
+                                 ("gate", gate), ("out", out)])
+    ps = _status_ptr(d_status, q_sig.device)
     rc = load_library().gdla_attn_fwd(*ptrs, B, T, Hs, Hn, Hkv, d, int(window), int(bool(causal)),
                                       float(scale), ps, _stream_ptr(q_sig.device, stream))
     if rc != GDLA_OK:
         raise GDLAError(rc, "gdla_attn_fwd")
+    if _sync_check_enabled():
+        check_status(q_sig.device, d_status)
     return out
 
 

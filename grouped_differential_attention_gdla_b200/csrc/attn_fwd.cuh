@@ -69,10 +69,6 @@ struct RegSplit {
 };
 constexpr int kSlotThreads = 128;          // one warpgroup per slot
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: O is rescaled only if the max grows by > 2^8
-// Of every 16 score pairs in a 32-column chunk of an unmasked tile, this many
-// take 2^x from the FMA-pipe polynomial instead of the MUFU ex2 unit, which
-// would otherwise cap the softmax at one exponential per MMA-consumed score.
-constexpr int kPolyPairs = 0;
 
 struct AttnParams {
   const __nv_bfloat16 *lam;   // [B, T, Hs]
@@ -1001,13 +997,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                   float t0v, t1v;
                   f2_split(f2_fma(f2_from_bits(raw[2 * e], raw[2 * e + 1]), sl2x2, negm2), t0v,
                            t1v);
-                  float p0, p1;
-                  if (e >= 16 - kPolyPairs) {
-                    exp2_poly_x2(t0v, t1v, p0, p1);
-                  } else {
-                    p0 = ex2_approx(t0v);
-                    p1 = ex2_approx(t1v);
-                  }
+                  const float p0 = ex2_approx(t0v);
+                  const float p1 = ex2_approx(t1v);
                   rs2 = f2_add(rs2, f2_make(p0, p1));
                   pk[e] = pack_bf16x2(p0, p1);
                 }

@@ -4,6 +4,7 @@
 // point fetched through the runtime, so the library links no libcuda), and
 // kernel launches on the caller's stream.  The library never allocates,
 // frees or synchronises.
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -39,6 +40,61 @@ EncodeTiledFn encode_tiled_fn() {
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+// Devices whose ordinal fits the 64-bit masks below get their one-time
+// kernel set-up and attribute queries cached; others redo them per call.
+constexpr int kCachedDevices = 64;
+
+int current_device(int *dev) {
+  return cudaGetDevice(dev) == cudaSuccess ? GDLA_OK : GDLA_ERR_CUDA;
+}
+
+// Number of SMs of the current device (queried once per device).
+int sm_count(int *sms) {
+  static std::atomic<int> cache[kCachedDevices];
+  int dev = 0;
+  if (current_device(&dev) != GDLA_OK) return GDLA_ERR_CUDA;
+  if (dev >= 0 && dev < kCachedDevices) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c > 0) {
+      *sms = c;
+      return GDLA_OK;
+    }
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return GDLA_ERR_CUDA;
+  if (dev >= 0 && dev < kCachedDevices) cache[dev].store(n, std::memory_order_relaxed);
+  *sms = n;
+  return GDLA_OK;
+}
+
+// One-time set-up of kernel `Kern` on the current device: its dynamic
+// shared-memory limit and, when `want_regs` > 0, the check that the build
+// uses exactly that many registers per thread (kernels that re-split their
+// register pool with setmaxnreg are only sound for the count they were
+// written for).  Both are properties of the device context and the binary,
+// so they are done once per device; two threads racing here only repeat
+// idempotent work.
+template <auto Kern>
+int prepare_kernel(uint32_t smem, int want_regs) {
+  static std::atomic<uint64_t> ready{0};
+  int dev = 0;
+  if (current_device(&dev) != GDLA_OK) return GDLA_ERR_CUDA;
+  const uint64_t bit = (dev >= 0 && dev < kCachedDevices) ? (1ull << dev) : 0ull;
+  if (bit && (ready.load(std::memory_order_acquire) & bit)) return GDLA_OK;
+  if (cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return GDLA_ERR_CUDA;
+  if (want_regs > 0) {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, Kern) != cudaSuccess) return GDLA_ERR_CUDA;
+    if (fa.numRegs != want_regs) return GDLA_ERR_UNSUPPORTED;
+  }
+  if (bit) ready.fetch_or(bit, std::memory_order_release);
+  return GDLA_OK;
+}
 
 // Row-major bf16 tensor of `rank` dims given innermost-first; box innermost-first.
 bool make_map(CUtensorMap *map, const void *base, int rank, const uint64_t *dims,
@@ -88,11 +144,8 @@ int launch_attn(const void *q_sig, const void *q_noise, const void *k, const voi
   // attention items differ in length; one CTA each lets the hardware balance.
   uint64_t grid = items;
   if (prm.window > 0) {
-    int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        sms <= 0)
-      return GDLA_ERR_CUDA;
+    int sms = 0;
+    if (sm_count(&sms) != GDLA_OK) return GDLA_ERR_CUDA;
     if (grid > static_cast<uint64_t>(sms)) grid = static_cast<uint64_t>(sms);
   }
   // every CTA allocates all 512 TMEM columns: at least 116 KB of shared
@@ -102,26 +155,25 @@ int launch_attn(const void *q_sig, const void *q_noise, const void *k, const voi
     // windows of at most one K/V tile: the union-row kernel
     using LW = gdla::WinSmemLayout<D>;
     const uint32_t smem = LW::kBytes > kMinSmem ? LW::kBytes : kMinSmem;
-    auto kern = gdla::gdla_attn_win_kernel<D>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-      return GDLA_ERR_CUDA;
+    constexpr auto kern = gdla::gdla_attn_win_kernel<D>;
+    const int rc = prepare_kernel<kern>(smem, 0);
+    if (rc != GDLA_OK) return rc;
     kern<<<static_cast<unsigned>(grid), gdla::kWinThreads, smem, stream>>>(
         tm_qs, tm_qn, tm_k, tm_v, tm_gate, tm_out, run);
     return cudaGetLastError() == cudaSuccess ? GDLA_OK : GDLA_ERR_CUDA;
   }
   const uint32_t smem = L::kBytes > kMinSmem ? L::kBytes : kMinSmem;
-  auto kern = prm.window > 0 ? gdla::gdla_attn_fwd_kernel<D, true>
-                              : gdla::gdla_attn_fwd_kernel<D, false>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
-    return GDLA_ERR_CUDA;
   // The kernel re-splits its register pool between warpgroups (setmaxnreg);
   // that is only sound for the per-thread count it was written for, so any
   // other build is refused rather than launched.
-  cudaFuncAttributes fa;
-  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return GDLA_ERR_CUDA;
-  if (fa.numRegs != static_cast<int>(gdla::kLaunchRegs)) return GDLA_ERR_UNSUPPORTED;
+  const int rc = prm.window > 0
+                     ? prepare_kernel<gdla::gdla_attn_fwd_kernel<D, true>>(
+                           smem, static_cast<int>(gdla::kLaunchRegs))
+                     : prepare_kernel<gdla::gdla_attn_fwd_kernel<D, false>>(
+                           smem, static_cast<int>(gdla::kLaunchRegs));
+  if (rc != GDLA_OK) return rc;
+  auto kern = prm.window > 0 ? gdla::gdla_attn_fwd_kernel<D, true>
+                              : gdla::gdla_attn_fwd_kernel<D, false>;
   kern<<<static_cast<unsigned>(grid), gdla::kAttnThreads, smem, stream>>>(
       tm_qs, tm_qn, tm_k, tm_v, tm_gate, tm_out, run);
   return cudaGetLastError() == cudaSuccess ? GDLA_OK : GDLA_ERR_CUDA;
@@ -139,10 +191,9 @@ int launch_expand(const void *c_kv, const void *w_kvb, const gdla::ExpandParams 
   const uint32_t wbox[2] = {64, gdla::kExpKC};
   if (!make_map(&tm_c, c_kv, 2, dc, cbox) || !make_map(&tm_w, w_kvb, 2, dw, wbox))
     return GDLA_ERR_CUDA;
-  auto kern = gdla::gdla_kv_expand_kernel<DH>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(L::kAlloc)) != cudaSuccess)
-    return GDLA_ERR_CUDA;
+  constexpr auto kern = gdla::gdla_kv_expand_kernel<DH>;
+  const int rc = prepare_kernel<kern>(L::kAlloc, 0);
+  if (rc != GDLA_OK) return rc;
   const uint64_t blocks = (static_cast<uint64_t>(prm.n_tokens) + gdla::kExpBM - 1) / gdla::kExpBM;
   if (blocks > 0x7fffffffull) return GDLA_ERR_UNSUPPORTED;
   kern<<<static_cast<unsigned>(blocks), gdla::kExpThreads, L::kAlloc, stream>>>(tm_c, tm_w, prm);
@@ -160,7 +211,8 @@ const char *gdla_status_string(int code) {
     case GDLA_OK: return "ok";
     case GDLA_ERR_INVALID_ARG: return "invalid argument (null pointer, negative size or bad flag)";
     case GDLA_ERR_UNSUPPORTED: return "unsupported shape for the sm_100a kernels";
-    case GDLA_ERR_ALIGNMENT: return "a tensor pointer is not 16-byte aligned";
+    case GDLA_ERR_ALIGNMENT:
+      return "a pointer is misaligned (tensors need 16 bytes, the status word 4)";
     case GDLA_ERR_CUDA: return "a CUDA runtime or driver call failed";
     case GDLA_ERR_TIMEOUT: return "a device-side pipeline wait timed out";
     default: return "unknown status code";
@@ -179,7 +231,7 @@ int gdla_kv_expand(const void *c_kv, const void *rms_w, const void *w_kvb, float
   if (n_tokens > 0x7fffffffll) return GDLA_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(n_kv_heads) * 2 * d_head > 0x7fffffffll) return GDLA_ERR_UNSUPPORTED;
   if (!aligned16(c_kv) || !aligned16(w_kvb) || !aligned16(k_out) || !aligned16(v_out) ||
-      (rms_w && !aligned16(rms_w)))
+      (rms_w && !aligned16(rms_w)) || (d_status && !aligned4(d_status)))
     return GDLA_ERR_ALIGNMENT;
   gdla::ExpandParams prm;
   prm.rms_w = static_cast<const __nv_bfloat16 *>(rms_w);
@@ -210,7 +262,8 @@ int gdla_attn_fwd(const void *q_sig, const void *q_noise, const void *k, const v
   if (T > 0x7fffffffll - gdla::kBM) return GDLA_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(Hs) * d > 0x7fffffffll) return GDLA_ERR_UNSUPPORTED;
   if (!aligned16(q_sig) || !aligned16(q_noise) || !aligned16(k) || !aligned16(v) ||
-      !aligned16(lambda) || !aligned16(gate) || !aligned16(out))
+      !aligned16(lambda) || !aligned16(gate) || !aligned16(out) ||
+      (d_status && !aligned4(d_status)))
     return GDLA_ERR_ALIGNMENT;
   gdla::AttnParams prm;
   prm.lam = static_cast<const __nv_bfloat16 *>(lambda);
@@ -234,7 +287,7 @@ int gdla_attn_fwd(const void *q_sig, const void *q_noise, const void *k, const v
 
 int gdla_selftest_wait_timeout(int *d_status, int64_t limit_ns, void *stream) {
   if (!d_status || limit_ns <= 0 || limit_ns > 1000000000ll) return GDLA_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(d_status) & 3u) != 0) return GDLA_ERR_ALIGNMENT;
+  if (!aligned4(d_status)) return GDLA_ERR_ALIGNMENT;
   gdla::gdla_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
       d_status, static_cast<uint64_t>(limit_ns));
   return cudaGetLastError() == cudaSuccess ? GDLA_OK : GDLA_ERR_CUDA;

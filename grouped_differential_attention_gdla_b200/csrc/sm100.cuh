@@ -30,47 +30,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe, for two values at once (Cody-Waite style range
-// reduction plus a minimax polynomial, fitted for this library by a Remez
-// exchange on relative error):
-//   x = n + f, n = floor(x), f in [0, 1);  2^f ~ c0 + c1 f + c2 f^2 + c3 f^3
-//   (max relative error 7.5e-5 on [0, 1));  2^x = 2^f with n added to the
-//   exponent field.
-// floor(x) comes from one round-toward-minus-infinity add of 1.5 * 2^23: the
-// sum's integer ulp leaves floor(x) in the low mantissa bits, whose low nine
-// bits shifted up by 23 add n to the exponent (two's complement for n < 0).
-// Inputs are clamped to [-125, +inf) so the result stays a normal float;
-// the caller guarantees x <= 126.
-constexpr float kExp2C0 = 0.99992520f;
-constexpr float kExp2C1 = 0.69583356f;
-constexpr float kExp2C2 = 0.22606716f;
-constexpr float kExp2C3 = 0.07802452f;
-constexpr float kRoundShift = 12582912.0f;  // 1.5 * 2^23
-
-__device__ __forceinline__ void exp2_poly_x2(float x0, float x1, float &y0, float &y1) {
-  x0 = fmaxf(x0, -125.f);
-  x1 = fmaxf(x1, -125.f);
-  uint64_t x, t, n, f, q, shift;
-  asm("mov.b64 %0, {%1, %1};" : "=l"(shift) : "f"(kRoundShift));
-  asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(x0), "f"(x1));
-  asm("add.rm.f32x2 %0, %1, %2;" : "=l"(t) : "l"(x), "l"(shift));
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(n) : "l"(t), "l"(shift));
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(f) : "l"(x), "l"(n));
-  uint64_t c3, c2, c1, c0;
-  asm("mov.b64 %0, {%1, %1};" : "=l"(c3) : "f"(kExp2C3));
-  asm("mov.b64 %0, {%1, %1};" : "=l"(c2) : "f"(kExp2C2));
-  asm("mov.b64 %0, {%1, %1};" : "=l"(c1) : "f"(kExp2C1));
-  asm("mov.b64 %0, {%1, %1};" : "=l"(c0) : "f"(kExp2C0));
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(q) : "l"(c3), "l"(f), "l"(c2));
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(q) : "l"(q), "l"(f), "l"(c1));
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(q) : "l"(q), "l"(f), "l"(c0));
-  uint32_t q0, q1, t0, t1;
-  asm("mov.b64 {%0, %1}, %2;" : "=r"(q0), "=r"(q1) : "l"(q));
-  asm("mov.b64 {%0, %1}, %2;" : "=r"(t0), "=r"(t1) : "l"(t));
-  y0 = __uint_as_float(q0 + (t0 << 23));
-  y1 = __uint_as_float(q1 + (t1 << 23));
-}
-
 // 2^k for an integral float k <= 0, exactly (0 below the normal range).
 __device__ __forceinline__ float exp2_int(float k) {
   return k < -126.f ? 0.f : __int_as_float((127 + static_cast<int>(k)) << 23);

@@ -33,12 +33,15 @@
  *     returns.  Results are ready when that stream reaches the call.
  *   - Argument errors are reported before anything is enqueued; in that case
  *     the call has no effect.
- *   - d_status (optional, may be NULL): a device int that a kernel sets to
- *     GDLA_ERR_TIMEOUT if one of its internal pipeline waits gives up (after
- *     about two seconds); the kernel then stops early and its output is
- *     undefined.  The library never clears it; the caller zeroes it.
- *   - The library keeps no mutable global state; calls from several host
- *     threads are safe.
+ *   - d_status (optional, may be NULL): a device int, 4-byte aligned
+ *     (otherwise GDLA_ERR_ALIGNMENT), that a kernel sets to GDLA_ERR_TIMEOUT
+ *     if one of its internal pipeline waits gives up (after about two
+ *     seconds); the kernel then stops early and its output is undefined.  The
+ *     library never clears it; the caller zeroes it and reads it once the
+ *     stream has passed the call.
+ *   - The only state the library keeps is a per-device record that a
+ *     kernel's launch attributes (its shared-memory limit) have been set and
+ *     the device's SM count; calls from several host threads are safe.
  */
 #ifndef GDLA_H_
 #define GDLA_H_
@@ -53,7 +56,7 @@ extern "C" {
 #define GDLA_OK 0
 #define GDLA_ERR_INVALID_ARG (-1) /* null pointer, negative size, bad flag  */
 #define GDLA_ERR_UNSUPPORTED (-2) /* valid but not a shape the kernels take */
-#define GDLA_ERR_ALIGNMENT (-3)   /* a pointer is not 16-byte aligned        */
+#define GDLA_ERR_ALIGNMENT (-3)   /* a pointer is misaligned (16 B; d_status 4 B) */
 #define GDLA_ERR_CUDA (-4)        /* a CUDA runtime/driver call failed       */
 #define GDLA_ERR_TIMEOUT (-5)     /* a device-side wait gave up (d_status)   */
 

@@ -1,7 +1,14 @@
 """Shared helpers for the GPU parity tests: the per-tensor tolerance and row
 sampling.  The tolerance is the one the forward pass is held to everywhere:
-max|gpu - oracle| <= 1e-2 * max|oracle| + 1e-3 over each checked tensor."""
+max|gpu - oracle| <= 1e-2 * max|oracle| + 1e-3 over each checked tensor.
+
+With GDLA_PARITY_LOG=<path> set, every checked tensor's error statistics are
+appended to <path> as one JSON line (tests/parity_report.py turns the file
+into a table)."""
 from __future__ import annotations
+
+import json
+import os
 
 import numpy as np
 import torch
@@ -25,9 +32,20 @@ def error_stats(gpu, ref) -> dict:
     }
 
 
+def _log(what: str, st: dict, tol: float, n_rows: int) -> None:
+    path = os.environ.get("GDLA_PARITY_LOG")
+    if not path:
+        return
+    rec = {"what": what, "elements": n_rows, "tol": tol,
+           **{k: (list(map(int, v)) if k == "argmax" else v) for k, v in st.items()}}
+    with open(path, "a") as f:
+        f.write(json.dumps(rec) + "\n")
+
+
 def assert_parity(gpu, ref, what: str) -> dict:
     st = error_stats(gpu, ref)
     tol = RTOL * st["max_abs_ref"] + ATOL
+    _log(what, st, tol, int(np.asarray(ref).size))
     assert st["finite"], f"{what}: non-finite GPU output"
     assert st["max_abs_err"] <= tol, (
         f"{what}: max|gpu-oracle| = {st['max_abs_err']:.4e} > tol {tol:.4e} "

@@ -49,9 +49,9 @@ def test_version_and_status_strings(lib):
 
 
 def _attn(lib, q=A, qn=A, k=A, v=A, lam=A, gate=A, out=A, B=1, T=256, Hs=8, Hn=2, Hkv=2, d=64,
-          window=0, causal=1, scale=0.0):
+          window=0, causal=1, scale=0.0, status=None):
     return lib.gdla_attn_fwd(q, qn, k, v, lam, gate, out, B, T, Hs, Hn, Hkv, d, window, causal,
-                             ctypes.c_float(scale), None, None)
+                             ctypes.c_float(scale), status, None)
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -66,14 +66,16 @@ def _attn(lib, q=A, qn=A, k=A, v=A, lam=A, gate=A, out=A, B=1, T=256, Hs=8, Hn=2
     (dict(d=32), UNSUPPORTED), (dict(d=96), UNSUPPORTED), (dict(T=2 ** 31), UNSUPPORTED),
     (dict(q=M), ALIGN), (dict(qn=M), ALIGN), (dict(k=M), ALIGN), (dict(v=M), ALIGN),
     (dict(lam=M), ALIGN), (dict(gate=M), ALIGN), (dict(out=M), ALIGN),
+    (dict(status=0x100002), ALIGN), (dict(status=0x100001), ALIGN),
     (dict(T=0), OK), (dict(B=0), OK), (dict(T=0, q=None, out=None), OK),
 ])
 def test_attn_argument_errors(lib, kw, code):
     assert _attn(lib, **kw) == code
 
 
-def _expand(lib, c=A, w=None, wk=A, eps=1e-6, k=A, v=A, n=300, dl=512, hkv=16, dh=128):
-    return lib.gdla_kv_expand(c, w, wk, ctypes.c_float(eps), k, v, n, dl, hkv, dh, None, None)
+def _expand(lib, c=A, w=None, wk=A, eps=1e-6, k=A, v=A, n=300, dl=512, hkv=16, dh=128,
+            status=None):
+    return lib.gdla_kv_expand(c, w, wk, ctypes.c_float(eps), k, v, n, dl, hkv, dh, status, None)
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -84,7 +86,7 @@ def _expand(lib, c=A, w=None, wk=A, eps=1e-6, k=A, v=A, n=300, dl=512, hkv=16, d
     (dict(dl=100), UNSUPPORTED), (dict(dl=576), UNSUPPORTED), (dict(dh=96), UNSUPPORTED),
     (dict(n=2 ** 31), UNSUPPORTED),
     (dict(c=M), ALIGN), (dict(wk=M), ALIGN), (dict(k=M), ALIGN), (dict(v=M), ALIGN),
-    (dict(w=M), ALIGN),
+    (dict(w=M), ALIGN), (dict(status=0x100002), ALIGN),
     (dict(n=0), OK), (dict(n=0, c=None), OK),
 ])
 def test_expand_argument_errors(lib, kw, code):

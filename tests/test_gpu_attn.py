@@ -33,6 +33,7 @@ def _run(x, window, causal, status=None, out=None):
 
 
 def _check_rows(x, out, wl, rows, window, causal, what):
+    gdla.check_status()  # calls that passed no status word share the default one
     ref = oracle.gdla_attn_rows(gather_rows(x["q_sig"], rows), gather_rows(x["q_noise"], rows),
                                 x["k"].cpu(), x["v"].cpu(), gather_rows(x["lam"], rows),
                                 gather_rows(x["gate"], rows), rows, window=window, causal=causal)
@@ -41,6 +42,7 @@ def _check_rows(x, out, wl, rows, window, causal, what):
 
 
 def _check_full(x, out, window, causal, what):
+    gdla.check_status()
     cpu = {k: v.cpu() for k, v in x.items()}
     ref = oracle.gdla_attn(cpu["q_sig"], cpu["q_noise"], cpu["k"], cpu["v"], cpu["lam"],
                            cpu["gate"], window=window, causal=causal)
@@ -70,12 +72,14 @@ def test_workload_sampled_rows(name, n_random):
     _check_rows(x, out, wl, rows, wl.window, wl.causal, name)
 
 
-@pytest.mark.parametrize("name,n_random", [("long_full", 6), ("long_window", 200)])
+@pytest.mark.parametrize("name,n_random", [("long_full", 6), ("long_window", 300)])
 def test_long_context_sampled_rows(name, n_random):
     wl = WORKLOADS[name]
     x = make_inputs(wl, seed=0, device="cuda")
-    out = _run(x, wl.window, wl.causal)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = _run(x, wl.window, wl.causal, status)
     torch.cuda.synchronize()
+    assert int(status.item()) == 0
     rows = sample_rows(wl.B, wl.T, n_random, seed=2)
     _check_rows(x, out, wl, rows, wl.window, wl.causal, name)
     del x, out

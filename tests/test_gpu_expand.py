@@ -78,7 +78,11 @@ def test_latent_config_chained_attention():
                              v.view(wl.B, wl.T, wl.Hkv, wl.d), x["lam"], x["gate"],
                              window=wl.window, causal=wl.causal)
     torch.cuda.synchronize()
-    rows = sample_rows(wl.B, wl.T, 12, seed=4)
+    # every query block's first and last rows up to token 8191, block edges
+    # across the sequence and random rows: 256+ rows, keys up to the last one
+    rows = sample_rows(wl.B, wl.T, 96, seed=4,
+                       extra=[q + o for q in range(0, 8192, 128) for o in (0, 127)])
+    assert rows.size >= 256
     t_max = int(rows.max()) + 1
     rk, rv = _oracle_kv(x["c_kv"][:t_max].cpu(), x["w_kvb"].cpu(), None, wl.eps, wl.Hkv, wl.d)
     ref = oracle.gdla_attn_rows(gather_rows(x["q_sig"], rows), gather_rows(x["q_noise"], rows),

@@ -31,3 +31,24 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     ref = oracle.gdla_attn(cpu["q_sig"], cpu["q_noise"], cpu["k"], cpu["v"], cpu["lam"],
                            cpu["gate"])
     assert_parity(out.reshape(ref.shape).float().cpu().numpy(), ref, "after timeout")
+
+
+def test_binding_status_word_checks():
+    """The binding refuses a status word of the wrong dtype or device, and
+    check_status() raises on a word a kernel has set, then clears it."""
+    wl = custom(1, 64, 8, 2, 2, 64)
+    x = {k: v.cuda() for k, v in make_inputs(wl, seed=4).items()}
+    args = (x["q_sig"], x["q_noise"], x["k"], x["v"], x["lam"], x["gate"])
+    with pytest.raises(ValueError):
+        gdla.gdla_attn_fwd(*args, d_status=torch.zeros(1, dtype=torch.int16, device="cuda"))
+    with pytest.raises(ValueError):
+        gdla.gdla_attn_fwd(*args, d_status=torch.zeros(1, dtype=torch.int32))
+    with pytest.raises(ValueError):
+        gdla.gdla_attn_fwd(x["q_sig"], x["q_noise"].cpu(), *args[2:])
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    gdla.gdla_selftest_wait_timeout(status, 1_000_000)
+    with pytest.raises(gdla.GDLAError):
+        gdla.check_status(d_status=status)
+    gdla.check_status(d_status=status)  # cleared by the first check
+    gdla.gdla_attn_fwd(*args)            # default status word
+    gdla.check_status()
