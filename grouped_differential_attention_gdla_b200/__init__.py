@@ -6,11 +6,13 @@ device memory and streams only.
 
     gdla_kv_expand(c_kv, w_kvb, rms_w=None, eps=1e-6) -> (K, V)
     gdla_attn_fwd(q_sig, q_noise, k, v, lam, gate, window=0, causal=True) -> out
+    gdla_attn_fwd_sp(...)   the sliding window on one shard of a sequence (halo.py
+                            exchanges the shards' halo rows between ranks)
 """
 from ._binding import (GDLAError, EXPORTED, LIB_PATH, check_status, gdla_attn_fwd,
-                       gdla_kv_expand, gdla_selftest_wait_timeout, gdla_status_string,
-                       gdla_version, load_library)
+                       gdla_attn_fwd_sp, gdla_kv_expand, gdla_selftest_wait_timeout,
+                       gdla_status_string, gdla_version, load_library)
 
 __all__ = ["GDLAError", "EXPORTED", "LIB_PATH", "check_status", "gdla_attn_fwd",
-           "gdla_kv_expand", "gdla_selftest_wait_timeout", "gdla_status_string", "gdla_version",
-           "load_library"]
+           "gdla_attn_fwd_sp", "gdla_kv_expand", "gdla_selftest_wait_timeout",
+           "gdla_status_string", "gdla_version", "load_library"]

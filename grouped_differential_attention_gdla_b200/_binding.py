@@ -31,7 +31,7 @@ GDLA_ERR_TIMEOUT = -5
 
 # every symbol include/gdla.h declares
 EXPORTED = ("gdla_version", "gdla_status_string", "gdla_kv_expand", "gdla_attn_fwd",
-            "gdla_selftest_wait_timeout")
+            "gdla_attn_fwd_sp", "gdla_selftest_wait_timeout")
 
 _lib = None
 # One status word per device, used when a caller passes none (see check_status).
@@ -65,6 +65,9 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.gdla_attn_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32, i64,
                                   i32, f32, vp, vp]
     lib.gdla_attn_fwd.restype = i32
+    lib.gdla_attn_fwd_sp.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i64, i32, i32, i32,
+                                     i32, i64, f32, vp, vp]
+    lib.gdla_attn_fwd_sp.restype = i32
     lib.gdla_selftest_wait_timeout.argtypes = [vp, i64, vp]
     lib.gdla_selftest_wait_timeout.restype = i32
     if path is None:
@@ -210,6 +213,45 @@ def gdla_attn_fwd(q_sig: torch.Tensor, q_noise: torch.Tensor, k: torch.Tensor, v
                                       float(scale), ps, _stream_ptr(q_sig.device, stream))
     if rc != GDLA_OK:
         raise GDLAError(rc, "gdla_attn_fwd")
+    if _sync_check_enabled():
+        check_status(q_sig.device, d_status)
+    return out
+
+
+def gdla_attn_fwd_sp(q_sig: torch.Tensor, q_noise: torch.Tensor, k: torch.Tensor,
+                     v: torch.Tensor, lam: torch.Tensor, gate: torch.Tensor, window: int,
+                     kv_prefix: int, scale: float = 0.0, out: Optional[torch.Tensor] = None,
+                     d_status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Sliding-window GDLA forward on one shard of a sequence split across GPUs.
+
+    q_sig [B,T,Hs,d], q_noise [B,T,Hn,d], lam [B,T,Hs], gate [B,T,Hs*d] hold
+    the shard's T tokens; k/v [B, kv_prefix+T, Hkv, d] hold kv_prefix halo
+    rows (the previous shard's last keys; 0 on the first shard) and then the
+    shard's own.  window in 1..128.  Returns out [B, T, Hs*d].
+    """
+    if q_sig.dim() != 4:
+        raise ValueError("q_sig must be [B, T, Hs, d]")
+    B, T, Hs, d = q_sig.shape
+    Hn = q_noise.shape[2] if q_noise.dim() == 4 else -1
+    Hkv = k.shape[2] if k.dim() == 4 else -1
+    if out is None:
+        out = torch.empty((B, T, Hs * d), dtype=torch.bfloat16, device=q_sig.device)
+    ptrs = [
+        _check(q_sig, "q_sig"),
+        _check(q_noise, "q_noise", (B, T, Hn, d)),
+        _check(k, "k", (B, kv_prefix + T, Hkv, d)),
+        _check(v, "v", (B, kv_prefix + T, Hkv, d)),
+        _check(lam, "lam", (B, T, Hs)),
+        _check(gate, "gate", (B, T, Hs * d)),
+        _check(out, "out", (B, T, Hs * d)),
+    ]
+    _same_device(q_sig.device, [("q_noise", q_noise), ("k", k), ("v", v), ("lam", lam),
+                                 ("gate", gate), ("out", out)])
+    ps = _status_ptr(d_status, q_sig.device)
+    rc = load_library().gdla_attn_fwd_sp(*ptrs, B, T, int(kv_prefix), Hs, Hn, Hkv, d, int(window),
+                                         float(scale), ps, _stream_ptr(q_sig.device, stream))
+    if rc != GDLA_OK:
+        raise GDLAError(rc, "gdla_attn_fwd_sp")
     if _sync_check_enabled():
         check_status(q_sig.device, d_status)
     return out

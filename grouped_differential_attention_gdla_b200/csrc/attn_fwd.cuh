@@ -23,14 +23,15 @@
 // nor H_N reaches global memory.  Full attention launches one CTA per item;
 // sliding-window items are walked by one persistent CTA per SM.
 //
-// Warp roles (512 threads, registers re-split with setmaxnreg):
-//   warps  0-3   softmax for slot A (TMEM lanes 0..127)             152 regs
-//   warps  4-7   softmax for slot B                                  152 regs
-//   warps  8-11  epilogue for both slots: O / l, H_N, gate, output   96 regs
-//   warp  12     TMA producer (Q tiles, K/V ring)                    } 112 regs
-//   warp  13     TMEM allocator, MMA issuer for slot A               }
-//   warp  14     MMA issuer for slot B                               }
-//   warp  15     idle (completes the fourth warpgroup)               }
+// Warp roles (512 threads, registers re-split with setmaxnreg; full
+// attention / sliding windows wider than one tile):
+//   warps  0-3   softmax for slot A (TMEM lanes 0..127)        168 / 144 regs
+//   warps  4-7   softmax for slot B                             168 / 144 regs
+//   warps  8-11  epilogue for both slots: O / l, H_N, gate, output 88 / 112 regs
+//   warp  12     TMA producer (Q tiles, K/V ring)               }  88 / 112 regs
+//   warp  13     TMEM allocator, MMA issuer for slot A          }
+//   warp  14     MMA issuer for slot B                          }
+//   warp  15     idle (completes the fourth warpgroup)          }
 // A softmax warpgroup hands each finished head to the epilogue warpgroup
 // (row sums and maxima through shared memory) and goes straight on to the
 // next phase; the next PV into the same O columns waits for the epilogue.
@@ -54,15 +55,16 @@ constexpr int kAttnThreads = 16 * 32;
 // epilogue warpgroups give registers back and the softmax warpgroups take
 // them, within the launch pool.  The host refuses to launch a build whose
 // per-thread register count differs from kLaunchRegs.
-// The sliding-window kernel's softmax has no unmasked-tile path and its
+// Full attention's softmax reads a whole score row (128 registers) per
+// tile; the sliding-window instantiation reads chunk by chunk and its
 // epilogue stages tiles through shared memory, so it moves registers from
-// the softmax to the epilogue.
+// the softmax to the epilogue and the control warps.
 constexpr uint32_t kLaunchRegs = 128;
 template <bool kWin>
 struct RegSplit {
-  static constexpr uint32_t kSoftmax = kWin ? 144 : 152;
-  static constexpr uint32_t kEpilogue = kWin ? 112 : 96;
-  static constexpr uint32_t kControl = 112;
+  static constexpr uint32_t kSoftmax = kWin ? 144 : 168;
+  static constexpr uint32_t kEpilogue = kWin ? 112 : 88;
+  static constexpr uint32_t kControl = kWin ? 112 : 88;
   static_assert(2 * 128 * kSoftmax + 128 * kEpilogue + 128 * kControl <=
                     kAttnThreads * kLaunchRegs,
                 "register split must fit in the launch pool");
@@ -82,6 +84,8 @@ struct AttnParams {
   int g;
   int n_qblk;
   int n_items;     // B * Hn * n_qblk work items; CTA c runs c, c + grid, ...
+  int band;        // full attention: KV groups ordered heaviest-first together
+  int kv_prefix;   // K/V rows before query row 0 (sequence-parallel halo; 0 or 128)
   int64_t window;  // 0 = full
   int causal;
   float scale_log2;  // softmax scale * log2(e)
@@ -157,15 +161,24 @@ struct WorkItem {
   int b, kvh, q0, j_lo, n_tiles;
 };
 
-// Heaviest query blocks first.  Full attention: KV groups one after another,
-// so CTAs running at the same time stream the same group's K/V tiles and
-// those stay in L2.  Sliding window: all groups of a query block together, so
-// the block's query/gate/output rows are read and written as whole token rows.
+// Heaviest query blocks first.  Full attention: the KV groups are taken in
+// bands of p.band groups, and within a band the query blocks run heaviest
+// first across the band's groups: CTAs running at the same time stream the
+// K/V tiles of a few groups, which stay in L2, while the light blocks of
+// every band come last and fill the tail.  Sliding window: all groups of a
+// query block together, so the block's query/gate/output rows are read and
+// written as whole token rows.
 __device__ __forceinline__ WorkItem work_item(const AttnParams &p, int item) {
   int grp, qblk;
   if (p.window == 0) {
-    grp = item / p.n_qblk;
-    qblk = p.n_qblk - 1 - item % p.n_qblk;
+    const int groups = p.B * p.Hn;
+    const int per_band = p.band * p.n_qblk;
+    const int bi = item / per_band;
+    const int g0 = bi * p.band;
+    const int gb = min(p.band, groups - g0);  // groups in this band
+    const int rr = item - bi * per_band;
+    grp = g0 + rr % gb;
+    qblk = p.n_qblk - 1 - rr / gb;
   } else {
     const int groups = p.B * p.Hn;
     grp = item % groups;
@@ -882,61 +895,65 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           } else {
             masked = kbase + kBN > p.T;
           }
-          // pass 1: row max of the tile (64 columns live at a time)
-          float mt;
-          if (!kWin && !masked) {
+          // Full attention reads the whole score row of the tile in one TMEM
+          // round trip for the row max; chunks 0 and 1 stay in registers for
+          // the exponentials while chunks 2 and 3 are read again behind them.
+          // Columns the mask drops become -inf (a warp classifies each chunk
+          // warp-uniformly: every column kept, none kept, or mixed).  Sliding
+          // windows wider than one tile go chunk by chunk and skip the chunks
+          // no row of the warp keeps.
+          auto mask_chunk = [&](uint32_t (&v)[32], int cc) {
+            const int cls = chunk_class(cc, c_lo, c_hi);
+            if (cls == kChunkFull) return;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int c = cc * 32 + e;
+              if (cls == kChunkEmpty || c < c_lo || c > c_hi) v[e] = 0xff800000u;
+            }
+          };
+          float mt_raw = -INFINITY;
+          uint32_t s0[32], s1[32], s2[32], s3[32];
+          if constexpr (!kWin) {
+            tmem_ld32x4_sync(t_s(x) + lane_off, s0, s1, s2, s3);
+            if (masked) {
+              mask_chunk(s0, 0);
+              mask_chunk(s1, 1);
+              mask_chunk(s2, 2);
+              mask_chunk(s3, 3);
+            }
             float ma = -INFINITY, mb = -INFINITY;
 #pragma unroll
-            for (int cc = 0; cc < kBN / 32; cc += 2) {
-              uint32_t r0[32], r1[32];
-              tmem_ld32x2_sync(t_s(x) + lane_off + cc * 32, t_s(x) + lane_off + cc * 32 + 32, r0, r1);
-#pragma unroll
-              for (int e = 0; e < 32; e += 2) {
-                ma = fmax3(ma, __uint_as_float(r0[e]), __uint_as_float(r0[e + 1]));
-                mb = fmax3(mb, __uint_as_float(r1[e]), __uint_as_float(r1[e + 1]));
-              }
+            for (int e = 0; e < 32; e += 2) {
+              ma = fmax3(ma, __uint_as_float(s0[e]), __uint_as_float(s0[e + 1]));
+              mb = fmax3(mb, __uint_as_float(s1[e]), __uint_as_float(s1[e + 1]));
+              ma = fmax3(ma, __uint_as_float(s2[e]), __uint_as_float(s2[e + 1]));
+              mb = fmax3(mb, __uint_as_float(s3[e]), __uint_as_float(s3[e + 1]));
             }
-            mt = fmaxf(ma, mb);
+            // chunk 2 is read again while chunks 0 and 1 are exponentiated
+            tmem_ld32(t_s(x) + lane_off + 64, s2);
+            mt_raw = fmaxf(ma, mb);
           } else {
-            mt = -INFINITY;
-            if (kWin) {
-              // chunks no row of the warp keeps are not even read
+            // chunks no row of the warp keeps are not even read
 #pragma unroll 1
-              for (int cc = 0; cc < kBN / 32; ++cc) {
-                const int cls = chunk_class(cc, c_lo, c_hi);
-                if (cls == kChunkEmpty) continue;
-                uint32_t raw[32];
-                tmem_ld32_sync(t_s(x) + lane_off + cc * 32, raw);
-                if (cls == kChunkFull) {
+            for (int cc = 0; cc < kBN / 32; ++cc) {
+              const int cls = chunk_class(cc, c_lo, c_hi);
+              if (cls == kChunkEmpty) continue;
+              uint32_t raw[32];
+              tmem_ld32_sync(t_s(x) + lane_off + cc * 32, raw);
+              if (cls == kChunkFull) {
 #pragma unroll
-                  for (int e = 0; e < 32; e += 2)
-                    mt = fmax3(mt, __uint_as_float(raw[e]), __uint_as_float(raw[e + 1]));
-                } else {
+                for (int e = 0; e < 32; e += 2)
+                  mt_raw = fmax3(mt_raw, __uint_as_float(raw[e]), __uint_as_float(raw[e + 1]));
+              } else {
 #pragma unroll
-                  for (int e = 0; e < 32; ++e) {
-                    const int c = cc * 32 + e;
-                    if (c >= c_lo && c <= c_hi) mt = fmaxf(mt, __uint_as_float(raw[e]));
-                  }
-                }
-              }
-            } else {
-#pragma unroll
-              for (int cp = 0; cp < kBN / 64; ++cp) {
-                uint32_t r2[2][32];
-                tmem_ld32x2_sync(t_s(x) + lane_off + cp * 64, t_s(x) + lane_off + cp * 64 + 32,
-                                 r2[0], r2[1]);
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-#pragma unroll
-                  for (int e = 0; e < 32; ++e) {
-                    const int c = (cp * 2 + hh) * 32 + e;
-                    if (c >= c_lo && c <= c_hi) mt = fmaxf(mt, __uint_as_float(r2[hh][e]));
-                  }
+                for (int e = 0; e < 32; ++e) {
+                  const int c = cc * 32 + e;
+                  if (c >= c_lo && c <= c_hi) mt_raw = fmaxf(mt_raw, __uint_as_float(raw[e]));
                 }
               }
             }
           }
-          mt = mt * sl2;  // scale > 0 keeps the arg max
+          const float mt = mt_raw * sl2;  // scale > 0 keeps the arg max
           const float m_new = fmaxf(m_run, mt);
           float alpha = 1.f;
           float m_use = m_run;
@@ -945,12 +962,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             alpha = (m_run == -INFINITY) ? 0.f : exp2_int(m_run - m_use);
           }
           const float m_safe = (m_use == -INFINITY) ? 0.f : m_use;
-          // pass 2: P = exp2(S*c - m) as bf16 pairs; chunk cc ([16cc, 16cc+16))
-          // lies below the S columns still to be read.
           const uint64_t sl2x2 = f2_make(sl2, sl2);
           const uint64_t negm2 = f2_make(-m_safe, -m_safe);
           uint64_t rs2 = f2_make(0.f, 0.f);
-          if (kWin) {
+          if constexpr (!kWin) {
+            // P = exp2(S*c - m) as bf16 pairs; chunk cc lands in columns
+            // [16cc, 16cc+16), below the S columns still to be read
+            auto exp_chunk = [&](const uint32_t (&v)[32], int cc) {
+              uint32_t pk[16];
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                float t0v, t1v;
+                f2_split(f2_fma(f2_from_bits(v[2 * e], v[2 * e + 1]), sl2x2, negm2), t0v, t1v);
+                const float p0 = ex2_approx(t0v);
+                const float p1 = ex2_approx(t1v);
+                rs2 = f2_add(rs2, f2_make(p0, p1));
+                pk[e] = pack_bf16x2(p0, p1);
+              }
+              tmem_st16(t_s(x) + lane_off + cc * 16, pk);
+            };
+            exp_chunk(s0, 0);
+            exp_chunk(s1, 1);
+            tmem_wait_ld_fence(s2);
+            tmem_ld32(t_s(x) + lane_off + 96, s3);
+            if (masked) mask_chunk(s2, 2);
+            exp_chunk(s2, 2);
+            tmem_wait_ld_fence(s3);
+            if (masked) mask_chunk(s3, 3);
+            exp_chunk(s3, 3);
+          } else {
             // sliding window: chunks no row of the warp keeps are neither read
             // nor exponentiated (their P is zero)
 #pragma unroll 1
@@ -979,55 +1019,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 }
               }
               tmem_st16(t_s(x) + lane_off + cc * 16, pk);
-            }
-          } else {
-            // full attention: the load of chunk cc+1 is in flight while chunk
-            // cc is exponentiated
-            uint32_t ra[32], rb[32];
-            tmem_ld32_sync(t_s(x) + lane_off, ra);
-            if (!masked) {
-#pragma unroll
-              for (int cc = 0; cc < kBN / 32; ++cc) {
-                uint32_t(&raw)[32] = (cc & 1) ? rb : ra;
-                uint32_t(&nxt)[32] = (cc & 1) ? ra : rb;
-                if (cc + 1 < kBN / 32) tmem_ld32(t_s(x) + lane_off + (cc + 1) * 32, nxt);
-                uint32_t pk[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                  float t0v, t1v;
-                  f2_split(f2_fma(f2_from_bits(raw[2 * e], raw[2 * e + 1]), sl2x2, negm2), t0v,
-                           t1v);
-                  const float p0 = ex2_approx(t0v);
-                  const float p1 = ex2_approx(t1v);
-                  rs2 = f2_add(rs2, f2_make(p0, p1));
-                  pk[e] = pack_bf16x2(p0, p1);
-                }
-                tmem_st16(t_s(x) + lane_off + cc * 16, pk);
-                if (cc + 1 < kBN / 32) tmem_wait_ld_fence(nxt);
-              }
-            } else {
-#pragma unroll
-              for (int cc = 0; cc < kBN / 32; ++cc) {
-                uint32_t(&raw)[32] = (cc & 1) ? rb : ra;
-                uint32_t(&nxt)[32] = (cc & 1) ? ra : rb;
-                if (cc + 1 < kBN / 32) tmem_ld32(t_s(x) + lane_off + (cc + 1) * 32, nxt);
-                uint32_t pk[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                  float t0v, t1v;
-                  f2_split(f2_fma(f2_from_bits(raw[2 * e], raw[2 * e + 1]), sl2x2, negm2), t0v,
-                           t1v);
-                  const int c0 = cc * 32 + 2 * e;
-                  if (!(c0 >= c_lo && c0 <= c_hi)) t0v = -INFINITY;
-                  if (!(c0 + 1 >= c_lo && c0 + 1 <= c_hi)) t1v = -INFINITY;
-                  const float p0 = ex2_approx(t0v);
-                  const float p1 = ex2_approx(t1v);
-                  rs2 = f2_add(rs2, f2_make(p0, p1));
-                  pk[e] = pack_bf16x2(p0, p1);
-                }
-                tmem_st16(t_s(x) + lane_off + cc * 16, pk);
-                if (cc + 1 < kBN / 32) tmem_wait_ld_fence(nxt);
-              }
             }
           }
           float rs0, rs1;

@@ -8,28 +8,42 @@
 // A work item is (batch b, KV group k, query block q0 .. q0+127).  Query row
 // r (token i = q0 + r) keeps the keys i-W+1 .. i, all inside two K/V tiles:
 // the edge tile E = keys [q0-128, q0) and the diagonal tile G = keys
-// [q0, q0+128).  Column c of a row's "union" row is key q0 + c when c <= r
-// (from G) and key q0 - 128 + c when c > r (from E), so the 128 union
+// [q0, q0+128).  On a shard of a sequence split across GPUs, the K/V tensors
+// start kv_prefix (0 or 128) rows before the shard's first query (the halo
+// of the previous shard), and query row i reads K/V row i + kv_prefix.
+// Column c of a row's "union" row is key q0 + c when c <= r (from G) and key
+// q0 - 128 + c when c > r (from E), so the 128 union
 // columns of every row hold exactly its W <= 128 kept keys (plus masked
 // ones when W < 128).  Per head:
 //   S_E = Q K_E^T, S_G = Q K_G^T        two tcgen05.mma (A, B in smem)
 //   union row max and P = exp2(S*c - m) one pass per head, one thread per row;
 //                                       P_E = P where c > r, P_G where c <= r
 //   O = P_E V_E + P_G V_G               two tcgen05.mma (A = P from TMEM)
-// Every warp reads four union chunks (plus both tiles of the one chunk its
-// diagonal crosses), so the softmax is balanced across warps and a head
-// needs no running-max rescale.  K_E, K_G, V_E, V_G stay in shared memory for
-// the item's g+1 heads; query tiles stream through a two-deep ring.  The
-// noise head's H_N = O / l stays in TMEM next to O, and every signal head's
-// epilogue computes G (.) (O/l - lambda H_N) with the gate and output moved
-// as whole tiles by TMA.
+// K_E, K_G, V_E, V_G stay in shared memory for the item's g+1 heads; query
+// tiles stream through a two-deep ring.
 //
-// Warp roles (384 threads, no register re-split):
-//   warps 0-3   softmax (TMEM lanes 0..127)
-//   warps 4-7   epilogue
-//   warp  8     TMA producer
-//   warp  9     TMEM allocator and MMA issuer
-//   warps 10-11 idle
+// Softmax: each warp owns 32 rows, so of the four 32-column union chunks the
+// warp's own chunk (columns 32w .. 32w+31) mixes both tiles and the other
+// three each come whole from one tile (G left of it, E right of it).  A warp
+// reads its whole union row with two TMEM round trips (the mixed chunk from
+// both tiles, then the three whole chunks), takes the row max and writes P
+// in one pass, with no running-max rescale (a head is one tile).
+//
+// Epilogue: the noise head's H_N = O / l stays in TMEM next to O.  For a
+// signal head the epilogue reads O and H_N into registers as
+// D = O/l - lambda H_N (fp32) and releases O at once, so the next head's PV
+// never waits for the gate; it then multiplies by the gate tile, which a
+// dedicated TMA warp streams through a 128B-swizzled staging buffer (loaded
+// as soon as the previous output tile's store has read the buffer) and
+// stores back as the output tile.
+//
+// Warp roles (384 threads; registers re-split with setmaxnreg):
+//   warps 0-3   softmax (TMEM lanes 0..127)                         176 regs
+//   warps 4-7   epilogue                                            216 regs
+//   warp  8     TMA producer: query tiles, K/V                      } 112 regs
+//   warp  9     TMEM allocator and MMA issuer                       }
+//   warp  10    TMA for the gate / output staging tile              }
+//   warp  11    idle                                                }
 // TMEM (512 columns): S_E [0,128) S_G [128,256) O [256,256+d) H_N [256+d,256+2d).
 // P_E / P_G occupy the first 64 columns of S_E / S_G as packed bf16 pairs.
 #pragma once
@@ -42,6 +56,19 @@ constexpr int kWinThreads = 12 * 32;
 constexpr int kWinEpiWarp0 = 4;
 constexpr int kWinProducerWarp = 8;
 constexpr int kWinMmaWarp = 9;
+constexpr int kWinGateWarp = 10;
+// Register split: the block launches with kWinLaunchRegs per thread (the
+// compiler's cap for 12 warps on one SM); the control warpgroup gives
+// registers back, and the softmax (a whole union row in registers) and the
+// epilogue (a head's D in registers) take them.  The host refuses a build with another per-thread count.
+constexpr uint32_t kWinLaunchRegs = 168;
+constexpr uint32_t kWinSoftmaxRegs = 176;
+constexpr uint32_t kWinEpilogueRegs = 216;
+constexpr uint32_t kWinControlRegs = 112;
+static_assert(128 * (kWinSoftmaxRegs + kWinEpilogueRegs + kWinControlRegs) <=
+                  kWinThreads * kWinLaunchRegs,
+              "register split must fit in the launch pool");
+constexpr uint32_t kNegInfBits = 0xff800000u;
 
 template <int D>
 struct WinSmemLayout {
@@ -51,12 +78,20 @@ struct WinSmemLayout {
   static constexpr uint32_t kVOff = kKOff + 2 * kTile;  // V_E, V_G
   static constexpr uint32_t kGOff = kVOff + 2 * kTile;  // gate / output staging
   static constexpr uint32_t kHalf = kBM * 128;          // one [128][64] swizzled half
-  static constexpr uint32_t kStatOff = kGOff + kTile;   // float l[kBM]
-  static constexpr uint32_t kBarOff = kStatOff + kBM * 4;
-  static constexpr uint32_t kNumBars = 16;
+  static constexpr uint32_t kStatOff = kGOff + kTile;   // float l[2][kBM]
+  static constexpr uint32_t kBarOff = kStatOff + 2 * kBM * 4;
+  static constexpr uint32_t kNumBars = 18;
   static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;
   static constexpr uint32_t kBytes = kMiscOff + 16;
+  static_assert(kBytes <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
 };
+
+// One arrival per warp: every lane's earlier writes (ordered before this call
+// by the lane's own fences) are made visible to the lane that arrives.
+__device__ __forceinline__ void warp_arrive(uint32_t bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31u) == 0) mbar_arrive(bar);
+}
 
 template <int D>
 __global__ void __launch_bounds__(kWinThreads, 1)
@@ -81,16 +116,17 @@ __global__ void __launch_bounds__(kWinThreads, 1)
   const uint32_t v_full = bar0 + 8u * 6;    // V_E, V_G landed
   const uint32_t v_free = bar0 + 8u * 7;    // last PV of the item done
   const uint32_t s_full = bar0 + 8u * 8;    // S_E, S_G of a head written
-  const uint32_t p_full = bar0 + 8u * 9;    // P_E, P_G written (softmax threads)
+  const uint32_t p_full = bar0 + 8u * 9;    // P_E, P_G written (softmax warps)
   const uint32_t o_done = bar0 + 8u * 10;   // O of a head complete
-  const uint32_t o_free = bar0 + 8u * 11;   // epilogue has read O (epilogue threads)
-  const uint32_t epi_go = bar0 + 8u * 12;   // row sums handed over (softmax threads)
-  const uint32_t stat_free = bar0 + 8u * 13;  // row sums read (epilogue threads)
-  const uint32_t g_full = bar0 + 8u * 14;   // gate tile landed
-  const uint32_t g_done = bar0 + 8u * 15;   // output tile written (epilogue threads)
+  const uint32_t o_free = bar0 + 8u * 11;   // epilogue has read O (epilogue warps)
+  const uint32_t g_full = bar0 + 8u * 12;   // gate tile landed
+  const uint32_t g_done = bar0 + 8u * 13;   // output tile written (epilogue warps)
+  // row sums handed over through two slots (softmax warps) / read (epilogue warps)
+  auto epi_go = [&](uint32_t s) { return bar0 + 8u * (14 + s); };
+  auto stat_free = [&](uint32_t s) { return bar0 + 8u * (16 + s); };
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
-  float *stat = reinterpret_cast<float *>(smem + L::kStatOff);
+  float *stat = reinterpret_cast<float *>(smem + L::kStatOff);  // [2][kBM]
   const int warp = threadIdx.x >> 5;
   const int n_heads = p.g + 1;  // noise head + g signal heads
   const int W = static_cast<int>(p.window);
@@ -105,13 +141,15 @@ __global__ void __launch_bounds__(kWinThreads, 1)
     mbar_init(v_full, 1);
     mbar_init(v_free, 1);
     mbar_init(s_full, 1);
-    mbar_init(p_full, kSlotThreads);
+    mbar_init(p_full, 4);
     mbar_init(o_done, 1);
-    mbar_init(o_free, kSlotThreads);
-    mbar_init(epi_go, kSlotThreads);
-    mbar_init(stat_free, kSlotThreads);
+    mbar_init(o_free, 4);
+    for (uint32_t s = 0; s < 2; ++s) {
+      mbar_init(epi_go(s), 4);
+      mbar_init(stat_free(s), 4);
+    }
     mbar_init(g_full, 1);
-    mbar_init(g_done, kSlotThreads);
+    mbar_init(g_done, 4);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -126,6 +164,9 @@ __global__ void __launch_bounds__(kWinThreads, 1)
   const uint32_t t_se = tmem, t_sg = tmem + 128u, t_o = tmem + 256u, t_hn = tmem + 256u + D;
   auto p_col = [](int k) -> uint32_t { return 8u * k; };
 
+  if (warp >= kWinProducerWarp) {
+  // =============================== control warpgroup (warps 8-11)
+  regs_decrease<kWinControlRegs>();
   if (warp == kWinProducerWarp) {
     // =============================== TMA producer
     // Per item: K_E, K_G once the previous item's last S is done, the first
@@ -151,14 +192,15 @@ __global__ void __launch_bounds__(kWinThreads, 1)
     };
     for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
       const WorkItem w = work_item(p, item);
-      const bool has_edge = w.q0 > 0;
+      const bool has_edge = w.q0 + p.kv_prefix > 0;
+      const int kv0 = w.q0 + p.kv_prefix;  // K/V row of query row q0
       const uint32_t n_kv = has_edge ? 2u : 1u;
       ok = __all_sync(0xffffffffu, mbar_wait(k_free, (kv_uses & 1u) ^ 1u, abort_flag));
       if (!ok) break;
       if (leader) {
         mbar_arrive_expect_tx(k_full, n_kv * L::kTile);
-        if (has_edge) load_tile(sbase + L::kKOff, &tm_k, k_full, w.kvh * D, w.q0 - kBN, w.b);
-        load_tile(sbase + L::kKOff + L::kTile, &tm_k, k_full, w.kvh * D, w.q0, w.b);
+        if (has_edge) load_tile(sbase + L::kKOff, &tm_k, k_full, w.kvh * D, kv0 - kBN, w.b);
+        load_tile(sbase + L::kKOff + L::kTile, &tm_k, k_full, w.kvh * D, kv0, w.b);
       }
       ++k_issued;
       for (int hh = 0; hh < n_heads && ok; ++hh) {
@@ -178,8 +220,8 @@ __global__ void __launch_bounds__(kWinThreads, 1)
           if (!ok) break;
           if (leader) {
             mbar_arrive_expect_tx(v_full, n_kv * L::kTile);
-            if (has_edge) load_tile(sbase + L::kVOff, &tm_v, v_full, w.kvh * D, w.q0 - kBN, w.b);
-            load_tile(sbase + L::kVOff + L::kTile, &tm_v, v_full, w.kvh * D, w.q0, w.b);
+            if (has_edge) load_tile(sbase + L::kVOff, &tm_v, v_full, w.kvh * D, kv0 - kBN, w.b);
+            load_tile(sbase + L::kVOff + L::kTile, &tm_v, v_full, w.kvh * D, kv0, w.b);
           }
           ++v_issued;
         }
@@ -227,7 +269,7 @@ __global__ void __launch_bounds__(kWinThreads, 1)
     };
     for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
       const WorkItem w = work_item(p, item);
-      const bool has_edge = w.q0 > 0;
+      const bool has_edge = w.q0 + p.kv_prefix > 0;
       ok = __all_sync(0xffffffffu, mbar_wait(k_full, kv_uses & 1u, abort_flag));
       if (!ok) break;
       for (int hh = 0; hh < n_heads && ok; ++hh) {
@@ -267,167 +309,202 @@ __global__ void __launch_bounds__(kWinThreads, 1)
     }
     // drain: every MMA issued above must finish before TMEM is released
     if (leader && o_commits) mbar_wait_for(o_done, (o_commits - 1) & 1u, 100000000ull);
+  } else if (warp == kWinGateWarp) {
+    // =============================== gate / output staging (TMA)
+    // For every signal head in order: load its gate tile into the staging
+    // buffer once the previous output tile's store has read it, wait until
+    // the epilogue has overwritten the tile with the output, store it.
+    const bool leader = elect_one();
+    if (leader) {
+      tma_prefetch_desc(&tm_gate);
+      tma_prefetch_desc(&tm_out);
+    }
+    const uint32_t gbuf = sbase + L::kGOff;
+    uint32_t g_issued = 0, g_stored = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+      const WorkItem w = work_item(p, item);
+      for (int hh = 1; hh < n_heads && ok; ++hh) {
+        const int h = p.g * w.kvh + (hh - 1);
+        if (leader) {
+          if (g_stored) bulk_wait_group_read0();  // the previous store has read the buffer
+          mbar_arrive_expect_tx(g_full, (D / 64) * L::kHalf);
+#pragma unroll
+          for (int hf = 0; hf < D / 64; ++hf)
+            tma_load_3d(gbuf + hf * L::kHalf, &tm_gate, g_full, h * D + hf * 64, w.q0, w.b);
+        }
+        ++g_issued;
+        ok = __all_sync(0xffffffffu, mbar_wait(g_done, g_stored & 1u, abort_flag));
+        if (!ok) break;
+        if (leader) {
+#pragma unroll
+          for (int hf = 0; hf < D / 64; ++hf)
+            tma_store_3d(&tm_out, gbuf + hf * L::kHalf, h * D + hf * 64, w.q0, w.b);
+          bulk_commit_group();
+        }
+        ++g_stored;
+      }
+    }
+    if (leader) {
+      // a gate tile still in flight (after an abort) lands before the CTA
+      // exits; every output tile store completes
+      if (!ok && g_issued) mbar_wait_for(g_full, (g_issued - 1) & 1u, 100000000ull);
+      bulk_wait_group0();
+    }
+  }
   } else if (warp < kWinEpiWarp0) {
     // =============================== softmax (warps 0-3, one thread per row)
+    regs_increase<kWinSoftmaxRegs>();
     const int qw = warp & 3;
     const int r = threadIdx.x & 127;
     const uint32_t lane_off = static_cast<uint32_t>(qw * 32) << 16;
     const float sl2 = p.scale_log2;
     const uint64_t sl2x2 = f2_make(sl2, sl2);
+    const int cm = 32 * qw;       // this warp's mixed union chunk
+    const int dlo = r - W + 1;    // kept diagonal-tile columns: [dlo, r]
     uint32_t s_waits = 0, handoffs = 0;
     bool ok = true;
-    // Warp-uniform shape of union chunk c0 .. c0+31: does any lane keep a
-    // diagonal-tile (edge-tile) column in it, and does every lane keep all
-    // of the chunk from the diagonal (edge) tile?
-    struct ChunkShape {
-      bool g_any, e_any, g_all, e_all;
-    };
+    // the three whole chunks: chunk index, and whether it comes from the
+    // diagonal tile (left of the mixed chunk) or the edge tile (right of it)
+    int ccj[3];
+    bool from_g[3];
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+      ccj[j] = j + (j >= qw ? 1 : 0);
+      from_g[j] = ccj[j] < qw;
+    }
     for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
       const WorkItem w = work_item(p, item);
-      const bool has_edge = w.q0 > 0;
-      // kept union columns of row r: diagonal tile [dlo, r], edge tile [elo, 127]
-      const int dlo = r - W + 1;
+      const bool has_edge = w.q0 + p.kv_prefix > 0;
+      // kept edge-tile columns: [elo, 127]
       const int elo = has_edge ? max(r + 1, r + 129 - W) : 128;
-      auto shape = [&](int c0) -> ChunkShape {
-        ChunkShape s;
-        s.g_any = __any_sync(0xffffffffu, max(dlo, c0) <= min(r, c0 + 31));
-        s.e_any = __any_sync(0xffffffffu, max(elo, c0) <= c0 + 31);
-        s.g_all = __all_sync(0xffffffffu, dlo <= c0 && r >= c0 + 31);
-        s.e_all = __all_sync(0xffffffffu, elo <= c0);
-        return s;
-      };
-      // loads what chunk c0 needs of S_G / S_E (both in one round trip)
-      auto load = [&](int c0, const ChunkShape &s, uint32_t (&rg)[32], uint32_t (&re)[32]) {
-        if (s.g_any && s.e_any) {
-          tmem_ld32x2_sync(t_sg + lane_off + c0, t_se + lane_off + c0, rg, re);
-        } else if (s.g_any) {
-          tmem_ld32_sync(t_sg + lane_off + c0, rg);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) re[e] = 0u;
-        } else {
-          tmem_ld32_sync(t_se + lane_off + c0, re);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) rg[e] = 0u;
-        }
-      };
       for (int hh = 0; hh < n_heads && ok; ++hh) {
         ok = __all_sync(0xffffffffu, mbar_wait(s_full, s_waits & 1u, abort_flag));
         ++s_waits;
         if (!ok) break;
         tc_fence_after();
-        // pass 1: union row max
-        float mt = -INFINITY;
-#pragma unroll 1
-        for (int cc = 0; cc < kBN / 32; ++cc) {
-          const int c0 = cc * 32;
-          const ChunkShape s = shape(c0);
-          if (!s.g_any && !s.e_any) continue;
-          uint32_t rg[32], re[32];
-          if (s.g_all || s.e_all) {
-            if (s.g_all) {
-              tmem_ld32_sync(t_sg + lane_off + c0, rg);
-            } else {
-              tmem_ld32_sync(t_se + lane_off + c0, rg);
-            }
-#pragma unroll
-            for (int e = 0; e < 32; e += 2)
-              mt = fmax3(mt, __uint_as_float(rg[e]), __uint_as_float(rg[e + 1]));
+        // ---- round trip 1: the mixed chunk from both tiles
+        uint32_t um[32];
+        {
+          uint32_t mg[32], me[32];
+          if (has_edge) {
+            tmem_ld32x2_sync(t_sg + lane_off + cm, t_se + lane_off + cm, mg, me);
           } else {
-            load(c0, s, rg, re);
+            tmem_ld32_sync(t_sg + lane_off + cm, mg);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int c = c0 + e;
-              const bool diag = c <= r;
-              if (diag ? c >= dlo : c >= elo)
-                mt = fmaxf(mt, __uint_as_float(diag ? rg[e] : re[e]));
-            }
+            for (int e = 0; e < 32; ++e) me[e] = kNegInfBits;
           }
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int c = cm + e;
+            const bool diag = c <= r;
+            const bool kept = diag ? c >= dlo : c >= elo;
+            um[e] = kept ? (diag ? mg[e] : me[e]) : kNegInfBits;
+          }
+        }
+        // ---- round trip 2: the three whole chunks
+        uint32_t up[3][32];
+        tmem_ld32x3_sync((from_g[0] ? t_sg : t_se) + lane_off + 32 * ccj[0],
+                         (from_g[1] ? t_sg : t_se) + lane_off + 32 * ccj[1],
+                         (from_g[2] ? t_sg : t_se) + lane_off + 32 * ccj[2], up[0], up[1], up[2]);
+#pragma unroll
+        for (int j = 0; j < 3; ++j) {
+          // a whole chunk is cut only from below: G columns before dlo, E
+          // columns before elo (every E column when there is no edge tile)
+          const int lo = from_g[j] ? dlo : elo;
+          const int c0 = 32 * ccj[j];
+          if (__any_sync(0xffffffffu, lo > c0)) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (c0 + e < lo) up[j][e] = kNegInfBits;
+          }
+        }
+        // ---- row max (the diagonal key is always kept, so it is finite)
+        float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          m0 = fmax3(m0, __uint_as_float(um[e]), __uint_as_float(um[e + 1]));
+          m1 = fmax3(m1, __uint_as_float(up[0][e]), __uint_as_float(up[0][e + 1]));
+          m0 = fmax3(m0, __uint_as_float(up[1][e]), __uint_as_float(up[1][e + 1]));
+          m1 = fmax3(m1, __uint_as_float(up[2][e]), __uint_as_float(up[2][e + 1]));
         }
         // one tile per head: the reference max needs no later rescale; it is
         // rounded up to an integer like the other kernels' running max
-        mt = mt * sl2;
+        const float mt = fmaxf(m0, m1) * sl2;
         const float m_ref = mt == -INFINITY ? 0.f : ceilf(mt);
         const uint64_t negm2 = f2_make(-m_ref, -m_ref);
         uint64_t rs2 = f2_make(0.f, 0.f);
-        // pass 2: P_G and P_E (bf16 pairs) over the first 64 columns of S_G / S_E;
-        // P of chunk cc lands in columns [16cc, 16cc+16), below the S still unread
-#pragma unroll 1
-        for (int cc = 0; cc < kBN / 32; ++cc) {
-          const int c0 = cc * 32;
-          const ChunkShape s = shape(c0);
-          uint32_t pg[16], pe[16];
-          if (!s.g_any && !s.e_any) {
+        // ---- P = exp2(S*c - m) as bf16 pairs; chunk cc lands in columns
+        // [16cc, 16cc+16) of its tile's S (all of S is in registers already)
+        const uint32_t zero16[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u,
+                                     0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
 #pragma unroll
-            for (int e = 0; e < 16; ++e) pg[e] = pe[e] = 0u;
-          } else if (s.g_all || s.e_all) {
-            uint32_t rs[32];
-            tmem_ld32_sync((s.g_all ? t_sg : t_se) + lane_off + c0, rs);
-            uint32_t pk[16];
+        for (int j = 0; j < 3; ++j) {
+          uint32_t pk[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              float t0v, t1v;
-              f2_split(f2_fma(f2_from_bits(rs[2 * e], rs[2 * e + 1]), sl2x2, negm2), t0v, t1v);
-              const float p0 = ex2_approx(t0v);
-              const float p1 = ex2_approx(t1v);
-              rs2 = f2_add(rs2, f2_make(p0, p1));
-              pk[e] = pack_bf16x2(p0, p1);
-            }
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              pg[e] = s.g_all ? pk[e] : 0u;
-              pe[e] = s.g_all ? 0u : pk[e];
-            }
-          } else {
-            uint32_t rg[32], re[32];
-            load(c0, s, rg, re);
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int ca = c0 + 2 * e, cb = ca + 1;
-              const bool da = ca <= r, db = cb <= r;
-              float t0v, t1v;
-              f2_split(f2_fma(f2_from_bits(da ? rg[2 * e] : re[2 * e], db ? rg[2 * e + 1] : re[2 * e + 1]),
-                              sl2x2, negm2),
-                       t0v, t1v);
-              if (!(da ? ca >= dlo : ca >= elo)) t0v = -INFINITY;
-              if (!(db ? cb >= dlo : cb >= elo)) t1v = -INFINITY;
-              const float p0 = ex2_approx(t0v);
-              const float p1 = ex2_approx(t1v);
-              rs2 = f2_add(rs2, f2_make(p0, p1));
-              pg[e] = pack_bf16x2(da ? p0 : 0.f, db ? p1 : 0.f);
-              pe[e] = pack_bf16x2(da ? 0.f : p0, db ? 0.f : p1);
-            }
+          for (int e = 0; e < 16; ++e) {
+            float t0v, t1v;
+            f2_split(f2_fma(f2_from_bits(up[j][2 * e], up[j][2 * e + 1]), sl2x2, negm2), t0v, t1v);
+            const float p0 = ex2_approx(t0v);
+            const float p1 = ex2_approx(t1v);
+            rs2 = f2_add(rs2, f2_make(p0, p1));
+            pk[e] = pack_bf16x2(p0, p1);
           }
-          tmem_st16(t_sg + lane_off + cc * 16, pg);
-          if (has_edge) tmem_st16(t_se + lane_off + cc * 16, pe);
+          const uint32_t col = lane_off + 16 * ccj[j];
+          if (from_g[j]) {
+            tmem_st16(t_sg + col, pk);
+            if (has_edge) tmem_st16(t_se + col, zero16);
+          } else {
+            tmem_st16(t_sg + col, zero16);
+            if (has_edge) tmem_st16(t_se + col, pk);
+          }
+        }
+        {
+          uint32_t pg[16], pe[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            float t0v, t1v;
+            f2_split(f2_fma(f2_from_bits(um[2 * e], um[2 * e + 1]), sl2x2, negm2), t0v, t1v);
+            const float p0 = ex2_approx(t0v);
+            const float p1 = ex2_approx(t1v);
+            rs2 = f2_add(rs2, f2_make(p0, p1));
+            const bool d0 = cm + 2 * e <= r, d1 = cm + 2 * e + 1 <= r;
+            pg[e] = pack_bf16x2(d0 ? p0 : 0.f, d1 ? p1 : 0.f);
+            pe[e] = pack_bf16x2(d0 ? 0.f : p0, d1 ? 0.f : p1);
+          }
+          tmem_st16(t_sg + lane_off + 16 * qw, pg);
+          if (has_edge) tmem_st16(t_se + lane_off + 16 * qw, pe);
         }
         float rs0, rs1;
         f2_split(rs2, rs0, rs1);
         const float l = rs0 + rs1;
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(p_full);
-        // hand the row sum to the epilogue once it has read the previous one
-        if (handoffs > 0) {
-          ok = __all_sync(0xffffffffu, mbar_wait(stat_free, (handoffs - 1) & 1u, abort_flag));
+        warp_arrive(p_full);
+        // hand the row sum to the epilogue through slot handoffs % 2, once
+        // the epilogue has read what the slot held two heads ago
+        const uint32_t slot = handoffs & 1u;
+        if (handoffs >= 2) {
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait(stat_free(slot), ((handoffs >> 1) - 1) & 1u, abort_flag));
           if (!ok) break;
         }
         ++handoffs;
-        stat[r] = l;
-        mbar_arrive(epi_go);
+        stat[slot * kBM + r] = l;
+        warp_arrive(epi_go(slot));
       }
     }
-  } else if (warp < kWinProducerWarp) {
+  } else {
     // =============================== epilogue (warps 4-7)
-    // Noise head: H_N = O / l into its TMEM columns.  Signal head: the gate
-    // tile arrives by TMA in the 128B-swizzled staging buffer (issued before
-    // the wait for the head), each thread overwrites its row in place with
-    // G (.) (O/l - lambda H_N), and one thread stores the tile by TMA.
+    // Noise head: H_N = O / l into its TMEM columns.  Signal head:
+    // D = O/l - lambda H_N into registers (O released at once), then
+    // out = G (.) D over the row of the staged gate tile, in place.
+    regs_increase<kWinEpilogueRegs>();
     const int qw = warp & 3;
     const int r = threadIdx.x & 127;
     const uint32_t lane_off = static_cast<uint32_t>(qw * 32) << 16;
     const uint32_t gbuf = sbase + L::kGOff;
-    const bool issuer = warp == kWinEpiWarp0 ? elect_one() : false;
-    uint32_t go_waits = 0, o_seen = 0, g_issued = 0, g_seen = 0;
+    uint32_t go_waits = 0, o_seen = 0, g_seen = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
       const WorkItem w = work_item(p, item);
@@ -436,28 +513,18 @@ __global__ void __launch_bounds__(kWinThreads, 1)
       const int64_t row = static_cast<int64_t>(w.b) * p.T + i;
       for (int hh = 0; hh < n_heads && ok; ++hh) {
         const int h = p.g * w.kvh + (hh - 1);  // signal head (hh >= 1)
-        if (hh != 0) {
-          if (issuer) {
-            // the previous tile's stores must have read the buffer
-            bulk_wait_group_read0();
-            fence_proxy_async_smem();
-            mbar_arrive_expect_tx(g_full, (D / 64) * L::kHalf);
-#pragma unroll
-            for (int hf = 0; hf < D / 64; ++hf)
-              tma_load_3d(gbuf + hf * L::kHalf, &tm_gate, g_full, h * D + hf * 64, w.q0, w.b);
-          }
-          ++g_issued;
-          if (row_ok) prefetch_l2(p.lam + row * p.Hs + h);
-        }
-        bool okw = mbar_wait(epi_go, go_waits & 1u, abort_flag);
+        // lambda of a signal head: loaded now, used after the waits
+        const float lam = (hh != 0 && row_ok) ? __bfloat162float(p.lam[row * p.Hs + h]) : 0.f;
+        const uint32_t slot = go_waits & 1u;
+        bool okw = mbar_wait(epi_go(slot), (go_waits >> 1) & 1u, abort_flag);
         ++go_waits;
         if (okw) okw = mbar_wait(o_done, o_seen & 1u, abort_flag);
         ++o_seen;
         ok = __all_sync(0xffffffffu, okw);
         if (!ok) break;
         tc_fence_after();
-        const float l = stat[r];
-        mbar_arrive(stat_free);
+        const float l = stat[slot * kBM + r];
+        warp_arrive(stat_free(slot));
         const float inv_l = l > 0.f ? 1.f / l : 0.f;
         if (hh == 0) {
 #pragma unroll
@@ -470,24 +537,28 @@ __global__ void __launch_bounds__(kWinThreads, 1)
           }
           tmem_wait_st();
           tc_fence_before();
-          mbar_arrive(o_free);
+          warp_arrive(o_free);
           continue;
         }
-        const float lam = row_ok ? __bfloat162float(p.lam[row * p.Hs + h]) : 0.f;
+        float dv[D];
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32], hn[32];
+          tmem_ld32x2_sync(t_o + lane_off + cc * 32, t_hn + lane_off + cc * 32, o, hn);
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            dv[cc * 32 + e] = __uint_as_float(o[e]) * inv_l - lam * __uint_as_float(hn[e]);
+        }
+        // every column of O is in registers: the next head's PV may start
+        tc_fence_before();
+        warp_arrive(o_free);
         ok = __all_sync(0xffffffffu, mbar_wait(g_full, g_seen & 1u, abort_flag));
         ++g_seen;
         if (!ok) break;
         // row r of a 128B-swizzled [128][64] half: 16-byte unit j sits at j ^ (r % 8)
         const uint32_t rbase = gbuf + static_cast<uint32_t>(r) * 128u;
-#pragma unroll 1
+#pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t o[32], hn[32];
-          tmem_ld32x2_sync(t_o + lane_off + cc * 32, t_hn + lane_off + cc * 32, o, hn);
-          if (cc == D / 32 - 1) {
-            // every column of O is in registers: the next head's PV may start
-            tc_fence_before();
-            mbar_arrive(o_free);
-          }
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const int j = (cc & 1) * 4 + q;
@@ -498,35 +569,16 @@ __global__ void __launch_bounds__(kWinThreads, 1)
             uint32_t ow[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const int k0 = q * 8 + 2 * e;
-              const float d0 = __uint_as_float(o[k0]) * inv_l - lam * __uint_as_float(hn[k0]);
-              const float d1 =
-                  __uint_as_float(o[k0 + 1]) * inv_l - lam * __uint_as_float(hn[k0 + 1]);
-              ow[e] = pack_bf16x2(bf16lo_to_f32(gw[e]) * d0, bf16hi_to_f32(gw[e]) * d1);
+              const int k0 = cc * 32 + q * 8 + 2 * e;
+              ow[e] = pack_bf16x2(bf16lo_to_f32(gw[e]) * dv[k0], bf16hi_to_f32(gw[e]) * dv[k0 + 1]);
             }
             sts128(addr, make_uint4(ow[0], ow[1], ow[2], ow[3]));
           }
         }
         // every row written (generic proxy) before the TMA store reads the tile
         fence_proxy_async_smem();
-        mbar_arrive(g_done);
-        if (issuer) {
-          ok = mbar_wait(g_done, (g_seen - 1) & 1u, abort_flag);
-          if (ok) {
-#pragma unroll
-            for (int hf = 0; hf < D / 64; ++hf)
-              tma_store_3d(&tm_out, gbuf + hf * L::kHalf, h * D + hf * 64, w.q0, w.b);
-            bulk_commit_group();
-          }
-        }
-        ok = __all_sync(0xffffffffu, ok);
+        warp_arrive(g_done);
       }
-    }
-    if (issuer) {
-      // a gate tile still in flight (after an abort) lands before the CTA exits;
-      // every output tile store completes
-      if (g_issued > g_seen) mbar_wait_for(g_full, (g_issued - 1) & 1u, 100000000ull);
-      bulk_wait_group0();
     }
   }
 

@@ -129,10 +129,13 @@ int launch_attn(const void *q_sig, const void *q_noise, const void *k, const voi
   const uint64_t T = static_cast<uint64_t>(prm.T), B = static_cast<uint64_t>(prm.B);
   const uint64_t dqs[3] = {static_cast<uint64_t>(Hs) * D, T, B};
   const uint64_t dqn[3] = {static_cast<uint64_t>(Hn) * D, T, B};
+  // K and V hold kv_prefix rows (a sequence shard's halo) before query row 0
+  const uint64_t dkv[3] = {static_cast<uint64_t>(Hn) * D,
+                           T + static_cast<uint64_t>(prm.kv_prefix), B};
   const uint32_t qbox[3] = {64, gdla::kBM, 1};
   const uint32_t kvbox[3] = {64, gdla::kBN, 1};
   if (!make_map(&tm_qs, q_sig, 3, dqs, qbox) || !make_map(&tm_qn, q_noise, 3, dqn, qbox) ||
-      !make_map(&tm_k, k, 3, dqn, kvbox) || !make_map(&tm_v, v, 3, dqn, kvbox) ||
+      !make_map(&tm_k, k, 3, dkv, kvbox) || !make_map(&tm_v, v, 3, dkv, kvbox) ||
       !make_map(&tm_gate, prm.gate, 3, dqs, qbox) || !make_map(&tm_out, prm.out, 3, dqs, qbox))
     return GDLA_ERR_CUDA;
   const uint64_t items = static_cast<uint64_t>(prm.n_qblk) * B * static_cast<uint64_t>(Hn);
@@ -156,7 +159,7 @@ int launch_attn(const void *q_sig, const void *q_noise, const void *k, const voi
     using LW = gdla::WinSmemLayout<D>;
     const uint32_t smem = LW::kBytes > kMinSmem ? LW::kBytes : kMinSmem;
     constexpr auto kern = gdla::gdla_attn_win_kernel<D>;
-    const int rc = prepare_kernel<kern>(smem, 0);
+    const int rc = prepare_kernel<kern>(smem, static_cast<int>(gdla::kWinLaunchRegs));
     if (rc != GDLA_OK) return rc;
     kern<<<static_cast<unsigned>(grid), gdla::kWinThreads, smem, stream>>>(
         tm_qs, tm_qn, tm_k, tm_v, tm_gate, tm_out, run);
@@ -247,19 +250,27 @@ int gdla_kv_expand(const void *c_kv, const void *rms_w, const void *w_kvb, float
                        : launch_expand<64>(c_kv, w_kvb, prm, s);
 }
 
-int gdla_attn_fwd(const void *q_sig, const void *q_noise, const void *k, const void *v,
-                  const void *lambda, const void *gate, void *out, int B, int64_t T, int Hs,
-                  int Hn, int Hkv, int d, int64_t window, int causal, float scale,
-                  int *d_status, void *stream) {
+}  // extern "C"
+
+namespace {
+
+int attn_fwd_impl(const void *q_sig, const void *q_noise, const void *k, const void *v,
+                  const void *lambda, const void *gate, void *out, int B, int64_t T,
+                  int64_t kv_prefix, int Hs, int Hn, int Hkv, int d, int64_t window, int causal,
+                  float scale, int *d_status, void *stream) {
   if (B < 0 || T < 0 || Hs <= 0 || Hn <= 0 || Hkv <= 0 || d <= 0) return GDLA_ERR_INVALID_ARG;
   if (window < 0 || (causal != 0 && causal != 1) || (causal == 0 && window > 0))
+    return GDLA_ERR_INVALID_ARG;
+  // a shard's halo: one K/V tile, only for windows of at most one tile
+  if (kv_prefix != 0 && kv_prefix != gdla::kBN) return GDLA_ERR_INVALID_ARG;
+  if (kv_prefix != 0 && !(causal == 1 && window > 0 && window <= gdla::kBN))
     return GDLA_ERR_INVALID_ARG;
   if (std::isnan(scale) || std::isinf(scale)) return GDLA_ERR_INVALID_ARG;
   if (B == 0 || T == 0) return GDLA_OK;
   if (!q_sig || !q_noise || !k || !v || !lambda || !gate || !out) return GDLA_ERR_INVALID_ARG;
   if (Hn != Hkv || Hs % Hn != 0) return GDLA_ERR_UNSUPPORTED;
   if (d != 64 && d != 128) return GDLA_ERR_UNSUPPORTED;
-  if (T > 0x7fffffffll - gdla::kBM) return GDLA_ERR_UNSUPPORTED;
+  if (T + kv_prefix > 0x7fffffffll - gdla::kBM) return GDLA_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(Hs) * d > 0x7fffffffll) return GDLA_ERR_UNSUPPORTED;
   if (!aligned16(q_sig) || !aligned16(q_noise) || !aligned16(k) || !aligned16(v) ||
       !aligned16(lambda) || !aligned16(gate) || !aligned16(out) ||
@@ -276,13 +287,47 @@ int gdla_attn_fwd(const void *q_sig, const void *q_noise, const void *k, const v
   prm.Hn = Hn;
   prm.g = Hs / Hn;
   prm.n_qblk = static_cast<int>((T + gdla::kBM - 1) / gdla::kBM);
-  prm.window = (window >= T) ? 0 : window;  // a window covering every key is full causal
+  prm.kv_prefix = static_cast<int>(kv_prefix);
+  // a window covering every key is full causal (not so on a shard: its
+  // first rows still reach back into the halo)
+  prm.window = (kv_prefix == 0 && window >= T) ? 0 : window;
+  // Full attention orders its items heaviest-first within bands of KV groups
+  // whose K and V together fill about 32 MB of L2.
+  {
+    const int64_t groups = static_cast<int64_t>(B) * Hn;
+    const int64_t kv_group_bytes = T * static_cast<int64_t>(d) * 2 * 2;
+    int64_t band = (32ll << 20) / (kv_group_bytes > 0 ? kv_group_bytes : 1);
+    if (band < 1) band = 1;
+    if (band > groups) band = groups;
+    prm.band = static_cast<int>(band);
+  }
   prm.causal = causal;
   const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(d));
   prm.scale_log2 = sc * 1.4426950408889634f;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return d == 128 ? launch_attn<128>(q_sig, q_noise, k, v, prm, Hs, Hn, s)
                   : launch_attn<64>(q_sig, q_noise, k, v, prm, Hs, Hn, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+int gdla_attn_fwd(const void *q_sig, const void *q_noise, const void *k, const void *v,
+                  const void *lambda, const void *gate, void *out, int B, int64_t T, int Hs,
+                  int Hn, int Hkv, int d, int64_t window, int causal, float scale,
+                  int *d_status, void *stream) {
+  return attn_fwd_impl(q_sig, q_noise, k, v, lambda, gate, out, B, T, 0, Hs, Hn, Hkv, d, window,
+                       causal, scale, d_status, stream);
+}
+
+int gdla_attn_fwd_sp(const void *q_sig, const void *q_noise, const void *k, const void *v,
+                     const void *lambda, const void *gate, void *out, int B, int64_t T,
+                     int64_t kv_prefix, int Hs, int Hn, int Hkv, int d, int64_t window,
+                     float scale, int *d_status, void *stream) {
+  if (window <= 0 || window > gdla::kBN) return GDLA_ERR_INVALID_ARG;
+  return attn_fwd_impl(q_sig, q_noise, k, v, lambda, gate, out, B, T, kv_prefix, Hs, Hn, Hkv, d,
+                       window, 1, scale, d_status, stream);
 }
 
 int gdla_selftest_wait_timeout(int *d_status, int64_t limit_ns, void *stream) {

@@ -120,6 +120,34 @@ int gdla_attn_fwd(const void *q_sig, const void *q_noise, const void *k,
                   void *stream);
 
 /*
+ * gdla_attn_fwd_sp - gdla_attn_fwd with a sliding window on one shard of a
+ * sequence split across GPUs ("Motif 3: Technical Report", paper.rainbus.top:
+ * its long-context training step and "technical novelty" paragraph describe
+ * window-aware ring attention for the sliding-window layers, where one halo
+ * exchange of the previous shard's last keys replaces the ring's rotations).
+ *
+ * The shard holds T consecutive query tokens.  K and V hold kv_prefix rows
+ * before the shard's first token, the halo copied from the previous shard,
+ * then the shard's own T rows: query row i reads K/V row i + kv_prefix and
+ * keeps keys j with i + kv_prefix - window < j <= i + kv_prefix.  The first
+ * shard of a sequence passes kv_prefix = 0 (no keys before it).
+ *
+ * q_sig, q_noise, lambda, gate, out   as in gdla_attn_fwd ([B, T, ...])
+ * k, v       [B, kv_prefix + T, Hkv, d]  bf16, read
+ * kv_prefix  0 or 128 (one K/V tile; 128 >= window - 1 covers any window)
+ * window     1 .. 128, causal
+ * Returns GDLA_ERR_INVALID_ARG for another kv_prefix or window; otherwise as
+ * gdla_attn_fwd.  Each output row equals, bit for bit, the row the unsharded
+ * call computes for the same token when the shard starts on a multiple of
+ * 128 tokens (and the window is shorter than the whole sequence).
+ */
+int gdla_attn_fwd_sp(const void *q_sig, const void *q_noise, const void *k,
+                     const void *v, const void *lambda, const void *gate,
+                     void *out, int B, int64_t T, int64_t kv_prefix, int Hs,
+                     int Hn, int Hkv, int d, int64_t window, float scale,
+                     int *d_status, void *stream);
+
+/*
  * gdla_selftest_wait_timeout - device-side check of the failure path.
  *
  * Every pipeline wait inside the kernels above polls an mbarrier with a time

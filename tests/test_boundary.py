@@ -34,7 +34,7 @@ def _declared_functions():
 def test_exports_every_declared_symbol(lib):
     declared = _declared_functions()
     assert set(declared) == {"gdla_version", "gdla_status_string", "gdla_kv_expand",
-                             "gdla_attn_fwd", "gdla_selftest_wait_timeout"}
+                             "gdla_attn_fwd", "gdla_attn_fwd_sp", "gdla_selftest_wait_timeout"}
     for name in declared:
         assert hasattr(lib, name), f"{name} missing from libgdla.so"
     assert set(declared) == set(_binding.EXPORTED)
@@ -113,3 +113,23 @@ def test_missing_library_fails_loudly(tmp_path):
 ])
 def test_selftest_argument_errors(lib, status, limit, code):
     assert lib.gdla_selftest_wait_timeout(status, limit, None) == code
+
+
+def _sp(lib, q=A, qn=A, k=A, v=A, lam=A, gate=A, out=A, B=1, T=256, kv_prefix=128, Hs=8, Hn=2,
+        Hkv=2, d=64, window=128, scale=0.0, status=None):
+    return lib.gdla_attn_fwd_sp(q, qn, k, v, lam, gate, out, B, T, kv_prefix, Hs, Hn, Hkv, d,
+                                window, ctypes.c_float(scale), status, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(kv_prefix=64), INVALID), (dict(kv_prefix=-128), INVALID), (dict(kv_prefix=256), INVALID),
+    (dict(window=0), INVALID), (dict(window=129), INVALID), (dict(window=-1), INVALID),
+    (dict(window=129, kv_prefix=0), INVALID), (dict(window=0, kv_prefix=0), INVALID),
+    (dict(k=None), INVALID), (dict(out=None), INVALID), (dict(T=-1), INVALID),
+    (dict(Hn=2, Hkv=4), UNSUPPORTED), (dict(d=96), UNSUPPORTED),
+    (dict(T=2 ** 31 - 200), UNSUPPORTED),
+    (dict(k=M), ALIGN), (dict(v=M), ALIGN), (dict(status=0x100002), ALIGN),
+    (dict(T=0), OK), (dict(B=0), OK),
+])
+def test_sp_argument_errors(lib, kw, code):
+    assert _sp(lib, **kw) == code
