@@ -105,6 +105,10 @@ class Oracle:
                                                  i32, i64, i32, i32, i32, i32, i64, i32, f64, vp,
                                                  i64, vp]
         lib.gdla_oracle_attn_compact.restype = ctypes.c_int
+        lib.gdla_oracle_decode.argtypes = [vp, i32, vp, i32, vp, i32, vp, vp, i32, f64, vp, i32,
+                                           vp, i32, vp, i32, i32, i64, i32, i32, i32, i32, i32,
+                                           i64, f64, vp]
+        lib.gdla_oracle_decode.restype = ctypes.c_int
         lib.gdla_oracle_version.restype = ctypes.c_int
         self.lib = lib
         self.path = lib_path
@@ -236,6 +240,41 @@ class Oracle:
         return out
 
 
+    # decode: the newest token of each sequence over its latent cache
+    def decode(self, q_sig, q_noise, c_kv, cache_len, w_kvb, lam, gate, rms_w=None,
+               eps: float = 1e-6, window: int = 0, scale=None) -> np.ndarray:
+        """O[B, Hs*d] for the query token of each sequence (its position is
+        cache_len[b] - 1), from the raw KV latents c_kv [B, L_max, d_latent]:
+        RMSNorm, W^KV_b expand, then the GDLA forward for that one row.
+
+        q_sig [B,Hs,d], q_noise [B,Hn,d], lam [B,Hs], gate [B,Hs*d];
+        cache_len: B integers in 1..L_max.
+        """
+        qs, qsp, qsdt = _arr(q_sig)
+        qn, qnp, qndt = _arr(q_noise)
+        ca, cp, cdt = _arr(c_kv)
+        wa, wp, wdt = _arr(w_kvb)
+        la, lp, ldt = _arr(lam)
+        ga, gp, gdt = _arr(gate)
+        ra, rp, rdt = (None, None, F64) if rms_w is None else _arr(rms_w)
+        B, Hs, d = qs.shape
+        Hn = qn.shape[1]
+        L_max, dl = ca.shape[1], ca.shape[2]
+        Hkv = wa.shape[1] // (2 * d)
+        lens = np.ascontiguousarray(np.asarray(cache_len, dtype=np.int64).reshape(-1))
+        if lens.size != B or lens.min() < 1 or lens.max() > L_max:
+            raise ValueError("cache_len must hold B lengths in 1..L_max")
+        if scale is None:
+            scale = 1.0 / np.sqrt(d)
+        out = np.empty((B, Hs * d), dtype=np.float64)
+        rc = self.lib.gdla_oracle_decode(qsp, qsdt, qnp, qndt, cp, cdt, lens.ctypes.data, rp, rdt,
+                                         float(eps), wp, wdt, lp, ldt, gp, gdt, B, L_max, dl, Hs,
+                                         Hn, Hkv, d, int(window), float(scale), out.ctypes.data)
+        if rc != 0:
+            raise ValueError("oracle rejected the decode arguments (rc %d)" % rc)
+        return out
+
+
 _default = None
 
 
@@ -269,3 +308,7 @@ def gdla_attn(*a, **k):
 
 def gdla_attn_rows(*a, **k):
     return default().gdla_attn_rows(*a, **k)
+
+
+def decode(*a, **k):
+    return default().decode(*a, **k)

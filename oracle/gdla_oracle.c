@@ -286,3 +286,75 @@ int gdla_oracle_attn_compact(const void *q_sig, int qs_dt, const void *q_noise,
                    gate, gate_dt, 1, T, Hs, Hn, Hkv, d, window, causal, scale,
                    rows, n_rows, out);
 }
+
+/*
+ * Decode over the latent cache ([R] "technical novelty" paragraph: the two
+ * query paths share one up-projected KV, so the inference cache is the KV
+ * latent alone, the same size as MLA's).  Sequence b has cache_len[b] tokens
+ * whose KV latents c_KV are cached; its newest token, i = cache_len[b] - 1,
+ * is the query.  The result is the forward pass of [R] step 2 for that one
+ * row, written out as the definition:
+ *   c_hat = RMSNorm(c_KV[b, 0..i])                 (gdla_oracle_rmsnorm)
+ *   K, V  = c_hat W^KV_b                           (gdla_oracle_kv_expand)
+ *   O[b]  = G (.) (H_S - lambda Repeat_g(H_N))     for row i (attn_impl)
+ * q_sig [B, Hs, d], q_noise [B, Hn, d], lambda [B, Hs], gate [B, Hs*d] hold
+ * the query token of each sequence; c_kv is [B, L_max, d_latent].  Only the
+ * keys J(i) of the window enter (window 0 = full causal).  out: [B, Hs*d].
+ * Returns 0, -1 for bad head counts or lengths, -2 when out of memory.
+ */
+int gdla_oracle_decode(const void *q_sig, int qs_dt, const void *q_noise,
+                       int qn_dt, const void *c_kv, int c_dt,
+                       const int64_t *cache_len, const void *rms_w, int w_dt,
+                       double eps, const void *w_kvb, int wk_dt,
+                       const void *lam, int lam_dt, const void *gate,
+                       int gate_dt, int B, int64_t L_max, int d_latent,
+                       int Hs, int Hn, int Hkv, int d, int64_t window,
+                       double scale, double *out) {
+  if (Hn <= 0 || Hkv <= 0 || Hs % Hn != 0 || Hn != Hkv) return -1;
+  for (int b = 0; b < B; ++b) {
+    const int64_t Lb = cache_len[b];
+    if (Lb < 1 || Lb > L_max) return -1;
+    /* only the cached tokens the query's mask keeps are normalised and
+     * expanded: [first, Lb) with first = Lb - window under a window */
+    const int64_t first = (window > 0 && Lb > window) ? Lb - window : 0;
+    const int64_t L = Lb - first;
+    double *chat = (double *)malloc(sizeof(double) * (size_t)(L * d_latent));
+    double *k = (double *)malloc(sizeof(double) * (size_t)(L * Hkv * d));
+    double *v = (double *)malloc(sizeof(double) * (size_t)(L * Hkv * d));
+    if (!chat || !k || !v) {
+      free(chat);
+      free(k);
+      free(v);
+      return -2;
+    }
+    /* the kept cache rows of sequence b */
+    const int64_t c_off = ((int64_t)b * L_max + first) * d_latent;
+    const void *cb;
+    if (c_dt == ORACLE_F64) cb = (const double *)c_kv + c_off;
+    else if (c_dt == ORACLE_F32) cb = (const float *)c_kv + c_off;
+    else cb = (const uint16_t *)c_kv + c_off;
+    gdla_oracle_rmsnorm(cb, c_dt, rms_w, w_dt, eps, L, d_latent, chat);
+    gdla_oracle_kv_expand(chat, w_kvb, wk_dt, L, d_latent, Hkv, d, d, k, v);
+    /* the query token's inputs, addressed as the one evaluated row; it is
+     * the last of the L kept tokens */
+    const int64_t row = L - 1;
+    const void *qs_b, *qn_b, *lam_b, *gate_b;
+#define ORACLE_AT(ptr, dt, off) \
+    ((dt) == ORACLE_F64 ? (const void *)((const double *)(ptr) + (off)) : \
+     (dt) == ORACLE_F32 ? (const void *)((const float *)(ptr) + (off)) : \
+                          (const void *)((const uint16_t *)(ptr) + (off)))
+    qs_b = ORACLE_AT(q_sig, qs_dt, (int64_t)b * Hs * d);
+    qn_b = ORACLE_AT(q_noise, qn_dt, (int64_t)b * Hn * d);
+    lam_b = ORACLE_AT(lam, lam_dt, (int64_t)b * Hs);
+    gate_b = ORACLE_AT(gate, gate_dt, (int64_t)b * Hs * d);
+#undef ORACLE_AT
+    const int rc = attn_impl(qs_b, qs_dt, qn_b, qn_dt, k, ORACLE_F64, v, ORACLE_F64,
+                             lam_b, lam_dt, gate_b, gate_dt, 1, L, Hs, Hn, Hkv, d,
+                             window, 1, scale, &row, 1, out + (int64_t)b * Hs * d);
+    free(chat);
+    free(k);
+    free(v);
+    if (rc != 0) return rc;
+  }
+  return 0;
+}

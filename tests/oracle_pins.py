@@ -317,4 +317,129 @@ def pin_scale_placement(o):
     assert np.array_equal(a, c), "default scale must be 1/sqrt(d)"
 
 
+# ---------------------------------------------------------------- decode
+# The decode reads the KV latent cache ("Motif 3: Technical Report",
+# paper.rainbus.top, "technical novelty" paragraph: the inference cache is the
+# latent, the size of MLA's) and computes the forward pass for each
+# sequence's newest token.
+
+
+def _decode_case(B=3, L_max=37, Hs=8, Hn=2, d=16, dl=64, seed=5):
+    g = torch.Generator().manual_seed(seed)
+    bf = lambda *shape, s=1.0: (torch.randn(*shape, generator=g) * s).to(torch.bfloat16)
+    x = {
+        "q_sig": bf(B, Hs, d), "q_noise": bf(B, Hn, d), "c_kv": bf(B, L_max, dl),
+        "w_kvb": bf(dl, Hn * 2 * d, s=dl ** -0.5),
+        "lam": torch.sigmoid(torch.randn(B, Hs, generator=g)).to(torch.bfloat16),
+        "gate": torch.sigmoid(torch.randn(B, Hs * d, generator=g)).to(torch.bfloat16),
+        "rms_w": (torch.rand(dl, generator=g) + 0.5).to(torch.bfloat16),
+    }
+    return x, (B, L_max, Hs, Hn, d, dl)
+
+
+def _decode_torch(x, lens, window, eps=1e-6, use_w=True):
+    """The decode by torch library routines in float64: rms_norm, matmul,
+    SDPA for the one query row, then the differential combine and gate."""
+    B, Hs, d = x["q_sig"].shape
+    Hn = x["q_noise"].shape[1]
+    g = Hs // Hn
+    w = _f64(x["w_kvb"])
+    out = []
+    for b in range(B):
+        L = int(lens[b])
+        c = _f64(x["c_kv"][b, :L])
+        chat = F.rms_norm(c, (c.shape[-1],), weight=_f64(x["rms_w"]) if use_w else None, eps=eps)
+        kv = (chat @ w).view(L, Hn, 2 * d)
+        k, v = kv[..., :d], kv[..., d:]
+        lo = max(0, L - window) if window > 0 else 0
+
+        def attend(q, heads_per_kv):  # q [H, d] -> [H, d]
+            kk = k[lo:].repeat_interleave(heads_per_kv, dim=1).permute(1, 0, 2)
+            vv = v[lo:].repeat_interleave(heads_per_kv, dim=1).permute(1, 0, 2)
+            return F.scaled_dot_product_attention(q.unsqueeze(1), kk, vv,
+                                                  scale=1.0 / math.sqrt(d)).squeeze(1)
+        hs = attend(_f64(x["q_sig"][b]), g)
+        hn = attend(_f64(x["q_noise"][b]), 1)
+        dd = hs - _f64(x["lam"][b]).unsqueeze(1) * hn.repeat_interleave(g, dim=0)
+        out.append((_f64(x["gate"][b]).view(Hs, d) * dd).reshape(-1))
+    return torch.stack(out).numpy()
+
+
+def pin_decode_matches_torch_expand_sdpa(o):
+    x, (B, L_max, Hs, Hn, d, dl) = _decode_case()
+    lens = [37, 1, 20]
+    for window in (0, 5):
+        got = o.decode(x["q_sig"], x["q_noise"], x["c_kv"], lens, x["w_kvb"], x["lam"],
+                       x["gate"], rms_w=x["rms_w"], window=window)
+        _close(got, _decode_torch(x, lens, window), rtol=1e-10, atol=1e-12,
+               what=f"decode vs torch (window {window})")
+
+
+def pin_decode_absorbed_latent_form(o):
+    """W^KV_b absorbed into the query and the output: scores q.(c_hat W_K)
+    = (W_K q).c_hat and sum_j p_j (c_hat_j W_V) = (sum_j p_j c_hat_j) W_V,
+    so the decode can run in the 512-d latent space.  Written out here in
+    numpy, it must equal the oracle's expand-then-attend decode."""
+    x, (B, L_max, Hs, Hn, d, dl) = _decode_case(seed=8)
+    lens = [30, 37, 2]
+    got = o.decode(x["q_sig"], x["q_noise"], x["c_kv"], lens, x["w_kvb"], x["lam"], x["gate"],
+                   rms_w=x["rms_w"])
+    W = x["w_kvb"].double().numpy().reshape(dl, Hn, 2 * d)
+    g = Hs // Hn
+    rw = x["rms_w"].double().numpy()
+    for b in range(B):
+        L = lens[b]
+        c = x["c_kv"][b, :L].double().numpy()
+        chat = c / np.sqrt((c * c).mean(axis=1, keepdims=True) + 1e-6) * rw
+
+        def latent_head(q, kvh):
+            qt = W[:, kvh, :d] @ q                 # absorbed query, [dl]
+            s = chat @ qt / math.sqrt(d)
+            p = np.exp(s - s.max())
+            z = p @ chat / p.sum()                 # attention in latent space, [dl]
+            return z @ W[:, kvh, d:]               # absorbed output projection
+        hn = [latent_head(x["q_noise"][b, n].double().numpy(), n) for n in range(Hn)]
+        for h in range(Hs):
+            hs = latent_head(x["q_sig"][b, h].double().numpy(), h // g)
+            want = x["gate"][b, h * d:(h + 1) * d].double().numpy() * (
+                hs - float(x["lam"][b, h]) * hn[h // g])
+            _close(got[b, h * d:(h + 1) * d], want, rtol=1e-10, atol=1e-12,
+                   what=f"absorbed decode b={b} h={h}")
+
+
+def pin_decode_single_token_and_window_one(o):
+    """One cached token, or a window of 1: O = G (.) (1 - lambda) V_last with
+    V_last = RMSNorm(c_last) W_V of the head's KV group."""
+    x, (B, L_max, Hs, Hn, d, dl) = _decode_case(seed=9)
+    g = Hs // Hn
+    W = x["w_kvb"].double().numpy().reshape(dl, Hn, 2 * d)
+    rw = x["rms_w"].double().numpy()
+    for lens, window in (([1, 1, 1], 0), ([37, 12, 3], 1)):
+        got = o.decode(x["q_sig"], x["q_noise"], x["c_kv"], lens, x["w_kvb"], x["lam"],
+                       x["gate"], rms_w=x["rms_w"], window=window)
+        for b in range(B):
+            c = x["c_kv"][b, lens[b] - 1].double().numpy()
+            chat = c / np.sqrt((c * c).mean() + 1e-6) * rw
+            for h in range(Hs):
+                v = chat @ W[:, h // g, d:]
+                want = x["gate"][b, h * d:(h + 1) * d].double().numpy() * \
+                    (1.0 - float(x["lam"][b, h])) * v
+                _close(got[b, h * d:(h + 1) * d], want, rtol=1e-12, atol=1e-13,
+                       what=f"decode closed form lens={lens} b={b} h={h}")
+
+
+def pin_decode_ignores_rows_past_the_length(o):
+    x, _ = _decode_case(seed=10)
+    lens = [10, 37, 25]
+    a = o.decode(x["q_sig"], x["q_noise"], x["c_kv"], lens, x["w_kvb"], x["lam"], x["gate"])
+    c2 = x["c_kv"].clone()
+    for b, L in enumerate(lens):
+        c2[b, L:] = 1e3
+    bb = o.decode(x["q_sig"], x["q_noise"], c2, lens, x["w_kvb"], x["lam"], x["gate"])
+    assert np.array_equal(a, bb), "decode read cache rows past the sequence length"
+    c2[1, 36] += 1.0  # the query token's own latent does count
+    cc = o.decode(x["q_sig"], x["q_noise"], c2, lens, x["w_kvb"], x["lam"], x["gate"])
+    assert not np.array_equal(a[1], cc[1])
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -33,6 +33,11 @@ MUTANTS = {
     "rms_sum_not_mean": ("sqrt(ss / (double)d_latent + eps)", "sqrt(ss + eps)"),
     "expand_w_transposed": ("(int64_t)k * ncol + col)", "col * d_latent + k)"),
     "expand_k_v_swapped": ("if (x < dk)\n        k_out", "if (x >= dk)\n        k_out"),
+    "decode_query_is_first_token": ("const int64_t row = L - 1;", "const int64_t row = 0;"),
+    "decode_window_slice_drops_oldest_key": ("(window > 0 && Lb > window) ? Lb - window : 0",
+                                             "(window > 0 && Lb >= window) ? Lb - window + 1 : 0"),
+    "decode_cache_stride_by_length": ("((int64_t)b * L_max + first) * d_latent",
+                                      "((int64_t)b * Lb + first) * d_latent"),
 }
 
 
