@@ -51,6 +51,8 @@ STEPS = {
     "tiny": ("tiny",),
     "long_full": ("long_full",),
     "long_window": ("long_window",),
+    "decode": ("decode",),
+    "decode_window": ("decode_window",),
 }
 # A timed region at least this long runs tensor-bound kernels under the power
 # cap, so their fraction is taken against the sustained bf16 peak.
@@ -161,29 +163,52 @@ def _gpu_id(torch, dev):
 class Layer:
     """One layer of a step: its inputs, output buffer and launches."""
 
-    def __init__(self, wl, x, dev):
+    def __init__(self, wl, x, dev, gdla=None):
         import torch
         self.wl = wl
         self.x = x
         n_tok = wl.B * wl.T
         self.kbuf = self.vbuf = None
+        # the inputs a step brings from the host (decode: the query side; the
+        # latent cache and W^KV_b stay resident)
+        self.step_inputs = [n for n in x if not (wl.decode and n in ("c_kv", "w_kvb"))]
+        # (label, kernel, flops, bytes, kernel launches) per library call
+        self.launches = []
+        if wl.decode:
+            self.c_hat = gdla.gdla_latent_rmsnorm(x["c_kv"], None, wl.eps)
+            self.cache_len = torch.full((wl.B,), wl.T, dtype=torch.int32, device=dev)
+            self.ws = torch.empty(gdla.gdla_decode_workspace_bytes(wl.B, wl.T, wl.Hs, wl.Hn,
+                                                                   wl.d_latent, wl.window),
+                                  dtype=torch.uint8, device=dev)
+            self.out = torch.empty((wl.B, wl.Hs * wl.d), dtype=torch.bfloat16, device=dev)
+            self.launches.append(("%s/decode" % wl.name, "gdla_decode_attn_kernel",
+                                  wl.attn_flops(), wl.decode_bytes(), 3))
+            return
         if wl.latent:
             self.kbuf = torch.empty((n_tok, wl.Hkv, wl.d), dtype=torch.bfloat16, device=dev)
             self.vbuf = torch.empty_like(self.kbuf)
         self.out = torch.empty((wl.B, wl.T, wl.Hs * wl.d), dtype=torch.bfloat16, device=dev)
-        # (label, kernel, flops, bytes) per launch, in launch order
-        self.launches = []
         if wl.latent:
             self.launches.append(("%s/expand" % wl.name, "gdla_kv_expand_kernel",
-                                  wl.expand_flops(), wl.expand_bytes()))
+                                  wl.expand_flops(), wl.expand_bytes(), 1))
         self.launches.append(("%s/attn" % wl.name, attn_kernel_name(wl), wl.attn_flops(),
-                              wl.attn_bytes()))
+                              wl.attn_bytes(), 1))
 
-    def run(self, gdla, status, stream, inp=None, out=None, events=None):
+    def run(self, gdla, status, stream, inp=None, out=None, events=None, cache_len=None):
         """Enqueue the layer; events[i] = (start, end) for launch i."""
         wl = self.wl
         inp = self.x if inp is None else inp
         out = self.out if out is None else out
+        if wl.decode:
+            if events is not None:
+                events[0][0].record(stream)
+            gdla.gdla_decode_fwd(inp["q_sig"], inp["q_noise"], self.c_hat,
+                                 self.cache_len if cache_len is None else cache_len,
+                                 self.x["w_kvb"], inp["lam"], inp["gate"], window=wl.window,
+                                 out=out, workspace=self.ws, d_status=status, stream=stream)
+            if events is not None:
+                events[0][1].record(stream)
+            return
         li = 0
         if wl.latent:
             if events is not None:
@@ -256,7 +281,7 @@ def run_ours(args):
     dev = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
     torch.cuda.set_device(dev)
     layers = [Layer(WORKLOADS[n], make_inputs(WORKLOADS[n], seed=replica_seed(rank), device=dev),
-                    dev) for n in STEPS[args.workload]]
+                    dev, gdla) for n in STEPS[args.workload]]
     stream = torch.cuda.current_stream(dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     n_launch = sum(len(L.launches) for L in layers)
@@ -300,12 +325,22 @@ def run_ours(args):
         raise RuntimeError("kernel reported status %d" % int(status.item()))
     ms = max_over_ranks(ms, world, dev)
     # the first tokens of each output, for the parity figures of the CPU sample
-    head_out = [L.out[:1, :min(L.wl.T, SAMPLE_SPAN)].float().cpu() for L in layers]
+    # (decode: every sequence's output over the first SAMPLE_SPAN cache rows)
+    head_out = []
+    for L in layers:
+        if L.wl.decode:
+            span = torch.full_like(L.cache_len, min(L.wl.T, SAMPLE_SPAN))
+            o = torch.empty_like(L.out)
+            L.run(gdla, status, stream, out=o, cache_len=span)
+            head_out.append(o.float().cpu())
+        else:
+            head_out.append(L.out[:1, :min(L.wl.T, SAMPLE_SPAN)].float().cpu())
 
     e2e_ms, e2e_steps, h2d, d2h = _e2e(args, layers, step, stream, dev, world)
 
-    step_flops = sum(f for L in layers for (_, _, f, _) in L.launches)
-    n_tok = sum(L.wl.B * L.wl.T for L in layers)
+    step_flops = sum(f for L in layers for (_, _, f, _, _) in L.launches)
+    # tokens a step produces: every token of a prefill layer, one per sequence in decode
+    n_tok = sum(L.wl.B * (1 if L.wl.decode else L.wl.T) for L in layers)
     value = step_flops * args.steps * world / (ms * 1e-3) / 1e12
     e2e_value = step_flops * e2e_steps * world / (e2e_ms * 1e-3) / 1e12
     peaks, peak_src = _peaks()
@@ -313,7 +348,7 @@ def run_ours(args):
     entries = []
     j = 0
     for L in layers:
-        for (label, kernel, flops, nbytes) in L.launches:
+        for (label, kernel, flops, nbytes, _) in L.launches:
             traffic = _traffic_from_profiles(L.wl.name, kernel)
             entries.append(_roofline_entry(label, kernel, flops, nbytes, launch_ms[j], peaks,
                                            peak_src, sustained, traffic))
@@ -340,11 +375,12 @@ def run_ours(args):
         "config": {
             "workload": args.workload,
             "layers": [{"name": L.wl.name, "B": L.wl.B, "T": L.wl.T, "window": L.wl.window,
-                        "causal": L.wl.causal, "latent_kv": L.wl.latent} for L in layers],
+                        "causal": L.wl.causal, "latent_kv": L.wl.latent or L.wl.decode,
+                        "decode": L.wl.decode} for L in layers],
             "Hs": wl0.Hs, "Hn": wl0.Hn, "Hkv": wl0.Hkv, "d": wl0.d,
             "parallelism": "replicas" if world > 1 else "single GPU",
             "l2": "inputs larger than L2 (%.0f MB per step)" % (
-                sum(nb for L in layers for (_, _, _, nb) in L.launches) / 1e6),
+                sum(nb for L in layers for (_, _, _, nb, _) in L.launches) / 1e6),
         },
         "roofline": top,
         "rooflines": entries,
@@ -352,7 +388,7 @@ def run_ours(args):
         "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "mode": "pinned host buffers, copies pipelined with compute over 3 streams"},
-        "gpu_launches": n_launch * args.steps,
+        "gpu_launches": sum(k for L in layers for (_, _, _, _, k) in L.launches) * args.steps,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -379,11 +415,11 @@ def _e2e(args, layers, step, stream, dev, world):
         h.copy_(t)
         return h
 
-    host = [{n: pinned_copy(t) for n, t in L.x.items()} for L in layers]
+    host = [{n: pinned_copy(L.x[n]) for n in L.step_inputs} for L in layers]
     out_host = [torch.empty(L.out.shape, dtype=L.out.dtype, pin_memory=True) for L in layers]
     h2d = sum(t.numel() * t.element_size() for hs in host for t in hs.values())
     d2h = sum(L.out.numel() * L.out.element_size() for L in layers)
-    dev_in = [[L.x for L in layers], [{n: torch.empty_like(t) for n, t in L.x.items()}
+    dev_in = [[L.x for L in layers], [{n: torch.empty_like(L.x[n]) for n in L.step_inputs}
                                       for L in layers]]
     dev_out = [[L.out for L in layers], [torch.empty_like(L.out) for L in layers]]
     s_up, s_run, s_down = (torch.cuda.Stream(dev) for _ in range(3))
@@ -482,6 +518,8 @@ def _oracle_sample(wl, x, seconds, rng):
     import oracle
 
     span = min(wl.T, SAMPLE_SPAN)
+    if wl.decode:
+        return _oracle_decode_sample(wl, x, seconds, rng, span)
     # rows per pass: a sliding-window row costs W pairs, a causal row up to span
     n_rows = 256 if wl.window > 0 else 8
     total_flops, total_s = 0, 0.0
@@ -521,6 +559,37 @@ def _oracle_sample(wl, x, seconds, rng):
     return total_flops, total_s, desc, np.concatenate(all_rows), np.concatenate(all_ref)
 
 
+def _oracle_decode_sample(wl, x, seconds, rng, span):
+    """The decode sample: sequences drawn uniformly, each decoding its token
+    at cache length `span` (RMSNorm + expand of the kept cache rows and the
+    forward pass for the one query row).  Rows are sequence indices."""
+    import numpy as np
+
+    import oracle
+
+    n_seq = 16 if wl.window > 0 else 1
+    total_flops, total_s = 0, 0.0
+    all_rows, all_ref = [], []
+    w = x["w_kvb"].cpu()
+    while total_s < seconds:
+        rows = np.sort(rng.integers(0, x["q_sig"].shape[0], n_seq))
+        t0 = time.perf_counter()
+        sub = {n: x[n][rows].cpu() for n in ("q_sig", "q_noise", "lam", "gate")}
+        c = x["c_kv"][rows, :span].cpu()
+        ref = oracle.decode(sub["q_sig"], sub["q_noise"], c, [span] * n_seq, w, sub["lam"],
+                            sub["gate"], eps=wl.eps, window=wl.window)
+        total_s += time.perf_counter() - t0
+        kept = min(span, wl.window) if wl.window > 0 else span
+        total_flops += n_seq * 4 * wl.d * (wl.Hs + wl.Hn) * kept
+        all_rows.append(rows)
+        all_ref.append(ref)
+    n_done = sum(len(r) for r in all_rows)
+    desc = ("%s: %d sequences drawn uniformly, each decoding at cache length %d (RMSNorm + "
+            "W^KV_b expand of the kept cache rows, then the forward pass of the query token)" % (
+                wl.name, n_done, span))
+    return total_flops, total_s, desc, np.concatenate(all_rows), np.concatenate(all_ref)
+
+
 def _parity(gpu_rows, ref):
     """Error statistics of GPU output rows against the oracle's (per tensor
     tolerance max|gpu - oracle| <= 1e-2 * max|oracle| + 1e-3)."""
@@ -546,7 +615,7 @@ def cpu_baseline(layers, head_out, seconds=15.0):
         flops += f
         secs += s
         descs.append(d)
-        gpu_rows = ho[0].numpy()[rows].astype(np.float64)
+        gpu_rows = (ho if L.wl.decode else ho[0]).numpy()[rows].astype(np.float64)
         parity[L.wl.name] = _parity(gpu_rows, ref)
     threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
     return ({"value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s", "cores": threads,
@@ -567,7 +636,8 @@ def run_reference(args):
     oracle.build()
     wls = [WORKLOADS[n] for n in STEPS[args.workload]]
     # inputs drawn on the CPU in the same recipe; only the sampled slices are used
-    xs = [make_inputs(wl, seed=0, device="cpu", T=min(wl.T, SAMPLE_SPAN), B=1) for wl in wls]
+    xs = [make_inputs(wl, seed=0, device="cpu", T=min(wl.T, SAMPLE_SPAN),
+                      B=(min(wl.B, 16) if wl.decode else 1)) for wl in wls]
     per_step = max(2.0, min(20.0, 60.0 / max(1, args.steps + args.warmup)))
     rng = np.random.default_rng(0)
     for _ in range(args.warmup):
@@ -584,7 +654,7 @@ def run_reference(args):
             descs.append(d)
     value = flops / secs / 1e12
     threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    n_tok = sum(wl.B * wl.T for wl in wls)
+    n_tok = sum(wl.B * (1 if wl.decode else wl.T) for wl in wls)
     step_flops = sum(wl.attn_flops() + (wl.expand_flops() if wl.latent else 0) for wl in wls)
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
@@ -594,7 +664,8 @@ def run_reference(args):
         "data": "synthetic (same recipe, CPU draw)",
         "config": {"workload": args.workload,
                    "layers": [{"name": wl.name, "B": wl.B, "T": wl.T, "window": wl.window,
-                               "causal": wl.causal, "latent_kv": wl.latent} for wl in wls],
+                               "causal": wl.causal, "latent_kv": wl.latent or wl.decode,
+                               "decode": wl.decode} for wl in wls],
                    "Hs": wls[0].Hs, "Hn": wls[0].Hn, "Hkv": wls[0].Hkv, "d": wls[0].d},
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": threads,
                          "kind": "oracle", "sample": "; ".join(descs) + " (per step)"},

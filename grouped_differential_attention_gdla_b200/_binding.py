@@ -31,7 +31,8 @@ GDLA_ERR_TIMEOUT = -5
 
 # every symbol include/gdla.h declares
 EXPORTED = ("gdla_version", "gdla_status_string", "gdla_kv_expand", "gdla_attn_fwd",
-            "gdla_attn_fwd_sp", "gdla_selftest_wait_timeout")
+            "gdla_attn_fwd_sp", "gdla_latent_rmsnorm", "gdla_decode_workspace_bytes",
+            "gdla_decode_fwd", "gdla_selftest_wait_timeout")
 
 _lib = None
 # One status word per device, used when a caller passes none (see check_status).
@@ -68,6 +69,13 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.gdla_attn_fwd_sp.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i64, i32, i32, i32,
                                      i32, i64, f32, vp, vp]
     lib.gdla_attn_fwd_sp.restype = i32
+    lib.gdla_latent_rmsnorm.argtypes = [vp, vp, f32, vp, i64, i32, vp, vp]
+    lib.gdla_latent_rmsnorm.restype = i32
+    lib.gdla_decode_workspace_bytes.argtypes = [i32, i64, i32, i32, i32, i64]
+    lib.gdla_decode_workspace_bytes.restype = ctypes.c_size_t
+    lib.gdla_decode_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32,
+                                    i32, i64, f32, vp, ctypes.c_size_t, vp, vp]
+    lib.gdla_decode_fwd.restype = i32
     lib.gdla_selftest_wait_timeout.argtypes = [vp, i64, vp]
     lib.gdla_selftest_wait_timeout.restype = i32
     if path is None:
@@ -252,6 +260,87 @@ def gdla_attn_fwd_sp(q_sig: torch.Tensor, q_noise: torch.Tensor, k: torch.Tensor
                                          float(scale), ps, _stream_ptr(q_sig.device, stream))
     if rc != GDLA_OK:
         raise GDLAError(rc, "gdla_attn_fwd_sp")
+    if _sync_check_enabled():
+        check_status(q_sig.device, d_status)
+    return out
+
+
+def gdla_latent_rmsnorm(c_kv: torch.Tensor, rms_w: Optional[torch.Tensor] = None,
+                        eps: float = 1e-6, out: Optional[torch.Tensor] = None,
+                        d_status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """RMSNorm of KV latents entering the decode cache: c_kv [..., d_latent]
+    (bf16, CUDA) -> out of the same shape (may be a view into the cache)."""
+    dl = c_kv.shape[-1]
+    n = c_kv.numel() // dl if dl else 0
+    if out is None:
+        out = torch.empty_like(c_kv)
+    pc = _check(c_kv, "c_kv")
+    po = _check(out, "out", tuple(c_kv.shape))
+    pr = _check(rms_w, "rms_w", (dl,)) if rms_w is not None else None
+    _same_device(c_kv.device, [("rms_w", rms_w), ("out", out)])
+    ps = _status_ptr(d_status, c_kv.device)
+    rc = load_library().gdla_latent_rmsnorm(pc, pr, float(eps), po, n, dl, ps,
+                                            _stream_ptr(c_kv.device, stream))
+    if rc != GDLA_OK:
+        raise GDLAError(rc, "gdla_latent_rmsnorm")
+    return out
+
+
+def gdla_decode_workspace_bytes(B: int, L_max: int, Hs: int, Hn: int, d_latent: int = 512,
+                                window: int = 0) -> int:
+    """Device scratch bytes gdla_decode_fwd needs for these shapes."""
+    return int(load_library().gdla_decode_workspace_bytes(B, L_max, Hs, Hn, d_latent,
+                                                         int(window)))
+
+
+def gdla_decode_fwd(q_sig: torch.Tensor, q_noise: torch.Tensor, c_hat: torch.Tensor,
+                    cache_len: torch.Tensor, w_kvb: torch.Tensor, lam: torch.Tensor,
+                    gate: torch.Tensor, window: int = 0, scale: float = 0.0,
+                    out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                    d_status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """GDLA forward of the newest token of each sequence over its latent cache.
+
+    q_sig [B,Hs,d], q_noise [B,Hn,d], c_hat [B,L_max,d_latent] (RMSNorm'd
+    latents, gdla_latent_rmsnorm), cache_len int32 [B] on the device,
+    w_kvb [d_latent, Hn*2d], lam [B,Hs], gate [B,Hs*d].  Returns out [B, Hs*d].
+    The scratch comes from `workspace` (a uint8 CUDA tensor) or, when None,
+    is allocated here with torch (the library itself never allocates).
+    """
+    if q_sig.dim() != 3 or c_hat.dim() != 3:
+        raise ValueError("q_sig must be [B, Hs, d] and c_hat [B, L_max, d_latent]")
+    B, Hs, d = q_sig.shape
+    Hn = q_noise.shape[1] if q_noise.dim() == 3 else -1
+    L_max, dl = c_hat.shape[1], c_hat.shape[2]
+    hkv = w_kvb.shape[1] // (2 * d) if w_kvb.dim() == 2 else -1
+    if out is None:
+        out = torch.empty((B, Hs * d), dtype=torch.bfloat16, device=q_sig.device)
+    need = gdla_decode_workspace_bytes(B, L_max, Hs, Hn, dl, window) if B > 0 else 0
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q_sig.device)
+    if workspace.dtype != torch.uint8 or workspace.device != q_sig.device or \
+            not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous uint8 tensor on the inputs' device")
+    if cache_len.dtype != torch.int32 or tuple(cache_len.shape) != (B,) or \
+            not cache_len.is_contiguous():
+        raise ValueError("cache_len must be a contiguous int32 tensor of shape [B]")
+    ptrs = [
+        _check(q_sig, "q_sig"),
+        _check(q_noise, "q_noise", (B, Hn, d)),
+        _check(c_hat, "c_hat"),
+    ]
+    pw = _check(w_kvb, "w_kvb", (dl, hkv * 2 * d))
+    pl = _check(lam, "lam", (B, Hs))
+    pg = _check(gate, "gate", (B, Hs * d))
+    po = _check(out, "out", (B, Hs * d))
+    _same_device(q_sig.device, [("q_noise", q_noise), ("c_hat", c_hat), ("cache_len", cache_len),
+                                 ("w_kvb", w_kvb), ("lam", lam), ("gate", gate), ("out", out)])
+    ps = _status_ptr(d_status, q_sig.device)
+    rc = load_library().gdla_decode_fwd(*ptrs, cache_len.data_ptr(), pw, pl, pg, po, B, L_max, Hs,
+                                        Hn, hkv, d, dl, int(window), float(scale),
+                                        workspace.data_ptr(), workspace.numel(), ps,
+                                        _stream_ptr(q_sig.device, stream))
+    if rc != GDLA_OK:
+        raise GDLAError(rc, "gdla_decode_fwd")
     if _sync_check_enabled():
         check_status(q_sig.device, d_status)
     return out

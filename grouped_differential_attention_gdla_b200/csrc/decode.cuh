@@ -1,0 +1,550 @@
+// decode.cuh - GDLA decode over the KV latent cache, sm_100a.
+//
+// Operation ("Motif 3: Technical Report", paper.rainbus.top, step 2 "GDLA
+// forward" and the "technical novelty" paragraph: the two query paths share
+// one up-projected KV, so the inference cache holds only the 512-d KV latent
+// per token, the size of MLA's).  Sequence b has cache_len[b] cached tokens
+// whose RMSNorm'd latents c_hat are in the cache; its newest token is the
+// query.  Per head h of KV group k, with W_K = W^KV_b[:, k*2d : k*2d+d] and
+// W_V = W^KV_b[:, k*2d+d : (k+1)*2d]:
+//   s_j = q_h . (c_hat_j W_K) = (W_K q_h) . c_hat_j      absorbed query q~_h
+//   H_h = sum_j p_j (c_hat_j W_V) = (sum_j p_j c_hat_j) W_V
+// so attention runs in the latent space and reads 1 KB per cached token for
+// all 80 heads at once.  Three kernels:
+//   absorb   q~ = (scale log2 e) W_K q for every head, bf16, into workspace;
+//   attn     split-KV attention over the cache (tcgen05): per chunk of 128
+//            cached tokens, S^T = c_hat q~^T (M = 128 tokens, N = heads,
+//            K = latent), a per-head online softmax across tokens, and
+//            z^T += c_hat^T P (M = latent, N = heads, K = tokens); each CTA
+//            leaves (max, sum, z) of its chunks in workspace;
+//   combine  merges the splits per head, H = z W_V, then
+//            out = G (.) (H_S - lambda Repeat_g(H_N)).
+#pragma once
+
+#include "sm100.cuh"
+
+namespace gdla {
+
+constexpr int kDecTok = 128;    // cached tokens per chunk (MMA M of S^T)
+constexpr int kDecUnit = 128;   // latent columns per ring unit (MMA M of z^T)
+constexpr int kDecRing = 3;     // ring depth (units of [128 tokens][128 latent])
+constexpr int kDecThreads = 192;  // warps 0-3 softmax / partials, 4 TMA, 5 MMA
+constexpr int kDecMaxLatent = 512;
+constexpr int kDecMaxGroup = 8;   // signal heads per KV group in the decode kernels
+constexpr float kDecRescale = 8.0f;  // log2 units: a head's reference moves only past 2^8
+
+struct DecodeParams {
+  const __nv_bfloat16 *q_sig;    // [B, Hs, d]
+  const __nv_bfloat16 *q_noise;  // [B, Hn, d]
+  const __nv_bfloat16 *w_kvb;    // [dl, Hn * 2d]
+  const __nv_bfloat16 *lam;      // [B, Hs]
+  const __nv_bfloat16 *gate;     // [B, Hs * d]
+  __nv_bfloat16 *out;            // [B, Hs * d]
+  const int32_t *cache_len;      // [B], device
+  __nv_bfloat16 *qt;             // workspace: absorbed queries [B, Np, dl]
+  float *part;                   // workspace: per (b, split): m[Np], l[Np], z[Np][dl]
+  int *status;
+  int B, Hs, Hn, d, dl, Np, n_split, cps;
+  int64_t L_max, window;
+  float qscale;  // softmax scale * log2(e)
+};
+
+// The cached tokens sequence b's query keeps, and the chunks split s covers.
+struct DecodeRange {
+  int64_t len, t_lo;     // keys [t_lo, len)
+  int64_t c_begin, c_end;  // chunks [c_begin, c_end) of this split
+  bool bad_len;
+};
+
+__device__ __forceinline__ DecodeRange decode_range(const DecodeParams &p, int b, int s) {
+  DecodeRange r;
+  int64_t L = p.cache_len[b];
+  r.bad_len = L < 1 || L > p.L_max;
+  if (r.bad_len) L = L < 1 ? 1 : p.L_max;
+  r.len = L;
+  r.t_lo = (p.window > 0 && L > p.window) ? L - p.window : 0;
+  const int64_t c_first = r.t_lo / kDecTok, c_last = (L - 1) / kDecTok;
+  r.c_begin = c_first + static_cast<int64_t>(s) * p.cps;
+  const int64_t e = r.c_begin + p.cps;
+  r.c_end = e < c_last + 1 ? e : c_last + 1;
+  if (r.c_end < r.c_begin) r.c_end = r.c_begin;
+  return r;
+}
+
+__device__ __forceinline__ float *decode_part(const DecodeParams &p, int b, int s) {
+  return p.part + (static_cast<size_t>(b) * p.n_split + s) * p.Np * (p.dl + 2);
+}
+
+// ---------------------------------------------------------------- absorb
+// One CTA per (KV group k, sequence b): q~ rows of the group's heads (signal
+// heads h -> row h, noise head k -> row Hs + k), q~[x] = qscale * sum_c
+// W^KV_b[x, k*2d + c] q[c].  Rows Hs + Hn .. Np - 1 are zero padding.
+__global__ void __launch_bounds__(256) gdla_decode_absorb_kernel(const DecodeParams p) {
+  const int k = blockIdx.x, b = blockIdx.y;
+  const int g = p.Hs / p.Hn, nh = g + 1, d = p.d, dl = p.dl;
+  __shared__ float qs[(kDecMaxGroup + 1) * 128];
+  for (int i = threadIdx.x; i < nh * d; i += blockDim.x) {
+    const int j = i / d, c = i % d;
+    const __nv_bfloat16 *src =
+        j < g ? p.q_sig + (static_cast<int64_t>(b) * p.Hs + g * k + j) * d
+              : p.q_noise + (static_cast<int64_t>(b) * p.Hn + k) * d;
+    qs[i] = __bfloat162float(src[c]);
+  }
+  __syncthreads();
+  const int64_t ldw = static_cast<int64_t>(p.Hn) * 2 * d;
+  __nv_bfloat16 *qt = p.qt + static_cast<int64_t>(b) * p.Np * dl;
+  for (int x = threadIdx.x; x < dl; x += blockDim.x) {
+    const __nv_bfloat16 *wr = p.w_kvb + x * ldw + static_cast<int64_t>(k) * 2 * d;
+    for (int j = 0; j < nh; ++j) {
+      float acc = 0.f;
+      for (int c = 0; c < d; ++c) acc = fmaf(__bfloat162float(wr[c]), qs[j * d + c], acc);
+      const int row = j < g ? g * k + j : p.Hs + k;
+      qt[static_cast<int64_t>(row) * dl + x] = __float2bfloat16(acc * p.qscale);
+    }
+    if (k == 0)
+      for (int row = p.Hs + p.Hn; row < p.Np; ++row)
+        qt[static_cast<int64_t>(row) * dl + x] = __float2bfloat16(0.f);
+  }
+}
+
+// ---------------------------------------------------------------- attention
+template <int NP>
+struct DecSmem {
+  static constexpr uint32_t kUnitBytes = kDecTok * kDecUnit * 2;  // 32 KB
+  static constexpr uint32_t kQtOff = 0;  // q~: [dl/64 blocks][NP rows][128 B], K-major
+  static constexpr uint32_t kQtBytes = NP * kDecMaxLatent * 2;
+  static constexpr uint32_t kRingOff = kQtOff + kQtBytes;
+  static constexpr uint32_t kPOff = kRingOff + kDecRing * kUnitBytes;  // P: [2][NP][128 B]
+  static constexpr uint32_t kPBytes = 2 * NP * 128;
+  static constexpr uint32_t kRedOff = kPOff + kPBytes;     // int red[2][4][NP]; float lred[4][NP]
+  static constexpr uint32_t kRedBytes = 2 * 4 * NP * 4 + 4 * NP * 4;
+  static constexpr uint32_t kRefOff = kRedOff + kRedBytes;  // int ref[2][4][NP] (per warp, per chunk parity)
+  static constexpr uint32_t kBarOff = kRefOff + 2 * 4 * NP * 4;
+  static constexpr int kZStride = (NP + 31) / 32 * 32;        // TMEM columns per z^T block
+  static constexpr uint32_t kNumBars = 2 * kDecRing + 6;
+  static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr uint32_t kBytes = kMiscOff + 16;
+  static_assert(kQtBytes % 1024 == 0 && kRingOff % 1024 == 0 && kPOff % 1024 == 0,
+                "swizzled operands need 1024-byte alignment");
+  static_assert(kBytes <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
+  static_assert(NP % 16 == 0 && NP <= 80, "head rows: a multiple of 16, at most 80");
+};
+
+// One arrival per warp after the lanes' own writes.
+__device__ __forceinline__ void dec_warp_arrive(uint32_t bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31u) == 0) mbar_arrive(bar);
+}
+
+// One CTA per (split s, sequence b); NP = head rows (Hs + Hn padded to 16).
+// Warps 0-3: softmax (thread t = token t of the chunk = TMEM lane t) and the
+// partial results; warp 4: TMA; warp 5: TMEM allocation and MMA issue.
+// TMEM: S^T [0, NP), z^T block u (latent rows 128u..128u+127) at
+// [Z (1 + u), Z (1 + u) + NP) with Z = NP rounded up to 32 columns.
+template <int NP>
+__global__ void __launch_bounds__(kDecThreads, 1)
+    gdla_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_qt,
+                            const __grid_constant__ CUtensorMap tm_c, const DecodeParams p) {
+  using L = DecSmem<NP>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int s = blockIdx.x, b = blockIdx.y;
+  if ((smem_u32(smem) & 1023u) != 0) {
+    if (threadIdx.x == 0 && p.status) atomicExch(p.status, -4 /* GDLA_ERR_CUDA */);
+    return;
+  }
+  const DecodeRange rg = decode_range(p, b, s);
+  if (rg.bad_len && s == 0 && threadIdx.x == 0 && p.status)
+    atomicExch(p.status, -1 /* GDLA_ERR_INVALID_ARG: cache_len out of 1..L_max */);
+  const int n_chunks = static_cast<int>(rg.c_end - rg.c_begin);
+  float *part = decode_part(p, b, s);
+  if (n_chunks == 0) {  // nothing for this split: a partial that weighs nothing
+    for (int h = threadIdx.x; h < NP; h += blockDim.x) {
+      part[h] = -INFINITY;
+      part[NP + h] = 0.f;
+    }
+    return;
+  }
+  const int U = p.dl / kDecUnit;  // ring units per chunk
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + L::kBarOff;
+  auto ring_full = [&](int i) { return bar0 + 8u * i; };
+  auto ring_empty = [&](int i) { return bar0 + 8u * (kDecRing + i); };
+  const uint32_t qt_full = bar0 + 8u * (2 * kDecRing);
+  const uint32_t s_full = bar0 + 8u * (2 * kDecRing + 1);   // S^T of a chunk written
+  const uint32_t p_full = bar0 + 8u * (2 * kDecRing + 2);   // P written, z^T rescaled
+  const uint32_t z_done = bar0 + 8u * (2 * kDecRing + 3);   // z^T MMAs of a chunk done
+  auto red_full = [&](int i) { return bar0 + 8u * (2 * kDecRing + 4 + i); };  // maxima exchanged
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
+  int *red = reinterpret_cast<int *>(smem + L::kRedOff);                  // [2][4][NP]
+  float *lred = reinterpret_cast<float *>(smem + L::kRedOff + 2 * 4 * NP * 4);  // [4][NP]
+  int *refw = reinterpret_cast<int *>(smem + L::kRefOff);                 // [2][4][NP]
+  const int warp = threadIdx.x >> 5;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kDecRing; ++i) {
+      mbar_init(ring_full(i), 1);
+      mbar_init(ring_empty(i), 1);
+    }
+    mbar_init(qt_full, 1);
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 4);
+    mbar_init(z_done, 1);
+    mbar_init(red_full(0), 4);
+    mbar_init(red_full(1), 4);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t t_s = tmem;
+  auto t_z = [&](int u) { return tmem + static_cast<uint32_t>(L::kZStride * (1 + u)); };
+  const uint32_t sP = sbase + L::kPOff;
+
+  if (warp == 4) {
+    // =============================== TMA: q~ once, then per chunk the units
+    // of pass 1 (scores) and of pass 2 (z^T; the same rows again, from L2)
+    const bool leader = elect_one();
+    if (leader) {
+      tma_prefetch_desc(&tm_qt);
+      tma_prefetch_desc(&tm_c);
+      mbar_arrive_expect_tx(qt_full, static_cast<uint32_t>(NP * p.dl * 2));
+      for (int kb = 0; kb < p.dl / 64; ++kb)
+        tma_load_2d(sbase + L::kQtOff + kb * (NP * 128), &tm_qt, qt_full, kb * 64, b * NP);
+    }
+    uint32_t c = 0;
+    bool ok = true;
+    for (int ch = 0; ch < n_chunks && ok; ++ch) {
+      const int32_t tok0 = static_cast<int32_t>((rg.c_begin + ch) * kDecTok);
+      for (int pass = 0; pass < 2 && ok; ++pass) {
+        for (int u = 0; u < U; ++u) {
+          const int slot = static_cast<int>(c % kDecRing);
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait(ring_empty(slot), ((c / kDecRing) & 1u) ^ 1u, abort_flag));
+          if (!ok) break;
+          if (leader) {
+            const uint32_t dst = sbase + L::kRingOff + slot * L::kUnitBytes;
+            mbar_arrive_expect_tx(ring_full(slot), L::kUnitBytes);
+            tma_load_3d(dst, &tm_c, ring_full(slot), u * kDecUnit, tok0, b);
+            tma_load_3d(dst + kDecTok * 128, &tm_c, ring_full(slot), u * kDecUnit + 64, tok0, b);
+          }
+          ++c;
+        }
+      }
+    }
+    if (!ok && leader) {
+      for (int i = 0; i < kDecRing; ++i) {
+        const uint32_t issued = c > static_cast<uint32_t>(i) ? (c - 1 - i) / kDecRing + 1 : 0;
+        if (issued) mbar_wait_for(ring_full(i), (issued - 1) & 1u, 100000000ull);
+      }
+      mbar_wait_for(qt_full, 0, 100000000ull);
+    }
+  } else if (warp == 5) {
+    // =============================== MMA issue (one elected lane)
+    const bool leader = elect_one();
+    const uint32_t idesc_s = idesc_bf16_f32(kDecTok, NP, false, false);
+    const uint32_t idesc_z = idesc_bf16_f32(kDecUnit, NP, true, false);
+    bool ok = __all_sync(0xffffffffu, mbar_wait(qt_full, 0, abort_flag));
+    uint32_t c = 0, commits = 0;
+    for (int ch = 0; ch < n_chunks && ok; ++ch) {
+      // pass 1: S^T = c_hat q~^T over the latent, one unit (two K-blocks) at a time
+      for (int u = 0; u < U && ok; ++u) {
+        const int slot = static_cast<int>(c % kDecRing);
+        ok = __all_sync(0xffffffffu, mbar_wait(ring_full(slot), (c / kDecRing) & 1u, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        if (leader) {
+          const uint32_t a0 = sbase + L::kRingOff + slot * L::kUnitBytes;
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const uint64_t ad = sdesc_sw128(a0 + half * (kDecTok * 128), 16, 1024);
+            const uint64_t bd =
+                sdesc_sw128(sbase + L::kQtOff + (2 * u + half) * (NP * 128), 16, 1024);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              umma_ss(t_s, ad + ((k * 32) >> 4), bd + ((k * 32) >> 4), idesc_s,
+                      (u > 0 || half > 0 || k > 0) ? 1u : 0u);
+          }
+          umma_commit(ring_empty(slot));
+        }
+        ++c;
+      }
+      if (!ok) break;
+      if (leader) umma_commit(s_full);
+      ok = __all_sync(0xffffffffu, mbar_wait(p_full, ch & 1u, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      // pass 2: z^T[u] += c_hat_u^T P (A: the unit, MN-major over the latent;
+      // B: P, K-major over the tokens)
+      for (int u = 0; u < U && ok; ++u) {
+        const int slot = static_cast<int>(c % kDecRing);
+        ok = __all_sync(0xffffffffu, mbar_wait(ring_full(slot), (c / kDecRing) & 1u, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        if (leader) {
+          const uint64_t ad =
+              sdesc_sw128(sbase + L::kRingOff + slot * L::kUnitBytes, kDecTok * 128, 1024);
+#pragma unroll
+          for (int k = 0; k < kDecTok / 16; ++k) {
+            const uint64_t bd = sdesc_sw128(sP + (k >> 2) * (NP * 128), 16, 1024);
+            umma_ss(t_z(u), ad + ((k * 16 * 128) >> 4), bd + (((k & 3) * 32) >> 4), idesc_z,
+                    (ch > 0 || k > 0) ? 1u : 0u);
+          }
+          umma_commit(ring_empty(slot));
+        }
+        ++c;
+      }
+      if (!ok) break;
+      if (leader) umma_commit(z_done);
+      ++commits;
+    }
+    if (leader && commits) mbar_wait_for(z_done, (commits - 1) & 1u, 100000000ull);
+  } else {
+    // =============================== softmax over the chunk's tokens, per head
+    const int w = warp;
+    const int lane = threadIdx.x & 31;
+    const int t = threadIdx.x;  // token row of the chunk = TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>(w * 32) << 16;
+    float lsum[NP];
+#pragma unroll
+    for (int h = 0; h < NP; ++h) lsum[h] = 0.f;
+    for (int i = lane; i < NP; i += 32) refw[w * NP + i] = refw[(4 + w) * NP + i] = INT_MIN;
+    __syncwarp();
+    bool ok = true;
+    for (int ch = 0; ch < n_chunks && ok; ++ch) {
+      ok = __all_sync(0xffffffffu, mbar_wait(s_full, ch & 1u, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      float sv[NP];
+#pragma unroll
+      for (int i = 0; i < NP / 16; ++i) {
+        uint32_t r16[16];
+        tmem_ld16_sync(t_s + lane_off + 16 * i, r16);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) sv[16 * i + e] = __uint_as_float(r16[e]);
+      }
+      const int64_t tok = (rg.c_begin + ch) * kDecTok + t;
+      const bool valid = tok >= rg.t_lo && tok < rg.len;
+      // per head: the chunk's largest score rounded up to an integer, over the
+      // warp (one redux each), then over the four warps through shared memory
+      int *rb = red + (ch & 1) * 4 * NP;
+#pragma unroll
+      for (int h = 0; h < NP; ++h) {
+        const int mi = valid ? static_cast<int>(ceilf(sv[h])) : INT_MIN;
+        const int wm = __reduce_max_sync(0xffffffffu, mi);
+        if (lane == 0) rb[w * NP + h] = wm;
+      }
+      dec_warp_arrive(red_full(ch & 1));
+      ok = __all_sync(0xffffffffu, mbar_wait(red_full(ch & 1), (ch >> 1) & 1u, abort_flag));
+      if (!ok) break;
+      // the previous chunk's z^T MMAs must be done before P is overwritten or
+      // z^T rescaled
+      if (ch > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(z_done, (ch - 1) & 1u, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+      }
+      // new integral reference per head: the lanes compute it for heads
+      // lane, lane + 32, ... into this warp's copy for the chunk (every warp
+      // computes the same values); a head's reference moves only when its
+      // maximum passes it by more than 2^8
+      const int *ref_old = refw + ((ch & 1) * 4 + w) * NP;
+      int *ref_new = refw + (((ch & 1) ^ 1) * 4 + w) * NP;
+      bool moved = false;
+      for (int h = lane; h < NP; h += 32) {
+        const int cm = max(max(rb[h], rb[NP + h]), max(rb[2 * NP + h], rb[3 * NP + h]));
+        const int old = ref_old[h];
+        const bool move =
+            old == INT_MIN || static_cast<float>(cm) > static_cast<float>(old) + kDecRescale;
+        ref_new[h] = move ? cm : old;
+        moved = moved || (move && old != INT_MIN);
+      }
+      __syncwarp();
+      if (__any_sync(0xffffffffu, moved) && ch > 0) {
+        // z^T and the row sums hold earlier chunks at the old references
+#pragma unroll
+        for (int h = 0; h < NP; ++h) lsum[h] *= exp2_int(static_cast<float>(ref_old[h] - ref_new[h]));
+        for (int u = 0; u < U; ++u) {
+#pragma unroll
+          for (int i = 0; i < NP / 16; ++i) {
+            uint32_t r16[16];
+            tmem_ld16_sync(t_z(u) + lane_off + 16 * i, r16);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int h = 16 * i + e;
+              const float a = exp2_int(static_cast<float>(ref_old[h] - ref_new[h]));
+              r16[e] = __float_as_uint(__uint_as_float(r16[e]) * a);
+            }
+            tmem_st16(t_z(u) + lane_off + 16 * i, r16);
+          }
+        }
+        tmem_wait_st();
+      }
+      // P[h][t] = 2^(s - ref) (bf16), K-major over the tokens: block t / 64,
+      // row h, 16-byte unit ((t % 64) / 8) ^ (h % 8)
+      const uint32_t pb = sP + static_cast<uint32_t>(t >> 6) * (NP * 128) +
+                          static_cast<uint32_t>((t & 7) * 2);
+      const uint32_t unit = static_cast<uint32_t>((t & 63) >> 3);
+#pragma unroll
+      for (int h = 0; h < NP; ++h) {
+        const float pv = valid ? ex2_approx(sv[h] - static_cast<float>(ref_new[h])) : 0.f;
+        lsum[h] += pv;
+        const uint32_t addr = pb + static_cast<uint32_t>(h) * 128u +
+                              ((unit ^ static_cast<uint32_t>(h & 7)) << 4);
+        const unsigned short bits = __bfloat16_as_ushort(__float2bfloat16(pv));
+        asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(bits) : "memory");
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      dec_warp_arrive(p_full);
+    }
+    // ---- partial results of this split: reference, row sums, z^T
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(z_done, (n_chunks - 1) & 1u, abort_flag));
+    if (ok) {
+      tc_fence_after();
+#pragma unroll
+      for (int h = 0; h < NP; ++h) {
+        float v = lsum[h];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0) lred[w * NP + h] = v;
+      }
+      dec_warp_arrive(red_full(n_chunks & 1));
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(red_full(n_chunks & 1), (n_chunks >> 1) & 1u, abort_flag));
+    }
+    if (ok) {
+      const int *ref_last = refw + ((n_chunks & 1) * 4 + w) * NP;
+      for (int h = t; h < NP; h += kDecTok) {
+        part[h] = static_cast<float>(ref_last[h]);  // this warp's copy; all copies agree
+        part[NP + h] = lred[h] + lred[NP + h] + lred[2 * NP + h] + lred[3 * NP + h];
+      }
+      float *zp = part + 2 * NP;
+      for (int u = 0; u < U; ++u) {
+#pragma unroll
+        for (int i = 0; i < NP / 16; ++i) {
+          uint32_t r16[16];
+          tmem_ld16_sync(t_z(u) + lane_off + 16 * i, r16);
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            zp[static_cast<size_t>(16 * i + e) * p.dl + u * kDecUnit + t] = __uint_as_float(r16[e]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0 && p.status) atomicExch(p.status, -5 /* GDLA_ERR_TIMEOUT */);
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- combine
+// One CTA per (KV group k, sequence b): merge the splits of the group's heads
+// (weights 2^(m_s - M)), z = sum / l, H = z W_V, then
+// out = G (.) (H_S - lambda H_N) for the group's signal heads.
+__global__ void __launch_bounds__(128) gdla_decode_combine_kernel(const DecodeParams p) {
+  const int k = blockIdx.x, b = blockIdx.y;
+  const int g = p.Hs / p.Hn, nh = g + 1, d = p.d, dl = p.dl;
+  __shared__ float zs[(kDecMaxGroup + 1) * kDecMaxLatent];
+  __shared__ float hsm[(kDecMaxGroup + 1) * 128];
+  for (int j = 0; j < nh; ++j) {
+    const int row = j < g ? g * k + j : p.Hs + k;
+    float M = -INFINITY;
+    for (int sp = 0; sp < p.n_split; ++sp) M = fmaxf(M, decode_part(p, b, sp)[row]);
+    float l = 0.f;
+    for (int sp = 0; sp < p.n_split; ++sp) {
+      const float *pp = decode_part(p, b, sp);
+      if (pp[row] != -INFINITY) l += exp2f(pp[row] - M) * pp[p.Np + row];
+    }
+    const float inv_l = l > 0.f ? 1.f / l : 0.f;
+    for (int x = threadIdx.x; x < dl; x += blockDim.x) {
+      float acc = 0.f;
+      for (int sp = 0; sp < p.n_split; ++sp) {
+        const float *pp = decode_part(p, b, sp);
+        if (pp[row] != -INFINITY)
+          acc = fmaf(exp2f(pp[row] - M), pp[2 * p.Np + static_cast<size_t>(row) * dl + x], acc);
+      }
+      zs[j * dl + x] = acc * inv_l;
+    }
+  }
+  __syncthreads();
+  const int64_t ldw = static_cast<int64_t>(p.Hn) * 2 * d;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+    float acc[kDecMaxGroup + 1];
+#pragma unroll
+    for (int j = 0; j < kDecMaxGroup + 1; ++j) acc[j] = 0.f;
+    const __nv_bfloat16 *wv = p.w_kvb + static_cast<int64_t>(k) * 2 * d + d + c;
+    for (int x = 0; x < dl; ++x) {
+      const float wx = __bfloat162float(wv[x * ldw]);
+#pragma unroll
+      for (int j = 0; j < kDecMaxGroup + 1; ++j)
+        if (j < nh) acc[j] = fmaf(zs[j * dl + x], wx, acc[j]);
+    }
+#pragma unroll
+    for (int j = 0; j < kDecMaxGroup + 1; ++j)
+      if (j < nh) hsm[j * d + c] = acc[j];
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < g * d; i += blockDim.x) {
+    const int j = i / d, c = i % d;
+    const int h = g * k + j;
+    const float lamv = __bfloat162float(p.lam[static_cast<int64_t>(b) * p.Hs + h]);
+    const int64_t o = (static_cast<int64_t>(b) * p.Hs + h) * d + c;
+    const float dv = hsm[j * d + c] - lamv * hsm[g * d + c];
+    p.out[o] = __float2bfloat16(__bfloat162float(p.gate[o]) * dv);
+  }
+}
+
+// ---------------------------------------------------------------- cache write
+// RMSNorm of the KV latent of tokens entering the cache: one warp per token,
+// fp32 sum of squares, c / sqrt(mean c^2 + eps) * w rounded to bf16.
+__global__ void __launch_bounds__(256) gdla_latent_rmsnorm_kernel(
+    const __nv_bfloat16 *c, const __nv_bfloat16 *w, float eps, __nv_bfloat16 *out,
+    int64_t n_tokens, int dl) {
+  const int64_t tkn = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (tkn >= n_tokens) return;
+  const __nv_bfloat16 *row = c + tkn * dl;
+  float ss = 0.f;
+  for (int x = lane * 8; x < dl; x += 32 * 8) {
+    const uint4 v = *reinterpret_cast<const uint4 *>(row + x);
+    const uint32_t q[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float a = bf16lo_to_f32(q[e]), bb = bf16hi_to_f32(q[e]);
+      ss = fmaf(a, a, ss);
+      ss = fmaf(bb, bb, ss);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float rinv = rsqrtf(ss / static_cast<float>(dl) + eps);
+  __nv_bfloat16 *orow = out + tkn * dl;
+  for (int x = lane * 8; x < dl; x += 32 * 8) {
+    const uint4 v = *reinterpret_cast<const uint4 *>(row + x);
+    const uint32_t q[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o4[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float w0 = 1.f, w1 = 1.f;
+      if (w) {
+        w0 = __bfloat162float(w[x + 2 * e]);
+        w1 = __bfloat162float(w[x + 2 * e + 1]);
+      }
+      o4[e] = pack_bf16x2(bf16lo_to_f32(q[e]) * rinv * w0, bf16hi_to_f32(q[e]) * rinv * w1);
+    }
+    *reinterpret_cast<uint4 *>(orow + x) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+  }
+}
+
+}  // namespace gdla

@@ -15,6 +15,7 @@
 #include "gdla.h"
 #include "attn_fwd.cuh"
 #include "attn_win.cuh"
+#include "decode.cuh"
 #include "kv_expand.cuh"
 #include "selftest.cuh"
 
@@ -203,6 +204,61 @@ int launch_expand(const void *c_kv, const void *w_kvb, const gdla::ExpandParams 
   return cudaGetLastError() == cudaSuccess ? GDLA_OK : GDLA_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------- decode
+// Work split of the decode: each CTA of the attention kernel takes `cps`
+// chunks of 128 cached tokens of one sequence, enough of them that the grid
+// is about two CTAs per SM of a B200 and that each CTA's partial result
+// (Np * (d_latent + 2) floats) is small next to the cache it reads.  The
+// split depends on the shapes only, so the workspace size does too.
+constexpr int64_t kDecodeTargetCtas = 296;
+constexpr int64_t kDecodeMinChunks = 4;
+
+struct DecodePlan {
+  int Np, cps, n_split;
+  size_t qt_bytes, part_bytes;
+};
+
+bool decode_plan(int B, int64_t L_max, int Hs, int Hn, int d_latent, int64_t window,
+                 DecodePlan *pl) {
+  if (B <= 0 || L_max <= 0 || Hs <= 0 || Hn <= 0 || d_latent <= 0 || window < 0) return false;
+  const int64_t np = (static_cast<int64_t>(Hs) + Hn + 15) / 16 * 16;
+  int64_t chunks = (L_max + gdla::kDecTok - 1) / gdla::kDecTok;
+  if (window > 0) {
+    // the most 128-token chunks W consecutive keys can touch
+    const int64_t w = (window + gdla::kDecTok - 2) / gdla::kDecTok + 1;
+    if (w < chunks) chunks = w;
+  }
+  int64_t cps = (static_cast<int64_t>(B) * chunks + kDecodeTargetCtas - 1) / kDecodeTargetCtas;
+  if (cps < kDecodeMinChunks) cps = kDecodeMinChunks;
+  const int64_t n_split = (chunks + cps - 1) / cps;
+  if (np > 256 || n_split > 0x7fffffffll || cps > 0x7fffffffll) return false;
+  pl->Np = static_cast<int>(np);
+  pl->cps = static_cast<int>(cps);
+  pl->n_split = static_cast<int>(n_split);
+  pl->qt_bytes = (static_cast<size_t>(B) * np * d_latent * 2 + 255) / 256 * 256;
+  pl->part_bytes = static_cast<size_t>(B) * n_split * np * (d_latent + 2) * 4;
+  return true;
+}
+
+template <int NP>
+int launch_decode_attn(const gdla::DecodeParams &prm, const void *c_hat, cudaStream_t stream) {
+  using L = gdla::DecSmem<NP>;
+  CUtensorMap tm_qt, tm_c;
+  const uint64_t dq[2] = {static_cast<uint64_t>(prm.dl), static_cast<uint64_t>(prm.B) * NP};
+  const uint32_t qbox[2] = {64, NP};
+  const uint64_t dc[3] = {static_cast<uint64_t>(prm.dl), static_cast<uint64_t>(prm.L_max),
+                          static_cast<uint64_t>(prm.B)};
+  const uint32_t cbox[3] = {64, gdla::kDecTok, 1};
+  if (!make_map(&tm_qt, prm.qt, 2, dq, qbox) || !make_map(&tm_c, c_hat, 3, dc, cbox))
+    return GDLA_ERR_CUDA;
+  constexpr auto kern = gdla::gdla_decode_attn_kernel<NP>;
+  const int rc = prepare_kernel<kern>(L::kBytes, 0);
+  if (rc != GDLA_OK) return rc;
+  kern<<<dim3(static_cast<unsigned>(prm.n_split), static_cast<unsigned>(prm.B)), gdla::kDecThreads,
+         L::kBytes, stream>>>(tm_qt, tm_c, prm);
+  return cudaGetLastError() == cudaSuccess ? GDLA_OK : GDLA_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -328,6 +384,93 @@ int gdla_attn_fwd_sp(const void *q_sig, const void *q_noise, const void *k, cons
   if (window <= 0 || window > gdla::kBN) return GDLA_ERR_INVALID_ARG;
   return attn_fwd_impl(q_sig, q_noise, k, v, lambda, gate, out, B, T, kv_prefix, Hs, Hn, Hkv, d,
                        window, 1, scale, d_status, stream);
+}
+
+size_t gdla_decode_workspace_bytes(int B, int64_t L_max, int Hs, int Hn, int d_latent,
+                                   int64_t window) {
+  DecodePlan pl;
+  if (!decode_plan(B, L_max, Hs, Hn, d_latent, window, &pl)) return 0;
+  return pl.qt_bytes + pl.part_bytes;
+}
+
+int gdla_decode_fwd(const void *q_sig, const void *q_noise, const void *c_hat,
+                    const int32_t *cache_len, const void *w_kvb, const void *lambda,
+                    const void *gate, void *out, int B, int64_t L_max, int Hs, int Hn, int Hkv,
+                    int d, int d_latent, int64_t window, float scale, void *workspace,
+                    size_t workspace_bytes, int *d_status, void *stream) {
+  if (B < 0 || L_max <= 0 || Hs <= 0 || Hn <= 0 || Hkv <= 0 || d <= 0 || d_latent <= 0 ||
+      window < 0)
+    return GDLA_ERR_INVALID_ARG;
+  if (std::isnan(scale) || std::isinf(scale)) return GDLA_ERR_INVALID_ARG;
+  if (B == 0) return GDLA_OK;
+  if (!q_sig || !q_noise || !c_hat || !cache_len || !w_kvb || !lambda || !gate || !out ||
+      !workspace)
+    return GDLA_ERR_INVALID_ARG;
+  if (Hn != Hkv || Hs % Hn != 0 || Hs / Hn > gdla::kDecMaxGroup) return GDLA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return GDLA_ERR_UNSUPPORTED;
+  if (d_latent % gdla::kDecUnit != 0 || d_latent > gdla::kDecMaxLatent) return GDLA_ERR_UNSUPPORTED;
+  if (B > 65535 || L_max > 0x7fffffffll - gdla::kDecTok) return GDLA_ERR_UNSUPPORTED;
+  DecodePlan pl;
+  if (!decode_plan(B, L_max, Hs, Hn, d_latent, window, &pl)) return GDLA_ERR_UNSUPPORTED;
+  if (pl.Np != 16 && pl.Np != 80) return GDLA_ERR_UNSUPPORTED;
+  if (workspace_bytes < pl.qt_bytes + pl.part_bytes) return GDLA_ERR_INVALID_ARG;
+  if (!aligned16(q_sig) || !aligned16(q_noise) || !aligned16(c_hat) || !aligned16(w_kvb) ||
+      !aligned16(lambda) || !aligned16(gate) || !aligned16(out) || !aligned16(workspace) ||
+      !aligned4(cache_len) || (d_status && !aligned4(d_status)))
+    return GDLA_ERR_ALIGNMENT;
+  gdla::DecodeParams prm;
+  prm.q_sig = static_cast<const __nv_bfloat16 *>(q_sig);
+  prm.q_noise = static_cast<const __nv_bfloat16 *>(q_noise);
+  prm.w_kvb = static_cast<const __nv_bfloat16 *>(w_kvb);
+  prm.lam = static_cast<const __nv_bfloat16 *>(lambda);
+  prm.gate = static_cast<const __nv_bfloat16 *>(gate);
+  prm.out = static_cast<__nv_bfloat16 *>(out);
+  prm.cache_len = cache_len;
+  prm.qt = static_cast<__nv_bfloat16 *>(workspace);
+  prm.part = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + pl.qt_bytes);
+  prm.status = d_status;
+  prm.B = B;
+  prm.Hs = Hs;
+  prm.Hn = Hn;
+  prm.d = d;
+  prm.dl = d_latent;
+  prm.Np = pl.Np;
+  prm.n_split = pl.n_split;
+  prm.cps = pl.cps;
+  prm.L_max = L_max;
+  prm.window = window;
+  const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(d));
+  prm.qscale = sc * 1.4426950408889634f;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  gdla::gdla_decode_absorb_kernel<<<dim3(static_cast<unsigned>(Hn), static_cast<unsigned>(B)),
+                                    256, 0, s>>>(prm);
+  if (cudaGetLastError() != cudaSuccess) return GDLA_ERR_CUDA;
+  const int rc = pl.Np == 80 ? launch_decode_attn<80>(prm, c_hat, s)
+                             : launch_decode_attn<16>(prm, c_hat, s);
+  if (rc != GDLA_OK) return rc;
+  gdla::gdla_decode_combine_kernel<<<dim3(static_cast<unsigned>(Hn), static_cast<unsigned>(B)),
+                                     128, 0, s>>>(prm);
+  return cudaGetLastError() == cudaSuccess ? GDLA_OK : GDLA_ERR_CUDA;
+}
+
+int gdla_latent_rmsnorm(const void *c_kv, const void *rms_w, float eps, void *out,
+                        int64_t n_tokens, int d_latent, int *d_status, void *stream) {
+  (void)d_status;
+  if (n_tokens < 0 || d_latent <= 0) return GDLA_ERR_INVALID_ARG;
+  if (!std::isfinite(eps) || eps < 0.f) return GDLA_ERR_INVALID_ARG;
+  if (n_tokens == 0) return GDLA_OK;
+  if (!c_kv || !out) return GDLA_ERR_INVALID_ARG;
+  if (d_latent % 8 != 0 || d_latent > 8192) return GDLA_ERR_UNSUPPORTED;
+  if (n_tokens > 0x7fffffffll * 8) return GDLA_ERR_UNSUPPORTED;
+  if (!aligned16(c_kv) || !aligned16(out) || (rms_w && !aligned16(rms_w)) ||
+      (d_status && !aligned4(d_status)))
+    return GDLA_ERR_ALIGNMENT;
+  const uint64_t blocks = (static_cast<uint64_t>(n_tokens) + 7) / 8;
+  gdla::gdla_latent_rmsnorm_kernel<<<static_cast<unsigned>(blocks), 256, 0,
+                                     static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16 *>(c_kv), static_cast<const __nv_bfloat16 *>(rms_w), eps,
+      static_cast<__nv_bfloat16 *>(out), n_tokens, d_latent);
+  return cudaGetLastError() == cudaSuccess ? GDLA_OK : GDLA_ERR_CUDA;
 }
 
 int gdla_selftest_wait_timeout(int *d_status, int64_t limit_ns, void *stream) {

@@ -6,7 +6,9 @@ It holds none of the method's arithmetic (the sigmoid below prepares the
 already-activated lambda and gate inputs, which arrive at the attention
 boundary as given values).
 
-Recipe (fixed order, one ``torch.Generator`` seeded once):
+Recipe (fixed order, one ``torch.Generator`` seeded once; decode workloads
+draw Q_sig, Q_noise [B, H, d], lambda, gate, the cache's raw latents
+c_KV [B, T, 512] and W^KV_b in that order):
   Q_sig, Q_noise, K, V  ~ N(0, 1) rounded to bfloat16   (K, V skipped for the
                                                            latent workload)
   lambda = bf16(sigmoid(N(0, 1)))  shape [B, T, Hs]
@@ -43,6 +45,7 @@ class Workload:
     latent: bool = False     # K, V come from RMSNorm + W^KV_b of c_KV
     d_latent: int = 512
     eps: float = 1e-6
+    decode: bool = False     # one query token per sequence over a T-token latent cache
 
     @property
     def g(self) -> int:
@@ -51,6 +54,8 @@ class Workload:
     def pairs_per_batch(self) -> int:
         """(query, key) pairs the mask keeps in one batch element."""
         T, W = self.T, self.window
+        if self.decode:  # the newest token over a full cache of T tokens
+            return min(T, W) if W > 0 else T
         if not self.causal:
             return T * T
         if W <= 0 or W >= T:
@@ -61,6 +66,13 @@ class Workload:
     def attn_flops(self) -> int:
         """4*d FLOPs per kept pair per query head (QK^T and PV), all heads."""
         return 4 * self.d * (self.Hs + self.Hn) * self.B * self.pairs_per_batch()
+
+    def decode_bytes(self) -> int:
+        """The kept cache rows read once, W^KV_b, the query-side inputs and
+        the output, bfloat16 everywhere."""
+        per_seq = self.pairs_per_batch() * self.d_latent + (self.Hs + self.Hn) * self.d + \
+            self.Hs + 2 * self.Hs * self.d
+        return 2 * (self.B * per_seq + self.d_latent * self.Hkv * 2 * self.d)
 
     def attn_bytes(self) -> int:
         """Inputs read once plus output written once, bfloat16 everywhere."""
@@ -84,6 +96,10 @@ WORKLOADS: Dict[str, Workload] = {
     "latent": Workload("latent", B=1, T=32768, latent=True),
     "long_full": Workload("long_full", B=1, T=131072),
     "long_window": Workload("long_window", B=1, T=262144, window=128),
+    # decode: 64 sequences, each with a 32768-token latent cache (the 32K stage
+    # of the long-context schedule), every key or the 128-token window
+    "decode": Workload("decode", B=64, T=32768, decode=True),
+    "decode_window": Workload("decode_window", B=64, T=32768, window=128, decode=True),
 }
 
 
@@ -113,6 +129,16 @@ def make_inputs(wl: Workload, seed: int = 0, device="cpu",
     gen = torch.Generator(device=device)
     gen.manual_seed(seed)
     out = {}
+    if wl.decode:
+        # one query token per sequence; the cache holds raw KV latents
+        out["q_sig"] = _normal_bf16((B, wl.Hs, wl.d), gen, device)
+        out["q_noise"] = _normal_bf16((B, wl.Hn, wl.d), gen, device)
+        out["lam"] = _sigmoid_bf16((B, wl.Hs), gen, device)
+        out["gate"] = _sigmoid_bf16((B, wl.Hs * wl.d), gen, device)
+        out["c_kv"] = _normal_bf16((B, T, wl.d_latent), gen, device)
+        out["w_kvb"] = _normal_bf16((wl.d_latent, wl.Hkv * 2 * wl.d), gen, device,
+                                    std=(1.0 / wl.d_latent) ** 0.5)
+        return out
     out["q_sig"] = _normal_bf16((B, T, wl.Hs, wl.d), gen, device)
     out["q_noise"] = _normal_bf16((B, T, wl.Hn, wl.d), gen, device)
     if not wl.latent:

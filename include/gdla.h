@@ -46,6 +46,7 @@
 #ifndef GDLA_H_
 #define GDLA_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -146,6 +147,73 @@ int gdla_attn_fwd_sp(const void *q_sig, const void *q_noise, const void *k,
                      void *out, int B, int64_t T, int64_t kv_prefix, int Hs,
                      int Hn, int Hkv, int d, int64_t window, float scale,
                      int *d_status, void *stream);
+
+/*
+ * gdla_latent_rmsnorm - RMSNorm of KV latents entering the decode cache
+ * ("Motif 3: Technical Report", paper.rainbus.top, step 2: the KV latent
+ * c_KV,t goes through RMSNorm before W^KV_b; the "technical novelty"
+ * paragraph: the inference cache is this latent, the size of MLA's).
+ *
+ *   c_hat[t, k] = c_kv[t, k] / sqrt(mean_k c_kv[t, k]^2 + eps) * rms_w[k]
+ *
+ * c_kv   [n_tokens, d_latent]   bf16, read
+ * rms_w  [d_latent] or NULL     bf16, read (NULL: weight of ones)
+ * out    [n_tokens, d_latent]   bf16, written (may be a slice of the cache)
+ * Supported: d_latent a multiple of 8, at most 8192.  n_tokens == 0 is a
+ * no-op.  d_status is accepted for symmetry (this kernel has no waits).
+ */
+int gdla_latent_rmsnorm(const void *c_kv, const void *rms_w, float eps,
+                        void *out, int64_t n_tokens, int d_latent,
+                        int *d_status, void *stream);
+
+/*
+ * gdla_decode_workspace_bytes - bytes of device scratch gdla_decode_fwd needs
+ * for these shapes (absorbed queries and per-split partial results); 0 for
+ * shapes gdla_decode_fwd cannot take.  Depends on the shapes only.
+ */
+size_t gdla_decode_workspace_bytes(int B, int64_t L_max, int Hs, int Hn,
+                                   int d_latent, int64_t window);
+
+/*
+ * gdla_decode_fwd - GDLA forward for the newest token of B sequences over
+ * their cache of RMSNorm'd KV latents (same page, step 2 and the "technical
+ * novelty" paragraph: both query paths share one up-projected KV, so the
+ * cache holds only the latent).  For sequence b with L = cache_len[b]
+ * cached tokens, the query token is token L - 1 and the result equals the
+ * row gdla_kv_expand + gdla_attn_fwd would compute for it:
+ *   K, V = c_hat[b, 0..L-1] W^KV_b,   keys j in (L-1-window, L-1] (0: all)
+ *   out[b] = G (.) (H_S - lambda Repeat_g(H_N))
+ * The kernels never expand K and V: W^KV_b's K columns are absorbed into the
+ * queries and its V columns applied after the attention, which runs in the
+ * d_latent-dimensional latent space and reads the cache once for all heads.
+ *
+ * q_sig      [B, Hs, d]                  bf16, read
+ * q_noise    [B, Hn, d]                  bf16, read
+ * c_hat      [B, L_max, d_latent]        bf16, read (gdla_latent_rmsnorm output)
+ * cache_len  [B] int32, device           1 .. L_max (a value out of range sets
+ *                                        d_status to GDLA_ERR_INVALID_ARG and
+ *                                        is clamped)
+ * w_kvb      [d_latent, Hkv * 2 * d]     bf16, read (per head [K_h | V_h])
+ * lambda     [B, Hs], gate [B, Hs * d]   bf16, read
+ * out        [B, Hs * d]                 bf16, written
+ * workspace  device scratch of at least gdla_decode_workspace_bytes(...)
+ *            bytes, 16-byte aligned, owned by the caller; its contents on
+ *            entry do not matter, and calls that overlap on the GPU must not
+ *            share it
+ * window     0 = every cached token; W > 0 = the last W
+ * scale      softmax scale on q.k; <= 0 selects 1/sqrt(d)
+ * Cache rows the query does not keep (past cache_len, before the window)
+ * are read and multiplied by zero weights: they must hold finite values.
+ * Supported: Hn == Hkv, Hs / Hn <= 8, Hs + Hn rounded up to 16 equal to 16
+ * or 80, d in {64, 128}, d_latent in {128, 256, 384, 512}, B <= 65535.
+ */
+int gdla_decode_fwd(const void *q_sig, const void *q_noise, const void *c_hat,
+                    const int32_t *cache_len, const void *w_kvb,
+                    const void *lambda, const void *gate, void *out, int B,
+                    int64_t L_max, int Hs, int Hn, int Hkv, int d,
+                    int d_latent, int64_t window, float scale,
+                    void *workspace, size_t workspace_bytes, int *d_status,
+                    void *stream);
 
 /*
  * gdla_selftest_wait_timeout - device-side check of the failure path.

@@ -34,7 +34,9 @@ def _declared_functions():
 def test_exports_every_declared_symbol(lib):
     declared = _declared_functions()
     assert set(declared) == {"gdla_version", "gdla_status_string", "gdla_kv_expand",
-                             "gdla_attn_fwd", "gdla_attn_fwd_sp", "gdla_selftest_wait_timeout"}
+                             "gdla_attn_fwd", "gdla_attn_fwd_sp", "gdla_latent_rmsnorm",
+                             "gdla_decode_workspace_bytes", "gdla_decode_fwd",
+                             "gdla_selftest_wait_timeout"}
     for name in declared:
         assert hasattr(lib, name), f"{name} missing from libgdla.so"
     assert set(declared) == set(_binding.EXPORTED)
@@ -133,3 +135,54 @@ def _sp(lib, q=A, qn=A, k=A, v=A, lam=A, gate=A, out=A, B=1, T=256, kv_prefix=12
 ])
 def test_sp_argument_errors(lib, kw, code):
     assert _sp(lib, **kw) == code
+
+
+WS = 1 << 30  # a workspace size larger than any case below needs
+
+
+def _dec(lib, q=A, qn=A, c=A, cl=A, w=A, lam=A, gate=A, out=A, B=2, L=300, Hs=8, Hn=2, Hkv=2,
+         d=64, dl=512, window=0, scale=0.0, ws=A, ws_bytes=WS, status=None):
+    return lib.gdla_decode_fwd(q, qn, c, cl, w, lam, gate, out, B, L, Hs, Hn, Hkv, d, dl, window,
+                               ctypes.c_float(scale), ws, ws_bytes, status, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), INVALID), (dict(c=None), INVALID), (dict(cl=None), INVALID),
+    (dict(w=None), INVALID), (dict(out=None), INVALID), (dict(ws=None), INVALID),
+    (dict(B=-1), INVALID), (dict(L=0), INVALID), (dict(Hs=0), INVALID), (dict(d=0), INVALID),
+    (dict(dl=0), INVALID), (dict(window=-1), INVALID), (dict(scale=float("nan")), INVALID),
+    (dict(ws_bytes=1000), INVALID),
+    (dict(Hn=2, Hkv=4), UNSUPPORTED), (dict(Hs=6, Hn=4, Hkv=4), UNSUPPORTED),
+    (dict(Hs=18, Hn=2, Hkv=2), UNSUPPORTED),   # 10 signal heads per group
+    (dict(Hs=32, Hn=8, Hkv=8), UNSUPPORTED),   # 40 head rows: neither 16 nor 80
+    (dict(d=96), UNSUPPORTED), (dict(dl=448), UNSUPPORTED), (dict(dl=640), UNSUPPORTED),
+    (dict(B=70000), UNSUPPORTED),
+    (dict(c=M), ALIGN), (dict(ws=M), ALIGN), (dict(out=M), ALIGN), (dict(cl=0x100002), ALIGN),
+    (dict(status=0x100002), ALIGN),
+    (dict(B=0), OK), (dict(B=0, q=None), OK),
+])
+def test_decode_argument_errors(lib, kw, code):
+    assert _dec(lib, **kw) == code
+
+
+def test_decode_workspace_size_follows_the_shapes(lib):
+    f = lib.gdla_decode_workspace_bytes
+    # 64 sequences x 32768 tokens, 64 + 16 heads: 56 chunks per split, 5 splits
+    assert f(64, 32768, 64, 16, 512, 0) == 64 * 80 * 512 * 2 + 64 * 5 * 80 * 514 * 4
+    # a 128-token window touches at most 2 chunks: one split per sequence
+    assert f(64, 32768, 64, 16, 512, 128) == 64 * 80 * 512 * 2 + 64 * 1 * 80 * 514 * 4
+    assert f(1, 100, 8, 2, 512, 0) == 16 * 512 * 2 + 1 * 1 * 16 * 514 * 4
+    assert f(0, 100, 8, 2, 512, 0) == 0 and f(1, 0, 8, 2, 512, 0) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(c=None), INVALID), (dict(out=None), INVALID), (dict(n=-1), INVALID),
+    (dict(dl=0), INVALID), (dict(eps=-1.0), INVALID), (dict(eps=float("nan")), INVALID),
+    (dict(dl=100), UNSUPPORTED), (dict(c=M), ALIGN), (dict(out=M), ALIGN), (dict(w=M), ALIGN),
+    (dict(n=0), OK),
+])
+def test_latent_rmsnorm_argument_errors(lib, kw, code):
+    args = dict(c=A, w=None, eps=1e-6, out=A, n=100, dl=512)
+    args.update(kw)
+    assert lib.gdla_latent_rmsnorm(args["c"], args["w"], ctypes.c_float(args["eps"]), args["out"],
+                                   args["n"], args["dl"], None, None) == code

@@ -80,7 +80,7 @@ def test_latent_config_chained_attention():
     torch.cuda.synchronize()
     # every query block's first and last rows up to token 8191, block edges
     # across the sequence and random rows: 256+ rows, keys up to the last one
-    rows = sample_rows(wl.B, wl.T, 96, seed=4,
+    rows = sample_rows(wl.B, wl.T, 140, seed=4,
                        extra=[q + o for q in range(0, 8192, 128) for o in (0, 127)])
     assert rows.size >= 256
     t_max = int(rows.max()) + 1
