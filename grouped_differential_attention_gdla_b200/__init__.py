@@ -11,13 +11,17 @@ device memory and streams only.
     gdla_latent_rmsnorm(c_kv) -> c_hat          cache write: RMSNorm'd KV latents
     gdla_decode_fwd(q_sig, q_noise, c_hat, cache_len, w_kvb, lam, gate) -> out
                             the newest token of each sequence over its latent cache
+    gdla_decode_fwd_noalloc(..., out)   the same, with the library's own scratch
+                            array, for callers that cannot allocate device memory
 """
 from ._binding import (GDLAError, EXPORTED, LIB_PATH, check_status, gdla_attn_fwd,
-                       gdla_attn_fwd_sp, gdla_decode_fwd, gdla_decode_workspace_bytes,
+                       gdla_attn_fwd_sp, gdla_decode_fwd, gdla_decode_fwd_noalloc,
+                       gdla_decode_workspace_bytes,
                        gdla_kv_expand, gdla_latent_rmsnorm, gdla_selftest_wait_timeout,
                        gdla_status_string, gdla_version, load_library)
 
 __all__ = ["GDLAError", "EXPORTED", "LIB_PATH", "check_status", "gdla_attn_fwd",
-           "gdla_attn_fwd_sp", "gdla_decode_fwd", "gdla_decode_workspace_bytes",
+           "gdla_attn_fwd_sp", "gdla_decode_fwd", "gdla_decode_fwd_noalloc",
+           "gdla_decode_workspace_bytes",
            "gdla_kv_expand", "gdla_latent_rmsnorm", "gdla_selftest_wait_timeout",
            "gdla_status_string", "gdla_version", "load_library"]

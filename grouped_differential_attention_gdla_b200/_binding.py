@@ -32,7 +32,7 @@ GDLA_ERR_TIMEOUT = -5
 # every symbol include/gdla.h declares
 EXPORTED = ("gdla_version", "gdla_status_string", "gdla_kv_expand", "gdla_attn_fwd",
             "gdla_attn_fwd_sp", "gdla_latent_rmsnorm", "gdla_decode_workspace_bytes",
-            "gdla_decode_fwd", "gdla_selftest_wait_timeout")
+            "gdla_decode_fwd", "gdla_selftest_wait_timeout", "gdla_decode_fwd_noalloc")
 
 _lib = None
 # One status word per device, used when a caller passes none (see check_status).
@@ -77,6 +77,9 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
                                     i32, i64, f32, vp, ctypes.c_size_t, vp, vp]
     lib.gdla_decode_fwd.restype = i32
     lib.gdla_selftest_wait_timeout.argtypes = [vp, i64, vp]
+    lib.gdla_decode_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32,
+                                            i32, i32, i32, i64, f32, vp, vp]
+    lib.gdla_decode_fwd_noalloc.restype = i32
     lib.gdla_selftest_wait_timeout.restype = i32
     if path is None:
         _lib = lib
@@ -343,6 +346,59 @@ def gdla_decode_fwd(q_sig: torch.Tensor, q_noise: torch.Tensor, c_hat: torch.Ten
         raise GDLAError(rc, "gdla_decode_fwd")
     if _sync_check_enabled():
         check_status(q_sig.device, d_status)
+    return out
+
+
+# Size of the scratch array compiled into libgdla.so for gdla_decode_fwd_noalloc.
+DECODE_NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def gdla_decode_fwd_noalloc(q_sig: torch.Tensor, q_noise: torch.Tensor, c_hat: torch.Tensor,
+                            cache_len: torch.Tensor, w_kvb: torch.Tensor, lam: torch.Tensor,
+                            gate: torch.Tensor, out: torch.Tensor, window: int = 0,
+                            scale: float = 0.0, d_status: Optional[torch.Tensor] = None,
+                            stream=None) -> torch.Tensor:
+    """gdla_decode_fwd without a workspace, for callers that cannot allocate.
+
+    The decode's scratch comes from an array compiled into the library
+    (DECODE_NOALLOC_SCRATCH_BYTES per GPU), so neither the library nor this
+    wrapper allocates device memory: the caller passes every input and `out`
+    [B, Hs*d].  A d_status of None passes no status word.  Shapes needing more
+    scratch than the array holds raise GDLAError (GDLA_ERR_UNSUPPORTED).  All
+    calls on a device share the array: calls that overlap on the GPU race.
+    """
+    if q_sig.dim() != 3 or c_hat.dim() != 3:
+        raise ValueError("q_sig must be [B, Hs, d] and c_hat [B, L_max, d_latent]")
+    B, Hs, d = q_sig.shape
+    Hn = q_noise.shape[1] if q_noise.dim() == 3 else -1
+    L_max, dl = c_hat.shape[1], c_hat.shape[2]
+    hkv = w_kvb.shape[1] // (2 * d) if w_kvb.dim() == 2 else -1
+    if cache_len.dtype != torch.int32 or tuple(cache_len.shape) != (B,) or \
+            not cache_len.is_contiguous():
+        raise ValueError("cache_len must be a contiguous int32 tensor of shape [B]")
+    ptrs = [
+        _check(q_sig, "q_sig"),
+        _check(q_noise, "q_noise", (B, Hn, d)),
+        _check(c_hat, "c_hat"),
+    ]
+    pw = _check(w_kvb, "w_kvb", (dl, hkv * 2 * d))
+    pl = _check(lam, "lam", (B, Hs))
+    pg = _check(gate, "gate", (B, Hs * d))
+    po = _check(out, "out", (B, Hs * d))
+    _same_device(q_sig.device, [("q_noise", q_noise), ("c_hat", c_hat), ("cache_len", cache_len),
+                                 ("w_kvb", w_kvb), ("lam", lam), ("gate", gate), ("out", out)])
+    ps = 0
+    if d_status is not None:
+        _same_device(q_sig.device, [("d_status", d_status)])
+        if d_status.dtype != torch.int32:
+            raise ValueError("d_status must be an int32 tensor")
+        ps = d_status.data_ptr()
+    rc = load_library().gdla_decode_fwd_noalloc(*ptrs, cache_len.data_ptr(), pw, pl, pg, po, B,
+                                                L_max, Hs, Hn, hkv, d, dl, int(window),
+                                                float(scale), ps,
+                                                _stream_ptr(q_sig.device, stream))
+    if rc != GDLA_OK:
+        raise GDLAError(rc, "gdla_decode_fwd_noalloc")
     return out
 
 

@@ -482,3 +482,54 @@ int gdla_selftest_wait_timeout(int *d_status, int64_t limit_ns, void *stream) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------- decode without allocation
+// Scratch for gdla_decode_fwd_noalloc, compiled into the library so that
+// callers which cannot allocate device memory still have a workspace.  Host
+// code must not pass `g_decode_scratch` itself to a kernel: on the host the
+// name stands for a host-side shadow, not the device address.  The device
+// address is looked up once per device, with that device current.
+static __device__ __align__(256) uint8_t g_decode_scratch[GDLA_DECODE_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+int decode_scratch_address(void **ptr) {
+  static std::atomic<void *> cache[kCachedDevices];
+  int dev = 0;
+  if (current_device(&dev) != GDLA_OK) return GDLA_ERR_CUDA;
+  if (dev >= 0 && dev < kCachedDevices) {
+    void *c = cache[dev].load(std::memory_order_acquire);
+    if (c) {
+      *ptr = c;
+      return GDLA_OK;
+    }
+  }
+  void *p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr)
+    return GDLA_ERR_CUDA;
+  if (dev >= 0 && dev < kCachedDevices) cache[dev].store(p, std::memory_order_release);
+  *ptr = p;
+  return GDLA_OK;
+}
+
+}  // namespace
+
+extern "C" int gdla_decode_fwd_noalloc(const void *q_sig, const void *q_noise, const void *c_hat,
+                                       const int32_t *cache_len, const void *w_kvb,
+                                       const void *lambda, const void *gate, void *out, int B,
+                                       int64_t L_max, int Hs, int Hn, int Hkv, int d,
+                                       int d_latent, int64_t window, float scale, int *d_status,
+                                       void *stream) {
+  // the size check comes first, so an oversized request touches no device
+  if (B > 0 && gdla_decode_workspace_bytes(B, L_max, Hs, Hn, d_latent, window) >
+                   GDLA_DECODE_NOALLOC_SCRATCH_BYTES)
+    return GDLA_ERR_UNSUPPORTED;
+  void *scratch = nullptr;
+  if (B > 0) {
+    const int rc = decode_scratch_address(&scratch);
+    if (rc != GDLA_OK) return rc;
+  }
+  return gdla_decode_fwd(q_sig, q_noise, c_hat, cache_len, w_kvb, lambda, gate, out, B, L_max,
+                         Hs, Hn, Hkv, d, d_latent, window, scale, scratch,
+                         GDLA_DECODE_NOALLOC_SCRATCH_BYTES, d_status, stream);
+}

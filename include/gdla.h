@@ -233,6 +233,45 @@ int gdla_decode_fwd(const void *q_sig, const void *q_noise, const void *c_hat,
  */
 int gdla_selftest_wait_timeout(int *d_status, int64_t limit_ns, void *stream);
 
+/*
+ * gdla_decode_fwd_noalloc - gdla_decode_fwd for callers that cannot allocate
+ * device memory.  The pages have no counterpart to this entry point: it
+ * exists for the library's users, not for the method.
+ *
+ * gdla_decode_fwd needs a device workspace for the absorbed queries and the
+ * per-split partial results.  Some callers have no way to obtain one: code
+ * that runs where the process's allocator is owned by someone else (a host
+ * framework that forbids cudaMalloc inside its callbacks, a plugin without
+ * an allocator handle), or a serving loop that must not allocate between
+ * requests.  This entry point takes the same arguments minus the workspace
+ * and uses instead a scratch array compiled into the library: a file-scope
+ * __device__ array of GDLA_DECODE_NOALLOC_SCRATCH_BYTES bytes (16 MiB), which
+ * every GPU that loads the library holds until the process exits.
+ *
+ *   - It allocates nothing (no cudaMalloc, cudaFree or allocating library
+ *     routine) and otherwise behaves exactly like gdla_decode_fwd.
+ *   - Shapes whose workspace (gdla_decode_workspace_bytes) exceeds
+ *     GDLA_DECODE_NOALLOC_SCRATCH_BYTES are refused with GDLA_ERR_UNSUPPORTED
+ *     before anything else happens; use gdla_decode_fwd for them.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and keeps it; make that
+ *     first call before any stream capture.  A failed look-up returns
+ *     GDLA_ERR_CUDA.
+ *   - Every call on a device shares the one array, which keeps the previous
+ *     call's contents.  Nothing in it needs to start at zero: the kernels
+ *     write each byte they read first.  Calls whose kernels overlap on the
+ *     GPU (other streams, other host threads) race on the array and give
+ *     undefined results: serialise them on one stream.
+ */
+#define GDLA_DECODE_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+int gdla_decode_fwd_noalloc(const void *q_sig, const void *q_noise,
+                            const void *c_hat, const int32_t *cache_len,
+                            const void *w_kvb, const void *lambda,
+                            const void *gate, void *out, int B, int64_t L_max,
+                            int Hs, int Hn, int Hkv, int d, int d_latent,
+                            int64_t window, float scale, int *d_status,
+                            void *stream);
+
 #ifdef __cplusplus
 } /* extern "C" */
 #endif

@@ -36,7 +36,7 @@ def test_exports_every_declared_symbol(lib):
     assert set(declared) == {"gdla_version", "gdla_status_string", "gdla_kv_expand",
                              "gdla_attn_fwd", "gdla_attn_fwd_sp", "gdla_latent_rmsnorm",
                              "gdla_decode_workspace_bytes", "gdla_decode_fwd",
-                             "gdla_selftest_wait_timeout"}
+                             "gdla_selftest_wait_timeout", "gdla_decode_fwd_noalloc"}
     for name in declared:
         assert hasattr(lib, name), f"{name} missing from libgdla.so"
     assert set(declared) == set(_binding.EXPORTED)
