@@ -48,8 +48,9 @@ def test_expand_every_element(n, dl, hkv, dh, with_w):
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     rk, rv = _oracle_kv(c, w, rw, 1e-6, hkv, dh)
-    assert_parity(k.float().cpu().numpy(), rk, "K")
-    assert_parity(v.float().cpu().numpy(), rv, "V")
+    shape = f"n={n} dl={dl} Hkv={hkv} d={dh}"
+    assert_parity(k.float().cpu().numpy(), rk, f"expand K {shape}")
+    assert_parity(v.float().cpu().numpy(), rv, f"expand V {shape}")
 
 
 def test_latent_config_expand_sampled_tokens():
