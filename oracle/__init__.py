@@ -105,9 +105,13 @@ class Oracle:
                                                  i32, i64, i32, i32, i32, i32, i64, i32, f64, vp,
                                                  i64, vp]
         lib.gdla_oracle_attn_compact.restype = ctypes.c_int
-        lib.gdla_oracle_decode.argtypes = [vp, i32, vp, i32, vp, i32, vp, vp, i32, f64, vp, i32,
-                                           vp, i32, vp, i32, i32, i64, i32, i32, i32, i32, i32,
-                                           i64, f64, vp]
+        lib.gdla_oracle_attn_rope.argtypes = [vp, i32, vp, i32, vp, i32, vp, i32, vp, i32, vp,
+                                              i32, i32, vp, i32, vp, i32, vp, i32, i32, i64, i32,
+                                              i32, i32, i32, i64, i32, f64, vp, i64, vp]
+        lib.gdla_oracle_attn_rope.restype = ctypes.c_int
+        lib.gdla_oracle_decode.argtypes = [vp, i32, vp, i32, vp, i32, vp, i32, vp, i32, vp, i32,
+                                           i32, vp, vp, i32, f64, vp, i32, vp, i32, vp, i32, i32,
+                                           i64, i32, i32, i32, i32, i32, i64, f64, vp]
         lib.gdla_oracle_decode.restype = ctypes.c_int
         lib.gdla_oracle_version.restype = ctypes.c_int
         self.lib = lib
@@ -181,12 +185,19 @@ class Oracle:
 
     # whole attention forward
     def gdla_attn(self, q_sig, q_noise, k, v, lam, gate, window: int = 0, causal: bool = True,
-                  scale=None, rows=None) -> np.ndarray:
+                  scale=None, rows=None, q_rope_sig=None, q_rope_noise=None,
+                  k_rope=None) -> np.ndarray:
         """O[n_rows, Hs*d] in float64 for flat rows b*T+i (all when None).
 
         q_sig [B,T,Hs,d], q_noise [B,T,Hn,d], k/v [B,T,Hkv,d], lam [B,T,Hs],
-        gate [B,T,Hs*d].
+        gate [B,T,Hs*d].  With the decoupled rotary term: q_rope_sig
+        [B,T,Hs,dr], q_rope_noise [B,T,Hn,dr] and k_rope [B,T,dr] (one rotary
+        key per token for every head); the default scale is then
+        1/sqrt(d + dr).
         """
+        if k_rope is not None:
+            return self._attn_rope(q_sig, q_noise, q_rope_sig, q_rope_noise, k, k_rope, v, lam,
+                                   gate, window, causal, scale, rows, compact=False)
         qs, qsp, qsdt = _arr(q_sig)
         qn, qnp, qndt = _arr(q_noise)
         ka, kp, kdt = _arr(k)
@@ -208,14 +219,54 @@ class Oracle:
         return out
 
 
+    def _attn_rope(self, q_sig, q_noise, qr_sig, qr_noise, k, k_rope, v, lam, gate, window,
+                   causal, scale, rows, compact):
+        qs, qsp, qsdt = _arr(q_sig)
+        qn, qnp, qndt = _arr(q_noise)
+        rs, rsp, rsdt = _arr(qr_sig)
+        rn, rnp, rndt = _arr(qr_noise)
+        ka, kp, kdt = _arr(k)
+        kr, krp, krdt = _arr(k_rope)
+        va, vp, vdt = _arr(v)
+        la, lp, ldt = _arr(lam)
+        ga, gp, gdt = _arr(gate)
+        B, T, Hkv, d = ka.shape
+        dr = kr.shape[-1]
+        Hs, Hn = qs.shape[-2], qn.shape[-2]
+        if tuple(kr.shape) != (B, T, dr) or rs.shape[-1] != dr or rn.shape[-1] != dr:
+            raise ValueError("k_rope must be [B,T,dr] and the rotary queries [..., H, dr]")
+        if rs.shape[:-1] != qs.shape[:-1] or rn.shape[:-1] != qn.shape[:-1]:
+            raise ValueError("rotary queries must be laid out like the queries")
+        if scale is None:
+            scale = 1.0 / np.sqrt(d + dr)
+        r, rp, n = _rows(rows, B * T)
+        if compact and (qs.shape[0] != n or la.shape[0] != n or ga.shape[0] != n):
+            raise ValueError("row-gathered inputs must have one entry per row")
+        out = np.empty((n, Hs * d), dtype=np.float64)
+        rc = self.lib.gdla_oracle_attn_rope(qsp, qsdt, qnp, qndt, rsp, rsdt, rnp, rndt, kp, kdt,
+                                            krp, krdt, dr, vp, vdt, lp, ldt, gp, gdt,
+                                            int(bool(compact)), T, Hs, Hn, Hkv, d, int(window),
+                                            int(bool(causal)), float(scale), rp, n,
+                                            out.ctypes.data)
+        if rc != 0:
+            raise ValueError("oracle rejected the head counts or the rotary inputs")
+        return out
+
     def gdla_attn_rows(self, q_sig_rows, q_noise_rows, k, v, lam_rows, gate_rows, rows,
-                       window: int = 0, causal: bool = True, scale=None) -> np.ndarray:
+                       window: int = 0, causal: bool = True, scale=None, q_rope_sig_rows=None,
+                       q_rope_noise_rows=None, k_rope=None) -> np.ndarray:
         """Same as gdla_attn, with the query-side inputs gathered per row.
 
         q_sig_rows [n,Hs,d], q_noise_rows [n,Hn,d], lam_rows [n,Hs] and
         gate_rows [n,Hs*d] hold only the evaluated rows (flat indices b*T+i in
-        ``rows``, same order); k and v stay full [B,T,Hkv,d].
+        ``rows``, same order); k and v stay full [B,T,Hkv,d].  With the
+        rotary term, q_rope_*_rows [n,H,dr] are gathered too and k_rope
+        [B,T,dr] stays full.
         """
+        if k_rope is not None:
+            return self._attn_rope(q_sig_rows, q_noise_rows, q_rope_sig_rows, q_rope_noise_rows,
+                                   k, k_rope, v, lam_rows, gate_rows, window, causal, scale,
+                                   rows, compact=True)
         qs, qsp, qsdt = _arr(q_sig_rows)
         qn, qnp, qndt = _arr(q_noise_rows)
         ka, kp, kdt = _arr(k)
@@ -242,16 +293,31 @@ class Oracle:
 
     # decode: the newest token of each sequence over its latent cache
     def decode(self, q_sig, q_noise, c_kv, cache_len, w_kvb, lam, gate, rms_w=None,
-               eps: float = 1e-6, window: int = 0, scale=None) -> np.ndarray:
+               eps: float = 1e-6, window: int = 0, scale=None, q_rope_sig=None,
+               q_rope_noise=None, k_rope=None) -> np.ndarray:
         """O[B, Hs*d] for the query token of each sequence (its position is
         cache_len[b] - 1), from the raw KV latents c_kv [B, L_max, d_latent]:
         RMSNorm, W^KV_b expand, then the GDLA forward for that one row.
 
         q_sig [B,Hs,d], q_noise [B,Hn,d], lam [B,Hs], gate [B,Hs*d];
-        cache_len: B integers in 1..L_max.
+        cache_len: B integers in 1..L_max.  With the rotary term: the cached
+        rotary keys k_rope [B,L_max,dr] and the query token's q_rope_sig
+        [B,Hs,dr], q_rope_noise [B,Hn,dr]; the default scale is then
+        1/sqrt(d + dr).
         """
         qs, qsp, qsdt = _arr(q_sig)
         qn, qnp, qndt = _arr(q_noise)
+        dr = 0
+        rsp = rnp = krp = None
+        rsdt = rndt = krdt = F64
+        if k_rope is not None:
+            rs, rsp, rsdt = _arr(q_rope_sig)
+            rn, rnp, rndt = _arr(q_rope_noise)
+            kr, krp, krdt = _arr(k_rope)
+            dr = kr.shape[-1]
+            if rs.shape != (qs.shape[0], qs.shape[1], dr) or \
+                    rn.shape != (qn.shape[0], qn.shape[1], dr):
+                raise ValueError("rotary queries must be [B, H, dr]")
         ca, cp, cdt = _arr(c_kv)
         wa, wp, wdt = _arr(w_kvb)
         la, lp, ldt = _arr(lam)
@@ -264,12 +330,15 @@ class Oracle:
         lens = np.ascontiguousarray(np.asarray(cache_len, dtype=np.int64).reshape(-1))
         if lens.size != B or lens.min() < 1 or lens.max() > L_max:
             raise ValueError("cache_len must hold B lengths in 1..L_max")
+        if dr and tuple(kr.shape) != (B, L_max, dr):
+            raise ValueError("k_rope must be [B, L_max, dr]")
         if scale is None:
-            scale = 1.0 / np.sqrt(d)
+            scale = 1.0 / np.sqrt(d + dr)
         out = np.empty((B, Hs * d), dtype=np.float64)
-        rc = self.lib.gdla_oracle_decode(qsp, qsdt, qnp, qndt, cp, cdt, lens.ctypes.data, rp, rdt,
-                                         float(eps), wp, wdt, lp, ldt, gp, gdt, B, L_max, dl, Hs,
-                                         Hn, Hkv, d, int(window), float(scale), out.ctypes.data)
+        rc = self.lib.gdla_oracle_decode(qsp, qsdt, qnp, qndt, rsp, rsdt, rnp, rndt, cp, cdt, krp,
+                                         krdt, dr, lens.ctypes.data, rp, rdt, float(eps), wp, wdt,
+                                         lp, ldt, gp, gdt, B, L_max, dl, Hs, Hn, Hkv, d,
+                                         int(window), float(scale), out.ctypes.data)
         if rc != 0:
             raise ValueError("oracle rejected the decode arguments (rc %d)" % rc)
         return out

@@ -29,7 +29,14 @@
  *     already passed through their sigmoids;
  *   - sliding window W keeps keys j with i-W < j <= i; W = 0 means full causal;
  *   - RMSNorm is c / sqrt(mean(c^2) + eps) * w;
- *   - the W^KV_b columns of KV head h are [K_h (dk) | V_h (dv)].
+ *   - the W^KV_b columns of KV head h are [K_h (dk) | V_h (dv)];
+ *   - decoupled rotary term ([R] "technical novelty" paragraph: both query
+ *     paths share the up-projected KV and one broadcast decoupled rotary
+ *     key): every head of both paths has its own rotary query q_r (d_rope
+ *     wide), every token one rotary key k_r shared by all heads, and the
+ *     score is scale * (q . k + q_r . k_r).  The rotation itself is applied
+ *     before the attention (q_r and k_r arrive rotated), as lambda and the
+ *     gate arrive after their sigmoids.  d_rope = 0 is the score without it.
  *
  * Every function computes in double, in the order the definition is written:
  * no tiling, no online softmax, no reassociation.  Inputs may be given as
@@ -129,14 +136,19 @@ static void key_range(int64_t i, int64_t T, int64_t window, int causal,
  *   p_j = exp(s_j - max_j s_j)
  *   H[row, h, :] = sum_j p_j V[b,j,kv(h),:] / sum_j p_j
  * kv(h) = h / (H / Hkv).  Q is [B,T,H,d], K and V are [B,T,Hkv,d].
+ * With the decoupled rotary term (dr > 0) the score of key j adds
+ *   sum_c Qr[b,i,h,c] Kr[b,j,c]                            c < dr
+ * inside the scale: Qr is [B,T,H,dr] (laid out like Q), Kr is [B,T,dr], one
+ * rotary key per token for every head.  dr == 0 leaves the score as above.
  * rows == NULL means every row (n_rows must then be B*T).
  */
 static void attention_path_impl(const void *q, int q_dt, int q_compact,
-                                const void *k, int k_dt, const void *v,
-                                int v_dt, int64_t T, int H, int Hkv, int d,
-                                int64_t window, int causal, double scale,
-                                const int64_t *rows, int64_t n_rows,
-                                double *out) {
+                                const void *qr, int qr_dt, const void *k,
+                                int k_dt, const void *kr, int kr_dt, int dr,
+                                const void *v, int v_dt, int64_t T, int H,
+                                int Hkv, int d, int64_t window, int causal,
+                                double scale, const int64_t *rows,
+                                int64_t n_rows, double *out) {
   const int group = H / Hkv;
   int64_t task;
 #pragma omp parallel
@@ -153,12 +165,17 @@ static void attention_path_impl(const void *q, int q_dt, int q_compact,
       int64_t lo, hi;
       key_range(i, T, window, causal, &lo, &hi);
       const int64_t qoff = ((q_compact ? ri : row) * H + h) * d;
+      const int64_t qroff = ((q_compact ? ri : row) * H + h) * (int64_t)dr;
       double m = -INFINITY;
       for (int64_t j = lo; j <= hi; ++j) {
         const int64_t koff = ((b * T + j) * Hkv + kvh) * d;
         double dot = 0.0;
         for (int c = 0; c < d; ++c)
           dot += load_elem(q, q_dt, qoff + c) * load_elem(k, k_dt, koff + c);
+        /* the rotary key of token j: one vector for every head */
+        for (int c = 0; c < dr; ++c)
+          dot += load_elem(qr, qr_dt, qroff + c) *
+                 load_elem(kr, kr_dt, (b * T + j) * (int64_t)dr + c);
         s[j - lo] = scale * dot;
         if (s[j - lo] > m) m = s[j - lo];
       }
@@ -185,8 +202,9 @@ void gdla_oracle_attention_path(const void *q, int q_dt, const void *k,
                                 const int64_t *rows, int64_t n_rows,
                                 double *out) {
   (void)B;
-  attention_path_impl(q, q_dt, 0, k, k_dt, v, v_dt, T, H, Hkv, d, window,
-                      causal, scale, rows, n_rows, out);
+  attention_path_impl(q, q_dt, 0, NULL, ORACLE_F64, k, k_dt, NULL, ORACLE_F64, 0,
+                      v, v_dt, T, H, Hkv, d, window, causal, scale, rows, n_rows,
+                      out);
 }
 
 /*
@@ -239,7 +257,9 @@ void gdla_oracle_differential_gate(const double *hs, const double *hn,
  * (Hs % Hn, Hn != Hkv).
  */
 static int attn_impl(const void *q_sig, int qs_dt, const void *q_noise,
-                     int qn_dt, const void *k, int k_dt, const void *v,
+                     int qn_dt, const void *qr_sig, int qrs_dt,
+                     const void *qr_noise, int qrn_dt, const void *k, int k_dt,
+                     const void *kr, int kr_dt, int dr, const void *v,
                      int v_dt, const void *lam, int lam_dt, const void *gate,
                      int gate_dt, int compact, int64_t T, int Hs, int Hn,
                      int Hkv, int d, int64_t window, int causal, double scale,
@@ -252,10 +272,12 @@ static int attn_impl(const void *q_sig, int qs_dt, const void *q_noise,
     free(hn);
     return -2;
   }
-  attention_path_impl(q_sig, qs_dt, compact, k, k_dt, v, v_dt, T, Hs, Hkv, d,
-                      window, causal, scale, rows, n_rows, hs);
-  attention_path_impl(q_noise, qn_dt, compact, k, k_dt, v, v_dt, T, Hn, Hkv,
-                      d, window, causal, scale, rows, n_rows, hn);
+  attention_path_impl(q_sig, qs_dt, compact, qr_sig, qrs_dt, k, k_dt, kr, kr_dt,
+                      dr, v, v_dt, T, Hs, Hkv, d, window, causal, scale, rows,
+                      n_rows, hs);
+  attention_path_impl(q_noise, qn_dt, compact, qr_noise, qrn_dt, k, k_dt, kr,
+                      kr_dt, dr, v, v_dt, T, Hn, Hkv, d, window, causal, scale,
+                      rows, n_rows, hn);
   differential_gate_impl(hs, hn, lam, lam_dt, gate, gate_dt, compact, Hs, Hn,
                          d, rows, n_rows, out);
   free(hs);
@@ -270,9 +292,10 @@ int gdla_oracle_attn(const void *q_sig, int qs_dt, const void *q_noise,
                      int d, int64_t window, int causal, double scale,
                      const int64_t *rows, int64_t n_rows, double *out) {
   (void)B;
-  return attn_impl(q_sig, qs_dt, q_noise, qn_dt, k, k_dt, v, v_dt, lam, lam_dt,
-                   gate, gate_dt, 0, T, Hs, Hn, Hkv, d, window, causal, scale,
-                   rows, n_rows, out);
+  return attn_impl(q_sig, qs_dt, q_noise, qn_dt, NULL, ORACLE_F64, NULL,
+                   ORACLE_F64, k, k_dt, NULL, ORACLE_F64, 0, v, v_dt, lam,
+                   lam_dt, gate, gate_dt, 0, T, Hs, Hn, Hkv, d, window, causal,
+                   scale, rows, n_rows, out);
 }
 
 int gdla_oracle_attn_compact(const void *q_sig, int qs_dt, const void *q_noise,
@@ -282,8 +305,32 @@ int gdla_oracle_attn_compact(const void *q_sig, int qs_dt, const void *q_noise,
                              int Hn, int Hkv, int d, int64_t window,
                              int causal, double scale, const int64_t *rows,
                              int64_t n_rows, double *out) {
-  return attn_impl(q_sig, qs_dt, q_noise, qn_dt, k, k_dt, v, v_dt, lam, lam_dt,
-                   gate, gate_dt, 1, T, Hs, Hn, Hkv, d, window, causal, scale,
+  return attn_impl(q_sig, qs_dt, q_noise, qn_dt, NULL, ORACLE_F64, NULL,
+                   ORACLE_F64, k, k_dt, NULL, ORACLE_F64, 0, v, v_dt, lam,
+                   lam_dt, gate, gate_dt, 1, T, Hs, Hn, Hkv, d, window, causal,
+                   scale, rows, n_rows, out);
+}
+
+/*
+ * gdla_oracle_attn with the decoupled rotary term ([R] "technical novelty"
+ * paragraph): qr_sig [.., Hs, dr] and qr_noise [.., Hn, dr] are laid out like
+ * q_sig and q_noise (full, or one entry per evaluated row when compact), kr
+ * is [B, T, dr], one rotary key per token shared by every head of both
+ * paths.  Returns as gdla_oracle_attn.
+ */
+int gdla_oracle_attn_rope(const void *q_sig, int qs_dt, const void *q_noise,
+                          int qn_dt, const void *qr_sig, int qrs_dt,
+                          const void *qr_noise, int qrn_dt, const void *k,
+                          int k_dt, const void *kr, int kr_dt, int dr,
+                          const void *v, int v_dt, const void *lam, int lam_dt,
+                          const void *gate, int gate_dt, int compact,
+                          int64_t T, int Hs, int Hn, int Hkv, int d,
+                          int64_t window, int causal, double scale,
+                          const int64_t *rows, int64_t n_rows, double *out) {
+  if (dr < 0 || (dr > 0 && (!qr_sig || !qr_noise || !kr))) return -1;
+  return attn_impl(q_sig, qs_dt, q_noise, qn_dt, qr_sig, qrs_dt, qr_noise,
+                   qrn_dt, k, k_dt, kr, kr_dt, dr, v, v_dt, lam, lam_dt, gate,
+                   gate_dt, compact, T, Hs, Hn, Hkv, d, window, causal, scale,
                    rows, n_rows, out);
 }
 
@@ -300,10 +347,16 @@ int gdla_oracle_attn_compact(const void *q_sig, int qs_dt, const void *q_noise,
  * q_sig [B, Hs, d], q_noise [B, Hn, d], lambda [B, Hs], gate [B, Hs*d] hold
  * the query token of each sequence; c_kv is [B, L_max, d_latent].  Only the
  * keys J(i) of the window enter (window 0 = full causal).  out: [B, Hs*d].
+ * With the decoupled rotary term (dr > 0) the cache also holds each token's
+ * rotary key, kr [B, L_max, dr] (cached beside the latent, as in MLA), and
+ * qr_sig [B, Hs, dr], qr_noise [B, Hn, dr] are the query token's rotary
+ * queries; dr == 0 ignores all three.
  * Returns 0, -1 for bad head counts or lengths, -2 when out of memory.
  */
 int gdla_oracle_decode(const void *q_sig, int qs_dt, const void *q_noise,
-                       int qn_dt, const void *c_kv, int c_dt,
+                       int qn_dt, const void *qr_sig, int qrs_dt,
+                       const void *qr_noise, int qrn_dt, const void *c_kv,
+                       int c_dt, const void *kr, int kr_dt, int dr,
                        const int64_t *cache_len, const void *rms_w, int w_dt,
                        double eps, const void *w_kvb, int wk_dt,
                        const void *lam, int lam_dt, const void *gate,
@@ -311,6 +364,7 @@ int gdla_oracle_decode(const void *q_sig, int qs_dt, const void *q_noise,
                        int Hs, int Hn, int Hkv, int d, int64_t window,
                        double scale, double *out) {
   if (Hn <= 0 || Hkv <= 0 || Hs % Hn != 0 || Hn != Hkv) return -1;
+  if (dr < 0 || (dr > 0 && (!qr_sig || !qr_noise || !kr))) return -1;
   for (int b = 0; b < B; ++b) {
     const int64_t Lb = cache_len[b];
     if (Lb < 1 || Lb > L_max) return -1;
@@ -347,10 +401,18 @@ int gdla_oracle_decode(const void *q_sig, int qs_dt, const void *q_noise,
     qn_b = ORACLE_AT(q_noise, qn_dt, (int64_t)b * Hn * d);
     lam_b = ORACLE_AT(lam, lam_dt, (int64_t)b * Hs);
     gate_b = ORACLE_AT(gate, gate_dt, (int64_t)b * Hs * d);
+    /* rotary queries of the query token, rotary keys of the kept tokens */
+    const void *qrs_b = NULL, *qrn_b = NULL, *kr_b = NULL;
+    if (dr > 0) {
+      qrs_b = ORACLE_AT(qr_sig, qrs_dt, (int64_t)b * Hs * dr);
+      qrn_b = ORACLE_AT(qr_noise, qrn_dt, (int64_t)b * Hn * dr);
+      kr_b = ORACLE_AT(kr, kr_dt, ((int64_t)b * L_max + first) * dr);
+    }
 #undef ORACLE_AT
-    const int rc = attn_impl(qs_b, qs_dt, qn_b, qn_dt, k, ORACLE_F64, v, ORACLE_F64,
-                             lam_b, lam_dt, gate_b, gate_dt, 1, L, Hs, Hn, Hkv, d,
-                             window, 1, scale, &row, 1, out + (int64_t)b * Hs * d);
+    const int rc = attn_impl(qs_b, qs_dt, qn_b, qn_dt, qrs_b, qrs_dt, qrn_b, qrn_dt,
+                             k, ORACLE_F64, kr_b, kr_dt, dr, v, ORACLE_F64, lam_b,
+                             lam_dt, gate_b, gate_dt, 1, L, Hs, Hn, Hkv, d, window,
+                             1, scale, &row, 1, out + (int64_t)b * Hs * d);
     free(chat);
     free(k);
     free(v);

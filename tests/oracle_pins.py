@@ -317,6 +317,132 @@ def pin_scale_placement(o):
     assert np.array_equal(a, c), "default scale must be 1/sqrt(d)"
 
 
+# ---------------------------------------------------------------- rotary term
+# "Motif 3: Technical Report" (paper.rainbus.top digest), "technical novelty"
+# paragraph: both query paths share the up-projected KV and one broadcast
+# decoupled rotary key.  Reading: score = scale * (q.k + q_r.k_r), one rotary
+# key per token for every head of both paths; default scale 1/sqrt(d + d_rope).
+
+def _golden_value(x):
+    if isinstance(x, str):
+        if x in ("LN2", "LN3"):
+            return math.log(2.0 if x == "LN2" else 3.0)
+        num, den = x.split("/")
+        return float(num) / float(den)
+    return x
+
+
+def _golden_array(a):
+    if isinstance(a, list):
+        return [_golden_array(e) for e in a]
+    return _golden_value(a)
+
+
+def _rope_small(B=2, T=19, Hs=8, Hn=2, Hkv=2, d=16, dr=8, seed=3, window=0, causal=True):
+    wl, x = _small(B, T, Hs, Hn, Hkv, d, seed=seed, window=window, causal=causal)
+    g = torch.Generator().manual_seed(seed + 1000)
+    x["q_rope_sig"] = torch.randn(B, T, Hs, dr, generator=g).to(torch.bfloat16)
+    x["q_rope_noise"] = torch.randn(B, T, Hn, dr, generator=g).to(torch.bfloat16)
+    x["k_rope"] = torch.randn(B, T, dr, generator=g).to(torch.bfloat16)
+    return wl, x
+
+
+def _rope_attn(o, x, **kw):
+    return o.gdla_attn(x["q_sig"], x["q_noise"], x["k"], x["v"], x["lam"], x["gate"],
+                       q_rope_sig=x["q_rope_sig"], q_rope_noise=x["q_rope_noise"],
+                       k_rope=x["k_rope"], **kw)
+
+
+def pin_rope_hand_example(o):
+    """Two-token case with the rotary term, derived by hand
+    (tests/golden/rope_hand_example.json)."""
+    with open(os.path.join(GOLDEN, "rope_hand_example.json")) as f:
+        g = json.load(f)
+    arr = lambda key: np.array(_golden_array(g[key]), dtype=np.float64)
+    args = dict(q_sig=arr("q_sig"), q_noise=arr("q_noise"), k=arr("k"), v=arr("v"),
+                lam=arr("lam"), gate=arr("gate"), q_rope_sig=arr("q_rope_sig"),
+                q_rope_noise=arr("q_rope_noise"), k_rope=arr("k_rope"),
+                scale=g["shape"]["scale"])
+    exp = {k: np.array(_golden_array(v)) for k, v in g["expected"].items()}
+    _close(o.gdla_attn(**args, window=0, causal=True), exp["causal"], what="rope causal")
+    _close(o.gdla_attn(**args, window=1, causal=True), exp["window1"], what="rope W=1")
+    _close(o.gdla_attn(**args, window=0, causal=False), exp["noncausal"],
+           what="rope non-causal")
+
+
+def pin_rope_matches_sdpa_on_concatenated_heads(o):
+    """torch SDPA on [q | q_r] against [k_h | k_r] (the one rotary key
+    concatenated to every KV head), then the differential and gate."""
+    for window, causal in ((0, True), (5, True), (0, False)):
+        wl, x = _rope_small(seed=41 + window, window=window, causal=causal)
+        dr = x["k_rope"].shape[-1]
+        sc = 1.0 / math.sqrt(wl.d + dr)
+        kr = _f64(x["k_rope"]).unsqueeze(2).expand(-1, -1, wl.Hkv, -1)
+        kcat = torch.cat([_f64(x["k"]), kr], dim=-1)
+        # SDPA takes a value width (d) other than the key width (d + d_rope)
+        hs = _sdpa(torch.cat([_f64(x["q_sig"]), _f64(x["q_rope_sig"])], -1), kcat, x["v"],
+                   wl.Hs // wl.Hkv, window, causal, sc)
+        hn = _sdpa(torch.cat([_f64(x["q_noise"]), _f64(x["q_rope_noise"])], -1), kcat, x["v"],
+                   1, window, causal, sc)
+        g = wl.Hs // wl.Hn
+        dd = hs - _f64(x["lam"]).unsqueeze(-1) * hn.repeat_interleave(g, dim=2)
+        want = (_f64(x["gate"]).view(wl.B, wl.T, wl.Hs, wl.d) * dd).reshape(wl.B * wl.T, -1)
+        _close(_rope_attn(o, x, window=window, causal=causal), want.numpy(), rtol=1e-10,
+               atol=1e-12, what=f"rope vs SDPA (window {window}, causal {causal})")
+
+
+def pin_rope_zero_terms_leave_plain_scores(o):
+    """Zero rotary queries and keys add nothing: with the same scale the
+    result equals the oracle without the rotary term, bit for bit."""
+    wl, x = _rope_small(seed=43)
+    sc = 1.0 / math.sqrt(wl.d)
+    plain = o.gdla_attn(x["q_sig"], x["q_noise"], x["k"], x["v"], x["lam"], x["gate"], scale=sc)
+    for name in ("q_rope_sig", "q_rope_noise", "k_rope"):
+        x[name] = torch.zeros_like(x[name])
+    assert np.array_equal(_rope_attn(o, x, scale=sc), plain)
+
+
+def pin_rope_key_shift_invariance(o):
+    """Adding one vector c to every rotary key adds q_r.c to every score of a
+    row (per head), which the softmax removes: O is unchanged."""
+    wl, x = _rope_small(seed=44, window=4)
+    a = _rope_attn(o, x, window=4)
+    x["k_rope"] = _f64(x["k_rope"]) + torch.linspace(-2, 3, x["k_rope"].shape[-1],
+                                                     dtype=torch.float64)
+    _close(_rope_attn(o, x, window=4), a, rtol=1e-9, atol=1e-12, what="rope shift")
+
+
+def pin_rope_key_is_per_token_not_per_query(o):
+    """Row i's rotary scores use key j's rotary vector: changing the rotary
+    key of one earlier token changes row i, changing a later one does not."""
+    wl, x = _rope_small(B=1, seed=45)
+    a = _rope_attn(o, x)
+    kr = x["k_rope"].clone()
+    kr[0, 3] += 2.0
+    x2 = dict(x, k_rope=kr)
+    b = _rope_attn(o, x2)
+    assert np.array_equal(a[:3], b[:3]), "rows before the changed key must not move"
+    assert not np.allclose(a[10], b[10]), "a later row must see the changed rotary key"
+
+
+def pin_rope_default_scale(o):
+    """The default scale with the rotary term is 1/sqrt(d + d_rope)."""
+    wl, x = _rope_small(seed=46)
+    dr = x["k_rope"].shape[-1]
+    assert np.array_equal(_rope_attn(o, x), _rope_attn(o, x, scale=1 / math.sqrt(wl.d + dr)))
+
+
+def pin_rope_rows_match_full(o):
+    wl, x = _rope_small(seed=47, window=6)
+    rows = np.array([3, 0, 20, 21, 37, 33])
+    full = _rope_attn(o, x, window=6)
+    flat = lambda t: t.reshape(wl.B * wl.T, *t.shape[2:])[torch.as_tensor(rows)]
+    got = o.gdla_attn_rows(flat(x["q_sig"]), flat(x["q_noise"]), x["k"], x["v"], flat(x["lam"]),
+                           flat(x["gate"]), rows, window=6, q_rope_sig_rows=flat(x["q_rope_sig"]),
+                           q_rope_noise_rows=flat(x["q_rope_noise"]), k_rope=x["k_rope"])
+    assert np.array_equal(full[rows], got)
+
+
 # ---------------------------------------------------------------- decode
 # The decode reads the KV latent cache ("Motif 3: Technical Report",
 # paper.rainbus.top, "technical novelty" paragraph: the inference cache is the
@@ -373,6 +499,44 @@ def pin_decode_matches_torch_expand_sdpa(o):
                        x["gate"], rms_w=x["rms_w"], window=window)
         _close(got, _decode_torch(x, lens, window), rtol=1e-10, atol=1e-12,
                what=f"decode vs torch (window {window})")
+
+
+def pin_decode_rope_matches_torch(o):
+    """Decode with the rotary term: the cache holds each token's rotary key
+    beside its latent (as MLA caches it); torch float64 rms_norm, matmul and
+    SDPA on the concatenated [q | q_r] / [k_h | k_r] give the same row."""
+    x, (B, L_max, Hs, Hn, d, dl) = _decode_case(seed=12)
+    dr = 8
+    g_ = torch.Generator().manual_seed(99)
+    qrs = torch.randn(B, Hs, dr, generator=g_).to(torch.bfloat16)
+    qrn = torch.randn(B, Hn, dr, generator=g_).to(torch.bfloat16)
+    kr = torch.randn(B, L_max, dr, generator=g_).to(torch.bfloat16)
+    g = Hs // Hn
+    w = _f64(x["w_kvb"])
+    for window, lens in ((0, [37, 1, 20]), (5, [37, 4, 20])):
+        got = o.decode(x["q_sig"], x["q_noise"], x["c_kv"], lens, x["w_kvb"], x["lam"],
+                       x["gate"], rms_w=x["rms_w"], window=window, q_rope_sig=qrs,
+                       q_rope_noise=qrn, k_rope=kr)
+        for b in range(B):
+            L = lens[b]
+            c = _f64(x["c_kv"][b, :L])
+            chat = F.rms_norm(c, (dl,), weight=_f64(x["rms_w"]), eps=1e-6)
+            kv = (chat @ w).view(L, Hn, 2 * d)
+            lo = max(0, L - window) if window > 0 else 0
+            k = torch.cat([kv[lo:, :, :d], _f64(kr[b, lo:L]).unsqueeze(1).expand(-1, Hn, -1)], -1)
+            v = kv[lo:, :, d:]
+
+            def attend(q, qr, rep):
+                kk = k.repeat_interleave(rep, dim=1).permute(1, 0, 2)
+                vv = v.repeat_interleave(rep, dim=1).permute(1, 0, 2)
+                qq = torch.cat([_f64(q), _f64(qr)], -1).unsqueeze(1)
+                return F.scaled_dot_product_attention(qq, kk, vv,
+                                                      scale=1 / math.sqrt(d + dr)).squeeze(1)
+            hs = attend(x["q_sig"][b], qrs[b], g)
+            hn = attend(x["q_noise"][b], qrn[b], 1)
+            dd = hs - _f64(x["lam"][b]).unsqueeze(1) * hn.repeat_interleave(g, dim=0)
+            want = (_f64(x["gate"][b]).view(Hs, d) * dd).reshape(-1).numpy()
+            _close(got[b], want, rtol=1e-10, atol=1e-12, what=f"rope decode W={window} b={b}")
 
 
 def pin_decode_absorbed_latent_form(o):

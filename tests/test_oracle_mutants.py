@@ -33,6 +33,16 @@ MUTANTS = {
     "rms_sum_not_mean": ("sqrt(ss / (double)d_latent + eps)", "sqrt(ss + eps)"),
     "expand_w_transposed": ("(int64_t)k * ncol + col)", "col * d_latent + k)"),
     "expand_k_v_swapped": ("if (x < dk)\n        k_out", "if (x >= dk)\n        k_out"),
+    "rope_term_dropped": ("        for (int c = 0; c < dr; ++c)\n          dot +=",
+                          "        for (int c = 0; c < 0; ++c)\n          dot +="),
+    "rope_key_of_the_query_token": ("load_elem(kr, kr_dt, (b * T + j) * (int64_t)dr + c);",
+                                    "load_elem(kr, kr_dt, (b * T + i) * (int64_t)dr + c);"),
+    "rope_query_of_head_zero": ("const int64_t qroff = ((q_compact ? ri : row) * H + h)",
+                                "const int64_t qroff = ((q_compact ? ri : row) * H + 0)"),
+    "rope_sign": ("          dot += load_elem(qr, qr_dt, qroff + c) *",
+                  "          dot -= load_elem(qr, qr_dt, qroff + c) *"),
+    "decode_rope_key_of_first_cached_token": ("kr_b = ORACLE_AT(kr, kr_dt, ((int64_t)b * L_max + first) * dr);",
+                                              "kr_b = ORACLE_AT(kr, kr_dt, ((int64_t)b * L_max) * dr);"),
     "decode_query_is_first_token": ("const int64_t row = L - 1;", "const int64_t row = 0;"),
     "decode_window_slice_drops_oldest_key": ("(window > 0 && Lb > window) ? Lb - window : 0",
                                              "(window > 0 && Lb >= window) ? Lb - window + 1 : 0"),
