@@ -53,6 +53,8 @@ STEPS = {
     "long_window": ("long_window",),
     "decode": ("decode",),
     "decode_window": ("decode_window",),
+    "full_rope": ("full_rope",),
+    "window_rope": ("window_rope",),
 }
 # A timed region at least this long runs tensor-bound kernels under the power
 # cap, so their fraction is taken against the sustained bf16 peak.
@@ -81,6 +83,8 @@ def _dist():
 def attn_kernel_name(wl) -> str:
     """The kernel gdla_attn_fwd dispatches this layer to (window >= T is full
     causal; windows of 1..128 keys take the union-row kernel)."""
+    if wl.d_rope:
+        return "gdla_attn_rope_kernel"
     if wl.causal and 0 < wl.window < wl.T:
         return "gdla_attn_win_kernel" if wl.window <= 128 else "gdla_attn_fwd_kernel<window>"
     return "gdla_attn_fwd_kernel"
@@ -224,9 +228,15 @@ class Layer:
             k, v = inp["k"], inp["v"]
         if events is not None:
             events[li][0].record(stream)
-        gdla.gdla_attn_fwd(inp["q_sig"], inp["q_noise"], k, v, inp["lam"], inp["gate"],
-                           window=wl.window, causal=wl.causal, out=out, d_status=status,
-                           stream=stream)
+        if wl.d_rope:
+            gdla.gdla_attn_fwd_rope(inp["q_sig"], inp["q_noise"], inp["q_rope_sig"],
+                                    inp["q_rope_noise"], k, v, inp["k_rope"], inp["lam"],
+                                    inp["gate"], window=wl.window, causal=wl.causal, out=out,
+                                    d_status=status, stream=stream)
+        else:
+            gdla.gdla_attn_fwd(inp["q_sig"], inp["q_noise"], k, v, inp["lam"], inp["gate"],
+                               window=wl.window, causal=wl.causal, out=out, d_status=status,
+                               stream=stream)
         if events is not None:
             events[li][1].record(stream)
 
@@ -524,10 +534,11 @@ def _oracle_sample(wl, x, seconds, rng):
     n_rows = 256 if wl.window > 0 else 8
     total_flops, total_s = 0, 0.0
     cpu = {}
-    for n in ("c_kv", "w_kvb", "k", "v"):
+    for n in ("c_kv", "w_kvb", "k", "v", "k_rope"):
         if n in x:
             t = x[n]
-            cpu[n] = (t[:span] if n == "c_kv" else (t[:1, :span] if n in ("k", "v") else t)).cpu()
+            cpu[n] = (t[:span] if n == "c_kv" else
+                      (t[:1, :span] if n in ("k", "v", "k_rope") else t)).cpu()
     all_rows, all_ref = [], []
     while total_s < seconds:
         t0 = time.perf_counter()
@@ -543,11 +554,15 @@ def _oracle_sample(wl, x, seconds, rng):
         rows = np.sort(rng.integers(0, span, n_rows))
         idx = torch.as_tensor(rows, device=x["q_sig"].device)
         g = lambda t: t[0].index_select(0, idx).cpu()
+        rope = {}
+        if wl.d_rope:
+            rope = dict(q_rope_sig_rows=g(x["q_rope_sig"]), q_rope_noise_rows=g(x["q_rope_noise"]),
+                        k_rope=cpu["k_rope"])
         ref = oracle.gdla_attn_rows(g(x["q_sig"]), g(x["q_noise"]), k, v, g(x["lam"]),
-                                    g(x["gate"]), rows, window=wl.window, causal=wl.causal)
+                                    g(x["gate"]), rows, window=wl.window, causal=wl.causal, **rope)
         for i in rows:
             kept = min(int(i) + 1, wl.window) if wl.window > 0 else int(i) + 1
-            flops += 4 * wl.d * (wl.Hs + wl.Hn) * kept
+            flops += (4 * wl.d + 2 * wl.d_rope) * (wl.Hs + wl.Hn) * kept
         total_s += time.perf_counter() - t0
         total_flops += flops
         all_rows.append(rows)

@@ -32,7 +32,8 @@ GDLA_ERR_TIMEOUT = -5
 # every symbol include/gdla.h declares
 EXPORTED = ("gdla_version", "gdla_status_string", "gdla_kv_expand", "gdla_attn_fwd",
             "gdla_attn_fwd_sp", "gdla_latent_rmsnorm", "gdla_decode_workspace_bytes",
-            "gdla_decode_fwd", "gdla_selftest_wait_timeout", "gdla_decode_fwd_noalloc")
+            "gdla_decode_fwd", "gdla_selftest_wait_timeout", "gdla_decode_fwd_noalloc",
+            "gdla_attn_fwd_rope")
 
 _lib = None
 # One status word per device, used when a caller passes none (see check_status).
@@ -69,6 +70,9 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.gdla_attn_fwd_sp.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i64, i32, i32, i32,
                                      i32, i64, f32, vp, vp]
     lib.gdla_attn_fwd_sp.restype = i32
+    lib.gdla_attn_fwd_rope.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32,
+                                       i32, i32, i32, i64, i32, f32, vp, vp]
+    lib.gdla_attn_fwd_rope.restype = i32
     lib.gdla_latent_rmsnorm.argtypes = [vp, vp, f32, vp, i64, i32, vp, vp]
     lib.gdla_latent_rmsnorm.restype = i32
     lib.gdla_decode_workspace_bytes.argtypes = [i32, i64, i32, i32, i32, i64]
@@ -224,6 +228,53 @@ def gdla_attn_fwd(q_sig: torch.Tensor, q_noise: torch.Tensor, k: torch.Tensor, v
                                       float(scale), ps, _stream_ptr(q_sig.device, stream))
     if rc != GDLA_OK:
         raise GDLAError(rc, "gdla_attn_fwd")
+    if _sync_check_enabled():
+        check_status(q_sig.device, d_status)
+    return out
+
+
+def gdla_attn_fwd_rope(q_sig: torch.Tensor, q_noise: torch.Tensor, q_rope_sig: torch.Tensor,
+                       q_rope_noise: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                       k_rope: torch.Tensor, lam: torch.Tensor, gate: torch.Tensor,
+                       window: int = 0, causal: bool = True, scale: float = 0.0,
+                       out: Optional[torch.Tensor] = None,
+                       d_status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """GDLA attention forward with the decoupled rotary term; returns out
+    [B, T, Hs*d].
+
+    As gdla_attn_fwd, plus q_rope_sig [B,T,Hs,dr], q_rope_noise [B,T,Hn,dr]
+    and k_rope [B,T,dr] (one rotary key per token shared by every head;
+    dr = 64).  scale <= 0 means 1/sqrt(d + dr).
+    """
+    if q_sig.dim() != 4 or k_rope.dim() != 3:
+        raise ValueError("q_sig must be [B, T, Hs, d] and k_rope [B, T, d_rope]")
+    B, T, Hs, d = q_sig.shape
+    Hn = q_noise.shape[2] if q_noise.dim() == 4 else -1
+    Hkv = k.shape[2] if k.dim() == 4 else -1
+    dr = k_rope.shape[2]
+    if out is None:
+        out = torch.empty((B, T, Hs * d), dtype=torch.bfloat16, device=q_sig.device)
+    ptrs = [
+        _check(q_sig, "q_sig"),
+        _check(q_noise, "q_noise", (B, T, Hn, d)),
+        _check(q_rope_sig, "q_rope_sig", (B, T, Hs, dr)),
+        _check(q_rope_noise, "q_rope_noise", (B, T, Hn, dr)),
+        _check(k, "k", (B, T, Hkv, d)),
+        _check(v, "v", (B, T, Hkv, d)),
+        _check(k_rope, "k_rope", (B, T, dr)),
+        _check(lam, "lam", (B, T, Hs)),
+        _check(gate, "gate", (B, T, Hs * d)),
+        _check(out, "out", (B, T, Hs * d)),
+    ]
+    _same_device(q_sig.device, [("q_noise", q_noise), ("q_rope_sig", q_rope_sig),
+                                 ("q_rope_noise", q_rope_noise), ("k", k), ("v", v),
+                                 ("k_rope", k_rope), ("lam", lam), ("gate", gate), ("out", out)])
+    ps = _status_ptr(d_status, q_sig.device)
+    rc = load_library().gdla_attn_fwd_rope(*ptrs, B, T, Hs, Hn, Hkv, d, dr, int(window),
+                                           int(bool(causal)), float(scale), ps,
+                                           _stream_ptr(q_sig.device, stream))
+    if rc != GDLA_OK:
+        raise GDLAError(rc, "gdla_attn_fwd_rope")
     if _sync_check_enabled():
         check_status(q_sig.device, d_status)
     return out

@@ -14,6 +14,7 @@
 
 #include "gdla.h"
 #include "attn_fwd.cuh"
+#include "attn_rope.cuh"
 #include "attn_win.cuh"
 #include "decode.cuh"
 #include "kv_expand.cuh"
@@ -183,6 +184,44 @@ int launch_attn(const void *q_sig, const void *q_noise, const void *k, const voi
   return cudaGetLastError() == cudaSuccess ? GDLA_OK : GDLA_ERR_CUDA;
 }
 
+// The decoupled rotary term: q_rope_* are [B, T, H, kRope], k_rope [B, T, kRope].
+template <int D>
+int launch_attn_rope(const void *q_sig, const void *q_noise, const void *q_rope_sig,
+                     const void *q_rope_noise, const void *k, const void *v, const void *k_rope,
+                     const gdla::AttnParams &prm, int Hs, int Hn, cudaStream_t stream) {
+  using L = gdla::RopeSmemLayout<D>;
+  CUtensorMap tm_qs, tm_qn, tm_qrs, tm_qrn, tm_k, tm_kr, tm_v;
+  const uint64_t T = static_cast<uint64_t>(prm.T), B = static_cast<uint64_t>(prm.B);
+  const uint64_t dqs[3] = {static_cast<uint64_t>(Hs) * D, T, B};
+  const uint64_t dqn[3] = {static_cast<uint64_t>(Hn) * D, T, B};
+  const uint64_t dqrs[3] = {static_cast<uint64_t>(Hs) * gdla::kRope, T, B};
+  const uint64_t dqrn[3] = {static_cast<uint64_t>(Hn) * gdla::kRope, T, B};
+  const uint64_t dkv[3] = {static_cast<uint64_t>(Hn) * D, T, B};
+  const uint64_t dkr[3] = {static_cast<uint64_t>(gdla::kRope), T, B};
+  const uint32_t box[3] = {64, gdla::kBM, 1};
+  if (!make_map(&tm_qs, q_sig, 3, dqs, box) || !make_map(&tm_qn, q_noise, 3, dqn, box) ||
+      !make_map(&tm_qrs, q_rope_sig, 3, dqrs, box) ||
+      !make_map(&tm_qrn, q_rope_noise, 3, dqrn, box) || !make_map(&tm_k, k, 3, dkv, box) ||
+      !make_map(&tm_kr, k_rope, 3, dkr, box) || !make_map(&tm_v, v, 3, dkv, box))
+    return GDLA_ERR_CUDA;
+  const uint64_t items = static_cast<uint64_t>(prm.n_qblk) * B * static_cast<uint64_t>(Hn);
+  if (items > 0x7fffffffull) return GDLA_ERR_UNSUPPORTED;
+  gdla::AttnParams run = prm;
+  run.n_items = static_cast<int>(items);
+  uint64_t grid = items;
+  if (prm.window > 0) {
+    int sms = 0;
+    if (sm_count(&sms) != GDLA_OK) return GDLA_ERR_CUDA;
+    if (grid > static_cast<uint64_t>(sms)) grid = static_cast<uint64_t>(sms);
+  }
+  constexpr auto kern = gdla::gdla_attn_rope_kernel<D>;
+  const int rc = prepare_kernel<kern>(L::kBytes, 0);
+  if (rc != GDLA_OK) return rc;
+  kern<<<static_cast<unsigned>(grid), gdla::kRopeThreads, L::kBytes, stream>>>(
+      tm_qs, tm_qn, tm_qrs, tm_qrn, tm_k, tm_kr, tm_v, run);
+  return cudaGetLastError() == cudaSuccess ? GDLA_OK : GDLA_ERR_CUDA;
+}
+
 template <int DH>
 int launch_expand(const void *c_kv, const void *w_kvb, const gdla::ExpandParams &prm,
                   cudaStream_t stream) {
@@ -310,11 +349,15 @@ int gdla_kv_expand(const void *c_kv, const void *rms_w, const void *w_kvb, float
 
 namespace {
 
+// q_rope_sig, q_rope_noise and k_rope are read only when d_rope > 0.
 int attn_fwd_impl(const void *q_sig, const void *q_noise, const void *k, const void *v,
                   const void *lambda, const void *gate, void *out, int B, int64_t T,
                   int64_t kv_prefix, int Hs, int Hn, int Hkv, int d, int64_t window, int causal,
-                  float scale, int *d_status, void *stream) {
+                  float scale, int *d_status, void *stream, const void *q_rope_sig = nullptr,
+                  const void *q_rope_noise = nullptr, const void *k_rope = nullptr,
+                  int d_rope = 0) {
   if (B < 0 || T < 0 || Hs <= 0 || Hn <= 0 || Hkv <= 0 || d <= 0) return GDLA_ERR_INVALID_ARG;
+  if (d_rope < 0 || (d_rope > 0 && kv_prefix != 0)) return GDLA_ERR_INVALID_ARG;
   if (window < 0 || (causal != 0 && causal != 1) || (causal == 0 && window > 0))
     return GDLA_ERR_INVALID_ARG;
   // a shard's halo: one K/V tile, only for windows of at most one tile
@@ -324,8 +367,12 @@ int attn_fwd_impl(const void *q_sig, const void *q_noise, const void *k, const v
   if (std::isnan(scale) || std::isinf(scale)) return GDLA_ERR_INVALID_ARG;
   if (B == 0 || T == 0) return GDLA_OK;
   if (!q_sig || !q_noise || !k || !v || !lambda || !gate || !out) return GDLA_ERR_INVALID_ARG;
+  if (d_rope > 0 && (!q_rope_sig || !q_rope_noise || !k_rope)) return GDLA_ERR_INVALID_ARG;
   if (Hn != Hkv || Hs % Hn != 0) return GDLA_ERR_UNSUPPORTED;
   if (d != 64 && d != 128) return GDLA_ERR_UNSUPPORTED;
+  if (d_rope != 0 && d_rope != gdla::kRope) return GDLA_ERR_UNSUPPORTED;
+  if (d_rope > 0 && (!aligned16(q_rope_sig) || !aligned16(q_rope_noise) || !aligned16(k_rope)))
+    return GDLA_ERR_ALIGNMENT;
   if (T + kv_prefix > 0x7fffffffll - gdla::kBM) return GDLA_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(Hs) * d > 0x7fffffffll) return GDLA_ERR_UNSUPPORTED;
   if (!aligned16(q_sig) || !aligned16(q_noise) || !aligned16(k) || !aligned16(v) ||
@@ -358,9 +405,14 @@ int attn_fwd_impl(const void *q_sig, const void *q_noise, const void *k, const v
     prm.band = static_cast<int>(band);
   }
   prm.causal = causal;
-  const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(d));
+  const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(d + d_rope));
   prm.scale_log2 = sc * 1.4426950408889634f;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d_rope > 0)
+    return d == 128 ? launch_attn_rope<128>(q_sig, q_noise, q_rope_sig, q_rope_noise, k, v,
+                                            k_rope, prm, Hs, Hn, s)
+                    : launch_attn_rope<64>(q_sig, q_noise, q_rope_sig, q_rope_noise, k, v,
+                                           k_rope, prm, Hs, Hn, s);
   return d == 128 ? launch_attn<128>(q_sig, q_noise, k, v, prm, Hs, Hn, s)
                   : launch_attn<64>(q_sig, q_noise, k, v, prm, Hs, Hn, s);
 }
@@ -384,6 +436,15 @@ int gdla_attn_fwd_sp(const void *q_sig, const void *q_noise, const void *k, cons
   if (window <= 0 || window > gdla::kBN) return GDLA_ERR_INVALID_ARG;
   return attn_fwd_impl(q_sig, q_noise, k, v, lambda, gate, out, B, T, kv_prefix, Hs, Hn, Hkv, d,
                        window, 1, scale, d_status, stream);
+}
+
+int gdla_attn_fwd_rope(const void *q_sig, const void *q_noise, const void *q_rope_sig,
+                       const void *q_rope_noise, const void *k, const void *v,
+                       const void *k_rope, const void *lambda, const void *gate, void *out, int B,
+                       int64_t T, int Hs, int Hn, int Hkv, int d, int d_rope, int64_t window,
+                       int causal, float scale, int *d_status, void *stream) {
+  return attn_fwd_impl(q_sig, q_noise, k, v, lambda, gate, out, B, T, 0, Hs, Hn, Hkv, d, window,
+                       causal, scale, d_status, stream, q_rope_sig, q_rope_noise, k_rope, d_rope);
 }
 
 size_t gdla_decode_workspace_bytes(int B, int64_t L_max, int Hs, int Hn, int d_latent,

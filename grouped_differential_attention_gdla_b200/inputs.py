@@ -15,6 +15,10 @@ c_KV [B, T, 512] and W^KV_b in that order):
   gate   = bf16(sigmoid(N(0, 1)))  shape [B, T, Hs*d]
   c_KV   ~ N(0, 1) bf16            shape [B*T, 512]      (latent workload)
   W^KV_b ~ N(0, 1/512) bf16        shape [512, Hkv*(dk+dv)]
+and, for workloads with the decoupled rotary term (d_rope > 0), drawn after
+everything above so the other inputs do not change:
+  Q_rope_sig, Q_rope_noise ~ N(0, 1) bf16  shape [B, T, H, d_rope]
+  K_rope                   ~ N(0, 1) bf16  shape [B, T, d_rope]
 The same seed on a different device gives a different (but again fixed)
 stream; tests that compare against the oracle copy the device draw to the host.
 
@@ -46,6 +50,7 @@ class Workload:
     d_latent: int = 512
     eps: float = 1e-6
     decode: bool = False     # one query token per sequence over a T-token latent cache
+    d_rope: int = 0          # width of the decoupled rotary term (0: none)
 
     @property
     def g(self) -> int:
@@ -64,8 +69,10 @@ class Workload:
         return W * (W + 1) // 2 + (T - W) * W
 
     def attn_flops(self) -> int:
-        """4*d FLOPs per kept pair per query head (QK^T and PV), all heads."""
-        return 4 * self.d * (self.Hs + self.Hn) * self.B * self.pairs_per_batch()
+        """2*(d + d_rope) + 2*d FLOPs per kept pair per query head (QK^T with
+        the rotary term, and PV), all heads."""
+        per_pair = 2 * (self.d + self.d_rope) + 2 * self.d
+        return per_pair * (self.Hs + self.Hn) * self.B * self.pairs_per_batch()
 
     def decode_bytes(self) -> int:
         """The kept cache rows read once, W^KV_b, the query-side inputs and
@@ -77,7 +84,8 @@ class Workload:
     def attn_bytes(self) -> int:
         """Inputs read once plus output written once, bfloat16 everywhere."""
         per_tok = 2 * (self.Hs * self.d + self.Hn * self.d + 2 * self.Hkv * self.d
-                       + self.Hs + 2 * self.Hs * self.d)
+                       + self.Hs + 2 * self.Hs * self.d
+                       + (self.Hs + self.Hn + 1) * self.d_rope)
         return per_tok * self.B * self.T
 
     def expand_flops(self) -> int:
@@ -100,6 +108,10 @@ WORKLOADS: Dict[str, Workload] = {
     # of the long-context schedule), every key or the 128-token window
     "decode": Workload("decode", B=64, T=32768, decode=True),
     "decode_window": Workload("decode_window", B=64, T=32768, window=128, decode=True),
+    # the two attention layers with the decoupled rotary term (64 wide, the
+    # width that keeps the latent cache the size of MLA's: 512 + 64)
+    "full_rope": Workload("full_rope", B=2, T=8192, d_rope=64),
+    "window_rope": Workload("window_rope", B=8, T=4096, window=128, d_rope=64),
 }
 
 
@@ -150,11 +162,16 @@ def make_inputs(wl: Workload, seed: int = 0, device="cpu",
         out["c_kv"] = _normal_bf16((B * T, wl.d_latent), gen, device)
         out["w_kvb"] = _normal_bf16((wl.d_latent, wl.Hkv * 2 * wl.d), gen, device,
                                     std=(1.0 / wl.d_latent) ** 0.5)
+    if wl.d_rope:
+        out["q_rope_sig"] = _normal_bf16((B, T, wl.Hs, wl.d_rope), gen, device)
+        out["q_rope_noise"] = _normal_bf16((B, T, wl.Hn, wl.d_rope), gen, device)
+        out["k_rope"] = _normal_bf16((B, T, wl.d_rope), gen, device)
     return out
 
 
 def custom(B: int, T: int, Hs: int, Hn: int, Hkv: int, d: int, window: int = 0,
-           causal: bool = True, latent: bool = False, name: str = "custom") -> Workload:
+           causal: bool = True, latent: bool = False, name: str = "custom",
+           d_rope: int = 0) -> Workload:
     """A workload with arbitrary shapes (edge-case tests)."""
     return Workload(name, B=B, T=T, Hs=Hs, Hn=Hn, Hkv=Hkv, d=d, window=window,
-                    causal=causal, latent=latent)
+                    causal=causal, latent=latent, d_rope=d_rope)

@@ -121,6 +121,36 @@ int gdla_attn_fwd(const void *q_sig, const void *q_noise, const void *k,
                   void *stream);
 
 /*
+ * gdla_attn_fwd_rope - gdla_attn_fwd with the decoupled rotary term in the
+ * score ("Motif 3: Technical Report", paper.rainbus.top, "technical novelty"
+ * paragraph: both query paths share the up-projected KV and one broadcast
+ * decoupled rotary key):
+ *
+ *   s_ij = scale * (q_i . k_j + q_rope_i . k_rope_j)
+ *
+ * Every head of both paths has its own rotary query; every token has one
+ * rotary key that all heads share.  The rotation by position is applied
+ * before this call (q_rope and k_rope arrive rotated), as lambda and the gate
+ * arrive after their sigmoids.
+ *
+ * q_sig, q_noise, k, v, lambda, gate, out   as in gdla_attn_fwd
+ * q_rope_sig    [B, T, Hs, d_rope]   bf16, read
+ * q_rope_noise  [B, T, Hn, d_rope]   bf16, read
+ * k_rope        [B, T, d_rope]       bf16, read
+ * d_rope        64, or 0 (the rotary pointers are then ignored and the call is
+ *               gdla_attn_fwd); other widths give GDLA_ERR_UNSUPPORTED
+ * scale         <= 0 selects 1/sqrt(d + d_rope)
+ * Same masks, shapes, alignment and errors as gdla_attn_fwd.
+ */
+int gdla_attn_fwd_rope(const void *q_sig, const void *q_noise,
+                       const void *q_rope_sig, const void *q_rope_noise,
+                       const void *k, const void *v, const void *k_rope,
+                       const void *lambda, const void *gate, void *out, int B,
+                       int64_t T, int Hs, int Hn, int Hkv, int d, int d_rope,
+                       int64_t window, int causal, float scale, int *d_status,
+                       void *stream);
+
+/*
  * gdla_attn_fwd_sp - gdla_attn_fwd with a sliding window on one shard of a
  * sequence split across GPUs ("Motif 3: Technical Report", paper.rainbus.top:
  * its long-context training step and "technical novelty" paragraph describe

@@ -36,7 +36,8 @@ def test_exports_every_declared_symbol(lib):
     assert set(declared) == {"gdla_version", "gdla_status_string", "gdla_kv_expand",
                              "gdla_attn_fwd", "gdla_attn_fwd_sp", "gdla_latent_rmsnorm",
                              "gdla_decode_workspace_bytes", "gdla_decode_fwd",
-                             "gdla_selftest_wait_timeout", "gdla_decode_fwd_noalloc"}
+                             "gdla_selftest_wait_timeout", "gdla_decode_fwd_noalloc",
+                             "gdla_attn_fwd_rope"}
     for name in declared:
         assert hasattr(lib, name), f"{name} missing from libgdla.so"
     assert set(declared) == set(_binding.EXPORTED)
@@ -73,6 +74,28 @@ def _attn(lib, q=A, qn=A, k=A, v=A, lam=A, gate=A, out=A, B=1, T=256, Hs=8, Hn=2
 ])
 def test_attn_argument_errors(lib, kw, code):
     assert _attn(lib, **kw) == code
+
+
+def _rope(lib, q=A, qn=A, qr=A, qrn=A, k=A, v=A, kr=A, lam=A, gate=A, out=A, B=1, T=256, Hs=8,
+          Hn=2, Hkv=2, d=64, dr=64, window=0, causal=1, scale=0.0, status=None):
+    return lib.gdla_attn_fwd_rope(q, qn, qr, qrn, k, v, kr, lam, gate, out, B, T, Hs, Hn, Hkv, d,
+                                  dr, window, causal, ctypes.c_float(scale), status, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(qr=None), INVALID), (dict(qrn=None), INVALID), (dict(kr=None), INVALID),
+    (dict(q=None), INVALID), (dict(dr=-64), INVALID), (dict(causal=0, window=3), INVALID),
+    (dict(dr=32), UNSUPPORTED), (dict(dr=128), UNSUPPORTED), (dict(d=96), UNSUPPORTED),
+    (dict(Hn=2, Hkv=4), UNSUPPORTED),
+    (dict(qr=M), ALIGN), (dict(qrn=M), ALIGN), (dict(kr=M), ALIGN), (dict(q=M), ALIGN),
+    (dict(status=0x100002), ALIGN),
+    (dict(T=0), OK), (dict(B=0), OK),
+    # d_rope = 0 ignores the rotary pointers and validates like gdla_attn_fwd
+    (dict(dr=0, qr=None, qrn=None, kr=None, out=None), INVALID),
+    (dict(dr=0, qr=None, qrn=None, kr=None, B=0), OK),
+])
+def test_rope_argument_errors(lib, kw, code):
+    assert _rope(lib, **kw) == code
 
 
 def _expand(lib, c=A, w=None, wk=A, eps=1e-6, k=A, v=A, n=300, dl=512, hkv=16, dh=128,
