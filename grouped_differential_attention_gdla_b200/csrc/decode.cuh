@@ -31,6 +31,7 @@ constexpr int kDecRing = 3;     // ring depth (units of [128 tokens][128 latent]
 constexpr int kDecThreads = 192;  // warps 0-3 softmax / partials, 4 TMA, 5 MMA
 constexpr int kDecMaxLatent = 512;
 constexpr int kDecMaxGroup = 8;   // signal heads per KV group in the decode kernels
+constexpr int kDecMaxSplit = 256;  // splits per sequence (the host plan stays below)
 constexpr float kDecRescale = 8.0f;  // log2 units: a head's reference moves only past 2^8
 
 struct DecodeParams {
@@ -76,30 +77,72 @@ __device__ __forceinline__ float *decode_part(const DecodeParams &p, int b, int 
 }
 
 // ---------------------------------------------------------------- absorb
-// One CTA per (KV group k, sequence b): q~ rows of the group's heads (signal
-// heads h -> row h, noise head k -> row Hs + k), q~[x] = qscale * sum_c
-// W^KV_b[x, k*2d + c] q[c].  Rows Hs + Hn .. Np - 1 are zero padding.
-__global__ void __launch_bounds__(256) gdla_decode_absorb_kernel(const DecodeParams p) {
-  const int k = blockIdx.x, b = blockIdx.y;
+// q~ rows of KV group k (signal heads h -> row h, noise head k -> row Hs + k),
+// q~[x] = qscale * sum_c W^KV_b[x, k*2d + c] q[c]; rows Hs + Hn .. Np - 1 are
+// zero padding.  One CTA per (group k, block of 128 latent rows x, block of
+// kAbsorbSeqs sequences); thread x keeps its row of W_K in registers and
+// takes every query vector of the block's sequences from shared memory
+// (a broadcast read), so no chain waits on a global load.
+constexpr int kAbsorbSeqs = 2;
+__global__ void __launch_bounds__(128) gdla_decode_absorb_kernel(const DecodeParams p) {
+  const int k = blockIdx.x;
+  const int x = blockIdx.y * 128 + threadIdx.x;  // latent row
+  const int b0 = blockIdx.z * kAbsorbSeqs;
   const int g = p.Hs / p.Hn, nh = g + 1, d = p.d, dl = p.dl;
-  __shared__ float qs[(kDecMaxGroup + 1) * 128];
-  for (int i = threadIdx.x; i < nh * d; i += blockDim.x) {
-    const int j = i / d, c = i % d;
+  const int nb = min(kAbsorbSeqs, p.B - b0);
+  // query vectors [sequence][head of the group][d] as bf16 pairs
+  __shared__ __align__(16) uint32_t qs[kAbsorbSeqs * (kDecMaxGroup + 1) * 64];
+  // 16-byte pieces: d / 8 per query vector
+  const int pieces = d / 8;
+  for (int i = threadIdx.x; i < nb * nh * pieces; i += blockDim.x) {
+    const int bb = i / (nh * pieces), j = (i / pieces) % nh, v = i % pieces;
+    const int b = b0 + bb;
     const __nv_bfloat16 *src =
         j < g ? p.q_sig + (static_cast<int64_t>(b) * p.Hs + g * k + j) * d
               : p.q_noise + (static_cast<int64_t>(b) * p.Hn + k) * d;
-    qs[i] = __bfloat162float(src[c]);
+    reinterpret_cast<uint4 *>(qs + (bb * (kDecMaxGroup + 1) + j) * 64)[v] =
+        __ldg(reinterpret_cast<const uint4 *>(src) + v);
   }
   __syncthreads();
+  if (x >= dl) return;
+  // W_K row x of group k: d contiguous bf16 (16-byte aligned: 2d divides the row stride)
   const int64_t ldw = static_cast<int64_t>(p.Hn) * 2 * d;
-  __nv_bfloat16 *qt = p.qt + static_cast<int64_t>(b) * p.Np * dl;
-  for (int x = threadIdx.x; x < dl; x += blockDim.x) {
-    const __nv_bfloat16 *wr = p.w_kvb + x * ldw + static_cast<int64_t>(k) * 2 * d;
+  const uint4 *wr = reinterpret_cast<const uint4 *>(p.w_kvb + x * ldw + static_cast<int64_t>(k) * 2 * d);
+  uint32_t w[64];
+#pragma unroll
+  for (int v = 0; v < 16; ++v) {
+    if (v < d / 8) {
+      const uint4 t = __ldg(wr + v);
+      w[4 * v] = t.x;
+      w[4 * v + 1] = t.y;
+      w[4 * v + 2] = t.z;
+      w[4 * v + 3] = t.w;
+    } else {
+      w[4 * v] = w[4 * v + 1] = w[4 * v + 2] = w[4 * v + 3] = 0u;
+    }
+  }
+  for (int bb = 0; bb < nb; ++bb) {
+    const int64_t b = b0 + bb;
+    __nv_bfloat16 *qt = p.qt + b * p.Np * dl;
     for (int j = 0; j < nh; ++j) {
-      float acc = 0.f;
-      for (int c = 0; c < d; ++c) acc = fmaf(__bfloat162float(wr[c]), qs[j * d + c], acc);
+      const uint4 *q4 = reinterpret_cast<const uint4 *>(qs + (bb * (kDecMaxGroup + 1) + j) * 64);
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+      for (int v = 0; v < 16; ++v) {
+        if (v < d / 8) {
+          const uint4 q = q4[v];
+          a0 = fmaf(bf16lo_to_f32(w[4 * v]), bf16lo_to_f32(q.x), a0);
+          a1 = fmaf(bf16hi_to_f32(w[4 * v]), bf16hi_to_f32(q.x), a1);
+          a2 = fmaf(bf16lo_to_f32(w[4 * v + 1]), bf16lo_to_f32(q.y), a2);
+          a3 = fmaf(bf16hi_to_f32(w[4 * v + 1]), bf16hi_to_f32(q.y), a3);
+          a0 = fmaf(bf16lo_to_f32(w[4 * v + 2]), bf16lo_to_f32(q.z), a0);
+          a1 = fmaf(bf16hi_to_f32(w[4 * v + 2]), bf16hi_to_f32(q.z), a1);
+          a2 = fmaf(bf16lo_to_f32(w[4 * v + 3]), bf16lo_to_f32(q.w), a2);
+          a3 = fmaf(bf16hi_to_f32(w[4 * v + 3]), bf16hi_to_f32(q.w), a3);
+        }
+      }
       const int row = j < g ? g * k + j : p.Hs + k;
-      qt[static_cast<int64_t>(row) * dl + x] = __float2bfloat16(acc * p.qscale);
+      qt[static_cast<int64_t>(row) * dl + x] = __float2bfloat16(((a0 + a1) + (a2 + a3)) * p.qscale);
     }
     if (k == 0)
       for (int row = p.Hs + p.Hn; row < p.Np; ++row)
@@ -457,25 +500,64 @@ __global__ void __launch_bounds__(128) gdla_decode_combine_kernel(const DecodePa
   const int g = p.Hs / p.Hn, nh = g + 1, d = p.d, dl = p.dl;
   __shared__ float zs[(kDecMaxGroup + 1) * kDecMaxLatent];
   __shared__ float hsm[(kDecMaxGroup + 1) * 128];
-  for (int j = 0; j < nh; ++j) {
+  __shared__ float wsp[(kDecMaxGroup + 1) * kDecMaxSplit];  // weight of split s for head j
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // one warp per head row: M = max_s m_s, l = sum_s 2^(m_s - M) l_s, and the
+  // weight 2^(m_s - M) / l of every split (0 for a split that saw no key)
+  for (int j = warp; j < nh; j += 4) {
     const int row = j < g ? g * k + j : p.Hs + k;
     float M = -INFINITY;
-    for (int sp = 0; sp < p.n_split; ++sp) M = fmaxf(M, decode_part(p, b, sp)[row]);
+    for (int sp = lane; sp < p.n_split; sp += 32) M = fmaxf(M, decode_part(p, b, sp)[row]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float l = 0.f;
-    for (int sp = 0; sp < p.n_split; ++sp) {
+    for (int sp = lane; sp < p.n_split; sp += 32) {
       const float *pp = decode_part(p, b, sp);
-      if (pp[row] != -INFINITY) l += exp2f(pp[row] - M) * pp[p.Np + row];
+      const float e = pp[row] == -INFINITY ? 0.f : exp2f(pp[row] - M);
+      wsp[j * kDecMaxSplit + sp] = e;
+      l += e * pp[p.Np + row];
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
     const float inv_l = l > 0.f ? 1.f / l : 0.f;
-    for (int x = threadIdx.x; x < dl; x += blockDim.x) {
-      float acc = 0.f;
-      for (int sp = 0; sp < p.n_split; ++sp) {
-        const float *pp = decode_part(p, b, sp);
-        if (pp[row] != -INFINITY)
-          acc = fmaf(exp2f(pp[row] - M), pp[2 * p.Np + static_cast<size_t>(row) * dl + x], acc);
+    __syncwarp();
+    for (int sp = lane; sp < p.n_split; sp += 32) wsp[j * kDecMaxSplit + sp] *= inv_l;
+  }
+  __syncthreads();
+  // z = sum_s weight_s z_s for the group's heads.  Thread t owns latent
+  // columns t, t + 128, ... (dl / 128 of them); per split it issues the loads
+  // of every head and column it owns at once.
+  {
+    const int nx = dl / 128;
+    float acc[kDecMaxGroup + 1][kDecMaxLatent / 128];
+#pragma unroll
+    for (int j = 0; j < kDecMaxGroup + 1; ++j)
+#pragma unroll
+      for (int xi = 0; xi < kDecMaxLatent / 128; ++xi) acc[j][xi] = 0.f;
+    for (int sp = 0; sp < p.n_split; ++sp) {
+      const float *zp = decode_part(p, b, sp) + 2 * p.Np;
+      float z[kDecMaxGroup + 1][kDecMaxLatent / 128];
+#pragma unroll
+      for (int j = 0; j < kDecMaxGroup + 1; ++j) {
+        const int row = j < g ? g * k + j : p.Hs + k;
+#pragma unroll
+        for (int xi = 0; xi < kDecMaxLatent / 128; ++xi)
+          z[j][xi] = (j < nh && xi < nx)
+                         ? zp[static_cast<size_t>(row) * dl + xi * 128 + threadIdx.x]
+                         : 0.f;
       }
-      zs[j * dl + x] = acc * inv_l;
+#pragma unroll
+      for (int j = 0; j < kDecMaxGroup + 1; ++j) {
+        const float wgt = j < nh ? wsp[j * kDecMaxSplit + sp] : 0.f;
+#pragma unroll
+        for (int xi = 0; xi < kDecMaxLatent / 128; ++xi) acc[j][xi] = fmaf(wgt, z[j][xi], acc[j][xi]);
+      }
     }
+#pragma unroll
+    for (int j = 0; j < kDecMaxGroup + 1; ++j)
+#pragma unroll
+      for (int xi = 0; xi < kDecMaxLatent / 128; ++xi)
+        if (j < nh && xi < nx) zs[j * dl + xi * 128 + threadIdx.x] = acc[j][xi];
   }
   __syncthreads();
   const int64_t ldw = static_cast<int64_t>(p.Hn) * 2 * d;
@@ -484,11 +566,16 @@ __global__ void __launch_bounds__(128) gdla_decode_combine_kernel(const DecodePa
 #pragma unroll
     for (int j = 0; j < kDecMaxGroup + 1; ++j) acc[j] = 0.f;
     const __nv_bfloat16 *wv = p.w_kvb + static_cast<int64_t>(k) * 2 * d + d + c;
-    for (int x = 0; x < dl; ++x) {
-      const float wx = __bfloat162float(wv[x * ldw]);
+    // 32 loads in flight per batch of latent rows (dl is a multiple of 128)
+    for (int x0 = 0; x0 < dl; x0 += 32) {
+      float wx[32];
 #pragma unroll
-      for (int j = 0; j < kDecMaxGroup + 1; ++j)
-        if (j < nh) acc[j] = fmaf(zs[j * dl + x], wx, acc[j]);
+      for (int u = 0; u < 32; ++u) wx[u] = __bfloat162float(wv[(x0 + u) * ldw]);
+#pragma unroll
+      for (int u = 0; u < 32; ++u)
+#pragma unroll
+        for (int j = 0; j < kDecMaxGroup + 1; ++j)
+          if (j < nh) acc[j] = fmaf(zs[j * dl + x0 + u], wx[u], acc[j]);
     }
 #pragma unroll
     for (int j = 0; j < kDecMaxGroup + 1; ++j)

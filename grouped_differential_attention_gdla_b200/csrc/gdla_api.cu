@@ -245,12 +245,15 @@ int launch_expand(const void *c_kv, const void *w_kvb, const gdla::ExpandParams 
 
 // ---------------------------------------------------------------- decode
 // Work split of the decode: each CTA of the attention kernel takes `cps`
-// chunks of 128 cached tokens of one sequence, enough of them that the grid
-// is about two CTAs per SM of a B200 and that each CTA's partial result
-// (Np * (d_latent + 2) floats) is small next to the cache it reads.  The
-// split depends on the shapes only, so the workspace size does too.
-constexpr int64_t kDecodeTargetCtas = 296;
+// chunks of 128 cached tokens of one sequence.  One CTA fits an SM (it holds
+// all of TMEM), so the grid runs in waves of 148 CTAs on a B200; the split
+// minimises waves * (cps + kDecodeCtaOverhead), the second term standing for
+// what every CTA pays besides its chunks (loading q~, filling the pipeline,
+// writing its partial result of Np * (d_latent + 2) floats), in chunk units.
+// The split depends on the shapes only, so the workspace size does too.
+constexpr int64_t kDecodeSms = 148;
 constexpr int64_t kDecodeMinChunks = 4;
+constexpr int64_t kDecodeCtaOverhead = 3;
 
 struct DecodePlan {
   int Np, cps, n_split;
@@ -267,10 +270,21 @@ bool decode_plan(int B, int64_t L_max, int Hs, int Hn, int d_latent, int64_t win
     const int64_t w = (window + gdla::kDecTok - 2) / gdla::kDecTok + 1;
     if (w < chunks) chunks = w;
   }
-  int64_t cps = (static_cast<int64_t>(B) * chunks + kDecodeTargetCtas - 1) / kDecodeTargetCtas;
-  if (cps < kDecodeMinChunks) cps = kDecodeMinChunks;
+  int64_t cps = chunks, best = -1;
+  int64_t max_split = 8 * kDecodeSms / B + 1;
+  if (max_split > gdla::kDecMaxSplit) max_split = gdla::kDecMaxSplit;
+  for (int64_t ns = 1; ns <= chunks && ns <= max_split; ++ns) {
+    int64_t c = (chunks + ns - 1) / ns;
+    if (c < kDecodeMinChunks) c = kDecodeMinChunks;
+    const int64_t ctas = static_cast<int64_t>(B) * ((chunks + c - 1) / c);
+    const int64_t cost = (ctas + kDecodeSms - 1) / kDecodeSms * (c + kDecodeCtaOverhead);
+    if (best < 0 || cost < best) {
+      best = cost;
+      cps = c;
+    }
+  }
   const int64_t n_split = (chunks + cps - 1) / cps;
-  if (np > 256 || n_split > 0x7fffffffll || cps > 0x7fffffffll) return false;
+  if (np > 256 || n_split > gdla::kDecMaxSplit || cps > 0x7fffffffll) return false;
   pl->Np = static_cast<int>(np);
   pl->cps = static_cast<int>(cps);
   pl->n_split = static_cast<int>(n_split);
@@ -503,8 +517,11 @@ int gdla_decode_fwd(const void *q_sig, const void *q_noise, const void *c_hat,
   const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(d));
   prm.qscale = sc * 1.4426950408889634f;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  gdla::gdla_decode_absorb_kernel<<<dim3(static_cast<unsigned>(Hn), static_cast<unsigned>(B)),
-                                    256, 0, s>>>(prm);
+  gdla::gdla_decode_absorb_kernel<<<dim3(static_cast<unsigned>(Hn),
+                                         static_cast<unsigned>(d_latent / gdla::kDecUnit),
+                                         static_cast<unsigned>((B + gdla::kAbsorbSeqs - 1) /
+                                                               gdla::kAbsorbSeqs)),
+                                    128, 0, s>>>(prm);
   if (cudaGetLastError() != cudaSuccess) return GDLA_ERR_CUDA;
   const int rc = pl.Np == 80 ? launch_decode_attn<80>(prm, c_hat, s)
                              : launch_decode_attn<16>(prm, c_hat, s);

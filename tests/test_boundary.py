@@ -190,8 +190,9 @@ def test_decode_argument_errors(lib, kw, code):
 
 def test_decode_workspace_size_follows_the_shapes(lib):
     f = lib.gdla_decode_workspace_bytes
-    # 64 sequences x 32768 tokens, 64 + 16 heads: 56 chunks per split, 5 splits
-    assert f(64, 32768, 64, 16, 512, 0) == 64 * 80 * 512 * 2 + 64 * 5 * 80 * 514 * 4
+    # 64 sequences x 32768 tokens (256 chunks each), 64 + 16 heads: 9 splits of
+    # 29 chunks, 576 CTAs, the fewest waves x (chunks + 3) on 148 SMs
+    assert f(64, 32768, 64, 16, 512, 0) == 64 * 80 * 512 * 2 + 64 * 9 * 80 * 514 * 4
     # a 128-token window touches at most 2 chunks: one split per sequence
     assert f(64, 32768, 64, 16, 512, 128) == 64 * 80 * 512 * 2 + 64 * 1 * 80 * 514 * 4
     assert f(1, 100, 8, 2, 512, 0) == 16 * 512 * 2 + 1 * 1 * 16 * 514 * 4
