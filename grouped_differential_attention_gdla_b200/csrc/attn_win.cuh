@@ -22,28 +22,29 @@
 // K_E, K_G, V_E, V_G stay in shared memory for the item's g+1 heads; query
 // tiles stream through a two-deep ring.
 //
-// Softmax: each warp owns 32 rows, so of the four 32-column union chunks the
-// warp's own chunk (columns 32w .. 32w+31) mixes both tiles and the other
-// three each come whole from one tile (G left of it, E right of it).  A warp
-// reads its whole union row with two TMEM round trips (the mixed chunk from
-// both tiles, then the three whole chunks), takes the row max and writes P
-// in one pass, with no running-max rescale (a head is one tile).
+// Softmax: two warpgroups share every row, each taking two of the four
+// 32-column union chunks.  Warp quarter qw owns rows 32qw .. 32qw+31, so its
+// chunk qw mixes both tiles and the other chunks each come whole from one
+// tile (G left of it, E right of it).  A warp reads its two chunks in one
+// TMEM round trip; the two halves of a row agree on the (integral) reference
+// maximum through shared memory and an mbarrier per pair of warps, then each
+// writes P for its columns in one pass, with no running-max rescale (a head
+// is one tile).  Each half hands its partial row sum to the epilogue.
 //
 // Epilogue: the noise head's H_N = O / l stays in TMEM next to O.  For a
-// signal head the epilogue reads O and H_N into registers as
-// D = O/l - lambda H_N (fp32) and releases O at once, so the next head's PV
-// never waits for the gate; it then multiplies by the gate tile, which a
-// dedicated TMA warp streams through a 128B-swizzled staging buffer (loaded
-// as soon as the previous output tile's store has read the buffer) and
-// stores back as the output tile.
+// signal head the epilogue combines O and H_N with lambda and the gate tile,
+// which a dedicated TMA warp streams through a 128B-swizzled staging buffer
+// (loaded as soon as the previous output tile's store has read the buffer),
+// writes the output over the gate tile in place and releases O.
 //
-// Warp roles (384 threads; registers re-split with setmaxnreg):
-//   warps 0-3   softmax (TMEM lanes 0..127)                         176 regs
-//   warps 4-7   epilogue                                            216 regs
-//   warp  8     TMA producer: query tiles, K/V                      } 112 regs
-//   warp  9     TMEM allocator and MMA issuer                       }
-//   warp  10    TMA for the gate / output staging tile              }
-//   warp  11    idle                                                }
+// Warp roles (512 threads, 128 registers each):
+//   warps 0-3   softmax, union chunks 0-1 (TMEM lanes 0..127)
+//   warps 4-7   softmax, union chunks 2-3
+//   warps 8-11  epilogue
+//   warp  12    TMA producer: query tiles, K/V
+//   warp  13    TMEM allocator and MMA issuer
+//   warp  14    TMA for the gate / output staging tile
+//   warp  15    idle
 // TMEM (512 columns): S_E [0,128) S_G [128,256) O [256,256+d) H_N [256+d,256+2d).
 // P_E / P_G occupy the first 64 columns of S_E / S_G as packed bf16 pairs.
 #pragma once
@@ -52,22 +53,13 @@
 
 namespace gdla {
 
-constexpr int kWinThreads = 12 * 32;
-constexpr int kWinEpiWarp0 = 4;
-constexpr int kWinProducerWarp = 8;
-constexpr int kWinMmaWarp = 9;
-constexpr int kWinGateWarp = 10;
-// Register split: the block launches with kWinLaunchRegs per thread (the
-// compiler's cap for 12 warps on one SM); the control warpgroup gives
-// registers back, and the softmax (a whole union row in registers) and the
-// epilogue (a head's D in registers) take them.  The host refuses a build with another per-thread count.
-constexpr uint32_t kWinLaunchRegs = 168;
-constexpr uint32_t kWinSoftmaxRegs = 176;
-constexpr uint32_t kWinEpilogueRegs = 216;
-constexpr uint32_t kWinControlRegs = 112;
-static_assert(128 * (kWinSoftmaxRegs + kWinEpilogueRegs + kWinControlRegs) <=
-                  kWinThreads * kWinLaunchRegs,
-              "register split must fit in the launch pool");
+constexpr int kWinThreads = 16 * 32;
+constexpr int kWinEpiWarp0 = 8;
+constexpr int kWinProducerWarp = 12;
+constexpr int kWinMmaWarp = 13;
+constexpr int kWinGateWarp = 14;
+// Every role fits the 128 registers a thread of a 16-warp block gets (no
+// register re-split).
 constexpr uint32_t kNegInfBits = 0xff800000u;
 
 template <int D>
@@ -78,9 +70,10 @@ struct WinSmemLayout {
   static constexpr uint32_t kVOff = kKOff + 2 * kTile;  // V_E, V_G
   static constexpr uint32_t kGOff = kVOff + 2 * kTile;  // gate / output staging
   static constexpr uint32_t kHalf = kBM * 128;          // one [128][64] swizzled half
-  static constexpr uint32_t kStatOff = kGOff + kTile;   // float l[2][kBM]
-  static constexpr uint32_t kBarOff = kStatOff + 2 * kBM * 4;
-  static constexpr uint32_t kNumBars = 18;
+  static constexpr uint32_t kStatOff = kGOff + kTile;   // float l[2 slot][2 half][kBM]
+  static constexpr uint32_t kMxOff = kStatOff + 2 * 2 * kBM * 4;  // int16 [2 half][kBM]
+  static constexpr uint32_t kBarOff = kMxOff + 2 * kBM * 2;
+  static constexpr uint32_t kNumBars = 22;
   static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;
   static constexpr uint32_t kBytes = kMiscOff + 16;
   static_assert(kBytes <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
@@ -124,9 +117,12 @@ __global__ void __launch_bounds__(kWinThreads, 1)
   // row sums handed over through two slots (softmax warps) / read (epilogue warps)
   auto epi_go = [&](uint32_t s) { return bar0 + 8u * (14 + s); };
   auto stat_free = [&](uint32_t s) { return bar0 + 8u * (16 + s); };
+  // the two softmax halves of lane quarter wq meet here once per head
+  auto mx_bar = [&](uint32_t wq) { return bar0 + 8u * (18 + wq); };
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
-  float *stat = reinterpret_cast<float *>(smem + L::kStatOff);  // [2][kBM]
+  float *stat = reinterpret_cast<float *>(smem + L::kStatOff);  // [2 slot][2 half][kBM]
+  int16_t *mxs = reinterpret_cast<int16_t *>(smem + L::kMxOff);   // [2 half][kBM]
   const int warp = threadIdx.x >> 5;
   const int n_heads = p.g + 1;  // noise head + g signal heads
   const int W = static_cast<int>(p.window);
@@ -141,15 +137,16 @@ __global__ void __launch_bounds__(kWinThreads, 1)
     mbar_init(v_full, 1);
     mbar_init(v_free, 1);
     mbar_init(s_full, 1);
-    mbar_init(p_full, 4);
+    mbar_init(p_full, 8);  // one arrival per softmax warp
     mbar_init(o_done, 1);
     mbar_init(o_free, 4);
     for (uint32_t s = 0; s < 2; ++s) {
-      mbar_init(epi_go(s), 4);
+      mbar_init(epi_go(s), 8);
       mbar_init(stat_free(s), 4);
     }
     mbar_init(g_full, 1);
     mbar_init(g_done, 4);
+    for (uint32_t wq = 0; wq < 4; ++wq) mbar_init(mx_bar(wq), 2);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -165,8 +162,7 @@ __global__ void __launch_bounds__(kWinThreads, 1)
   auto p_col = [](int k) -> uint32_t { return 8u * k; };
 
   if (warp >= kWinProducerWarp) {
-  // =============================== control warpgroup (warps 8-11)
-  regs_decrease<kWinControlRegs>();
+  // =============================== control warpgroup (warps 12-15)
   if (warp == kWinProducerWarp) {
     // =============================== TMA producer
     // Per item: K_E, K_G once the previous item's last S is done, the first
@@ -353,136 +349,144 @@ __global__ void __launch_bounds__(kWinThreads, 1)
     }
   }
   } else if (warp < kWinEpiWarp0) {
-    // =============================== softmax (warps 0-3, one thread per row)
-    regs_increase<kWinSoftmaxRegs>();
+    // =============================== softmax (warps 0-7, one thread per row)
+    // Warpgroup `half` takes union chunks 2 half and 2 half + 1 of every row.
+    // Warp quarter qw's own chunk qw mixes both tiles (G left of the
+    // diagonal, E right of it); the other chunks come whole from one tile.
+    // The two halves of a row agree on the integral reference maximum once
+    // per head through shared memory and the pair's mbarrier.
+    const int half = warp >> 2;
     const int qw = warp & 3;
     const int r = threadIdx.x & 127;
     const uint32_t lane_off = static_cast<uint32_t>(qw * 32) << 16;
     const float sl2 = p.scale_log2;
     const uint64_t sl2x2 = f2_make(sl2, sl2);
-    const int cm = 32 * qw;       // this warp's mixed union chunk
-    const int dlo = r - W + 1;    // kept diagonal-tile columns: [dlo, r]
+    const int dlo = r - W + 1;  // kept diagonal-tile columns: [dlo, r]
+    const int ca = 2 * half, cb = 2 * half + 1;
+    const bool has_mixed = qw == ca || qw == cb;
+    const int other = qw == ca ? cb : ca;  // the whole chunk next to the mixed one
     uint32_t s_waits = 0, handoffs = 0;
     bool ok = true;
-    // the three whole chunks: chunk index, and whether it comes from the
-    // diagonal tile (left of the mixed chunk) or the edge tile (right of it)
-    int ccj[3];
-    bool from_g[3];
-#pragma unroll
-    for (int j = 0; j < 3; ++j) {
-      ccj[j] = j + (j >= qw ? 1 : 0);
-      from_g[j] = ccj[j] < qw;
-    }
+    const uint32_t zero16[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u,
+                                 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
     for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
       const WorkItem w = work_item(p, item);
       const bool has_edge = w.q0 + p.kv_prefix > 0;
       // kept edge-tile columns: [elo, 127]
       const int elo = has_edge ? max(r + 1, r + 129 - W) : 128;
+      // whole chunk cc (cc != qw): its tile and its lowest kept column
+      auto whole_src = [&](int cc) { return (cc < qw ? t_sg : t_se) + lane_off + 32 * cc; };
+      auto cut_whole = [&](uint32_t (&v)[32], int cc) {
+        const int lo = cc < qw ? dlo : elo;
+        const int c0 = 32 * cc;
+        if (__any_sync(0xffffffffu, lo > c0)) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (c0 + e < lo) v[e] = kNegInfBits;
+        }
+      };
       for (int hh = 0; hh < n_heads && ok; ++hh) {
         ok = __all_sync(0xffffffffu, mbar_wait(s_full, s_waits & 1u, abort_flag));
+        const uint32_t par = s_waits & 1u;
         ++s_waits;
         if (!ok) break;
         tc_fence_after();
-        // ---- round trip 1: the mixed chunk from both tiles
-        uint32_t um[32];
-        {
-          uint32_t mg[32], me[32];
+        // ---- this half's two chunks in one TMEM round trip: va holds chunk
+        // ka, vb chunk kb (the mixed chunk first when the half has it)
+        uint32_t va[32], vb[32];
+        const int ka = has_mixed ? qw : ca, kb = has_mixed ? other : cb;
+        if (has_mixed) {
+          uint32_t me[32];
           if (has_edge) {
-            tmem_ld32x2_sync(t_sg + lane_off + cm, t_se + lane_off + cm, mg, me);
+            tmem_ld32x3_sync(t_sg + lane_off + 32 * qw, t_se + lane_off + 32 * qw,
+                             whole_src(other), va, me, vb);
           } else {
-            tmem_ld32_sync(t_sg + lane_off + cm, mg);
+            tmem_ld32x2_sync(t_sg + lane_off + 32 * qw, whole_src(other), va, vb);
 #pragma unroll
             for (int e = 0; e < 32; ++e) me[e] = kNegInfBits;
           }
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            const int c = cm + e;
+            const int c = 32 * qw + e;
             const bool diag = c <= r;
             const bool kept = diag ? c >= dlo : c >= elo;
-            um[e] = kept ? (diag ? mg[e] : me[e]) : kNegInfBits;
+            va[e] = kept ? (diag ? va[e] : me[e]) : kNegInfBits;
           }
+        } else {
+          tmem_ld32x2_sync(whole_src(ca), whole_src(cb), va, vb);
+          cut_whole(va, ca);
         }
-        // ---- round trip 2: the three whole chunks
-        uint32_t up[3][32];
-        tmem_ld32x3_sync((from_g[0] ? t_sg : t_se) + lane_off + 32 * ccj[0],
-                         (from_g[1] ? t_sg : t_se) + lane_off + 32 * ccj[1],
-                         (from_g[2] ? t_sg : t_se) + lane_off + 32 * ccj[2], up[0], up[1], up[2]);
-#pragma unroll
-        for (int j = 0; j < 3; ++j) {
-          // a whole chunk is cut only from below: G columns before dlo, E
-          // columns before elo (every E column when there is no edge tile)
-          const int lo = from_g[j] ? dlo : elo;
-          const int c0 = 32 * ccj[j];
-          if (__any_sync(0xffffffffu, lo > c0)) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (c0 + e < lo) up[j][e] = kNegInfBits;
-          }
-        }
-        // ---- row max (the diagonal key is always kept, so it is finite)
+        cut_whole(vb, kb);
+        // ---- this half's maximum, as the integral reference it implies
         float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          m0 = fmax3(m0, __uint_as_float(um[e]), __uint_as_float(um[e + 1]));
-          m1 = fmax3(m1, __uint_as_float(up[0][e]), __uint_as_float(up[0][e + 1]));
-          m0 = fmax3(m0, __uint_as_float(up[1][e]), __uint_as_float(up[1][e + 1]));
-          m1 = fmax3(m1, __uint_as_float(up[2][e]), __uint_as_float(up[2][e + 1]));
+          m0 = fmax3(m0, __uint_as_float(va[e]), __uint_as_float(va[e + 1]));
+          m1 = fmax3(m1, __uint_as_float(vb[e]), __uint_as_float(vb[e + 1]));
         }
-        // one tile per head: the reference max needs no later rescale; it is
-        // rounded up to an integer like the other kernels' running max
-        const float mt = fmaxf(m0, m1) * sl2;
-        const float m_ref = mt == -INFINITY ? 0.f : ceilf(mt);
+        const float mh = fmaxf(m0, m1) * sl2;
+        // ceil is monotone, so the row's reference is the larger of the two
+        // halves'; it travels as int16 (scaled logits beyond +-32767 saturate)
+        const int mi = mh == -INFINITY ? -32768 : static_cast<int>(fminf(fmaxf(ceilf(mh), -32767.f), 32767.f));
+        mxs[half * kBM + r] = static_cast<int16_t>(mi);
+        warp_arrive(mx_bar(qw));
+        ok = __all_sync(0xffffffffu, mbar_wait(mx_bar(qw), par, abort_flag));
+        if (!ok) break;
+        const int mref_i = max(static_cast<int>(mxs[r]), static_cast<int>(mxs[kBM + r]));
+        // one tile per head: no running max, nothing to rescale; a row with
+        // no kept key (padding rows) keeps reference 0
+        const float m_ref = mref_i == -32768 ? 0.f : static_cast<float>(mref_i);
         const uint64_t negm2 = f2_make(-m_ref, -m_ref);
         uint64_t rs2 = f2_make(0.f, 0.f);
         // ---- P = exp2(S*c - m) as bf16 pairs; chunk cc lands in columns
-        // [16cc, 16cc+16) of its tile's S (all of S is in registers already)
-        const uint32_t zero16[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u,
-                                     0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-#pragma unroll
-        for (int j = 0; j < 3; ++j) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            float t0v, t1v;
-            f2_split(f2_fma(f2_from_bits(up[j][2 * e], up[j][2 * e + 1]), sl2x2, negm2), t0v, t1v);
-            const float p0 = ex2_approx(t0v);
-            const float p1 = ex2_approx(t1v);
-            rs2 = f2_add(rs2, f2_make(p0, p1));
-            pk[e] = pack_bf16x2(p0, p1);
-          }
-          const uint32_t col = lane_off + 16 * ccj[j];
-          if (from_g[j]) {
-            tmem_st16(t_sg + col, pk);
-            if (has_edge) tmem_st16(t_se + col, zero16);
-          } else {
-            tmem_st16(t_sg + col, zero16);
-            if (has_edge) tmem_st16(t_se + col, pk);
-          }
-        }
-        {
+        // [16cc, 16cc+16) of its tile's S (the other half has read its S:
+        // it arrived at the pair's barrier above)
+        if (has_mixed) {
           uint32_t pg[16], pe[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             float t0v, t1v;
-            f2_split(f2_fma(f2_from_bits(um[2 * e], um[2 * e + 1]), sl2x2, negm2), t0v, t1v);
+            f2_split(f2_fma(f2_from_bits(va[2 * e], va[2 * e + 1]), sl2x2, negm2), t0v, t1v);
             const float p0 = ex2_approx(t0v);
             const float p1 = ex2_approx(t1v);
             rs2 = f2_add(rs2, f2_make(p0, p1));
-            const bool d0 = cm + 2 * e <= r, d1 = cm + 2 * e + 1 <= r;
+            const bool d0 = 32 * qw + 2 * e <= r, d1 = 32 * qw + 2 * e + 1 <= r;
             pg[e] = pack_bf16x2(d0 ? p0 : 0.f, d1 ? p1 : 0.f);
             pe[e] = pack_bf16x2(d0 ? 0.f : p0, d1 ? 0.f : p1);
           }
           tmem_st16(t_sg + lane_off + 16 * qw, pg);
           if (has_edge) tmem_st16(t_se + lane_off + 16 * qw, pe);
         }
+        auto exp_whole = [&](const uint32_t (&v)[32], int cc) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            float t0v, t1v;
+            f2_split(f2_fma(f2_from_bits(v[2 * e], v[2 * e + 1]), sl2x2, negm2), t0v, t1v);
+            const float p0 = ex2_approx(t0v);
+            const float p1 = ex2_approx(t1v);
+            rs2 = f2_add(rs2, f2_make(p0, p1));
+            pk[e] = pack_bf16x2(p0, p1);
+          }
+          const uint32_t col = lane_off + 16 * cc;
+          if (cc < qw) {
+            tmem_st16(t_sg + col, pk);
+            if (has_edge) tmem_st16(t_se + col, zero16);
+          } else {
+            tmem_st16(t_sg + col, zero16);
+            if (has_edge) tmem_st16(t_se + col, pk);
+          }
+        };
+        if (!has_mixed) exp_whole(va, ca);
+        exp_whole(vb, kb);
         float rs0, rs1;
         f2_split(rs2, rs0, rs1);
         const float l = rs0 + rs1;
         tmem_wait_st();
         tc_fence_before();
         warp_arrive(p_full);
-        // hand the row sum to the epilogue through slot handoffs % 2, once
-        // the epilogue has read what the slot held two heads ago
+        // hand this half's row sum to the epilogue through slot handoffs % 2,
+        // once the epilogue has read what the slot held two heads ago
         const uint32_t slot = handoffs & 1u;
         if (handoffs >= 2) {
           ok = __all_sync(0xffffffffu,
@@ -490,16 +494,15 @@ __global__ void __launch_bounds__(kWinThreads, 1)
           if (!ok) break;
         }
         ++handoffs;
-        stat[slot * kBM + r] = l;
+        stat[(slot * 2 + half) * kBM + r] = l;
         warp_arrive(epi_go(slot));
       }
     }
   } else {
-    // =============================== epilogue (warps 4-7)
+    // =============================== epilogue (warps 8-11)
     // Noise head: H_N = O / l into its TMEM columns.  Signal head:
     // D = O/l - lambda H_N into registers (O released at once), then
     // out = G (.) D over the row of the staged gate tile, in place.
-    regs_increase<kWinEpilogueRegs>();
     const int qw = warp & 3;
     const int r = threadIdx.x & 127;
     const uint32_t lane_off = static_cast<uint32_t>(qw * 32) << 16;
@@ -523,7 +526,7 @@ __global__ void __launch_bounds__(kWinThreads, 1)
         ok = __all_sync(0xffffffffu, okw);
         if (!ok) break;
         tc_fence_after();
-        const float l = stat[slot * kBM + r];
+        const float l = stat[(slot * 2 + 0) * kBM + r] + stat[(slot * 2 + 1) * kBM + r];
         warp_arrive(stat_free(slot));
         const float inv_l = l > 0.f ? 1.f / l : 0.f;
         if (hh == 0) {
@@ -540,25 +543,17 @@ __global__ void __launch_bounds__(kWinThreads, 1)
           warp_arrive(o_free);
           continue;
         }
-        float dv[D];
+        ok = __all_sync(0xffffffffu, mbar_wait(g_full, g_seen & 1u, abort_flag));
+        ++g_seen;
+        if (!ok) break;
+        // out = G (.) (O/l - lambda H_N), 32 columns at a time, in place over
+        // the staged gate tile: row r of a 128B-swizzled [128][64] half holds
+        // 16-byte unit j at j ^ (r % 8)
+        const uint32_t rbase = gbuf + static_cast<uint32_t>(r) * 128u;
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32], hn[32];
           tmem_ld32x2_sync(t_o + lane_off + cc * 32, t_hn + lane_off + cc * 32, o, hn);
-#pragma unroll
-          for (int e = 0; e < 32; ++e)
-            dv[cc * 32 + e] = __uint_as_float(o[e]) * inv_l - lam * __uint_as_float(hn[e]);
-        }
-        // every column of O is in registers: the next head's PV may start
-        tc_fence_before();
-        warp_arrive(o_free);
-        ok = __all_sync(0xffffffffu, mbar_wait(g_full, g_seen & 1u, abort_flag));
-        ++g_seen;
-        if (!ok) break;
-        // row r of a 128B-swizzled [128][64] half: 16-byte unit j sits at j ^ (r % 8)
-        const uint32_t rbase = gbuf + static_cast<uint32_t>(r) * 128u;
-#pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const int j = (cc & 1) * 4 + q;
@@ -569,12 +564,18 @@ __global__ void __launch_bounds__(kWinThreads, 1)
             uint32_t ow[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const int k0 = cc * 32 + q * 8 + 2 * e;
-              ow[e] = pack_bf16x2(bf16lo_to_f32(gw[e]) * dv[k0], bf16hi_to_f32(gw[e]) * dv[k0 + 1]);
+              const int k0 = q * 8 + 2 * e;
+              const float d0 = __uint_as_float(o[k0]) * inv_l - lam * __uint_as_float(hn[k0]);
+              const float d1 =
+                  __uint_as_float(o[k0 + 1]) * inv_l - lam * __uint_as_float(hn[k0 + 1]);
+              ow[e] = pack_bf16x2(bf16lo_to_f32(gw[e]) * d0, bf16hi_to_f32(gw[e]) * d1);
             }
             sts128(addr, make_uint4(ow[0], ow[1], ow[2], ow[3]));
           }
         }
+        // every column of O has been read: the next head's PV may start
+        tc_fence_before();
+        warp_arrive(o_free);
         // every row written (generic proxy) before the TMA store reads the tile
         fence_proxy_async_smem();
         warp_arrive(g_done);

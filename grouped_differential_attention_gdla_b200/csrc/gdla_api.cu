@@ -161,7 +161,7 @@ int launch_attn(const void *q_sig, const void *q_noise, const void *k, const voi
     using LW = gdla::WinSmemLayout<D>;
     const uint32_t smem = LW::kBytes > kMinSmem ? LW::kBytes : kMinSmem;
     constexpr auto kern = gdla::gdla_attn_win_kernel<D>;
-    const int rc = prepare_kernel<kern>(smem, static_cast<int>(gdla::kWinLaunchRegs));
+    const int rc = prepare_kernel<kern>(smem, 0);
     if (rc != GDLA_OK) return rc;
     kern<<<static_cast<unsigned>(grid), gdla::kWinThreads, smem, stream>>>(
         tm_qs, tm_qn, tm_k, tm_v, tm_gate, tm_out, run);
