@@ -113,6 +113,10 @@ class Oracle:
                                            i32, vp, vp, i32, f64, vp, i32, vp, i32, vp, i32, i32,
                                            i64, i32, i32, i32, i32, i32, i64, f64, vp]
         lib.gdla_oracle_decode.restype = ctypes.c_int
+        lib.gdla_oracle_attn_bwd.argtypes = [vp, i32, vp, i32, vp, i32, vp, i32, vp, i32, vp, i32,
+                                             vp, i32, i32, i64, i32, i32, i32, i32, i64, i32, f64,
+                                             vp, vp, vp, vp, vp, vp]
+        lib.gdla_oracle_attn_bwd.restype = ctypes.c_int
         lib.gdla_oracle_version.restype = ctypes.c_int
         self.lib = lib
         self.path = lib_path
@@ -344,6 +348,39 @@ class Oracle:
         return out
 
 
+    # backward: gradients of sum(d_out * O) with respect to every input
+    def gdla_attn_bwd(self, q_sig, q_noise, k, v, lam, gate, d_out, window: int = 0,
+                      causal: bool = True, scale=None) -> dict:
+        """Gradients of the GDLA forward for upstream gradient d_out [B,T,Hs*d].
+
+        Returns float64 arrays dq_sig [B,T,Hs,d], dq_noise [B,T,Hn,d],
+        dk, dv [B,T,Hkv,d], dlam [B,T,Hs], dgate [B,T,Hs*d].
+        """
+        qs, qsp, qsdt = _arr(q_sig)
+        qn, qnp, qndt = _arr(q_noise)
+        ka, kp, kdt = _arr(k)
+        va, vp, vdt = _arr(v)
+        la, lp, ldt = _arr(lam)
+        ga, gp, gdt = _arr(gate)
+        da, dp, ddt = _arr(d_out)
+        B, T, Hs, d = qs.shape
+        Hn = qn.shape[2]
+        Hkv = ka.shape[2]
+        if scale is None:
+            scale = 1.0 / np.sqrt(d)
+        out = {"dq_sig": np.empty((B, T, Hs, d)), "dq_noise": np.empty((B, T, Hn, d)),
+               "dk": np.empty((B, T, Hkv, d)), "dv": np.empty((B, T, Hkv, d)),
+               "dlam": np.empty((B, T, Hs)), "dgate": np.empty((B, T, Hs * d))}
+        rc = self.lib.gdla_oracle_attn_bwd(qsp, qsdt, qnp, qndt, kp, kdt, vp, vdt, lp, ldt, gp,
+                                           gdt, dp, ddt, B, T, Hs, Hn, Hkv, d, int(window),
+                                           int(bool(causal)), float(scale),
+                                           *(out[n].ctypes.data for n in
+                                             ("dq_sig", "dq_noise", "dk", "dv", "dlam", "dgate")))
+        if rc != 0:
+            raise ValueError("oracle rejected the backward arguments (rc %d)" % rc)
+        return out
+
+
 _default = None
 
 
@@ -381,3 +418,7 @@ def gdla_attn_rows(*a, **k):
 
 def decode(*a, **k):
     return default().decode(*a, **k)
+
+
+def gdla_attn_bwd(*a, **k):
+    return default().gdla_attn_bwd(*a, **k)

@@ -420,3 +420,153 @@ int gdla_oracle_decode(const void *q_sig, int qs_dt, const void *q_noise,
   }
   return 0;
 }
+
+/*
+ * Backward of the GDLA attention forward ([R] step 2; the model is trained
+ * with GDLA, "Вышла новая модель Motif 3", pikabu.ru).  The pages give the
+ * forward only; this is its gradient by the chain rule, written out in the
+ * forward's order, for the loss sum(dO (.) O) with dO given.  For each token:
+ *   dG[h]      = dO[h] (.) D[h],            D[h] = H_S[h] - lambda[h] H_N[h/g]
+ *   dD[h]      = dO[h] (.) G[h]
+ *   dlambda[h] = - sum_c dD[h][c] H_N[h/g][c]
+ *   dH_S[h]    = dD[h]
+ *   dH_N[n]    = - sum_{h : h/g = n} lambda[h] dD[h]
+ * and for every head x of either path (output H_x, upstream gradient dH_x),
+ * with s_ij = scale q_i . k_j and p_ij = softmax_j(s_ij) over J(i):
+ *   dp_ij      = dH_x[i] . V[j]
+ *   ds_ij      = p_ij (dp_ij - sum_{j' in J(i)} p_ij' dp_ij')   (softmax Jacobian)
+ *   dQ_x[i]    = scale sum_j ds_ij K[j]
+ *   dK[j]     += scale sum_i ds_ij Q_x[i]   (every head reading KV head kv(x))
+ *   dV[j]     += sum_i p_ij dH_x[i]
+ * Inputs as gdla_oracle_attn (full tensors, every row); d_out [B,T,Hs*d].
+ * Outputs (float64): dq_sig [B,T,Hs,d], dq_noise [B,T,Hn,d], dk, dv
+ * [B,T,Hkv,d], dlam [B,T,Hs], dgate [B,T,Hs*d].  Returns 0, -1 for bad head
+ * counts, -2 when out of memory.
+ */
+int gdla_oracle_attn_bwd(const void *q_sig, int qs_dt, const void *q_noise,
+                         int qn_dt, const void *k, int k_dt, const void *v,
+                         int v_dt, const void *lam, int lam_dt,
+                         const void *gate, int gate_dt, const void *d_out,
+                         int do_dt, int B, int64_t T, int Hs, int Hn, int Hkv,
+                         int d, int64_t window, int causal, double scale,
+                         double *dq_sig, double *dq_noise, double *dk,
+                         double *dv, double *dlam, double *dgate) {
+  if (Hn <= 0 || Hkv <= 0 || Hs % Hn != 0 || Hn != Hkv) return -1;
+  const int g = Hs / Hn;
+  const int64_t N = (int64_t)B * T;
+  double *hs = (double *)malloc(sizeof(double) * (size_t)(N * Hs * d));
+  double *hn = (double *)malloc(sizeof(double) * (size_t)(N * Hn * d));
+  double *dhs = (double *)malloc(sizeof(double) * (size_t)(N * Hs * d));
+  double *dhn = (double *)malloc(sizeof(double) * (size_t)(N * Hn * d));
+  if (!hs || !hn || !dhs || !dhn) {
+    free(hs);
+    free(hn);
+    free(dhs);
+    free(dhn);
+    return -2;
+  }
+  /* the forward's two attention paths, every row */
+  attention_path_impl(q_sig, qs_dt, 0, NULL, ORACLE_F64, k, k_dt, NULL,
+                      ORACLE_F64, 0, v, v_dt, T, Hs, Hkv, d, window, causal,
+                      scale, NULL, N, hs);
+  attention_path_impl(q_noise, qn_dt, 0, NULL, ORACLE_F64, k, k_dt, NULL,
+                      ORACLE_F64, 0, v, v_dt, T, Hn, Hkv, d, window, causal,
+                      scale, NULL, N, hn);
+  /* the gate and the differential, token by token */
+  int64_t row;
+#pragma omp parallel for schedule(static)
+  for (row = 0; row < N; ++row) {
+    for (int n = 0; n < Hn; ++n)
+      for (int c = 0; c < d; ++c) dhn[(row * Hn + n) * d + c] = 0.0;
+    for (int h = 0; h < Hs; ++h) {
+      const double l = load_elem(lam, lam_dt, row * Hs + h);
+      const int n = h / g;
+      double dl = 0.0;
+      for (int c = 0; c < d; ++c) {
+        const int64_t oc = row * (int64_t)Hs * d + (int64_t)h * d + c;
+        const double hnv = hn[(row * Hn + n) * d + c];
+        const double dd = hs[(row * Hs + h) * d + c] - l * hnv;
+        const double go = load_elem(d_out, do_dt, oc);
+        dgate[oc] = go * dd;
+        const double ddd = go * load_elem(gate, gate_dt, oc);
+        dhs[(row * Hs + h) * d + c] = ddd;
+        dl -= ddd * hnv;
+        dhn[(row * Hn + n) * d + c] -= l * ddd;
+      }
+      dlam[row * Hs + h] = dl;
+    }
+  }
+  for (int64_t i = 0; i < N * Hkv * d; ++i) {
+    dk[i] = 0.0;
+    dv[i] = 0.0;
+  }
+  /* the attention backward of every head; one task per (batch, KV group)
+   * so that the group's dK and dV are accumulated by one thread */
+  int64_t task;
+#pragma omp parallel
+  {
+    double *p = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+    double *dp = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+#pragma omp for schedule(dynamic, 1)
+    for (task = 0; task < (int64_t)B * Hkv; ++task) {
+      const int64_t b = task / Hkv;
+      const int kvh = (int)(task % Hkv);
+      for (int x = 0; x <= g; ++x) {
+        /* x < g: signal head g*kvh + x; x == g: noise head kvh */
+        const int noise = x == g;
+        const int H = noise ? Hn : Hs;
+        const int hh = noise ? kvh : g * kvh + x;
+        const void *q = noise ? q_noise : q_sig;
+        const int q_dt = noise ? qn_dt : qs_dt;
+        const double *dh = noise ? dhn : dhs;
+        double *dq = noise ? dq_noise : dq_sig;
+        for (int64_t i = 0; i < T; ++i) {
+          const int64_t r = b * T + i;
+          const int64_t qoff = (r * H + hh) * d;
+          int64_t lo, hi;
+          key_range(i, T, window, causal, &lo, &hi);
+          double m = -INFINITY;
+          for (int64_t j = lo; j <= hi; ++j) {
+            const int64_t koff = ((b * T + j) * Hkv + kvh) * d;
+            double dot = 0.0;
+            for (int c = 0; c < d; ++c)
+              dot += load_elem(q, q_dt, qoff + c) * load_elem(k, k_dt, koff + c);
+            p[j - lo] = scale * dot;
+            if (p[j - lo] > m) m = p[j - lo];
+          }
+          double denom = 0.0;
+          for (int64_t j = lo; j <= hi; ++j) {
+            p[j - lo] = exp(p[j - lo] - m);
+            denom += p[j - lo];
+          }
+          double delta = 0.0;
+          for (int64_t j = lo; j <= hi; ++j) {
+            const int64_t voff = ((b * T + j) * Hkv + kvh) * d;
+            p[j - lo] /= denom;
+            double dot = 0.0;
+            for (int c = 0; c < d; ++c) dot += dh[qoff + c] * load_elem(v, v_dt, voff + c);
+            dp[j - lo] = dot;
+            delta += p[j - lo] * dot;
+          }
+          for (int c = 0; c < d; ++c) dq[qoff + c] = 0.0;
+          for (int64_t j = lo; j <= hi; ++j) {
+            const int64_t koff = ((b * T + j) * Hkv + kvh) * d;
+            const double ds = p[j - lo] * (dp[j - lo] - delta);
+            for (int c = 0; c < d; ++c) {
+              dq[qoff + c] += scale * ds * load_elem(k, k_dt, koff + c);
+              dk[koff + c] += scale * ds * load_elem(q, q_dt, qoff + c);
+              dv[koff + c] += p[j - lo] * dh[qoff + c];
+            }
+          }
+        }
+      }
+    }
+    free(p);
+    free(dp);
+  }
+  free(hs);
+  free(hn);
+  free(dhs);
+  free(dhn);
+  return 0;
+}

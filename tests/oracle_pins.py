@@ -606,4 +606,70 @@ def pin_decode_ignores_rows_past_the_length(o):
     assert not np.array_equal(a[1], cc[1])
 
 
+# ---------------------------------------------------------------- backward
+# The model is trained with GDLA ("Вышла новая модель Motif 3", pikabu.ru);
+# the backward is the gradient of the forward of [R] step 2.
+
+
+def _bwd_case(B=1, T=6, Hs=4, Hn=2, Hkv=2, d=3, seed=21):
+    g = torch.Generator().manual_seed(seed)
+    f = lambda *shape: torch.randn(*shape, generator=g, dtype=torch.float64)
+    x = {"q_sig": f(B, T, Hs, d), "q_noise": f(B, T, Hn, d), "k": f(B, T, Hkv, d),
+         "v": f(B, T, Hkv, d),
+         "lam": torch.sigmoid(f(B, T, Hs)), "gate": torch.sigmoid(f(B, T, Hs * d))}
+    return x, f(B, T, Hs * d)
+
+
+def pin_bwd_finite_differences(o):
+    """Every gradient element against central differences of the (pinned)
+    forward oracle: d/dtheta sum(dO * O) ~ (L(theta + e) - L(theta - e)) / 2e."""
+    for window, causal in ((0, True), (2, True), (0, False)):
+        x, dout = _bwd_case(seed=21 + window + 5 * int(causal))
+        grads = o.gdla_attn_bwd(*(x[n] for n in ("q_sig", "q_noise", "k", "v", "lam", "gate")),
+                                dout, window=window, causal=causal, scale=0.7)
+        loss = lambda xx: float((o.gdla_attn(xx["q_sig"], xx["q_noise"], xx["k"], xx["v"],
+                                              xx["lam"], xx["gate"], window=window,
+                                              causal=causal, scale=0.7)
+                                 * dout.reshape(-1, dout.shape[-1]).numpy()).sum())
+        eps = 1e-6
+        for name, gname in (("q_sig", "dq_sig"), ("q_noise", "dq_noise"), ("k", "dk"),
+                            ("v", "dv"), ("lam", "dlam"), ("gate", "dgate")):
+            t = x[name]
+            num = np.empty(t.numel())
+            flat = t.view(-1)
+            for idx in range(t.numel()):
+                keep = float(flat[idx])
+                flat[idx] = keep + eps
+                lp = loss(x)
+                flat[idx] = keep - eps
+                lm = loss(x)
+                flat[idx] = keep
+                num[idx] = (lp - lm) / (2 * eps)
+            _close(grads[gname].reshape(-1), num, rtol=1e-6, atol=1e-7,
+                   what=f"{gname} vs finite differences (window {window}, causal {causal})")
+
+
+def pin_bwd_matches_torch_autograd(o):
+    """torch float64 autograd through SDPA (KV heads repeated per group), the
+    differential and the gate."""
+    for window, causal in ((0, True), (5, True), (0, False)):
+        wl, x = _small(seed=77 + window, window=window, causal=causal)
+        g = torch.Generator().manual_seed(5)
+        dout = torch.randn(wl.B, wl.T, wl.Hs * wl.d, generator=g, dtype=torch.float64)
+        leaves = {n: _f64(x[n]).clone().requires_grad_(True)
+                  for n in ("q_sig", "q_noise", "k", "v", "lam", "gate")}
+        sc = 1.0 / math.sqrt(wl.d)
+        hs = _sdpa(leaves["q_sig"], leaves["k"], leaves["v"], wl.Hs // wl.Hkv, window, causal, sc)
+        hn = _sdpa(leaves["q_noise"], leaves["k"], leaves["v"], 1, window, causal, sc)
+        dd = hs - leaves["lam"].unsqueeze(-1) * hn.repeat_interleave(wl.g, dim=2)
+        out = (leaves["gate"].view(wl.B, wl.T, wl.Hs, wl.d) * dd).reshape(wl.B, wl.T, -1)
+        (out * dout).sum().backward()
+        got = o.gdla_attn_bwd(*(x[n] for n in ("q_sig", "q_noise", "k", "v", "lam", "gate")),
+                              dout, window=window, causal=causal)
+        for name, gname in (("q_sig", "dq_sig"), ("q_noise", "dq_noise"), ("k", "dk"),
+                            ("v", "dv"), ("lam", "dlam"), ("gate", "dgate")):
+            _close(got[gname], leaves[name].grad.numpy(), rtol=1e-10, atol=1e-12,
+                   what=f"{gname} vs torch autograd (window {window}, causal {causal})")
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

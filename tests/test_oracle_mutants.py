@@ -43,6 +43,16 @@ MUTANTS = {
                   "          dot -= load_elem(qr, qr_dt, qroff + c) *"),
     "decode_rope_key_of_first_cached_token": ("kr_b = ORACLE_AT(kr, kr_dt, ((int64_t)b * L_max + first) * dr);",
                                               "kr_b = ORACLE_AT(kr, kr_dt, ((int64_t)b * L_max) * dr);"),
+    "bwd_softmax_jacobian_without_delta": ("const double ds = p[j - lo] * (dp[j - lo] - delta);",
+                                           "const double ds = p[j - lo] * dp[j - lo];"),
+    "bwd_dlambda_sign": ("dl -= ddd * hnv;", "dl += ddd * hnv;"),
+    "bwd_dhn_without_lambda": ("dhn[(row * Hn + n) * d + c] -= l * ddd;",
+                               "dhn[(row * Hn + n) * d + c] -= ddd;"),
+    "bwd_dk_unscaled": ("dk[koff + c] += scale * ds *", "dk[koff + c] += ds *"),
+    "bwd_dv_from_ds": ("dv[koff + c] += p[j - lo] * dh[qoff + c];",
+                       "dv[koff + c] += ds * dh[qoff + c];"),
+    "bwd_dgate_from_signal_only": ("dgate[oc] = go * dd;",
+                                   "dgate[oc] = go * hs[(row * Hs + h) * d + c];"),
     "decode_query_is_first_token": ("const int64_t row = L - 1;", "const int64_t row = 0;"),
     "decode_window_slice_drops_oldest_key": ("(window > 0 && Lb > window) ? Lb - window : 0",
                                              "(window > 0 && Lb >= window) ? Lb - window + 1 : 0"),
