@@ -484,14 +484,30 @@ def _strip_comments(src):
     return "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
 
 
-def _csrc_hash():
-    """Hash of the CUDA sources' code (comments excluded), to tell whether
-    profiled counters still apply to the kernels being timed."""
+# The sources each kernel is built from (its launch code included): a
+# profiled counter applies to a kernel only while these are unchanged.
+KERNEL_SOURCES = {
+    "gdla_attn_fwd_kernel": ("gdla_api.cu", "attn_fwd.cuh", "sm100.cuh"),
+    "gdla_attn_win_kernel": ("gdla_api.cu", "attn_win.cuh", "attn_fwd.cuh", "sm100.cuh"),
+    "gdla_attn_rope_kernel": ("gdla_api.cu", "attn_rope.cuh", "attn_win.cuh", "attn_fwd.cuh",
+                              "sm100.cuh"),
+    "gdla_kv_expand_kernel": ("gdla_api.cu", "kv_expand.cuh", "sm100.cuh"),
+    "gdla_decode_attn_kernel": ("gdla_api.cu", "decode.cuh", "sm100.cuh"),
+}
+
+
+def _csrc_hash(kernel=None):
+    """Hash of the code (comments excluded) of the CUDA sources `kernel` is
+    built from (every source when None), to tell whether profiled counters
+    still apply to the kernel being timed."""
     import glob
     import hashlib
+    csrc = os.path.join(ROOT, "grouped_differential_attention_gdla_b200", "csrc")
+    names = KERNEL_SOURCES.get(kernel.split("<")[0]) if kernel else None
+    files = [os.path.join(csrc, n) for n in names] if names else sorted(
+        glob.glob(os.path.join(csrc, "*")))
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "grouped_differential_attention_gdla_b200",
-                                           "csrc", "*"))):
+    for f in files:
         with open(f, encoding="utf-8") as fh:
             h.update(_strip_comments(fh.read()).encode())
     return h.hexdigest()[:16]
@@ -501,10 +517,10 @@ def _traffic_from_profiles(name, kernel):
     """DRAM bytes (read + write) per launch of `kernel` on workload `name`
     from a committed ncu summary under profiles/ (a line "traffic:
     workload=<w> kernel=<k> csrc=<hash> bytes=<n>"), or None when none
-    matches this workload, kernel and these sources."""
+    matches this workload, kernel and the kernel's current sources."""
     import glob
-    want = _csrc_hash()
     kname = kernel.split("<")[0]
+    want = _csrc_hash(kname)
     pat = re.compile(r"traffic: workload=(\S+) kernel=(\S+) csrc=(\S+) bytes=(\d+)")
     for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
         with open(path) as f:
