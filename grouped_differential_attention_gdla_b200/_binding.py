@@ -33,7 +33,7 @@ GDLA_ERR_TIMEOUT = -5
 EXPORTED = ("gdla_version", "gdla_status_string", "gdla_kv_expand", "gdla_attn_fwd",
             "gdla_attn_fwd_sp", "gdla_latent_rmsnorm", "gdla_decode_workspace_bytes",
             "gdla_decode_fwd", "gdla_selftest_wait_timeout", "gdla_decode_fwd_noalloc",
-            "gdla_attn_fwd_rope")
+            "gdla_attn_fwd_rope", "gdla_attn_bwd_workspace_bytes", "gdla_attn_bwd")
 
 _lib = None
 # One status word per device, used when a caller passes none (see check_status).
@@ -73,6 +73,11 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.gdla_attn_fwd_rope.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32,
                                        i32, i32, i32, i64, i32, f32, vp, vp]
     lib.gdla_attn_fwd_rope.restype = i32
+    lib.gdla_attn_bwd_workspace_bytes.argtypes = [i32, i64, i32, i32, i32]
+    lib.gdla_attn_bwd_workspace_bytes.restype = ctypes.c_size_t
+    lib.gdla_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i64,
+                                  i32, i32, i32, i32, i64, i32, f32, vp, ctypes.c_size_t, vp, vp]
+    lib.gdla_attn_bwd.restype = i32
     lib.gdla_latent_rmsnorm.argtypes = [vp, vp, f32, vp, i64, i32, vp, vp]
     lib.gdla_latent_rmsnorm.restype = i32
     lib.gdla_decode_workspace_bytes.argtypes = [i32, i64, i32, i32, i32, i64]
@@ -278,6 +283,59 @@ def gdla_attn_fwd_rope(q_sig: torch.Tensor, q_noise: torch.Tensor, q_rope_sig: t
     if _sync_check_enabled():
         check_status(q_sig.device, d_status)
     return out
+
+
+def gdla_attn_bwd_workspace_bytes(B: int, T: int, Hs: int, Hn: int, d: int) -> int:
+    """Device scratch bytes gdla_attn_bwd needs for these shapes."""
+    return int(load_library().gdla_attn_bwd_workspace_bytes(B, T, Hs, Hn, d))
+
+
+def gdla_attn_bwd(q_sig: torch.Tensor, q_noise: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                  lam: torch.Tensor, gate: torch.Tensor, d_out: torch.Tensor, window: int = 0,
+                  causal: bool = True, scale: float = 0.0, grads: Optional[dict] = None,
+                  workspace: Optional[torch.Tensor] = None,
+                  d_status: Optional[torch.Tensor] = None, stream=None) -> dict:
+    """Gradients of gdla_attn_fwd for the upstream gradient d_out [B,T,Hs*d].
+
+    Returns a dict of bf16 CUDA tensors dq_sig, dq_noise, dk, dv, dlam, dgate
+    (written into `grads` when given).  The scratch comes from `workspace` (a
+    uint8 CUDA tensor) or, when None, is allocated here with torch.
+    """
+    if q_sig.dim() != 4:
+        raise ValueError("q_sig must be [B, T, Hs, d]")
+    B, T, Hs, d = q_sig.shape
+    Hn = q_noise.shape[2] if q_noise.dim() == 4 else -1
+    Hkv = k.shape[2] if k.dim() == 4 else -1
+    dev = q_sig.device
+    shapes = {"dq_sig": (B, T, Hs, d), "dq_noise": (B, T, Hn, d), "dk": (B, T, Hkv, d),
+              "dv": (B, T, Hkv, d), "dlam": (B, T, Hs), "dgate": (B, T, Hs * d)}
+    if grads is None:
+        grads = {n: torch.empty(sh, dtype=torch.bfloat16, device=dev) for n, sh in shapes.items()}
+    need = gdla_attn_bwd_workspace_bytes(B, T, Hs, Hn, d) if B > 0 and T > 0 else 0
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    if workspace.dtype != torch.uint8 or workspace.device != dev or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous uint8 tensor on the inputs' device")
+    ptrs = [
+        _check(q_sig, "q_sig"),
+        _check(q_noise, "q_noise", (B, T, Hn, d)),
+        _check(k, "k", (B, T, Hkv, d)),
+        _check(v, "v", (B, T, Hkv, d)),
+        _check(lam, "lam", (B, T, Hs)),
+        _check(gate, "gate", (B, T, Hs * d)),
+        _check(d_out, "d_out", (B, T, Hs * d)),
+    ] + [_check(grads[n], n, shapes[n]) for n in shapes]
+    _same_device(dev, [("q_noise", q_noise), ("k", k), ("v", v), ("lam", lam), ("gate", gate),
+                       ("d_out", d_out)] + [(n, grads[n]) for n in shapes])
+    ps = _status_ptr(d_status, dev)
+    rc = load_library().gdla_attn_bwd(*ptrs, B, T, Hs, Hn, Hkv, d, int(window), int(bool(causal)),
+                                      float(scale), workspace.data_ptr(), workspace.numel(), ps,
+                                      _stream_ptr(dev, stream))
+    if rc != GDLA_OK:
+        raise GDLAError(rc, "gdla_attn_bwd")
+    if _sync_check_enabled():
+        check_status(dev, d_status)
+    return grads
 
 
 def gdla_attn_fwd_sp(q_sig: torch.Tensor, q_noise: torch.Tensor, k: torch.Tensor,

@@ -51,18 +51,29 @@ constexpr int kRopeProducerWarp = 12;
 constexpr int kRopeMmaWarp = 13;
 constexpr int kRopeStages = 3;
 
-template <int D>
+// Parameters of the save mode (the forward a backward pass starts from):
+// every head's output H = O / l (fp32, [B, T, Hs + Hn, d], signal heads first)
+// and its log-sum-exp in log2 units of the scaled scores, head-major with the
+// token axis padded to tp (a multiple of 128): [B, Hs + Hn, tp].
+struct AttnSaveParams : AttnParams {
+  float *h;
+  float *lse;
+  int tp;
+};
+
+// R: rotary width (kRope, or 0 without the rotary term).
+template <int D, int R = kRope>
 struct RopeSmemLayout {
   static constexpr uint32_t kSub = kBM * 128;          // one [128][64] bf16 swizzled sub-tile
-  static constexpr int kQkSubs = (D + kRope) / 64;     // sub-tiles of a query tile / K entry
+  static constexpr int kQkSubs = (D + R) / 64;         // sub-tiles of a query tile / K entry
   static constexpr uint32_t kQBytes = kQkSubs * kSub;  // [Q | Q_r]
   static constexpr uint32_t kEntry = kQkSubs * kSub;   // [K | K_r], or V in its first D/64
   static constexpr uint32_t kVBytes = (D / 64) * kSub;
   static constexpr uint32_t kQOff = 0;
   static constexpr uint32_t kRingOff = kQOff + kQBytes;
   static constexpr uint32_t kMaxOff = kRingOff + kRopeStages * kEntry;  // float [2 buf][2 half][kBM]
-  static constexpr uint32_t kStatOff = kMaxOff + 2 * 2 * kBM * 4;       // float [2 slot][2 half][kBM]
-  static constexpr uint32_t kBarOff = kStatOff + 2 * 2 * kBM * 4;
+  static constexpr uint32_t kStatOff = kMaxOff + 2 * 2 * kBM * 4;  // float [2 slot][l0, l1, m][kBM]
+  static constexpr uint32_t kBarOff = kStatOff + 2 * 3 * kBM * 4;
   // q_full q_empty kv_full[S] kv_empty[S] s_full[2] p_full[2] mx_bar[2][4]
   // o_done[2] acc_free[2] epi_go[2] stat_free[2] head_done
   static constexpr uint32_t kNumBars = 2 + 2 * kRopeStages + 2 + 2 + 8 + 2 + 2 + 2 + 2 + 1;
@@ -71,7 +82,10 @@ struct RopeSmemLayout {
   static_assert(kBytes <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
 };
 
-template <int D>
+// kSave (with R = 0): the save mode.  Every head, the noise head included,
+// accumulates in the O region, and the epilogue writes H and the log-sum-exp
+// of every head instead of the gated differential.
+template <int D, int R = kRope, bool kSave = false, typename Params = AttnParams>
 __global__ void __launch_bounds__(kRopeThreads, 1)
     gdla_attn_rope_kernel(const __grid_constant__ CUtensorMap tm_qs,
                           const __grid_constant__ CUtensorMap tm_qn,
@@ -79,8 +93,9 @@ __global__ void __launch_bounds__(kRopeThreads, 1)
                           const __grid_constant__ CUtensorMap tm_qrn,
                           const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_kr,
-                          const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
-  using L = RopeSmemLayout<D>;
+                          const __grid_constant__ CUtensorMap tm_v, const Params p) {
+  static_assert(!kSave || R == 0, "the save mode takes no rotary term");
+  using L = RopeSmemLayout<D, R>;
   extern __shared__ __align__(1024) uint8_t smem[];
   if ((smem_u32(smem) & 1023u) != 0) {
     if (threadIdx.x == 0) write_status(p.status, -4 /* GDLA_ERR_CUDA */);
@@ -105,7 +120,7 @@ __global__ void __launch_bounds__(kRopeThreads, 1)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
   float *mx = reinterpret_cast<float *>(smem + L::kMaxOff);    // [buf][half][row]
-  float *stat = reinterpret_cast<float *>(smem + L::kStatOff);  // [slot][half][row]
+  float *stat = reinterpret_cast<float *>(smem + L::kStatOff);  // [slot][l0, l1, m][row]
   const int warp = threadIdx.x >> 5;
   const int n_heads = p.g + 1;  // noise head + g signal heads
 
@@ -151,10 +166,12 @@ __global__ void __launch_bounds__(kRopeThreads, 1)
     if (leader) {
       tma_prefetch_desc(&tm_qs);
       tma_prefetch_desc(&tm_qn);
-      tma_prefetch_desc(&tm_qrs);
-      tma_prefetch_desc(&tm_qrn);
+      if (R > 0) {
+        tma_prefetch_desc(&tm_qrs);
+        tma_prefetch_desc(&tm_qrn);
+        tma_prefetch_desc(&tm_kr);
+      }
       tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_kr);
       tma_prefetch_desc(&tm_v);
     }
     uint32_t c = 0, q_uses = 0;
@@ -174,7 +191,8 @@ __global__ void __launch_bounds__(kRopeThreads, 1)
           for (int kb = 0; kb < D / 64; ++kb)
             tma_load_3d(dst + kb * L::kSub, is_v ? &tm_v : &tm_k, kv_full(s), w.kvh * D + kb * 64,
                         row, w.b);
-          if (!is_v) tma_load_3d(dst + (D / 64) * L::kSub, &tm_kr, kv_full(s), 0, row, w.b);
+          if (R > 0 && !is_v)
+            tma_load_3d(dst + (D / 64) * L::kSub, &tm_kr, kv_full(s), 0, row, w.b);
         }
         ++c;
       };
@@ -190,8 +208,9 @@ __global__ void __launch_bounds__(kRopeThreads, 1)
           for (int kb = 0; kb < D / 64; ++kb)
             tma_load_3d(sbase + L::kQOff + kb * L::kSub, noise ? &tm_qn : &tm_qs, q_full,
                         head * D + kb * 64, w.q0, w.b);
-          tma_load_3d(sbase + L::kQOff + (D / 64) * L::kSub, noise ? &tm_qrn : &tm_qrs, q_full,
-                      head * kRope, w.q0, w.b);
+          if (R > 0)
+            tma_load_3d(sbase + L::kQOff + (D / 64) * L::kSub, noise ? &tm_qrn : &tm_qrs, q_full,
+                        head * R, w.q0, w.b);
         }
         const int n = w.n_tiles;
         load_kv(0, false);
@@ -220,7 +239,7 @@ __global__ void __launch_bounds__(kRopeThreads, 1)
     const bool leader = elect_one();
     constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBN, false, false);
     constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, D, false, true);
-    constexpr int kSSteps = (D + kRope) / 16;
+    constexpr int kSSteps = (D + R) / 16;
     const uint64_t qd = sdesc_sw128(sbase + L::kQOff, 16, 1024);
     uint32_t c = 0, q_uses = 0, sc = 0;  // ring position, query tiles, S tiles issued
     // per S buffer / accumulator region (kept as scalars: runtime-indexed
@@ -251,7 +270,7 @@ __global__ void __launch_bounds__(kRopeThreads, 1)
       const WorkItem w = work_item(p, item);
       const int n = w.n_tiles;
       for (int hi = 0; hi < n_heads && ok; ++hi) {
-        const uint32_t a = hi == 0 ? 1u : 0u;
+        const uint32_t a = (hi == 0 && !kSave) ? 1u : 0u;
         ok = __all_sync(0xffffffffu, mbar_wait(q_full, q_uses & 1u, abort_flag));
         ++q_uses;
         if (!ok) break;
@@ -328,7 +347,7 @@ __global__ void __launch_bounds__(kRopeThreads, 1)
       float inv_ln = 0.f;
       for (int hi = 0; hi < n_heads && ok; ++hi) {
         const int h = p.g * w.kvh + (hi - 1);  // signal head (hi >= 1)
-        if (hi > 0 && row_ok) {
+        if (!kSave && hi > 0 && row_ok) {
           // the gate row heads for L2 while the head still computes
           const __nv_bfloat16 *gr = p.gate + (row * p.Hs + h) * static_cast<int64_t>(D);
 #pragma unroll
@@ -339,8 +358,40 @@ __global__ void __launch_bounds__(kRopeThreads, 1)
         ok = __all_sync(0xffffffffu, mbar_wait(epi_go(slot), (go >> 1) & 1u, abort_flag));
         ++go;
         if (!ok) break;
-        const float l = stat[(slot * 2 + 0) * kBM + r] + stat[(slot * 2 + 1) * kBM + r];
+        const float l = stat[(slot * 3 + 0) * kBM + r] + stat[(slot * 3 + 1) * kBM + r];
+        const float m_ref = stat[(slot * 3 + 2) * kBM + r];
         warp_arrive(stat_free(slot));
+        if constexpr (kSave) {
+          // H = O / l and the log-sum-exp of the head (noise heads after the
+          // signal heads in the [Hs + Hn] head index)
+          ok = __all_sync(0xffffffffu, mbar_wait(head_done, heads & 1u, abort_flag));
+          ++heads;
+          if (!ok) break;
+          tc_fence_after();
+          const int hx = hi == 0 ? p.Hs + w.kvh : h;
+          const int64_t hrow = row * (p.Hs + p.Hn) + hx;
+          const float inv_l = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            tmem_ld32_sync(t_acc(0) + lane_off + cc * 32, o);
+            if (row_ok) {
+              float4 *hp = reinterpret_cast<float4 *>(p.h + hrow * D + cc * 32);
+#pragma unroll
+              for (int v = 0; v < 8; ++v)
+                hp[v] = make_float4(__uint_as_float(o[4 * v]) * inv_l,
+                                    __uint_as_float(o[4 * v + 1]) * inv_l,
+                                    __uint_as_float(o[4 * v + 2]) * inv_l,
+                                    __uint_as_float(o[4 * v + 3]) * inv_l);
+            }
+          }
+          if (row_ok)
+            p.lse[(static_cast<int64_t>(w.b) * (p.Hs + p.Hn) + hx) * p.tp + i] =
+                l > 0.f ? m_ref + log2f(l) : -INFINITY;
+          tc_fence_before();
+          warp_arrive(acc_free(0));
+          continue;
+        }
         if (hi == 0) {
           inv_ln = l > 0.f ? 1.f / l : 0.f;
           continue;
@@ -403,7 +454,7 @@ __global__ void __launch_bounds__(kRopeThreads, 1)
       const int i = w.q0 + r;  // query token
       const int n = w.n_tiles;
       for (int hi = 0; hi < n_heads && ok; ++hi) {
-        const uint32_t a = hi == 0 ? 1u : 0u;
+        const uint32_t a = (hi == 0 && !kSave) ? 1u : 0u;
         float m_run = -INFINITY, l_run = 0.f;
         for (int t = 0; t < n; ++t) {
           const uint32_t b = sc & 1u, par = (sc >> 1) & 1u;
@@ -472,8 +523,14 @@ __global__ void __launch_bounds__(kRopeThreads, 1)
               f2_split(f2_fma(f2_from_bits(v[2 * e], v[2 * e + 1]), sl2x2, negm2), t0v, t1v);
               const float p0 = ex2_approx(t0v);
               const float p1 = ex2_approx(t1v);
-              rs2 = f2_add(rs2, f2_make(p0, p1));
               pk[e] = pack_bf16x2(p0, p1);
+              // the save mode sums the bf16 P the PV MMA reads, so that the
+              // saved H and log-sum-exp describe the same weights (a row
+              // with one key gets H = V exactly)
+              if constexpr (kSave)
+                rs2 = f2_add(rs2, f2_make(bf16lo_to_f32(pk[e]), bf16hi_to_f32(pk[e])));
+              else
+                rs2 = f2_add(rs2, f2_make(p0, p1));
             }
             tmem_st16(t_s(b) + lane_off + cc * 16, pk);
           };
@@ -514,7 +571,8 @@ __global__ void __launch_bounds__(kRopeThreads, 1)
           if (!ok) break;
         }
         ++handoffs;
-        stat[(slot * 2 + half) * kBM + r] = l_run;
+        stat[(slot * 3 + half) * kBM + r] = l_run;
+        if (half == 0) stat[(slot * 3 + 2) * kBM + r] = m_run;
         warp_arrive(epi_go(slot));
         if (a) pv_base1 += static_cast<uint32_t>(n); else pv_base0 += static_cast<uint32_t>(n);
       }

@@ -1,0 +1,724 @@
+// bwd.cuh - GDLA attention backward, sm_100a.
+//
+// The model is trained with GDLA ("Вышла новая модель Motif 3", pikabu.ru);
+// the backward is the gradient of the forward of "Motif 3: Technical Report"
+// (paper.rainbus.top), step 2, for an upstream gradient dO of the output:
+//   dG[h] = dO[h] (.) D[h],    dD[h] = dO[h] (.) G[h]
+//   dlambda[h] = -sum_c dD[h][c] H_N[h/g][c]
+//   dH_S[h] = dD[h],           dH_N[n] = -sum_{h/g = n} lambda[h] dD[h]
+// and per head x (upstream dH_x): P = softmax(scale Q K^T + mask),
+//   dP = dH_x V^T,  Delta_i = sum_j P_ij dP_ij = dH_x[i] . H_x[i],
+//   dS = P (.) (dP - Delta),  dQ_x = scale dS K,
+//   dK += scale dS^T Q_x,     dV += P^T dH_x       (every head of the group)
+//
+// Four launches (host: gdla_bwd.cu):
+//   1. the forward in save mode (attn_rope.cuh): H of every head (fp32) and
+//      its log-sum-exp (log2 units of the scaled scores);
+//   2. gdla_bwd_prep_kernel (CUDA cores): dG, dlambda, dH of every head
+//      (bf16, the MMA operand) and Delta;
+//   3. gdla_bwd_dq_kernel (tcgen05): per (head, query block), over the key
+//      tiles: S = Q K^T and dP = dH V^T in TMEM, P and dS by two warpgroups
+//      (half the key columns each), dQ += dS K with dS read from TMEM;
+//   4. gdla_bwd_dkdv_kernel (tcgen05): per (KV group, key block), over the
+//      group's g+1 heads and their query blocks: S^T = K Q^T and
+//      dP^T = V dH^T in TMEM, P^T and dS^T per key row, dV += P^T dH and
+//      dK += dS^T Q with both A operands read from TMEM.
+// The softmax statistics come from step 1, so neither kernel needs a running
+// maximum, and the two warpgroups that share a row never wait on each other:
+// each writes its packed bf16 operand into TMEM columns of its own half of the
+// tile (the MMA's A address skips to the second half for K-steps 4..7).
+#pragma once
+
+#include "attn_rope.cuh"
+
+namespace gdla {
+
+constexpr int kBwdThreads = 16 * 32;
+constexpr int kBwdProducerWarp = 12;
+constexpr int kBwdMmaWarp = 13;
+constexpr int kBwdMaxGroup = 8;  // signal heads per KV group the prep kernel takes
+
+struct BwdParams {
+  const __nv_bfloat16 *lam;   // [B, T, Hs]
+  const __nv_bfloat16 *gate;  // [B, T, Hs*d]
+  const __nv_bfloat16 *dout;  // [B, T, Hs*d]
+  __nv_bfloat16 *dq_sig;      // [B, T, Hs, d]
+  __nv_bfloat16 *dq_noise;    // [B, T, Hn, d]
+  __nv_bfloat16 *dk;          // [B, T, Hkv, d]
+  __nv_bfloat16 *dv;          // [B, T, Hkv, d]
+  __nv_bfloat16 *dlam;        // [B, T, Hs]
+  __nv_bfloat16 *dgate;       // [B, T, Hs*d]
+  const float *h;             // workspace: H [B, T, Hs+Hn, d]
+  const float *lse;           // workspace: [B, Hs+Hn, tp]
+  float *delta;               // workspace: [B, Hs+Hn, tp]
+  __nv_bfloat16 *dox;         // workspace: dH [B, T, Hs+Hn, d]
+  int *status;
+  int B, T, tp, Hs, Hn, g, n_qblk, n_kblk;
+  int64_t window;  // 0 = full
+  int causal;
+  float scale, scale_log2;
+};
+
+// Non-tensor bulk copy global -> shared, completion on `bar` (no multicast).
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// TMEM column (relative to the packed tile's base) of the bf16 pairs for
+// keys (or queries) 16k .. 16k+15: the two warpgroups pack their halves at
+// columns 0..31 and 64..95.
+__device__ __forceinline__ uint32_t split_col(int k) { return 8u * k + (k >= 4 ? 32u : 0u); }
+
+// ---------------------------------------------------------------- prep
+// One CTA per (token row, KV group k); thread c owns column c.  Per signal
+// head h of the group: dG, dD (bf16, the dQ/dK/dV operand), dlambda and
+// Delta_h = dD . H_S; then dH_N = -sum lambda dD and Delta_N = dH_N . H_N.
+// Delta uses the bf16-rounded dH the MMAs will read, so that sum_j dS_ij
+// stays zero for the gradients the kernels form.
+template <int D>
+__global__ void __launch_bounds__(128) gdla_bwd_prep_kernel(const BwdParams p) {
+  const int64_t row = blockIdx.x;
+  const int k = blockIdx.y;
+  const int c = threadIdx.x;
+  const int g = p.g, H80 = p.Hs + p.Hn;
+  const int64_t b = row / p.T, i = row % p.T;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __shared__ float red[4][2 * kBwdMaxGroup + 1];
+  float part[2 * kBwdMaxGroup + 1];
+#pragma unroll
+  for (int q = 0; q < 2 * kBwdMaxGroup + 1; ++q) part[q] = 0.f;
+  if (c < D) {
+    const float hn = p.h[(row * H80 + p.Hs + k) * D + c];
+    float dhn = 0.f;
+#pragma unroll
+    for (int j = 0; j < kBwdMaxGroup; ++j) {
+      if (j < g) {
+        const int h = g * k + j;
+        const int64_t oc = (row * p.Hs + h) * D + c;
+        const float lam = __bfloat162float(p.lam[row * p.Hs + h]);
+        const float hs = p.h[(row * H80 + h) * D + c];
+        const float go = __bfloat162float(p.dout[oc]);
+        const float dd = go * __bfloat162float(p.gate[oc]);
+        const __nv_bfloat16 ddb = __float2bfloat16(dd);
+        p.dgate[oc] = __float2bfloat16(go * (hs - lam * hn));
+        p.dox[(row * H80 + h) * D + c] = ddb;
+        dhn -= lam * dd;
+        part[2 * j] = -dd * hn;                              // dlambda
+        part[2 * j + 1] = __bfloat162float(ddb) * hs;        // Delta of the signal head
+      }
+    }
+    const __nv_bfloat16 dhnb = __float2bfloat16(dhn);
+    p.dox[(row * H80 + p.Hs + k) * D + c] = dhnb;
+    part[2 * kBwdMaxGroup] = __bfloat162float(dhnb) * hn;  // Delta of the noise head
+  }
+#pragma unroll
+  for (int q = 0; q < 2 * kBwdMaxGroup + 1; ++q) {
+    float v = part[q];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) red[warp][q] = v;
+  }
+  __syncthreads();
+  if (threadIdx.x < 2 * kBwdMaxGroup + 1) {
+    const int q = threadIdx.x;
+    const float v = red[0][q] + red[1][q] + red[2][q] + red[3][q];
+    if (q == 2 * kBwdMaxGroup) {
+      p.delta[(b * H80 + p.Hs + k) * p.tp + i] = v;
+    } else if (q / 2 < g) {
+      const int h = g * k + q / 2;
+      if (q & 1)
+        p.delta[(b * H80 + h) * p.tp + i] = v;
+      else
+        p.dlam[row * p.Hs + h] = __float2bfloat16(v);
+    }
+  }
+}
+
+// ---------------------------------------------------------------- dQ
+template <int D>
+struct DqSmemLayout {
+  static constexpr uint32_t kSub = kBM * 128;        // [128][64] bf16 swizzled
+  static constexpr uint32_t kTile = (D / 64) * kSub;  // [128][D]
+  static constexpr uint32_t kStages = 4;              // K/V ring (K_t, V_t alternate)
+  static constexpr uint32_t kQOff = 0;
+  static constexpr uint32_t kDoOff = kQOff + kTile;
+  static constexpr uint32_t kRingOff = kDoOff + kTile;
+  static constexpr uint32_t kBarOff = kRingOff + kStages * kTile;
+  // qd_full kv_full[S] kv_empty[S] s_full p_full dq_done
+  static constexpr uint32_t kNumBars = 1 + 2 * kStages + 3;
+  static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr uint32_t kBytes = kMiscOff + 16;
+  static_assert(kBytes <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
+};
+
+// One CTA per (batch b, head x of Hs + Hn, query block), heaviest blocks
+// first.  Warps 0-7: P and dS (warpgroup `half` takes key columns
+// [64 half, 64 half + 64)); 8-11: dQ epilogue; 12: TMA; 13: TMEM and MMA.
+// TMEM: S [0,128) (dS packed over it), dP [128,256), dQ [256, 256+D).
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    gdla_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qs,
+                       const __grid_constant__ CUtensorMap tm_qn,
+                       const __grid_constant__ CUtensorMap tm_dox,
+                       const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const BwdParams p) {
+  using L = DqSmemLayout<D>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if ((smem_u32(smem) & 1023u) != 0) {
+    if (threadIdx.x == 0) write_status(p.status, -4 /* GDLA_ERR_CUDA */);
+    return;
+  }
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + L::kBarOff;
+  const uint32_t qd_full = bar0;
+  auto kv_full = [&](uint32_t s) { return bar0 + 8u * (1 + s); };
+  auto kv_empty = [&](uint32_t s) { return bar0 + 8u * (1 + L::kStages + s); };
+  const uint32_t s_full = bar0 + 8u * (1 + 2 * L::kStages);
+  const uint32_t p_full = s_full + 8u;
+  const uint32_t dq_done = s_full + 16u;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
+  const int warp = threadIdx.x >> 5;
+  const int H80 = p.Hs + p.Hn;
+
+  // the item: heaviest query blocks first
+  const int item = blockIdx.x;
+  const int qb = p.n_qblk - 1 - item / (p.B * H80);
+  const int rest = item % (p.B * H80);
+  const int b = rest / H80, x = rest % H80;
+  const bool noise = x >= p.Hs;
+  const int kvh = noise ? x - p.Hs : x / p.g;
+  const int q0 = qb * kBM;
+  int j_lo = 0, j_hi;
+  if (p.causal) {
+    j_hi = min(q0 + kBM - 1, p.T - 1) / kBN;
+    if (p.window > 0) {
+      const int64_t first = static_cast<int64_t>(q0) - p.window + 1;
+      j_lo = first > 0 ? static_cast<int>(first / kBN) : 0;
+    }
+  } else {
+    j_hi = (p.T - 1) / kBN;
+  }
+  const int n = j_hi - j_lo + 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(qd_full, 1);
+    for (uint32_t s = 0; s < L::kStages; ++s) {
+      mbar_init(kv_full(s), 1);
+      mbar_init(kv_empty(s), 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 8);
+    mbar_init(dq_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kBwdMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t t_s = tmem, t_dp = tmem + 128u, t_dq = tmem + 256u;
+
+  if (warp == kBwdProducerWarp) {
+    // =============================== TMA: Q_x and dH_x, then K_t, V_t per tile
+    const bool leader = elect_one();
+    if (leader) {
+      mbar_arrive_expect_tx(qd_full, 2 * L::kTile);
+#pragma unroll
+      for (int kb = 0; kb < D / 64; ++kb) {
+        const int head = noise ? kvh : x;
+        tma_load_3d(sbase + L::kQOff + kb * L::kSub, noise ? &tm_qn : &tm_qs, qd_full,
+                    head * D + kb * 64, q0, b);
+        tma_load_3d(sbase + L::kDoOff + kb * L::kSub, &tm_dox, qd_full, x * D + kb * 64, q0, b);
+      }
+    }
+    uint32_t c = 0;
+    bool ok = true;
+    for (int t = 0; t < n && ok; ++t) {
+      for (int kv = 0; kv < 2 && ok; ++kv) {
+        const uint32_t s = c % L::kStages;
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait(kv_empty(s), ((c / L::kStages) & 1u) ^ 1u, abort_flag));
+        if (!ok) break;
+        if (leader) {
+          mbar_arrive_expect_tx(kv_full(s), L::kTile);
+#pragma unroll
+          for (int kb = 0; kb < D / 64; ++kb)
+            tma_load_3d(sbase + L::kRingOff + s * L::kTile + kb * L::kSub, kv ? &tm_v : &tm_k,
+                        kv_full(s), kvh * D + kb * 64, (j_lo + t) * kBN, b);
+        }
+        ++c;
+      }
+    }
+    if (!ok && leader) {
+      for (uint32_t s = 0; s < L::kStages; ++s) {
+        const uint32_t issued = c > s ? (c - 1 - s) / L::kStages + 1 : 0;
+        if (issued) mbar_wait_for(kv_full(s), (issued - 1) & 1u, 100000000ull);
+      }
+      mbar_wait_for(qd_full, 0, 100000000ull);
+    }
+  } else if (warp == kBwdMmaWarp) {
+    // =============================== MMA: S(t), dP(t); then dQ += dS(t) K_t
+    const bool leader = elect_one();
+    constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBN, false, false);
+    constexpr uint32_t kIdescQ = idesc_bf16_f32(kBM, D, false, true);
+    const uint64_t qd = sdesc_sw128(sbase + L::kQOff, 16, 1024);
+    const uint64_t dod = sdesc_sw128(sbase + L::kDoOff, 16, 1024);
+    bool ok = __all_sync(0xffffffffu, mbar_wait(qd_full, 0, abort_flag));
+    uint32_t c = 0;
+    uint32_t done = 0;
+    for (int t = 0; t < n && ok; ++t) {
+      // S = Q K_t^T, dP = dH V_t^T (K-major operands, D/16 K-steps each)
+      const uint32_t sk = c % L::kStages;
+      ok = __all_sync(0xffffffffu, mbar_wait(kv_full(sk), (c / L::kStages) & 1u, abort_flag));
+      ++c;
+      if (!ok) break;
+      const uint32_t sv = c % L::kStages;
+      ok = __all_sync(0xffffffffu, mbar_wait(kv_full(sv), (c / L::kStages) & 1u, abort_flag));
+      ++c;
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t kbase = sbase + L::kRingOff + sk * L::kTile;
+      const uint32_t vbase = sbase + L::kRingOff + sv * L::kTile;
+      if (leader) {
+        const uint64_t kd = sdesc_sw128(kbase, 16, 1024);
+        const uint64_t vd = sdesc_sw128(vbase, 16, 1024);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k >> 2) * L::kSub + (k & 3) * 32;
+          umma_ss(t_s, qd + (off >> 4), kd + (off >> 4), kIdescS, k > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k >> 2) * L::kSub + (k & 3) * 32;
+          umma_ss(t_dp, dod + (off >> 4), vd + (off >> 4), kIdescS, k > 0 ? 1u : 0u);
+        }
+        umma_commit(s_full);
+        umma_commit(kv_empty(sv));  // V_t is no longer needed
+      }
+      ok = __all_sync(0xffffffffu, mbar_wait(p_full, static_cast<uint32_t>(t) & 1u, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      // dQ += dS K_t: A = dS (TMEM, packed halves), B = K_t MN-major over d
+      if (leader) {
+        const uint64_t kmn = sdesc_sw128(kbase, kBN * 128, 1024);
+#pragma unroll
+        for (int k = 0; k < kBN / 16; ++k)
+          umma_ts(t_dq, t_s + split_col(k), kmn + ((k * (16 * 128)) >> 4), kIdescQ,
+                  (t > 0 || k > 0) ? 1u : 0u);
+        umma_commit(kv_empty(sk));
+        if (t == n - 1) umma_commit(dq_done);
+      }
+      if (t == n - 1) ++done;
+    }
+    if (leader && done) mbar_wait_for(dq_done, 0, 100000000ull);
+  } else if (warp >= 8 && warp < 12) {
+    // =============================== epilogue: dQ_x = scale * (dS K), bf16 rows
+    const int wq = warp & 3;
+    const int r = threadIdx.x & 127;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const int i = q0 + r;
+    bool ok = __all_sync(0xffffffffu, mbar_wait(dq_done, 0, abort_flag));
+    if (ok) {
+      tc_fence_after();
+      __nv_bfloat16 *dst = noise ? p.dq_noise + ((static_cast<int64_t>(b) * p.T + i) * p.Hn + kvh) * D
+                                 : p.dq_sig + ((static_cast<int64_t>(b) * p.T + i) * p.Hs + x) * D;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t v[32];
+        tmem_ld32_sync(t_dq + lane_off + cc * 32, v);
+        if (i < p.T) {
+          uint4 *op = reinterpret_cast<uint4 *>(dst + cc * 32);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            op[q] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * q]) * p.scale,
+                                           __uint_as_float(v[8 * q + 1]) * p.scale),
+                               pack_bf16x2(__uint_as_float(v[8 * q + 2]) * p.scale,
+                                           __uint_as_float(v[8 * q + 3]) * p.scale),
+                               pack_bf16x2(__uint_as_float(v[8 * q + 4]) * p.scale,
+                                           __uint_as_float(v[8 * q + 5]) * p.scale),
+                               pack_bf16x2(__uint_as_float(v[8 * q + 6]) * p.scale,
+                                           __uint_as_float(v[8 * q + 7]) * p.scale));
+        }
+      }
+    }
+  } else if (warp < 8) {
+    // =============================== P and dS, half a row per warpgroup
+    const int half = warp >> 2, wq = warp & 3;
+    const int r = threadIdx.x & 127;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const int i = q0 + r;
+    const bool row_ok = i < p.T;
+    const int64_t srow = (static_cast<int64_t>(b) * H80 + x) * p.tp + i;
+    const float lse = row_ok ? p.lse[srow] : 0.f;
+    const float dl = row_ok ? p.delta[srow] : 0.f;
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+    for (int t = 0; t < n && ok; ++t) {
+      ok = __all_sync(0xffffffffu, mbar_wait(s_full, static_cast<uint32_t>(t) & 1u, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      const int kbase = (j_lo + t) * kBN;
+      int c_lo, c_hi;  // kept key columns of this row in the tile
+      if (p.causal) {
+        c_hi = i - kbase;
+        c_lo = p.window > 0 ? static_cast<int>(static_cast<int64_t>(i) - p.window + 1 - kbase) : -1;
+      } else {
+        c_hi = p.T - 1 - kbase;
+        c_lo = -1;
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int cc = 2 * half + u;  // 32-column chunk of the tile
+        uint32_t sv[32], dpv[32];
+        tmem_ld32x2_sync(t_s + lane_off + 32 * cc, t_dp + lane_off + 32 * cc, sv, dpv);
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int c0 = 32 * cc + 2 * e;
+          const bool k0 = row_ok && c0 >= c_lo && c0 <= c_hi;
+          const bool k1 = row_ok && c0 + 1 >= c_lo && c0 + 1 <= c_hi;
+          const float p0 = k0 ? ex2_approx(__uint_as_float(sv[2 * e]) * sl2 - lse) : 0.f;
+          const float p1 = k1 ? ex2_approx(__uint_as_float(sv[2 * e + 1]) * sl2 - lse) : 0.f;
+          pk[e] = pack_bf16x2(p0 * (__uint_as_float(dpv[2 * e]) - dl),
+                              p1 * (__uint_as_float(dpv[2 * e + 1]) - dl));
+        }
+        // dS of this chunk, packed into this half's own S columns
+        tmem_st16(t_s + lane_off + 64 * half + 16 * u, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      warp_arrive(p_full);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0) write_status(p.status, -5 /* GDLA_ERR_TIMEOUT */);
+  if (warp == kBwdMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- dK, dV
+template <int D>
+struct DkdvSmemLayout {
+  static constexpr uint32_t kSub = kBM * 128;
+  static constexpr uint32_t kTile = (D / 64) * kSub;
+  static constexpr uint32_t kStages = 2;  // (Q_x, dH_x, lse, Delta) of one query block
+  static constexpr uint32_t kStatBytes = 2 * kBM * 4;
+  static constexpr uint32_t kEntry = 2 * kTile + 1024;  // tiles, then lse[128], Delta[128]
+  static constexpr uint32_t kKOff = 0;
+  static constexpr uint32_t kVOff = kKOff + kTile;
+  static constexpr uint32_t kRingOff = kVOff + kTile;
+  static constexpr uint32_t kBarOff = kRingOff + kStages * kEntry;
+  // kv_full ring_full[S] ring_empty[S] s_full p_full acc_done
+  static constexpr uint32_t kNumBars = 1 + 2 * kStages + 3;
+  static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr uint32_t kBytes = kMiscOff + 16;
+  static_assert(kBytes <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
+};
+
+// The query blocks that reach key block kb (tokens kb*128 .. kb*128+127).
+__device__ __forceinline__ void dkdv_qrange(const BwdParams &p, int kb, int &qlo, int &qhi) {
+  if (!p.causal) {
+    qlo = 0;
+    qhi = p.n_qblk - 1;
+    return;
+  }
+  qlo = kb;  // queries at or after the key
+  qhi = p.n_qblk - 1;
+  if (p.window > 0) {
+    // the last query that keeps key kb*128 + 127 is kb*128 + 127 + W - 1
+    const int64_t last = static_cast<int64_t>(kb) * kBN + kBN - 1 + p.window - 1;
+    const int64_t lb = last / kBM;
+    if (lb < qhi) qhi = static_cast<int>(lb);
+  }
+}
+
+// One CTA per (batch b, KV group k, key block kb), heaviest (earliest) key
+// blocks first.  Warps 0-7: P^T and dS^T (warpgroup `half` takes query
+// columns [64 half, 64 half + 64)); 8-11: dK, dV epilogue; 12: TMA;
+// 13: TMEM and MMA.  TMEM: S^T [0,128) (P^T packed over it), dP^T [128,256)
+// (dS^T packed over it), dV [256, 256+D), dK [256+D, 256+2D).
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    gdla_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qs,
+                         const __grid_constant__ CUtensorMap tm_qn,
+                         const __grid_constant__ CUtensorMap tm_dox,
+                         const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v, const BwdParams p) {
+  using L = DkdvSmemLayout<D>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if ((smem_u32(smem) & 1023u) != 0) {
+    if (threadIdx.x == 0) write_status(p.status, -4 /* GDLA_ERR_CUDA */);
+    return;
+  }
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + L::kBarOff;
+  const uint32_t kv_full = bar0;
+  auto ring_full = [&](uint32_t s) { return bar0 + 8u * (1 + s); };
+  auto ring_empty = [&](uint32_t s) { return bar0 + 8u * (1 + L::kStages + s); };
+  const uint32_t s_full = bar0 + 8u * (1 + 2 * L::kStages);
+  const uint32_t p_full = s_full + 8u;
+  const uint32_t acc_done = s_full + 16u;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
+  const int warp = threadIdx.x >> 5;
+  const int H80 = p.Hs + p.Hn;
+  const int n_heads = p.g + 1;
+
+  const int item = blockIdx.x;
+  const int kb = item / (p.B * p.Hn);
+  const int rest = item % (p.B * p.Hn);
+  const int b = rest / p.Hn, kvh = rest % p.Hn;
+  const int k0 = kb * kBN;
+  int qlo, qhi;
+  dkdv_qrange(p, kb, qlo, qhi);
+  const int nq = qhi - qlo + 1;
+  const int n_tiles = n_heads * nq;
+  // head of tile number tt (noise head first, then the group's signal heads)
+  auto tile_head = [&](int tt) {
+    const int hh = tt / nq;
+    return hh == 0 ? p.Hs + kvh : p.g * kvh + (hh - 1);
+  };
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (uint32_t s = 0; s < L::kStages; ++s) {
+      mbar_init(ring_full(s), 1);
+      mbar_init(ring_empty(s), 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 8);
+    mbar_init(acc_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kBwdMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t t_s = tmem, t_dp = tmem + 128u;
+  const uint32_t t_dv = tmem + 256u, t_dk = tmem + 256u + D;
+
+  if (warp == kBwdProducerWarp) {
+    // =============================== TMA: K, V once; then per tile the
+    // head's query block: Q_x, dH_x, its lse and Delta rows
+    const bool leader = elect_one();
+    if (leader) {
+      mbar_arrive_expect_tx(kv_full, 2 * L::kTile);
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        tma_load_3d(sbase + L::kKOff + c * L::kSub, &tm_k, kv_full, kvh * D + c * 64, k0, b);
+        tma_load_3d(sbase + L::kVOff + c * L::kSub, &tm_v, kv_full, kvh * D + c * 64, k0, b);
+      }
+    }
+    bool ok = true;
+    uint32_t issued = 0;
+    for (int tt = 0; tt < n_tiles && ok; ++tt) {
+      const uint32_t s = tt % L::kStages;
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(ring_empty(s), ((tt / L::kStages) & 1u) ^ 1u, abort_flag));
+      if (!ok) break;
+      const int xh = tile_head(tt);
+      const int q0 = (qlo + tt % nq) * kBM;
+      const uint32_t dst = sbase + L::kRingOff + s * L::kEntry;
+      if (leader) {
+        mbar_arrive_expect_tx(ring_full(s), 2 * L::kTile + L::kStatBytes);
+        const bool noise = xh >= p.Hs;
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_3d(dst + c * L::kSub, noise ? &tm_qn : &tm_qs, ring_full(s),
+                      (noise ? xh - p.Hs : xh) * D + c * 64, q0, b);
+          tma_load_3d(dst + L::kTile + c * L::kSub, &tm_dox, ring_full(s), xh * D + c * 64, q0,
+                      b);
+        }
+        const int64_t so = (static_cast<int64_t>(b) * H80 + xh) * p.tp + q0;
+        bulk_load(dst + 2 * L::kTile, p.lse + so, kBM * 4, ring_full(s));
+        bulk_load(dst + 2 * L::kTile + kBM * 4, p.delta + so, kBM * 4, ring_full(s));
+      }
+      ++issued;
+    }
+    if (!ok && leader) {
+      for (uint32_t s = 0; s < L::kStages; ++s) {
+        const uint32_t n_s = issued > s ? (issued - 1 - s) / L::kStages + 1 : 0;
+        if (n_s) mbar_wait_for(ring_full(s), (n_s - 1) & 1u, 100000000ull);
+      }
+      mbar_wait_for(kv_full, 0, 100000000ull);
+    }
+  } else if (warp == kBwdMmaWarp) {
+    // =============================== MMA: S^T, dP^T; then dV += P^T dH,
+    // dK += dS^T Q
+    const bool leader = elect_one();
+    constexpr uint32_t kIdescS = idesc_bf16_f32(kBN, kBM, false, false);
+    constexpr uint32_t kIdescA = idesc_bf16_f32(kBN, D, false, true);
+    const uint64_t kd = sdesc_sw128(sbase + L::kKOff, 16, 1024);
+    const uint64_t vd = sdesc_sw128(sbase + L::kVOff, 16, 1024);
+    bool ok = __all_sync(0xffffffffu, mbar_wait(kv_full, 0, abort_flag));
+    bool done = false;
+    for (int tt = 0; tt < n_tiles && ok; ++tt) {
+      const uint32_t s = tt % L::kStages;
+      ok = __all_sync(0xffffffffu, mbar_wait(ring_full(s), (tt / L::kStages) & 1u, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t qbase = sbase + L::kRingOff + s * L::kEntry;
+      const uint32_t dobase = qbase + L::kTile;
+      if (leader) {
+        const uint64_t qdk = sdesc_sw128(qbase, 16, 1024);
+        const uint64_t dodk = sdesc_sw128(dobase, 16, 1024);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k >> 2) * L::kSub + (k & 3) * 32;
+          umma_ss(t_s, kd + (off >> 4), qdk + (off >> 4), kIdescS, k > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k >> 2) * L::kSub + (k & 3) * 32;
+          umma_ss(t_dp, vd + (off >> 4), dodk + (off >> 4), kIdescS, k > 0 ? 1u : 0u);
+        }
+        umma_commit(s_full);
+      }
+      ok = __all_sync(0xffffffffu, mbar_wait(p_full, static_cast<uint32_t>(tt) & 1u, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      if (leader) {
+        // B operands MN-major over d: dH_x and Q_x, 16 query rows per K-step
+        const uint64_t domn = sdesc_sw128(dobase, kBM * 128, 1024);
+        const uint64_t qmn = sdesc_sw128(qbase, kBM * 128, 1024);
+#pragma unroll
+        for (int k = 0; k < kBM / 16; ++k)
+          umma_ts(t_dv, t_s + split_col(k), domn + ((k * (16 * 128)) >> 4), kIdescA,
+                  (tt > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+        for (int k = 0; k < kBM / 16; ++k)
+          umma_ts(t_dk, t_dp + split_col(k), qmn + ((k * (16 * 128)) >> 4), kIdescA,
+                  (tt > 0 || k > 0) ? 1u : 0u);
+        umma_commit(ring_empty(s));
+        if (tt == n_tiles - 1) umma_commit(acc_done);
+      }
+      if (tt == n_tiles - 1) done = true;
+    }
+    if (leader && done) mbar_wait_for(acc_done, 0, 100000000ull);
+  } else if (warp >= 8 && warp < 12) {
+    // =============================== epilogue: dK = scale * sum dS^T Q, dV
+    const int wq = warp & 3;
+    const int r = threadIdx.x & 127;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const int j = k0 + r;
+    bool ok = __all_sync(0xffffffffu, mbar_wait(acc_done, 0, abort_flag));
+    if (ok) {
+      tc_fence_after();
+      const int64_t off = ((static_cast<int64_t>(b) * p.T + j) * p.Hn + kvh) * D;
+#pragma unroll
+      for (int w2 = 0; w2 < 2; ++w2) {
+        const uint32_t src = w2 == 0 ? t_dk : t_dv;
+        const float f = w2 == 0 ? p.scale : 1.f;
+        __nv_bfloat16 *dst = (w2 == 0 ? p.dk : p.dv) + off;
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t v[32];
+          tmem_ld32_sync(src + lane_off + cc * 32, v);
+          if (j < p.T) {
+            uint4 *op = reinterpret_cast<uint4 *>(dst + cc * 32);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              op[q] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * q]) * f,
+                                             __uint_as_float(v[8 * q + 1]) * f),
+                                 pack_bf16x2(__uint_as_float(v[8 * q + 2]) * f,
+                                             __uint_as_float(v[8 * q + 3]) * f),
+                                 pack_bf16x2(__uint_as_float(v[8 * q + 4]) * f,
+                                             __uint_as_float(v[8 * q + 5]) * f),
+                                 pack_bf16x2(__uint_as_float(v[8 * q + 6]) * f,
+                                             __uint_as_float(v[8 * q + 7]) * f));
+          }
+        }
+      }
+    }
+  } else if (warp < 8) {
+    // =============================== P^T and dS^T, half the query columns each
+    const int half = warp >> 2, wq = warp & 3;
+    const int r = threadIdx.x & 127;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const int j = k0 + r;  // key token of this row
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+    for (int tt = 0; tt < n_tiles && ok; ++tt) {
+      const uint32_t s = tt % L::kStages;
+      ok = __all_sync(0xffffffffu, mbar_wait(s_full, static_cast<uint32_t>(tt) & 1u, abort_flag));
+      // the entry's lse and Delta rows came by bulk copy: observe their barrier
+      // too (complete already; the stage is not reloaded before this tile's
+      // dV and dK MMAs, which wait for these warps)
+      if (ok)
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait(ring_full(s), (static_cast<uint32_t>(tt) / L::kStages) & 1u,
+                                  abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      const float *lse = reinterpret_cast<const float *>(smem + L::kRingOff + s * L::kEntry +
+                                                         2 * L::kTile);
+      const float *dlt = lse + kBM;
+      const int q0 = (qlo + tt % nq) * kBM;
+      // query columns c of this tile that keep key j
+      int c_lo, c_hi;
+      if (p.causal) {
+        c_lo = j - q0;  // queries at or after the key
+        c_hi = p.window > 0 ? static_cast<int>(static_cast<int64_t>(j) + p.window - 1 - q0) : kBM;
+        c_hi = min(c_hi, p.T - 1 - q0);
+      } else {
+        c_lo = 0;
+        c_hi = p.T - 1 - q0;
+      }
+      if (j >= p.T) c_hi = -1;  // padding key rows keep nothing
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int cc = 2 * half + u;
+        uint32_t sv[32], dpv[32];
+        tmem_ld32x2_sync(t_s + lane_off + 32 * cc, t_dp + lane_off + 32 * cc, sv, dpv);
+        uint32_t pk[16], dk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int c0 = 32 * cc + 2 * e;
+          const bool a0 = c0 >= c_lo && c0 <= c_hi;
+          const bool a1 = c0 + 1 >= c_lo && c0 + 1 <= c_hi;
+          const float p0 = a0 ? ex2_approx(__uint_as_float(sv[2 * e]) * sl2 - lse[c0]) : 0.f;
+          const float p1 = a1 ? ex2_approx(__uint_as_float(sv[2 * e + 1]) * sl2 - lse[c0 + 1]) : 0.f;
+          pk[e] = pack_bf16x2(p0, p1);
+          // selected, not multiplied: a masked column's lse and Delta may be
+          // the unwritten padding past T
+          dk[e] = pack_bf16x2(a0 ? p0 * (__uint_as_float(dpv[2 * e]) - dlt[c0]) : 0.f,
+                              a1 ? p1 * (__uint_as_float(dpv[2 * e + 1]) - dlt[c0 + 1]) : 0.f);
+        }
+        tmem_st16(t_s + lane_off + 64 * half + 16 * u, pk);
+        tmem_st16(t_dp + lane_off + 64 * half + 16 * u, dk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      warp_arrive(p_full);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0) write_status(p.status, -5 /* GDLA_ERR_TIMEOUT */);
+  if (warp == kBwdMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace gdla

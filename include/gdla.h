@@ -246,6 +246,48 @@ int gdla_decode_fwd(const void *q_sig, const void *q_noise, const void *c_hat,
                     void *stream);
 
 /*
+ * gdla_attn_bwd_workspace_bytes - bytes of device scratch gdla_attn_bwd needs
+ * for these shapes: every head's output H (fp32), its log-sum-exp and the
+ * softmax-gradient term Delta (fp32), and its upstream gradient (bf16);
+ * about (Hs + Hn) * (6 d + 8) bytes per token.  0 for invalid shapes.
+ */
+size_t gdla_attn_bwd_workspace_bytes(int B, int64_t T, int Hs, int Hn, int d);
+
+/*
+ * gdla_attn_bwd - gradients of the GDLA attention forward (gdla_attn_fwd) for
+ * an upstream gradient d_out of its output.  The pages give the forward only
+ * ("Motif 3: Technical Report", paper.rainbus.top, step 2) and say the model
+ * is trained with it ("Вышла новая модель Motif 3", pikabu.ru); these are the
+ * chain-rule gradients of that forward:
+ *   dgate    = d_out (.) D,           dD = d_out (.) G
+ *   dlambda  = -sum_c dD (.) Repeat_g(H_N)        (per token and signal head)
+ *   dq_sig, dq_noise, dk, dv: the softmax-attention gradients of both paths
+ *   for upstream gradients dH_S = dD and dH_N = -sum_{group} lambda dD; dk and
+ *   dv add up the g signal heads and the noise head of each KV group.
+ * The forward is recomputed inside (H and the log-sum-exp of every head), so
+ * only the forward's inputs are needed.
+ *
+ * q_sig, q_noise, k, v, lambda, gate   as in gdla_attn_fwd, read
+ * d_out     [B, T, Hs * d]   bf16, read
+ * dq_sig    [B, T, Hs, d], dq_noise [B, T, Hn, d], dk, dv [B, T, Hkv, d],
+ * dlambda   [B, T, Hs], dgate [B, T, Hs * d]: bf16, written (fp32 accumulate,
+ *           one rounding); none may overlap another argument
+ * workspace device scratch of at least gdla_attn_bwd_workspace_bytes(...)
+ *           bytes, 16-byte aligned, owned by the caller; contents on entry do
+ *           not matter; calls that overlap on the GPU must not share it
+ * window, causal, scale, d_status, stream   as in gdla_attn_fwd
+ * Supported: Hn == Hkv, Hs / Hn <= 8, d in {64, 128}.  Four kernels are
+ * enqueued on `stream`.
+ */
+int gdla_attn_bwd(const void *q_sig, const void *q_noise, const void *k,
+                  const void *v, const void *lambda, const void *gate,
+                  const void *d_out, void *dq_sig, void *dq_noise, void *dk,
+                  void *dv, void *dlambda, void *dgate, int B, int64_t T,
+                  int Hs, int Hn, int Hkv, int d, int64_t window, int causal,
+                  float scale, void *workspace, size_t workspace_bytes,
+                  int *d_status, void *stream);
+
+/*
  * gdla_selftest_wait_timeout - device-side check of the failure path.
  *
  * Every pipeline wait inside the kernels above polls an mbarrier with a time

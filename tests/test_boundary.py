@@ -37,7 +37,8 @@ def test_exports_every_declared_symbol(lib):
                              "gdla_attn_fwd", "gdla_attn_fwd_sp", "gdla_latent_rmsnorm",
                              "gdla_decode_workspace_bytes", "gdla_decode_fwd",
                              "gdla_selftest_wait_timeout", "gdla_decode_fwd_noalloc",
-                             "gdla_attn_fwd_rope"}
+                             "gdla_attn_fwd_rope", "gdla_attn_bwd_workspace_bytes",
+                             "gdla_attn_bwd"}
     for name in declared:
         assert hasattr(lib, name), f"{name} missing from libgdla.so"
     assert set(declared) == set(_binding.EXPORTED)
@@ -96,6 +97,40 @@ def _rope(lib, q=A, qn=A, qr=A, qrn=A, k=A, v=A, kr=A, lam=A, gate=A, out=A, B=1
 ])
 def test_rope_argument_errors(lib, kw, code):
     assert _rope(lib, **kw) == code
+
+
+def _bwd(lib, q=A, qn=A, k=A, v=A, lam=A, gate=A, do=A, dqs=A, dqn=A, dk=A, dv=A, dl=A, dg=A,
+         B=1, T=256, Hs=8, Hn=2, Hkv=2, d=64, window=0, causal=1, scale=0.0, ws=A,
+         ws_bytes=1 << 40, status=None):
+    return lib.gdla_attn_bwd(q, qn, k, v, lam, gate, do, dqs, dqn, dk, dv, dl, dg, B, T, Hs, Hn,
+                             Hkv, d, window, causal, ctypes.c_float(scale), ws, ws_bytes, status,
+                             None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), INVALID), (dict(do=None), INVALID), (dict(dk=None), INVALID),
+    (dict(dg=None), INVALID), (dict(ws=None), INVALID), (dict(B=-1), INVALID),
+    (dict(window=-1), INVALID), (dict(causal=0, window=3), INVALID),
+    (dict(scale=float("nan")), INVALID), (dict(ws_bytes=1024), INVALID),
+    (dict(Hs=6, Hn=4, Hkv=4), UNSUPPORTED), (dict(Hs=18, Hn=2, Hkv=2), UNSUPPORTED),
+    (dict(d=96), UNSUPPORTED), (dict(Hn=2, Hkv=4), UNSUPPORTED),
+    (dict(q=M), ALIGN), (dict(do=M), ALIGN), (dict(dv=M), ALIGN), (dict(ws=M), ALIGN),
+    (dict(status=0x100002), ALIGN),
+    (dict(T=0), OK), (dict(B=0), OK),
+])
+def test_bwd_argument_errors(lib, kw, code):
+    assert _bwd(lib, **kw) == code
+
+
+def test_bwd_workspace_size_follows_the_shapes(lib):
+    f = lib.gdla_attn_bwd_workspace_bytes
+    up = lambda x: (x + 255) // 256 * 256
+    # B=2, T=300 (padded to 384 for the statistics), 8 + 2 heads, d=64
+    rows, h80, tp = 600, 10, 384
+    want = up(up(up(rows * h80 * 64 * 4) + 2 * h80 * tp * 4) + 2 * h80 * tp * 4) + \
+        rows * h80 * 64 * 2
+    assert f(2, 300, 8, 2, 64) == up(want)
+    assert f(0, 300, 8, 2, 64) == 0 and f(2, 0, 8, 2, 64) == 0
 
 
 def _expand(lib, c=A, w=None, wk=A, eps=1e-6, k=A, v=A, n=300, dl=512, hkv=16, dh=128,
