@@ -55,12 +55,20 @@ STEPS = {
     "decode_window": ("decode_window",),
     "full_rope": ("full_rope",),
     "window_rope": ("window_rope",),
+    "bwd_full": ("bwd_full",),
+    "bwd_window": ("bwd_window",),
 }
+# The gradients of a backward layer, in the order they sit in its output buffer.
+BWD_GRADS = ("dq_sig", "dq_noise", "dk", "dv", "dlam", "dgate")
 # A timed region at least this long runs tensor-bound kernels under the power
 # cap, so their fraction is taken against the sustained bf16 peak.
 SUSTAINED_AFTER_S = 2.0
 # Query rows the CPU sample draws from (the first tokens of batch element 0).
 SAMPLE_SPAN = 4096
+# Tokens of the causal prefix the oracle's backward runs on for the CPU sample;
+# its rows' dQ, dlambda and dG equal the full problem's (they depend on
+# earlier keys only).
+BWD_SPAN = 512
 
 
 def _peaks():
@@ -80,9 +88,29 @@ def _dist():
     return world, rank, local
 
 
+def bwd_grad_shapes(wl):
+    return {"dq_sig": (wl.B, wl.T, wl.Hs, wl.d), "dq_noise": (wl.B, wl.T, wl.Hn, wl.d),
+            "dk": (wl.B, wl.T, wl.Hkv, wl.d), "dv": (wl.B, wl.T, wl.Hkv, wl.d),
+            "dlam": (wl.B, wl.T, wl.Hs), "dgate": (wl.B, wl.T, wl.Hs * wl.d)}
+
+
+def bwd_grad_views(wl, flat):
+    """The six gradients as views of one flat bf16 buffer."""
+    out, o = {}, 0
+    for n, sh in bwd_grad_shapes(wl).items():
+        k = 1
+        for e in sh:
+            k *= e
+        out[n] = flat[o:o + k].view(sh)
+        o += k
+    return out
+
+
 def attn_kernel_name(wl) -> str:
     """The kernel gdla_attn_fwd dispatches this layer to (window >= T is full
     causal; windows of 1..128 keys take the union-row kernel)."""
+    if wl.bwd:
+        return "gdla_attn_bwd"
     if wl.d_rope:
         return "gdla_attn_rope_kernel"
     if wl.causal and 0 < wl.window < wl.T:
@@ -188,6 +216,21 @@ class Layer:
             self.launches.append(("%s/decode" % wl.name, "gdla_decode_attn_kernel",
                                   wl.attn_flops(), wl.decode_bytes(), 3))
             return
+        if wl.bwd:
+            # the six gradients in one buffer (the step's output), the scratch
+            n_out = 0
+            for sh in bwd_grad_shapes(wl).values():
+                k = 1
+                for e in sh:
+                    k *= e
+                n_out += k
+            self.out = torch.empty(n_out, dtype=torch.bfloat16, device=dev)
+            self.ws = torch.empty(gdla.gdla_attn_bwd_workspace_bytes(wl.B, wl.T, wl.Hs, wl.Hn,
+                                                                     wl.d),
+                                  dtype=torch.uint8, device=dev)
+            self.launches.append(("%s/bwd" % wl.name, "gdla_attn_bwd", wl.bwd_flops(),
+                                  wl.bwd_bytes(), 4))
+            return
         if wl.latent:
             self.kbuf = torch.empty((n_tok, wl.Hkv, wl.d), dtype=torch.bfloat16, device=dev)
             self.vbuf = torch.empty_like(self.kbuf)
@@ -210,6 +253,16 @@ class Layer:
                                  self.cache_len if cache_len is None else cache_len,
                                  self.x["w_kvb"], inp["lam"], inp["gate"], window=wl.window,
                                  out=out, workspace=self.ws, d_status=status, stream=stream)
+            if events is not None:
+                events[0][1].record(stream)
+            return
+        if wl.bwd:
+            if events is not None:
+                events[0][0].record(stream)
+            gdla.gdla_attn_bwd(inp["q_sig"], inp["q_noise"], inp["k"], inp["v"], inp["lam"],
+                               inp["gate"], inp["d_out"], window=wl.window, causal=wl.causal,
+                               grads=bwd_grad_views(wl, out), workspace=self.ws,
+                               d_status=status, stream=stream)
             if events is not None:
                 events[0][1].record(stream)
             return
@@ -343,6 +396,11 @@ def run_ours(args):
             o = torch.empty_like(L.out)
             L.run(gdla, status, stream, out=o, cache_len=span)
             head_out.append(o.float().cpu())
+        elif L.wl.bwd:
+            # the row-local gradients of the first BWD_SPAN tokens of batch 0
+            gv = bwd_grad_views(L.wl, L.out)
+            head_out.append({n: gv[n][:1, :min(L.wl.T, BWD_SPAN)].float().cpu()
+                             for n in ("dq_sig", "dq_noise", "dlam", "dgate")})
         else:
             head_out.append(L.out[:1, :min(L.wl.T, SAMPLE_SPAN)].float().cpu())
 
@@ -546,6 +604,8 @@ def _oracle_sample(wl, x, seconds, rng):
     span = min(wl.T, SAMPLE_SPAN)
     if wl.decode:
         return _oracle_decode_sample(wl, x, seconds, rng, span)
+    if wl.bwd:
+        return _oracle_bwd_sample(wl, x, seconds)
     # rows per pass: a sliding-window row costs W pairs, a causal row up to span
     n_rows = 256 if wl.window > 0 else 8
     total_flops, total_s = 0, 0.0
@@ -588,6 +648,28 @@ def _oracle_sample(wl, x, seconds, rng):
         wl.name, n_done, wl.Hs + wl.Hn, span,
         ", plus RMSNorm+W^KV_b expand of those %d tokens per pass" % span if wl.latent else ""))
     return total_flops, total_s, desc, np.concatenate(all_rows), np.concatenate(all_ref)
+
+
+def _oracle_bwd_sample(wl, x, seconds):
+    """The backward sample: the oracle's backward of the causal prefix of the
+    first BWD_SPAN tokens of batch element 0, repeated for the time budget.
+    Rows are token indices; ref holds the row-local gradients."""
+    import oracle
+    span = min(wl.T, BWD_SPAN)
+    cpu = {n: x[n][:1, :span].cpu() for n in ("q_sig", "q_noise", "k", "v", "lam", "gate", "d_out")}
+    sub = type(wl)(wl.name, B=1, T=span, Hs=wl.Hs, Hn=wl.Hn, Hkv=wl.Hkv, d=wl.d,
+                   window=wl.window, causal=wl.causal, bwd=True)
+    total_s, passes, ref = 0.0, 0, None
+    while total_s < seconds or passes == 0:
+        t0 = time.perf_counter()
+        ref = oracle.gdla_attn_bwd(*(cpu[n] for n in ("q_sig", "q_noise", "k", "v", "lam", "gate",
+                                                    "d_out")), window=wl.window,
+                                   causal=wl.causal)
+        total_s += time.perf_counter() - t0
+        passes += 1
+    desc = ("%s: the backward of the first %d tokens of batch element 0 (all %d heads), %d "
+            "passes" % (wl.name, span, wl.Hs + wl.Hn, passes))
+    return sub.bwd_flops() * passes, total_s, desc, None, ref
 
 
 def _oracle_decode_sample(wl, x, seconds, rng, span):
@@ -646,6 +728,13 @@ def cpu_baseline(layers, head_out, seconds=15.0):
         flops += f
         secs += s
         descs.append(d)
+        if L.wl.bwd:
+            for n, g in ho.items():
+                span = g.shape[1]
+                parity["%s/%s" % (L.wl.name, n)] = _parity(
+                    g[0].reshape(span, -1).numpy().astype(np.float64),
+                    ref[n][0].reshape(span, -1))
+            continue
         gpu_rows = (ho if L.wl.decode else ho[0]).numpy()[rows].astype(np.float64)
         parity[L.wl.name] = _parity(gpu_rows, ref)
     threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))

@@ -15,8 +15,9 @@ c_KV [B, T, 512] and W^KV_b in that order):
   gate   = bf16(sigmoid(N(0, 1)))  shape [B, T, Hs*d]
   c_KV   ~ N(0, 1) bf16            shape [B*T, 512]      (latent workload)
   W^KV_b ~ N(0, 1/512) bf16        shape [512, Hkv*(dk+dv)]
-and, for workloads with the decoupled rotary term (d_rope > 0), drawn after
-everything above so the other inputs do not change:
+then, for backward workloads, the upstream gradient dO ~ N(0, 1) bf16
+[B, T, Hs*d]; and, for workloads with the decoupled rotary term (d_rope > 0),
+drawn after everything above so the other inputs do not change:
   Q_rope_sig, Q_rope_noise ~ N(0, 1) bf16  shape [B, T, H, d_rope]
   K_rope                   ~ N(0, 1) bf16  shape [B, T, d_rope]
 The same seed on a different device gives a different (but again fixed)
@@ -51,6 +52,7 @@ class Workload:
     eps: float = 1e-6
     decode: bool = False     # one query token per sequence over a T-token latent cache
     d_rope: int = 0          # width of the decoupled rotary term (0: none)
+    bwd: bool = False        # the backward: gradients for an upstream dO
 
     @property
     def g(self) -> int:
@@ -88,6 +90,19 @@ class Workload:
                        + (self.Hs + self.Hn + 1) * self.d_rope)
         return per_tok * self.B * self.T
 
+    def bwd_flops(self) -> int:
+        """The backward's algorithmic work: S recomputed, dP, dS K, dS^T Q and
+        P^T dO, 2*d FLOPs each per kept pair per head (10*d, 2.5x the
+        forward's 4*d)."""
+        return 10 * self.d * (self.Hs + self.Hn) * self.B * self.pairs_per_batch()
+
+    def bwd_bytes(self) -> int:
+        """The forward's inputs and dO read once, the six gradients written
+        once, bfloat16 everywhere."""
+        per_tok = 2 * (2 * (self.Hs * self.d + self.Hn * self.d + 2 * self.Hkv * self.d
+                            + self.Hs + self.Hs * self.d) + self.Hs * self.d)
+        return per_tok * self.B * self.T
+
     def expand_flops(self) -> int:
         return 2 * self.B * self.T * self.d_latent * self.Hkv * 2 * self.d
 
@@ -112,6 +127,9 @@ WORKLOADS: Dict[str, Workload] = {
     # width that keeps the latent cache the size of MLA's: 512 + 64)
     "full_rope": Workload("full_rope", B=2, T=8192, d_rope=64),
     "window_rope": Workload("window_rope", B=8, T=4096, window=128, d_rope=64),
+    # the backward of the full-attention and sliding-window layers
+    "bwd_full": Workload("bwd_full", B=2, T=8192, bwd=True),
+    "bwd_window": Workload("bwd_window", B=8, T=4096, window=128, bwd=True),
 }
 
 
@@ -162,6 +180,8 @@ def make_inputs(wl: Workload, seed: int = 0, device="cpu",
         out["c_kv"] = _normal_bf16((B * T, wl.d_latent), gen, device)
         out["w_kvb"] = _normal_bf16((wl.d_latent, wl.Hkv * 2 * wl.d), gen, device,
                                     std=(1.0 / wl.d_latent) ** 0.5)
+    if wl.bwd:
+        out["d_out"] = _normal_bf16((B, T, wl.Hs * wl.d), gen, device)
     if wl.d_rope:
         out["q_rope_sig"] = _normal_bf16((B, T, wl.Hs, wl.d_rope), gen, device)
         out["q_rope_noise"] = _normal_bf16((B, T, wl.Hn, wl.d_rope), gen, device)
