@@ -28,7 +28,9 @@ namespace gdla {
 constexpr int kDecTok = 128;    // cached tokens per chunk (MMA M of S^T)
 constexpr int kDecUnit = 128;   // latent columns per ring unit (MMA M of z^T)
 constexpr int kDecRing = 3;     // ring depth (units of [128 tokens][128 latent])
-constexpr int kDecThreads = 192;  // warps 0-3 softmax / partials, 4 TMA, 5 MMA
+constexpr int kDecThreads = 320;  // warps 0-7 softmax / partials (two halves of the heads), 8 TMA, 9 MMA
+constexpr int kDecTmaWarp = 8;
+constexpr int kDecMmaWarp = 9;
 constexpr int kDecMaxLatent = 512;
 constexpr int kDecMaxGroup = 8;   // signal heads per KV group in the decode kernels
 constexpr int kDecMaxSplit = 256;  // splits per sequence (the host plan stays below)
@@ -164,7 +166,7 @@ struct DecSmem {
   static constexpr uint32_t kRefOff = kRedOff + kRedBytes;  // int ref[2][4][NP] (per warp, per chunk parity)
   static constexpr uint32_t kBarOff = kRefOff + 2 * 4 * NP * 4;
   static constexpr int kZStride = (NP + 31) / 32 * 32;        // TMEM columns per z^T block
-  static constexpr uint32_t kNumBars = 2 * kDecRing + 6;
+  static constexpr uint32_t kNumBars = 2 * kDecRing + 8;
   static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;
   static constexpr uint32_t kBytes = kMiscOff + 16;
   static_assert(kQtBytes % 1024 == 0 && kRingOff % 1024 == 0 && kPOff % 1024 == 0,
@@ -173,6 +175,24 @@ struct DecSmem {
   static_assert(NP % 16 == 0 && NP <= 80, "head rows: a multiple of 16, at most 80");
 };
 
+// Warp-collective load / store of 8 consecutive 32-bit TMEM columns of the
+// warp's 32 lanes (thread i: lane addr.lane + i).
+__device__ __forceinline__ void tmem_ld8_sync(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
+}
+
 // One arrival per warp after the lanes' own writes.
 __device__ __forceinline__ void dec_warp_arrive(uint32_t bar) {
   __syncwarp();
@@ -180,8 +200,10 @@ __device__ __forceinline__ void dec_warp_arrive(uint32_t bar) {
 }
 
 // One CTA per (split s, sequence b); NP = head rows (Hs + Hn padded to 16).
-// Warps 0-3: softmax (thread t = token t of the chunk = TMEM lane t) and the
-// partial results; warp 4: TMA; warp 5: TMEM allocation and MMA issue.
+// Warps 0-7: softmax (thread t = token t of the chunk = TMEM lane t) and the
+// partial results, warps 0-3 for heads 0 .. NP/2-1 and warps 4-7 for the
+// rest (the heads are independent, so the halves never wait on each other);
+// warp 8: TMA; warp 9: TMEM allocation and MMA issue.
 // TMEM: S^T [0, NP), z^T block u (latent rows 128u..128u+127) at
 // [Z (1 + u), Z (1 + u) + NP) with Z = NP rounded up to 32 columns.
 template <int NP>
@@ -216,7 +238,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   const uint32_t s_full = bar0 + 8u * (2 * kDecRing + 1);   // S^T of a chunk written
   const uint32_t p_full = bar0 + 8u * (2 * kDecRing + 2);   // P written, z^T rescaled
   const uint32_t z_done = bar0 + 8u * (2 * kDecRing + 3);   // z^T MMAs of a chunk done
-  auto red_full = [&](int i) { return bar0 + 8u * (2 * kDecRing + 4 + i); };  // maxima exchanged
+  // maxima exchanged among the four warps of one half of the heads
+  auto red_full = [&](int half, int i) { return bar0 + 8u * (2 * kDecRing + 4 + 2 * half + i); };
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
   int *red = reinterpret_cast<int *>(smem + L::kRedOff);                  // [2][4][NP]
@@ -231,14 +254,16 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     }
     mbar_init(qt_full, 1);
     mbar_init(s_full, 1);
-    mbar_init(p_full, 4);
+    mbar_init(p_full, 8);
     mbar_init(z_done, 1);
-    mbar_init(red_full(0), 4);
-    mbar_init(red_full(1), 4);
+    for (int hf = 0; hf < 2; ++hf) {
+      mbar_init(red_full(hf, 0), 4);
+      mbar_init(red_full(hf, 1), 4);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == kDecMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
@@ -250,7 +275,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   auto t_z = [&](int u) { return tmem + static_cast<uint32_t>(L::kZStride * (1 + u)); };
   const uint32_t sP = sbase + L::kPOff;
 
-  if (warp == 4) {
+  if (warp == kDecTmaWarp) {
     // =============================== TMA: q~ once, then per chunk the units
     // of pass 1 (scores) and of pass 2 (z^T; the same rows again, from L2)
     const bool leader = elect_one();
@@ -288,7 +313,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       }
       mbar_wait_for(qt_full, 0, 100000000ull);
     }
-  } else if (warp == 5) {
+  } else if (warp == kDecMmaWarp) {
     // =============================== MMA issue (one elected lane)
     const bool leader = elect_one();
     const uint32_t idesc_s = idesc_bf16_f32(kDecTok, NP, false, false);
@@ -350,41 +375,45 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     if (leader && commits) mbar_wait_for(z_done, (commits - 1) & 1u, 100000000ull);
   } else {
     // =============================== softmax over the chunk's tokens, per head
-    const int w = warp;
+    // (this half's heads hb .. hb + NH - 1)
+    constexpr int NH = NP / 2;
+    const int half = warp >> 2;
+    const int w = warp & 3;
+    const int hb = half * NH;
     const int lane = threadIdx.x & 31;
-    const int t = threadIdx.x;  // token row of the chunk = TMEM lane
+    const int t = threadIdx.x & 127;  // token row of the chunk = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(w * 32) << 16;
-    float lsum[NP];
+    float lsum[NH];
 #pragma unroll
-    for (int h = 0; h < NP; ++h) lsum[h] = 0.f;
-    for (int i = lane; i < NP; i += 32) refw[w * NP + i] = refw[(4 + w) * NP + i] = INT_MIN;
+    for (int h = 0; h < NH; ++h) lsum[h] = 0.f;
+    for (int i = hb + lane; i < hb + NH; i += 32) refw[w * NP + i] = refw[(4 + w) * NP + i] = INT_MIN;
     __syncwarp();
     bool ok = true;
     for (int ch = 0; ch < n_chunks && ok; ++ch) {
       ok = __all_sync(0xffffffffu, mbar_wait(s_full, ch & 1u, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      float sv[NP];
+      float sv[NH];
 #pragma unroll
-      for (int i = 0; i < NP / 16; ++i) {
-        uint32_t r16[16];
-        tmem_ld16_sync(t_s + lane_off + 16 * i, r16);
+      for (int i = 0; i < NH / 8; ++i) {
+        uint32_t r8[8];
+        tmem_ld8_sync(t_s + lane_off + hb + 8 * i, r8);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) sv[16 * i + e] = __uint_as_float(r16[e]);
+        for (int e = 0; e < 8; ++e) sv[8 * i + e] = __uint_as_float(r8[e]);
       }
       const int64_t tok = (rg.c_begin + ch) * kDecTok + t;
       const bool valid = tok >= rg.t_lo && tok < rg.len;
       // per head: the chunk's largest score rounded up to an integer, over the
-      // warp (one redux each), then over the four warps through shared memory
+      // warp (one redux each), then over the half's four warps through shared memory
       int *rb = red + (ch & 1) * 4 * NP;
 #pragma unroll
-      for (int h = 0; h < NP; ++h) {
+      for (int h = 0; h < NH; ++h) {
         const int mi = valid ? static_cast<int>(ceilf(sv[h])) : INT_MIN;
         const int wm = __reduce_max_sync(0xffffffffu, mi);
-        if (lane == 0) rb[w * NP + h] = wm;
+        if (lane == 0) rb[w * NP + hb + h] = wm;
       }
-      dec_warp_arrive(red_full(ch & 1));
-      ok = __all_sync(0xffffffffu, mbar_wait(red_full(ch & 1), (ch >> 1) & 1u, abort_flag));
+      dec_warp_arrive(red_full(half, ch & 1));
+      ok = __all_sync(0xffffffffu, mbar_wait(red_full(half, ch & 1), (ch >> 1) & 1u, abort_flag));
       if (!ok) break;
       // the previous chunk's z^T MMAs must be done before P is overwritten or
       // z^T rescaled
@@ -394,13 +423,13 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         tc_fence_after();
       }
       // new integral reference per head: the lanes compute it for heads
-      // lane, lane + 32, ... into this warp's copy for the chunk (every warp
-      // computes the same values); a head's reference moves only when its
-      // maximum passes it by more than 2^8
+      // hb + lane, hb + lane + 32, ... into this warp's copy for the chunk
+      // (every warp of the half computes the same values); a head's reference
+      // moves only when its maximum passes it by more than 2^8
       const int *ref_old = refw + ((ch & 1) * 4 + w) * NP;
       int *ref_new = refw + (((ch & 1) ^ 1) * 4 + w) * NP;
       bool moved = false;
-      for (int h = lane; h < NP; h += 32) {
+      for (int h = hb + lane; h < hb + NH; h += 32) {
         const int cm = max(max(rb[h], rb[NP + h]), max(rb[2 * NP + h], rb[3 * NP + h]));
         const int old = ref_old[h];
         const bool move =
@@ -412,19 +441,20 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       if (__any_sync(0xffffffffu, moved) && ch > 0) {
         // z^T and the row sums hold earlier chunks at the old references
 #pragma unroll
-        for (int h = 0; h < NP; ++h) lsum[h] *= exp2_int(static_cast<float>(ref_old[h] - ref_new[h]));
+        for (int h = 0; h < NH; ++h)
+          lsum[h] *= exp2_int(static_cast<float>(ref_old[hb + h] - ref_new[hb + h]));
         for (int u = 0; u < U; ++u) {
 #pragma unroll
-          for (int i = 0; i < NP / 16; ++i) {
-            uint32_t r16[16];
-            tmem_ld16_sync(t_z(u) + lane_off + 16 * i, r16);
+          for (int i = 0; i < NH / 8; ++i) {
+            uint32_t r8[8];
+            tmem_ld8_sync(t_z(u) + lane_off + hb + 8 * i, r8);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int h = 16 * i + e;
+            for (int e = 0; e < 8; ++e) {
+              const int h = hb + 8 * i + e;
               const float a = exp2_int(static_cast<float>(ref_old[h] - ref_new[h]));
-              r16[e] = __float_as_uint(__uint_as_float(r16[e]) * a);
+              r8[e] = __float_as_uint(__uint_as_float(r8[e]) * a);
             }
-            tmem_st16(t_z(u) + lane_off + 16 * i, r16);
+            tmem_st8(t_z(u) + lane_off + hb + 8 * i, r8);
           }
         }
         tmem_wait_st();
@@ -435,11 +465,12 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                           static_cast<uint32_t>((t & 7) * 2);
       const uint32_t unit = static_cast<uint32_t>((t & 63) >> 3);
 #pragma unroll
-      for (int h = 0; h < NP; ++h) {
-        const float pv = valid ? ex2_approx(sv[h] - static_cast<float>(ref_new[h])) : 0.f;
+      for (int h = 0; h < NH; ++h) {
+        const int hh = hb + h;
+        const float pv = valid ? ex2_approx(sv[h] - static_cast<float>(ref_new[hh])) : 0.f;
         lsum[h] += pv;
-        const uint32_t addr = pb + static_cast<uint32_t>(h) * 128u +
-                              ((unit ^ static_cast<uint32_t>(h & 7)) << 4);
+        const uint32_t addr = pb + static_cast<uint32_t>(hh) * 128u +
+                              ((unit ^ static_cast<uint32_t>(hh & 7)) << 4);
         const unsigned short bits = __bfloat16_as_ushort(__float2bfloat16(pv));
         asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(bits) : "memory");
       }
@@ -447,36 +478,37 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       tc_fence_before();
       dec_warp_arrive(p_full);
     }
-    // ---- partial results of this split: reference, row sums, z^T
+    // ---- partial results of this split for this half's heads: reference,
+    // row sums, z^T
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(z_done, (n_chunks - 1) & 1u, abort_flag));
     if (ok) {
       tc_fence_after();
 #pragma unroll
-      for (int h = 0; h < NP; ++h) {
+      for (int h = 0; h < NH; ++h) {
         float v = lsum[h];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0) lred[w * NP + h] = v;
+        if (lane == 0) lred[w * NP + hb + h] = v;
       }
-      dec_warp_arrive(red_full(n_chunks & 1));
+      dec_warp_arrive(red_full(half, n_chunks & 1));
       ok = __all_sync(0xffffffffu,
-                      mbar_wait(red_full(n_chunks & 1), (n_chunks >> 1) & 1u, abort_flag));
+                      mbar_wait(red_full(half, n_chunks & 1), (n_chunks >> 1) & 1u, abort_flag));
     }
     if (ok) {
       const int *ref_last = refw + ((n_chunks & 1) * 4 + w) * NP;
-      for (int h = t; h < NP; h += kDecTok) {
+      for (int h = hb + t; h < hb + NH; h += kDecTok) {
         part[h] = static_cast<float>(ref_last[h]);  // this warp's copy; all copies agree
         part[NP + h] = lred[h] + lred[NP + h] + lred[2 * NP + h] + lred[3 * NP + h];
       }
       float *zp = part + 2 * NP;
       for (int u = 0; u < U; ++u) {
 #pragma unroll
-        for (int i = 0; i < NP / 16; ++i) {
-          uint32_t r16[16];
-          tmem_ld16_sync(t_z(u) + lane_off + 16 * i, r16);
+        for (int i = 0; i < NH / 8; ++i) {
+          uint32_t r8[8];
+          tmem_ld8_sync(t_z(u) + lane_off + hb + 8 * i, r8);
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            zp[static_cast<size_t>(16 * i + e) * p.dl + u * kDecUnit + t] = __uint_as_float(r16[e]);
+          for (int e = 0; e < 8; ++e)
+            zp[static_cast<size_t>(hb + 8 * i + e) * p.dl + u * kDecUnit + t] = __uint_as_float(r8[e]);
         }
       }
     }
@@ -485,7 +517,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (*abort_flag && threadIdx.x == 0 && p.status) atomicExch(p.status, -5 /* GDLA_ERR_TIMEOUT */);
-  if (warp == 5) {
+  if (warp == kDecMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
