@@ -79,76 +79,134 @@ __device__ __forceinline__ float *decode_part(const DecodeParams &p, int b, int 
 }
 
 // ---------------------------------------------------------------- absorb
-// q~ rows of KV group k (signal heads h -> row h, noise head k -> row Hs + k),
-// q~[x] = qscale * sum_c W^KV_b[x, k*2d + c] q[c]; rows Hs + Hn .. Np - 1 are
-// zero padding.  One CTA per (group k, block of 128 latent rows x, block of
-// kAbsorbSeqs sequences); thread x keeps its row of W_K in registers and
-// takes every query vector of the block's sequences from shared memory
-// (a broadcast read), so no chain waits on a global load.
-constexpr int kAbsorbSeqs = 2;
-__global__ void __launch_bounds__(128) gdla_decode_absorb_kernel(const DecodeParams p) {
-  const int k = blockIdx.x;
-  const int x = blockIdx.y * 128 + threadIdx.x;  // latent row
-  const int b0 = blockIdx.z * kAbsorbSeqs;
-  const int g = p.Hs / p.Hn, nh = g + 1, d = p.d, dl = p.dl;
-  const int nb = min(kAbsorbSeqs, p.B - b0);
-  // query vectors [sequence][head of the group][d] as bf16 pairs
-  __shared__ __align__(16) uint32_t qs[kAbsorbSeqs * (kDecMaxGroup + 1) * 64];
-  // 16-byte pieces: d / 8 per query vector
-  const int pieces = d / 8;
-  for (int i = threadIdx.x; i < nb * nh * pieces; i += blockDim.x) {
-    const int bb = i / (nh * pieces), j = (i / pieces) % nh, v = i % pieces;
-    const int b = b0 + bb;
-    const __nv_bfloat16 *src =
-        j < g ? p.q_sig + (static_cast<int64_t>(b) * p.Hs + g * k + j) * d
-              : p.q_noise + (static_cast<int64_t>(b) * p.Hn + k) * d;
-    reinterpret_cast<uint4 *>(qs + (bb * (kDecMaxGroup + 1) + j) * 64)[v] =
-        __ldg(reinterpret_cast<const uint4 *>(src) + v);
+// q~ = (scale log2 e) W_K q for every head (signal head h -> row h, noise
+// head k -> row Hs + k; rows Hs + Hn .. Np - 1 are zero padding), as one
+// tcgen05 GEMM tile per (KV group k, tile of query rows, 128 latent columns):
+//   D[r][x] = sum_c Q[r][c] W_K[x][c],   A = Q rows, B = W_K rows (both K-major)
+// A signal tile holds the group's g signal heads of 128 / g sequences (one
+// TMA box of [sequences][heads][64]); a noise tile holds the noise head of
+// 128 sequences.  Warp 0 loads and issues; the four warps write the rows.
+constexpr int kAbsThreads = 128;
+
+struct AbsorbSmem {
+  static constexpr uint32_t kSub = 128 * 128;  // [128 rows][64] bf16, 128B swizzle
+  static constexpr uint32_t kAOff = 0;
+  static constexpr uint32_t kBOff = 2 * kSub;  // up to d = 128
+  static constexpr uint32_t kBarOff = kBOff + 2 * kSub;
+  static constexpr uint32_t kBytes = kBarOff + 16 + 16;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kAbsThreads, 1)
+    gdla_decode_absorb_kernel(const __grid_constant__ CUtensorMap tm_qs,
+                              const __grid_constant__ CUtensorMap tm_qn,
+                              const __grid_constant__ CUtensorMap tm_w, const DecodeParams p,
+                              int n_sig_tiles) {
+  using L = AbsorbSmem;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if ((smem_u32(smem) & 1023u) != 0) {
+    if (threadIdx.x == 0 && p.status) atomicExch(p.status, -4 /* GDLA_ERR_CUDA */);
+    return;
   }
+  const int x0 = blockIdx.x * 128;  // latent columns
+  const int k = blockIdx.y;         // KV group
+  const int g = p.Hs / p.Hn;
+  const int nb = 128 / g;           // sequences per signal tile
+  const bool noise = static_cast<int>(blockIdx.z) >= n_sig_tiles;
+  const int b0 = noise ? (blockIdx.z - n_sig_tiles) * 128 : blockIdx.z * nb;
+  const int rows = noise ? 128 : nb * g;  // A rows the box fills
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t full = sbase + L::kBarOff, done = full + 8u;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kBarOff + 16);
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    mbar_init(full, 1);
+    mbar_init(done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
-  if (x >= dl) return;
-  // W_K row x of group k: d contiguous bf16 (16-byte aligned: 2d divides the row stride)
-  const int64_t ldw = static_cast<int64_t>(p.Hn) * 2 * d;
-  const uint4 *wr = reinterpret_cast<const uint4 *>(p.w_kvb + x * ldw + static_cast<int64_t>(k) * 2 * d);
-  uint32_t w[64];
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  volatile int abort_local = 0;
+  bool ok = true;
+  if (warp == 0) {
+    const bool leader = elect_one();
+    if (leader) {
+      mbar_arrive_expect_tx(full, static_cast<uint32_t>((D / 64) * (rows + 128) * 128));
 #pragma unroll
-  for (int v = 0; v < 16; ++v) {
-    if (v < d / 8) {
-      const uint4 t = __ldg(wr + v);
-      w[4 * v] = t.x;
-      w[4 * v + 1] = t.y;
-      w[4 * v + 2] = t.z;
-      w[4 * v + 3] = t.w;
-    } else {
-      w[4 * v] = w[4 * v + 1] = w[4 * v + 2] = w[4 * v + 3] = 0u;
+      for (int kb = 0; kb < D / 64; ++kb) {
+        if (noise)
+          tma_load_3d(sbase + L::kAOff + kb * L::kSub, &tm_qn, full, kb * 64, k, b0);
+        else
+          tma_load_3d(sbase + L::kAOff + kb * L::kSub, &tm_qs, full, kb * 64, g * k, b0);
+        tma_load_2d(sbase + L::kBOff + kb * L::kSub, &tm_w, full, k * 2 * D + kb * 64, x0);
+      }
+    }
+    ok = __all_sync(0xffffffffu, mbar_wait(full, 0, &abort_local));
+    tc_fence_after();
+    if (ok && leader) {
+      constexpr uint32_t kIdesc = idesc_bf16_f32(128, 128, false, false);
+      const uint64_t ad = sdesc_sw128(sbase + L::kAOff, 16, 1024);
+      const uint64_t bd = sdesc_sw128(sbase + L::kBOff, 16, 1024);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * L::kSub + (kk & 3) * 32;
+        umma_ss(tmem, ad + (off >> 4), bd + (off >> 4), kIdesc, kk > 0 ? 1u : 0u);
+      }
+      umma_commit(done);
+    }
+    if (!ok && leader) mbar_wait_for(full, 0, 100000000ull);
+  }
+  ok = __all_sync(0xffffffffu, ok && mbar_wait(done, 0, &abort_local));
+  if (ok) {
+    tc_fence_after();
+    // row r of the tile: (sequence b0 + r / g, signal head g k + r % g), or
+    // (sequence b0 + r, noise head k)
+    const int r = threadIdx.x;
+    const int b = noise ? b0 + r : b0 + r / g;
+    const int row = noise ? p.Hs + k : g * k + r % g;
+    const bool valid = r < rows && b < p.B;
+    __nv_bfloat16 *qt = p.qt + (static_cast<int64_t>(b) * p.Np + row) * p.dl + x0;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+      uint32_t v[32];
+      tmem_ld32_sync(tmem + lane_off + cc * 32, v);
+      if (valid) {
+        uint4 *dst = reinterpret_cast<uint4 *>(qt + cc * 32);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          dst[q] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * q]) * p.qscale,
+                                         __uint_as_float(v[8 * q + 1]) * p.qscale),
+                              pack_bf16x2(__uint_as_float(v[8 * q + 2]) * p.qscale,
+                                          __uint_as_float(v[8 * q + 3]) * p.qscale),
+                              pack_bf16x2(__uint_as_float(v[8 * q + 4]) * p.qscale,
+                                          __uint_as_float(v[8 * q + 5]) * p.qscale),
+                              pack_bf16x2(__uint_as_float(v[8 * q + 6]) * p.qscale,
+                                          __uint_as_float(v[8 * q + 7]) * p.qscale));
+      }
+    }
+    // the padding rows of these sequences, once (group 0's noise tiles)
+    if (noise && k == 0 && b < p.B) {
+      const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+      for (int pr = p.Hs + p.Hn; pr < p.Np; ++pr) {
+        uint4 *dst = reinterpret_cast<uint4 *>(p.qt + (static_cast<int64_t>(b) * p.Np + pr) * p.dl + x0);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) dst[q] = z;
+      }
     }
   }
-  for (int bb = 0; bb < nb; ++bb) {
-    const int64_t b = b0 + bb;
-    __nv_bfloat16 *qt = p.qt + b * p.Np * dl;
-    for (int j = 0; j < nh; ++j) {
-      const uint4 *q4 = reinterpret_cast<const uint4 *>(qs + (bb * (kDecMaxGroup + 1) + j) * 64);
-      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-      for (int v = 0; v < 16; ++v) {
-        if (v < d / 8) {
-          const uint4 q = q4[v];
-          a0 = fmaf(bf16lo_to_f32(w[4 * v]), bf16lo_to_f32(q.x), a0);
-          a1 = fmaf(bf16hi_to_f32(w[4 * v]), bf16hi_to_f32(q.x), a1);
-          a2 = fmaf(bf16lo_to_f32(w[4 * v + 1]), bf16lo_to_f32(q.y), a2);
-          a3 = fmaf(bf16hi_to_f32(w[4 * v + 1]), bf16hi_to_f32(q.y), a3);
-          a0 = fmaf(bf16lo_to_f32(w[4 * v + 2]), bf16lo_to_f32(q.z), a0);
-          a1 = fmaf(bf16hi_to_f32(w[4 * v + 2]), bf16hi_to_f32(q.z), a1);
-          a2 = fmaf(bf16lo_to_f32(w[4 * v + 3]), bf16lo_to_f32(q.w), a2);
-          a3 = fmaf(bf16hi_to_f32(w[4 * v + 3]), bf16hi_to_f32(q.w), a3);
-        }
-      }
-      const int row = j < g ? g * k + j : p.Hs + k;
-      qt[static_cast<int64_t>(row) * dl + x] = __float2bfloat16(((a0 + a1) + (a2 + a3)) * p.qscale);
-    }
-    if (k == 0)
-      for (int row = p.Hs + p.Hn; row < p.Np; ++row)
-        qt[static_cast<int64_t>(row) * dl + x] = __float2bfloat16(0.f);
+  if (!ok && threadIdx.x == 0 && p.status) atomicExch(p.status, -5 /* GDLA_ERR_TIMEOUT */);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
   }
 }
 
@@ -527,10 +585,13 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 // One CTA per (KV group k, sequence b): merge the splits of the group's heads
 // (weights 2^(m_s - M)), z = sum / l, H = z W_V, then
 // out = G (.) (H_S - lambda H_N) for the group's signal heads.
+// NH = g + 1, the heads of a KV group.
+template <int NH>
 __global__ void __launch_bounds__(128) gdla_decode_combine_kernel(const DecodeParams p) {
   const int k = blockIdx.x, b = blockIdx.y;
-  const int g = p.Hs / p.Hn, nh = g + 1, d = p.d, dl = p.dl;
-  __shared__ float zs[(kDecMaxGroup + 1) * kDecMaxLatent];
+  constexpr int g = NH - 1, nh = NH;
+  const int d = p.d, dl = p.dl;
+  __shared__ __align__(16) float zs[(kDecMaxGroup + 1) * kDecMaxLatent];
   __shared__ float hsm[(kDecMaxGroup + 1) * 128];
   __shared__ float wsp[(kDecMaxGroup + 1) * kDecMaxSplit];  // weight of split s for head j
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -561,57 +622,63 @@ __global__ void __launch_bounds__(128) gdla_decode_combine_kernel(const DecodePa
   // of every head and column it owns at once.
   {
     const int nx = dl / 128;
-    float acc[kDecMaxGroup + 1][kDecMaxLatent / 128];
+    float acc[NH][kDecMaxLatent / 128];
 #pragma unroll
-    for (int j = 0; j < kDecMaxGroup + 1; ++j)
+    for (int j = 0; j < NH; ++j)
 #pragma unroll
       for (int xi = 0; xi < kDecMaxLatent / 128; ++xi) acc[j][xi] = 0.f;
     for (int sp = 0; sp < p.n_split; ++sp) {
       const float *zp = decode_part(p, b, sp) + 2 * p.Np;
-      float z[kDecMaxGroup + 1][kDecMaxLatent / 128];
+      float z[NH][kDecMaxLatent / 128];
 #pragma unroll
-      for (int j = 0; j < kDecMaxGroup + 1; ++j) {
+      for (int j = 0; j < NH; ++j) {
         const int row = j < g ? g * k + j : p.Hs + k;
 #pragma unroll
         for (int xi = 0; xi < kDecMaxLatent / 128; ++xi)
-          z[j][xi] = (j < nh && xi < nx)
+          z[j][xi] = xi < nx
                          ? zp[static_cast<size_t>(row) * dl + xi * 128 + threadIdx.x]
                          : 0.f;
       }
 #pragma unroll
-      for (int j = 0; j < kDecMaxGroup + 1; ++j) {
-        const float wgt = j < nh ? wsp[j * kDecMaxSplit + sp] : 0.f;
+      for (int j = 0; j < NH; ++j) {
+        const float wgt = wsp[j * kDecMaxSplit + sp];
 #pragma unroll
         for (int xi = 0; xi < kDecMaxLatent / 128; ++xi) acc[j][xi] = fmaf(wgt, z[j][xi], acc[j][xi]);
       }
     }
 #pragma unroll
-    for (int j = 0; j < kDecMaxGroup + 1; ++j)
+    for (int j = 0; j < NH; ++j)
 #pragma unroll
       for (int xi = 0; xi < kDecMaxLatent / 128; ++xi)
-        if (j < nh && xi < nx) zs[j * dl + xi * 128 + threadIdx.x] = acc[j][xi];
+        if (xi < nx) zs[j * dl + xi * 128 + threadIdx.x] = acc[j][xi];
   }
   __syncthreads();
   const int64_t ldw = static_cast<int64_t>(p.Hn) * 2 * d;
   for (int c = threadIdx.x; c < d; c += blockDim.x) {
-    float acc[kDecMaxGroup + 1];
+    float acc[NH];
 #pragma unroll
-    for (int j = 0; j < kDecMaxGroup + 1; ++j) acc[j] = 0.f;
+    for (int j = 0; j < NH; ++j) acc[j] = 0.f;
     const __nv_bfloat16 *wv = p.w_kvb + static_cast<int64_t>(k) * 2 * d + d + c;
-    // 32 loads in flight per batch of latent rows (dl is a multiple of 128)
+    // 32 loads in flight per batch of latent rows (dl is a multiple of 128);
+    // z comes four latent rows per shared-memory read
     for (int x0 = 0; x0 < dl; x0 += 32) {
       float wx[32];
 #pragma unroll
       for (int u = 0; u < 32; ++u) wx[u] = __bfloat162float(wv[(x0 + u) * ldw]);
 #pragma unroll
-      for (int u = 0; u < 32; ++u)
+      for (int u = 0; u < 32; u += 4)
 #pragma unroll
-        for (int j = 0; j < kDecMaxGroup + 1; ++j)
-          if (j < nh) acc[j] = fmaf(zs[j * dl + x0 + u], wx[u], acc[j]);
+        for (int j = 0; j < NH; ++j) {
+          const float4 z4 = *reinterpret_cast<const float4 *>(&zs[j * dl + x0 + u]);
+          acc[j] = fmaf(z4.x, wx[u], acc[j]);
+          acc[j] = fmaf(z4.y, wx[u + 1], acc[j]);
+          acc[j] = fmaf(z4.z, wx[u + 2], acc[j]);
+          acc[j] = fmaf(z4.w, wx[u + 3], acc[j]);
+        }
     }
 #pragma unroll
-    for (int j = 0; j < kDecMaxGroup + 1; ++j)
-      if (j < nh) hsm[j * d + c] = acc[j];
+    for (int j = 0; j < NH; ++j)
+      hsm[j * d + c] = acc[j];
   }
   __syncthreads();
   for (int i = threadIdx.x; i < g * d; i += blockDim.x) {

@@ -293,6 +293,34 @@ bool decode_plan(int B, int64_t L_max, int Hs, int Hn, int d_latent, int64_t win
   return true;
 }
 
+// The absorb GEMM tiles: signal tiles of 128 / g sequences (all g signal
+// heads of a group), noise tiles of 128 sequences, 128 latent columns each.
+template <int D>
+int launch_decode_absorb(const gdla::DecodeParams &prm, cudaStream_t stream) {
+  const int g = prm.Hs / prm.Hn;
+  const int nb = 128 / g;
+  CUtensorMap tm_qs, tm_qn, tm_w;
+  const uint64_t dqs[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(prm.Hs),
+                           static_cast<uint64_t>(prm.B)};
+  const uint32_t bqs[3] = {64, static_cast<uint32_t>(g), static_cast<uint32_t>(nb)};
+  const uint64_t dqn[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(prm.Hn),
+                           static_cast<uint64_t>(prm.B)};
+  const uint32_t bqn[3] = {64, 1, 128};
+  const uint64_t dw[2] = {static_cast<uint64_t>(prm.Hn) * 2 * D, static_cast<uint64_t>(prm.dl)};
+  const uint32_t bw[2] = {64, 128};
+  if (!make_map(&tm_qs, prm.q_sig, 3, dqs, bqs) || !make_map(&tm_qn, prm.q_noise, 3, dqn, bqn) ||
+      !make_map(&tm_w, prm.w_kvb, 2, dw, bw))
+    return GDLA_ERR_CUDA;
+  constexpr auto kern = gdla::gdla_decode_absorb_kernel<D>;
+  const int rc = prepare_kernel<kern>(gdla::AbsorbSmem::kBytes, 0);
+  if (rc != GDLA_OK) return rc;
+  const int n_sig = (prm.B + nb - 1) / nb, n_noise = (prm.B + 127) / 128;
+  kern<<<dim3(static_cast<unsigned>(prm.dl / 128), static_cast<unsigned>(prm.Hn),
+              static_cast<unsigned>(n_sig + n_noise)),
+         gdla::kAbsThreads, gdla::AbsorbSmem::kBytes, stream>>>(tm_qs, tm_qn, tm_w, prm, n_sig);
+  return cudaGetLastError() == cudaSuccess ? GDLA_OK : GDLA_ERR_CUDA;
+}
+
 template <int NP>
 int launch_decode_attn(const gdla::DecodeParams &prm, const void *c_hat, cudaStream_t stream) {
   using L = gdla::DecSmem<NP>;
@@ -517,17 +545,22 @@ int gdla_decode_fwd(const void *q_sig, const void *q_noise, const void *c_hat,
   const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(d));
   prm.qscale = sc * 1.4426950408889634f;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  gdla::gdla_decode_absorb_kernel<<<dim3(static_cast<unsigned>(Hn),
-                                         static_cast<unsigned>(d_latent / gdla::kDecUnit),
-                                         static_cast<unsigned>((B + gdla::kAbsorbSeqs - 1) /
-                                                               gdla::kAbsorbSeqs)),
-                                    128, 0, s>>>(prm);
-  if (cudaGetLastError() != cudaSuccess) return GDLA_ERR_CUDA;
+  const int arc = d == 128 ? launch_decode_absorb<128>(prm, s) : launch_decode_absorb<64>(prm, s);
+  if (arc != GDLA_OK) return arc;
   const int rc = pl.Np == 80 ? launch_decode_attn<80>(prm, c_hat, s)
                              : launch_decode_attn<16>(prm, c_hat, s);
   if (rc != GDLA_OK) return rc;
-  gdla::gdla_decode_combine_kernel<<<dim3(static_cast<unsigned>(Hn), static_cast<unsigned>(B)),
-                                     128, 0, s>>>(prm);
+  const dim3 cgrid(static_cast<unsigned>(Hn), static_cast<unsigned>(B));
+  switch (Hs / Hn) {  // the combine is specialised for the heads of a group
+    case 1: gdla::gdla_decode_combine_kernel<2><<<cgrid, 128, 0, s>>>(prm); break;
+    case 2: gdla::gdla_decode_combine_kernel<3><<<cgrid, 128, 0, s>>>(prm); break;
+    case 3: gdla::gdla_decode_combine_kernel<4><<<cgrid, 128, 0, s>>>(prm); break;
+    case 4: gdla::gdla_decode_combine_kernel<5><<<cgrid, 128, 0, s>>>(prm); break;
+    case 5: gdla::gdla_decode_combine_kernel<6><<<cgrid, 128, 0, s>>>(prm); break;
+    case 6: gdla::gdla_decode_combine_kernel<7><<<cgrid, 128, 0, s>>>(prm); break;
+    case 7: gdla::gdla_decode_combine_kernel<8><<<cgrid, 128, 0, s>>>(prm); break;
+    default: gdla::gdla_decode_combine_kernel<9><<<cgrid, 128, 0, s>>>(prm); break;
+  }
   return cudaGetLastError() == cudaSuccess ? GDLA_OK : GDLA_ERR_CUDA;
 }
 
