@@ -224,7 +224,7 @@ struct DecSmem {
   static constexpr uint32_t kRefOff = kRedOff + kRedBytes;  // int ref[2][4][NP] (per warp, per chunk parity)
   static constexpr uint32_t kBarOff = kRefOff + 2 * 4 * NP * 4;
   static constexpr int kZStride = (NP + 31) / 32 * 32;        // TMEM columns per z^T block
-  static constexpr uint32_t kNumBars = 2 * kDecRing + 8;
+  static constexpr uint32_t kNumBars = 2 * kDecRing + 9;
   static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;
   static constexpr uint32_t kBytes = kMiscOff + 16;
   static_assert(kQtBytes % 1024 == 0 && kRingOff % 1024 == 0 && kPOff % 1024 == 0,
@@ -298,6 +298,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   const uint32_t z_done = bar0 + 8u * (2 * kDecRing + 3);   // z^T MMAs of a chunk done
   // maxima exchanged among the four warps of one half of the heads
   auto red_full = [&](int half, int i) { return bar0 + 8u * (2 * kDecRing + 4 + 2 * half + i); };
+  const uint32_t s_free = bar0 + 8u * (2 * kDecRing + 8);   // S^T of a chunk read out
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
   int *red = reinterpret_cast<int *>(smem + L::kRedOff);                  // [2][4][NP]
@@ -314,6 +315,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     mbar_init(s_full, 1);
     mbar_init(p_full, 8);
     mbar_init(z_done, 1);
+    mbar_init(s_free, 8);
     for (int hf = 0; hf < 2; ++hf) {
       mbar_init(red_full(hf, 0), 4);
       mbar_init(red_full(hf, 1), 4);
@@ -344,24 +346,29 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       for (int kb = 0; kb < p.dl / 64; ++kb)
         tma_load_2d(sbase + L::kQtOff + kb * (NP * 128), &tm_qt, qt_full, kb * 64, b * NP);
     }
+    // chunk order of the loads: 0, then per chunk ch the scores pass of ch + 1
+    // ahead of the z^T pass of ch (0, 1, 0, 2, 1, ..., n-1, n-2, n-1), so the
+    // cache streams from HBM while the softmax of ch runs
     uint32_t c = 0;
     bool ok = true;
-    for (int ch = 0; ch < n_chunks && ok; ++ch) {
-      const int32_t tok0 = static_cast<int32_t>((rg.c_begin + ch) * kDecTok);
-      for (int pass = 0; pass < 2 && ok; ++pass) {
-        for (int u = 0; u < U; ++u) {
-          const int slot = static_cast<int>(c % kDecRing);
-          ok = __all_sync(0xffffffffu,
-                          mbar_wait(ring_empty(slot), ((c / kDecRing) & 1u) ^ 1u, abort_flag));
-          if (!ok) break;
-          if (leader) {
-            const uint32_t dst = sbase + L::kRingOff + slot * L::kUnitBytes;
-            mbar_arrive_expect_tx(ring_full(slot), L::kUnitBytes);
-            tma_load_3d(dst, &tm_c, ring_full(slot), u * kDecUnit, tok0, b);
-            tma_load_3d(dst + kDecTok * 128, &tm_c, ring_full(slot), u * kDecUnit + 64, tok0, b);
-          }
-          ++c;
+    for (int q = 0; q < 2 * n_chunks && ok; ++q) {
+      const int chx = q == 0                  ? 0
+                      : q == 2 * n_chunks - 1 ? n_chunks - 1
+                      : (q & 1)               ? (q + 1) / 2
+                                              : q / 2 - 1;
+      const int32_t tok0 = static_cast<int32_t>((rg.c_begin + chx) * kDecTok);
+      for (int u = 0; u < U; ++u) {
+        const int slot = static_cast<int>(c % kDecRing);
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait(ring_empty(slot), ((c / kDecRing) & 1u) ^ 1u, abort_flag));
+        if (!ok) break;
+        if (leader) {
+          const uint32_t dst = sbase + L::kRingOff + slot * L::kUnitBytes;
+          mbar_arrive_expect_tx(ring_full(slot), L::kUnitBytes);
+          tma_load_3d(dst, &tm_c, ring_full(slot), u * kDecUnit, tok0, b);
+          tma_load_3d(dst + kDecTok * 128, &tm_c, ring_full(slot), u * kDecUnit + 64, tok0, b);
         }
+        ++c;
       }
     }
     if (!ok && leader) {
@@ -378,8 +385,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     const uint32_t idesc_z = idesc_bf16_f32(kDecUnit, NP, true, false);
     bool ok = __all_sync(0xffffffffu, mbar_wait(qt_full, 0, abort_flag));
     uint32_t c = 0, commits = 0;
-    for (int ch = 0; ch < n_chunks && ok; ++ch) {
-      // pass 1: S^T = c_hat q~^T over the latent, one unit (two K-blocks) at a time
+    // pass 1: S^T = c_hat q~^T over the latent, one unit (two K-blocks) at a time
+    auto score_pass = [&]() {
       for (int u = 0; u < U && ok; ++u) {
         const int slot = static_cast<int>(c % kDecRing);
         ok = __all_sync(0xffffffffu, mbar_wait(ring_full(slot), (c / kDecRing) & 1u, abort_flag));
@@ -401,8 +408,18 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         }
         ++c;
       }
-      if (!ok) break;
-      if (leader) umma_commit(s_full);
+      if (ok && leader) umma_commit(s_full);
+    };
+    if (ok) score_pass();
+    for (int ch = 0; ch < n_chunks && ok; ++ch) {
+      // the scores of chunk ch + 1 as soon as the softmax has read those of ch
+      if (ch + 1 < n_chunks) {
+        ok = __all_sync(0xffffffffu, mbar_wait(s_free, ch & 1u, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        score_pass();
+        if (!ok) break;
+      }
       ok = __all_sync(0xffffffffu, mbar_wait(p_full, ch & 1u, abort_flag));
       if (!ok) break;
       tc_fence_after();
@@ -459,6 +476,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 #pragma unroll
         for (int e = 0; e < 8; ++e) sv[8 * i + e] = __uint_as_float(r8[e]);
       }
+      // S^T is in registers: the next chunk's scores may overwrite it
+      tc_fence_before();
+      dec_warp_arrive(s_free);
       const int64_t tok = (rg.c_begin + ch) * kDecTok + t;
       const bool valid = tok >= rg.t_lo && tok < rg.len;
       // per head: the chunk's largest score rounded up to an integer, over the
