@@ -391,10 +391,10 @@ __global__ void __launch_bounds__(kWinThreads, 1)
         ++s_waits;
         if (!ok) break;
         tc_fence_after();
-        // ---- this half's two chunks in one TMEM round trip: va holds chunk
-        // ka, vb chunk kb (the mixed chunk first when the half has it)
+        // ---- this half's two chunks in one TMEM round trip: va holds the
+        // first (the mixed chunk when the half has it), vb chunk kb
         uint32_t va[32], vb[32];
-        const int ka = has_mixed ? qw : ca, kb = has_mixed ? other : cb;
+        const int kb = has_mixed ? other : cb;
         if (has_mixed) {
           uint32_t me[32];
           if (has_edge) {

@@ -602,112 +602,263 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 }
 
 // ---------------------------------------------------------------- combine
-// One CTA per (KV group k, sequence b): merge the splits of the group's heads
-// (weights 2^(m_s - M)), z = sum / l, H = z W_V, then
-// out = G (.) (H_S - lambda H_N) for the group's signal heads.
-// NH = g + 1, the heads of a KV group.
+// Two kernels.  merge: one CTA per (KV group k, sequence b, head j of the
+// group; j < g: signal head g k + j, j = g: noise head k), thread = 4 latent
+// columns: over the splits, M = max_s m_s, l = sum_s 2^(m_s - M) l_s and
+// z = sum_s 2^(m_s - M) z_s / l (online over batches of 8 splits, so the loads
+// of a batch are in flight together; a split that saw no key weighs nothing),
+// written as bf16 row (k B + b) NH + j of Z (over the absorbed queries, which
+// the attention kernel no longer needs).  out: one CTA per (k, block of SB
+// sequences), one tcgen05 GEMM H^T = W_V^T Z^T (M = 128 value columns, N = the
+// block's NH SB rows padded to 16, K = latent; W_V MN-major and Z K-major, both
+// by TMA), then out = G (.) (H_S - lambda H_N) for the group's signal heads.
+// Merge of one Z row item (row, 4 latent columns) over the splits.
+struct MergeItem {
+  const float *pm, *pz;  // split 0's m of the head row, and its z at the item's columns
+  float M, l;
+  float4 acc;
+};
+
+// item < Hn B NH dl / 4 <= 80 * 65535 * 128 < 2^31 (the host limits B and the heads)
 template <int NH>
-__global__ void __launch_bounds__(128) gdla_decode_combine_kernel(const DecodeParams p) {
-  const int k = blockIdx.x, b = blockIdx.y;
-  constexpr int g = NH - 1, nh = NH;
+__device__ __forceinline__ void merge_item_init(const DecodeParams &p, uint32_t item, MergeItem &it,
+                                                __nv_bfloat16 *&dst) {
+  constexpr int g = NH - 1;
+  const uint32_t tpr = static_cast<uint32_t>(p.dl) / 4;
+  const uint32_t row = item / tpr;  // Z row (k B + b) NH + j
+  const int x = 4 * static_cast<int>(item - row * tpr);
+  const uint32_t kb = row / NH;
+  const int j = static_cast<int>(row - kb * NH);
+  const uint32_t k = kb / static_cast<uint32_t>(p.B);
+  const int b = static_cast<int>(kb - k * static_cast<uint32_t>(p.B));
+  const int prow = j < g ? g * static_cast<int>(k) + j : p.Hs + static_cast<int>(k);
+  const int64_t ss = static_cast<int64_t>(p.Np) * (p.dl + 2);
+  const float *pb = p.part + static_cast<int64_t>(b) * p.n_split * ss;
+  it.pm = pb + prow;
+  it.pz = pb + 2 * p.Np + static_cast<int64_t>(prow) * p.dl + x;
+  it.M = -INFINITY;
+  it.l = 0.f;
+  it.acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  dst = p.qt + static_cast<int64_t>(row) * p.dl + x;
+}
+
+// Folds the splits [s0, s0 + SPB) whose values are in m, lv, v into the item.
+template <int SPB>
+__device__ __forceinline__ void merge_fold(MergeItem &it, const float *m, const float *lv,
+                                           const float4 *v) {
+  float mn = it.M;
+#pragma unroll
+  for (int i = 0; i < SPB; ++i) mn = fmaxf(mn, m[i]);
+  if (mn == -INFINITY) return;  // no key so far
+  const float a = exp2f(it.M - mn);  // 0 while M is -inf
+  it.l *= a;
+  it.acc.x *= a, it.acc.y *= a, it.acc.z *= a, it.acc.w *= a;
+#pragma unroll
+  for (int i = 0; i < SPB; ++i) {
+    if (m[i] == -INFINITY) continue;  // a split that saw no key: its z was never written
+    const float w = exp2f(m[i] - mn);
+    it.l = fmaf(w, lv[i], it.l);
+    it.acc.x = fmaf(w, v[i].x, it.acc.x);
+    it.acc.y = fmaf(w, v[i].y, it.acc.y);
+    it.acc.z = fmaf(w, v[i].z, it.acc.z);
+    it.acc.w = fmaf(w, v[i].w, it.acc.w);
+  }
+  it.M = mn;
+}
+
+template <int SPB>
+__device__ __forceinline__ void merge_load(const DecodeParams &p, const MergeItem &it, bool live,
+                                           int s0, float *m, float *lv, float4 *v) {
+  const int64_t ss = static_cast<int64_t>(p.Np) * (p.dl + 2);
+#pragma unroll
+  for (int i = 0; i < SPB; ++i) {
+    const bool on = live && s0 + i < p.n_split;
+    const int64_t so = on ? (s0 + i) * ss : 0;
+    m[i] = on ? it.pm[so] : -INFINITY;
+    lv[i] = on ? it.pm[so + p.Np] : 0.f;
+    v[i] = on ? *reinterpret_cast<const float4 *>(it.pz + so) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+__device__ __forceinline__ void merge_store(const MergeItem &it, __nv_bfloat16 *dst) {
+  const float il = it.l > 0.f ? 1.f / it.l : 0.f;
+  uint2 o;
+  o.x = pack_bf16x2(it.acc.x * il, it.acc.y * il);
+  o.y = pack_bf16x2(it.acc.z * il, it.acc.w * il);
+  *reinterpret_cast<uint2 *>(dst) = o;
+}
+
+// One thread per IPT items (Hn B NH rows x dl / 4 column groups; a CTA's
+// threads take consecutive items, IPT blocks of 128), SPB splits of each per
+// batch, all IPT x SPB loads of a batch in flight together (IPT = 1, SPB = 8
+// for several splits; IPT = 4, SPB = 1 for one).  Few registers, so many
+// CTAs per SM keep many loads in flight.
+template <int NH, int IPT, int SPB>
+__global__ void __launch_bounds__(128) gdla_decode_merge_kernel(const DecodeParams p) {
+  const uint32_t items = static_cast<uint32_t>(p.Hn * NH) * static_cast<uint32_t>(p.B) *
+                         static_cast<uint32_t>(p.dl / 4);
+  const uint32_t i0 = blockIdx.x * (128 * IPT) + threadIdx.x;
+  MergeItem it[IPT];
+  __nv_bfloat16 *dst[IPT];
+  bool live[IPT];
+#pragma unroll
+  for (int u = 0; u < IPT; ++u) {
+    live[u] = i0 + u * 128 < items;
+    merge_item_init<NH>(p, live[u] ? i0 + u * 128 : 0, it[u], dst[u]);
+  }
+  for (int s0 = 0; s0 < p.n_split; s0 += SPB) {
+    float m[IPT][SPB], lv[IPT][SPB];
+    float4 v[IPT][SPB];
+#pragma unroll
+    for (int u = 0; u < IPT; ++u) merge_load<SPB>(p, it[u], live[u], s0, m[u], lv[u], v[u]);
+#pragma unroll
+    for (int u = 0; u < IPT; ++u) merge_fold<SPB>(it[u], m[u], lv[u], v[u]);
+  }
+#pragma unroll
+  for (int u = 0; u < IPT; ++u)
+    if (live[u]) merge_store(it[u], dst[u]);
+}
+
+constexpr int kCombThreads = 256;
+constexpr int kCombMaxRows = 80;  // N of the GEMM at most
+struct CombSmem {
+  static constexpr uint32_t kWOff = 0;  // W_V: [dl / 128][2 halves of 64 columns][128 x][128 B]
+  static constexpr uint32_t kWBytes = kDecMaxLatent / 128 * 32768;
+  static constexpr uint32_t kZOff = kWOff + kWBytes;  // Z: [dl / 64][Npad rows][128 B]
+  static constexpr uint32_t kZBytes = kCombMaxRows * kDecMaxLatent * 2;
+  static constexpr uint32_t kBarOff = kZOff + kZBytes;
+  static constexpr uint32_t kBytes = kBarOff + 32;
+  static_assert(kZOff % 1024 == 0, "swizzled operands need 1024-byte alignment");
+  static_assert(kBytes <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
+  // H [rows][128] fp32 overlays W_V once the GEMM is done
+  static_assert(kCombMaxRows * 128 * 4 <= kWBytes, "H must fit over W_V");
+};
+
+template <int NH>
+__global__ void __launch_bounds__(kCombThreads, 1)
+    gdla_decode_out_kernel(const __grid_constant__ CUtensorMap tm_w,
+                           const __grid_constant__ CUtensorMap tm_z, const DecodeParams p, int SB) {
+  using L = CombSmem;
+  constexpr int g = NH - 1;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if ((smem_u32(smem) & 1023u) != 0) {
+    if (threadIdx.x == 0 && p.status) atomicExch(p.status, -4 /* GDLA_ERR_CUDA */);
+    return;
+  }
+  const int k = blockIdx.x, b0 = blockIdx.y * SB;
   const int d = p.d, dl = p.dl;
-  __shared__ __align__(16) float zs[(kDecMaxGroup + 1) * kDecMaxLatent];
-  __shared__ float hsm[(kDecMaxGroup + 1) * 128];
-  __shared__ float wsp[(kDecMaxGroup + 1) * kDecMaxSplit];  // weight of split s for head j
+  const int Npad = (SB * NH + 15) / 16 * 16;  // N of the GEMM (host: SB NH <= kCombMaxRows)
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t full = sbase + L::kBarOff, mma_done = full + 8u;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kBarOff + 16);
+  volatile int abort_local = 0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // one warp per head row: M = max_s m_s, l = sum_s 2^(m_s - M) l_s, and the
-  // weight 2^(m_s - M) / l of every split (0 for a split that saw no key)
-  for (int j = warp; j < nh; j += 4) {
-    const int row = j < g ? g * k + j : p.Hs + k;
-    float M = -INFINITY;
-    for (int sp = lane; sp < p.n_split; sp += 32) M = fmaxf(M, decode_part(p, b, sp)[row]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float l = 0.f;
-    for (int sp = lane; sp < p.n_split; sp += 32) {
-      const float *pp = decode_part(p, b, sp);
-      const float e = pp[row] == -INFINITY ? 0.f : exp2f(pp[row] - M);
-      wsp[j * kDecMaxSplit + sp] = e;
-      l += e * pp[p.Np + row];
+  if (threadIdx.x == 0) {
+    mbar_init(full, 1);
+    mbar_init(mma_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  bool ok = true;
+  if (warp == 0) {
+    const bool leader = elect_one();
+    if (leader) {
+      // W_V of group k: value columns k 2d + d + [0, 128) (lanes past d unused);
+      // the block's Z rows (rows past them belong to other blocks or lie
+      // outside Z: their columns of H^T are not read)
+      mbar_arrive_expect_tx(full, static_cast<uint32_t>(dl / 128 * 32768 + dl / 64 * Npad * 128));
+      for (int kb = 0; kb < dl / 128; ++kb)
+        for (int hf = 0; hf < 2; ++hf)
+          tma_load_2d(sbase + L::kWOff + kb * 32768 + hf * 16384, &tm_w, full,
+                      k * 2 * d + d + 64 * hf, kb * 128);
+      const int row0 = (k * p.B + b0) * NH;
+      for (int kb = 0; kb < dl / 64; ++kb)
+        tma_load_2d(sbase + L::kZOff + kb * (Npad * 128), &tm_z, full, kb * 64, row0);
     }
+    ok = __all_sync(0xffffffffu, mbar_wait(full, 0, &abort_local));
+    tc_fence_after();
+    if (ok && leader) {
+      const uint32_t idesc = idesc_bf16_f32(128, Npad, true, false);
+      for (int kk = 0; kk < dl / 16; ++kk) {
+        const uint64_t ad = sdesc_sw128(sbase + L::kWOff + (kk >> 3) * 32768 + (kk & 7) * 2048,
+                                        16384, 1024);
+        const uint64_t bd =
+            sdesc_sw128(sbase + L::kZOff + (kk >> 2) * (Npad * 128) + (kk & 3) * 32, 16, 1024);
+        umma_ss(tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
+      }
+      umma_commit(mma_done);
+    }
+    if (!ok && leader) mbar_wait_for(full, 0, 100000000ull);
+  }
+  ok = __all_sync(0xffffffffu, ok && mbar_wait(mma_done, 0, &abort_local));
+  tc_fence_after();
+  // H^T in TMEM (lane = value column c, column = row r) -> H [r][c] in shared
+  // memory over W_V (the GEMM has read it)
+  __syncthreads();
+  float *hs = reinterpret_cast<float *>(smem + L::kWOff);
+  if (ok && warp < 4) {
+    const int c = warp * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    for (int q = 0; q < Npad / 8; ++q) {
+      uint32_t r8[8];
+      tmem_ld8_sync(tmem + lane_off + 8 * q, r8);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-    const float inv_l = l > 0.f ? 1.f / l : 0.f;
-    __syncwarp();
-    for (int sp = lane; sp < p.n_split; sp += 32) wsp[j * kDecMaxSplit + sp] *= inv_l;
+      for (int e = 0; e < 8; ++e) hs[(8 * q + e) * 128 + c] = __uint_as_float(r8[e]);
+    }
   }
   __syncthreads();
-  // z = sum_s weight_s z_s for the group's heads.  Thread t owns latent
-  // columns t, t + 128, ... (dl / 128 of them); per split it issues the loads
-  // of every head and column it owns at once.
-  {
-    const int nx = dl / 128;
-    float acc[NH][kDecMaxLatent / 128];
+  if (ok) {
+    // items of 8 value columns of one (sequence, signal head); per thread two
+    // items, their gate and lambda loads issued before any store
+    const int nb = min(SB, p.B - b0), nq = d / 8;
+    const int items = nb * g * nq;
+    for (int i0 = threadIdx.x; i0 < items; i0 += 2 * kCombThreads) {
+      uint4 gv[2];
+      float lamv[2];
+      int64_t o[2];
+      int hrow[2];
 #pragma unroll
-    for (int j = 0; j < NH; ++j)
-#pragma unroll
-      for (int xi = 0; xi < kDecMaxLatent / 128; ++xi) acc[j][xi] = 0.f;
-    for (int sp = 0; sp < p.n_split; ++sp) {
-      const float *zp = decode_part(p, b, sp) + 2 * p.Np;
-      float z[NH][kDecMaxLatent / 128];
-#pragma unroll
-      for (int j = 0; j < NH; ++j) {
-        const int row = j < g ? g * k + j : p.Hs + k;
-#pragma unroll
-        for (int xi = 0; xi < kDecMaxLatent / 128; ++xi)
-          z[j][xi] = xi < nx
-                         ? zp[static_cast<size_t>(row) * dl + xi * 128 + threadIdx.x]
-                         : 0.f;
+      for (int u = 0; u < 2; ++u) {
+        const int i = i0 + u * kCombThreads;
+        const bool on = i < items;
+        const int ii = on ? i : i0;
+        const int c8 = (ii % nq) * 8, j = (ii / nq) % g, bb = ii / (nq * g);
+        const int b = b0 + bb, h = g * k + j;
+        o[u] = (static_cast<int64_t>(b) * p.Hs + h) * d + c8;
+        hrow[u] = (bb * NH + j) * 128 + c8;
+        gv[u] = *reinterpret_cast<const uint4 *>(p.gate + o[u]);
+        lamv[u] = __bfloat162float(p.lam[static_cast<int64_t>(b) * p.Hs + h]);
       }
 #pragma unroll
-      for (int j = 0; j < NH; ++j) {
-        const float wgt = wsp[j * kDecMaxSplit + sp];
+      for (int u = 0; u < 2; ++u) {
+        if (i0 + u * kCombThreads >= items) break;
+        const float *hsg = hs + hrow[u];
+        const float *hno = hsg + (g - (hrow[u] / 128) % NH) * 128;  // the noise row of the sequence
+        const uint32_t gw[4] = {gv[u].x, gv[u].y, gv[u].z, gv[u].w};
+        uint32_t ow[4];
 #pragma unroll
-        for (int xi = 0; xi < kDecMaxLatent / 128; ++xi) acc[j][xi] = fmaf(wgt, z[j][xi], acc[j][xi]);
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < NH; ++j)
-#pragma unroll
-      for (int xi = 0; xi < kDecMaxLatent / 128; ++xi)
-        if (xi < nx) zs[j * dl + xi * 128 + threadIdx.x] = acc[j][xi];
-  }
-  __syncthreads();
-  const int64_t ldw = static_cast<int64_t>(p.Hn) * 2 * d;
-  for (int c = threadIdx.x; c < d; c += blockDim.x) {
-    float acc[NH];
-#pragma unroll
-    for (int j = 0; j < NH; ++j) acc[j] = 0.f;
-    const __nv_bfloat16 *wv = p.w_kvb + static_cast<int64_t>(k) * 2 * d + d + c;
-    // 32 loads in flight per batch of latent rows (dl is a multiple of 128);
-    // z comes four latent rows per shared-memory read
-    for (int x0 = 0; x0 < dl; x0 += 32) {
-      float wx[32];
-#pragma unroll
-      for (int u = 0; u < 32; ++u) wx[u] = __bfloat162float(wv[(x0 + u) * ldw]);
-#pragma unroll
-      for (int u = 0; u < 32; u += 4)
-#pragma unroll
-        for (int j = 0; j < NH; ++j) {
-          const float4 z4 = *reinterpret_cast<const float4 *>(&zs[j * dl + x0 + u]);
-          acc[j] = fmaf(z4.x, wx[u], acc[j]);
-          acc[j] = fmaf(z4.y, wx[u + 1], acc[j]);
-          acc[j] = fmaf(z4.z, wx[u + 2], acc[j]);
-          acc[j] = fmaf(z4.w, wx[u + 3], acc[j]);
+        for (int e = 0; e < 4; ++e) {
+          const float d0 = hsg[2 * e] - lamv[u] * hno[2 * e];
+          const float d1 = hsg[2 * e + 1] - lamv[u] * hno[2 * e + 1];
+          ow[e] = pack_bf16x2(bf16lo_to_f32(gw[e]) * d0, bf16hi_to_f32(gw[e]) * d1);
         }
+        *reinterpret_cast<uint4 *>(p.out + o[u]) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+      }
     }
-#pragma unroll
-    for (int j = 0; j < NH; ++j)
-      hsm[j * d + c] = acc[j];
   }
+  if (!ok && threadIdx.x == 0 && p.status) atomicExch(p.status, -5 /* GDLA_ERR_TIMEOUT */);
+  tc_fence_before();
   __syncthreads();
-  for (int i = threadIdx.x; i < g * d; i += blockDim.x) {
-    const int j = i / d, c = i % d;
-    const int h = g * k + j;
-    const float lamv = __bfloat162float(p.lam[static_cast<int64_t>(b) * p.Hs + h]);
-    const int64_t o = (static_cast<int64_t>(b) * p.Hs + h) * d + c;
-    const float dv = hsm[j * d + c] - lamv * hsm[g * d + c];
-    p.out[o] = __float2bfloat16(__bfloat162float(p.gate[o]) * dv);
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
   }
 }
 

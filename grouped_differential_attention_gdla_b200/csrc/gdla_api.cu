@@ -293,50 +293,89 @@ bool decode_plan(int B, int64_t L_max, int Hs, int Hn, int d_latent, int64_t win
   return true;
 }
 
+// Tensor maps of one decode call, all encoded before its first launch so the
+// four kernels go out back to back.
+struct DecodeMaps {
+  CUtensorMap qs, qn;  // queries [B, Hs | Hn, d]: absorb A tiles
+  CUtensorMap w;       // W^KV_b [dl, Hn 2d], boxes {64, 128}: absorb B, W_V of the output GEMM
+  CUtensorMap qt;      // absorbed queries [B Np, dl], boxes {64, Np}
+  CUtensorMap c;       // latent cache [B, L_max, dl], boxes {64, 128 tokens}
+  CUtensorMap z;       // merged z [Hn B NH, dl] over the absorbed queries, boxes {64, Npad}
+  int sb;              // sequences per CTA of the output GEMM
+};
+
+bool decode_maps(const gdla::DecodeParams &prm, const void *c_hat, DecodeMaps *m) {
+  const int g = prm.Hs / prm.Hn, nh = g + 1;
+  const int nb = 128 / g;
+  const uint64_t dqs[3] = {static_cast<uint64_t>(prm.d), static_cast<uint64_t>(prm.Hs),
+                           static_cast<uint64_t>(prm.B)};
+  const uint32_t bqs[3] = {64, static_cast<uint32_t>(g), static_cast<uint32_t>(nb)};
+  const uint64_t dqn[3] = {static_cast<uint64_t>(prm.d), static_cast<uint64_t>(prm.Hn),
+                           static_cast<uint64_t>(prm.B)};
+  const uint32_t bqn[3] = {64, 1, 128};
+  const uint64_t dw[2] = {static_cast<uint64_t>(prm.Hn) * 2 * prm.d, static_cast<uint64_t>(prm.dl)};
+  const uint32_t bw[2] = {64, 128};
+  const uint64_t dq[2] = {static_cast<uint64_t>(prm.dl), static_cast<uint64_t>(prm.B) * prm.Np};
+  const uint32_t qbox[2] = {64, static_cast<uint32_t>(prm.Np)};
+  const uint64_t dc[3] = {static_cast<uint64_t>(prm.dl), static_cast<uint64_t>(prm.L_max),
+                          static_cast<uint64_t>(prm.B)};
+  const uint32_t cbox[3] = {64, gdla::kDecTok, 1};
+  // output GEMM: about one wave of CTAs over the groups, at most
+  // kCombMaxRows head rows per CTA
+  const int per_group = std::max(1, static_cast<int>(kDecodeSms) / prm.Hn);
+  m->sb = std::min(std::max(1, (prm.B + per_group - 1) / per_group), gdla::kCombMaxRows / nh);
+  const int npad = (m->sb * nh + 15) / 16 * 16;
+  const uint64_t dz[2] = {static_cast<uint64_t>(prm.dl),
+                          static_cast<uint64_t>(prm.Hn) * prm.B * nh};
+  const uint32_t bz[2] = {64, static_cast<uint32_t>(npad)};
+  return make_map(&m->qs, prm.q_sig, 3, dqs, bqs) && make_map(&m->qn, prm.q_noise, 3, dqn, bqn) &&
+         make_map(&m->w, prm.w_kvb, 2, dw, bw) && make_map(&m->qt, prm.qt, 2, dq, qbox) &&
+         make_map(&m->c, c_hat, 3, dc, cbox) && make_map(&m->z, prm.qt, 2, dz, bz);
+}
+
 // The absorb GEMM tiles: signal tiles of 128 / g sequences (all g signal
 // heads of a group), noise tiles of 128 sequences, 128 latent columns each.
 template <int D>
-int launch_decode_absorb(const gdla::DecodeParams &prm, cudaStream_t stream) {
-  const int g = prm.Hs / prm.Hn;
-  const int nb = 128 / g;
-  CUtensorMap tm_qs, tm_qn, tm_w;
-  const uint64_t dqs[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(prm.Hs),
-                           static_cast<uint64_t>(prm.B)};
-  const uint32_t bqs[3] = {64, static_cast<uint32_t>(g), static_cast<uint32_t>(nb)};
-  const uint64_t dqn[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(prm.Hn),
-                           static_cast<uint64_t>(prm.B)};
-  const uint32_t bqn[3] = {64, 1, 128};
-  const uint64_t dw[2] = {static_cast<uint64_t>(prm.Hn) * 2 * D, static_cast<uint64_t>(prm.dl)};
-  const uint32_t bw[2] = {64, 128};
-  if (!make_map(&tm_qs, prm.q_sig, 3, dqs, bqs) || !make_map(&tm_qn, prm.q_noise, 3, dqn, bqn) ||
-      !make_map(&tm_w, prm.w_kvb, 2, dw, bw))
-    return GDLA_ERR_CUDA;
+int launch_decode_absorb(const gdla::DecodeParams &prm, const DecodeMaps &m, cudaStream_t stream) {
+  const int nb = 128 / (prm.Hs / prm.Hn);
   constexpr auto kern = gdla::gdla_decode_absorb_kernel<D>;
   const int rc = prepare_kernel<kern>(gdla::AbsorbSmem::kBytes, 0);
   if (rc != GDLA_OK) return rc;
   const int n_sig = (prm.B + nb - 1) / nb, n_noise = (prm.B + 127) / 128;
   kern<<<dim3(static_cast<unsigned>(prm.dl / 128), static_cast<unsigned>(prm.Hn),
               static_cast<unsigned>(n_sig + n_noise)),
-         gdla::kAbsThreads, gdla::AbsorbSmem::kBytes, stream>>>(tm_qs, tm_qn, tm_w, prm, n_sig);
+         gdla::kAbsThreads, gdla::AbsorbSmem::kBytes, stream>>>(m.qs, m.qn, m.w, prm, n_sig);
   return cudaGetLastError() == cudaSuccess ? GDLA_OK : GDLA_ERR_CUDA;
 }
 
 template <int NP>
-int launch_decode_attn(const gdla::DecodeParams &prm, const void *c_hat, cudaStream_t stream) {
+int launch_decode_attn(const gdla::DecodeParams &prm, const DecodeMaps &m, cudaStream_t stream) {
   using L = gdla::DecSmem<NP>;
-  CUtensorMap tm_qt, tm_c;
-  const uint64_t dq[2] = {static_cast<uint64_t>(prm.dl), static_cast<uint64_t>(prm.B) * NP};
-  const uint32_t qbox[2] = {64, NP};
-  const uint64_t dc[3] = {static_cast<uint64_t>(prm.dl), static_cast<uint64_t>(prm.L_max),
-                          static_cast<uint64_t>(prm.B)};
-  const uint32_t cbox[3] = {64, gdla::kDecTok, 1};
-  if (!make_map(&tm_qt, prm.qt, 2, dq, qbox) || !make_map(&tm_c, c_hat, 3, dc, cbox))
-    return GDLA_ERR_CUDA;
   constexpr auto kern = gdla::gdla_decode_attn_kernel<NP>;
   const int rc = prepare_kernel<kern>(L::kBytes, 0);
   if (rc != GDLA_OK) return rc;
   kern<<<dim3(static_cast<unsigned>(prm.n_split), static_cast<unsigned>(prm.B)), gdla::kDecThreads,
-         L::kBytes, stream>>>(tm_qt, tm_c, prm);
+         L::kBytes, stream>>>(m.qt, m.c, prm);
+  return cudaGetLastError() == cudaSuccess ? GDLA_OK : GDLA_ERR_CUDA;
+}
+
+// merge of the splits into Z, then the output GEMM and gate
+template <int NH>
+int launch_decode_combine(const gdla::DecodeParams &prm, const DecodeMaps &m,
+                          cudaStream_t stream) {
+  constexpr auto kout = gdla::gdla_decode_out_kernel<NH>;
+  const int rc = prepare_kernel<kout>(gdla::CombSmem::kBytes, 0);
+  if (rc != GDLA_OK) return rc;
+  const int64_t items = static_cast<int64_t>(prm.Hn) * prm.B * NH * (prm.dl / 4);
+  if (prm.n_split > 1)
+    gdla::gdla_decode_merge_kernel<NH, 1, 8>
+        <<<static_cast<unsigned>((items + 127) / 128), 128, 0, stream>>>(prm);
+  else
+    gdla::gdla_decode_merge_kernel<NH, 4, 1>
+        <<<static_cast<unsigned>((items + 511) / 512), 128, 0, stream>>>(prm);
+  if (cudaGetLastError() != cudaSuccess) return GDLA_ERR_CUDA;
+  kout<<<dim3(static_cast<unsigned>(prm.Hn), static_cast<unsigned>((prm.B + m.sb - 1) / m.sb)),
+         gdla::kCombThreads, gdla::CombSmem::kBytes, stream>>>(m.w, m.z, prm, m.sb);
   return cudaGetLastError() == cudaSuccess ? GDLA_OK : GDLA_ERR_CUDA;
 }
 
@@ -545,23 +584,24 @@ int gdla_decode_fwd(const void *q_sig, const void *q_noise, const void *c_hat,
   const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(d));
   prm.qscale = sc * 1.4426950408889634f;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int arc = d == 128 ? launch_decode_absorb<128>(prm, s) : launch_decode_absorb<64>(prm, s);
+  DecodeMaps maps;
+  if (!decode_maps(prm, c_hat, &maps)) return GDLA_ERR_CUDA;
+  const int arc =
+      d == 128 ? launch_decode_absorb<128>(prm, maps, s) : launch_decode_absorb<64>(prm, maps, s);
   if (arc != GDLA_OK) return arc;
-  const int rc = pl.Np == 80 ? launch_decode_attn<80>(prm, c_hat, s)
-                             : launch_decode_attn<16>(prm, c_hat, s);
+  const int rc = pl.Np == 80 ? launch_decode_attn<80>(prm, maps, s)
+                             : launch_decode_attn<16>(prm, maps, s);
   if (rc != GDLA_OK) return rc;
-  const dim3 cgrid(static_cast<unsigned>(Hn), static_cast<unsigned>(B));
   switch (Hs / Hn) {  // the combine is specialised for the heads of a group
-    case 1: gdla::gdla_decode_combine_kernel<2><<<cgrid, 128, 0, s>>>(prm); break;
-    case 2: gdla::gdla_decode_combine_kernel<3><<<cgrid, 128, 0, s>>>(prm); break;
-    case 3: gdla::gdla_decode_combine_kernel<4><<<cgrid, 128, 0, s>>>(prm); break;
-    case 4: gdla::gdla_decode_combine_kernel<5><<<cgrid, 128, 0, s>>>(prm); break;
-    case 5: gdla::gdla_decode_combine_kernel<6><<<cgrid, 128, 0, s>>>(prm); break;
-    case 6: gdla::gdla_decode_combine_kernel<7><<<cgrid, 128, 0, s>>>(prm); break;
-    case 7: gdla::gdla_decode_combine_kernel<8><<<cgrid, 128, 0, s>>>(prm); break;
-    default: gdla::gdla_decode_combine_kernel<9><<<cgrid, 128, 0, s>>>(prm); break;
+    case 1: return launch_decode_combine<2>(prm, maps, s);
+    case 2: return launch_decode_combine<3>(prm, maps, s);
+    case 3: return launch_decode_combine<4>(prm, maps, s);
+    case 4: return launch_decode_combine<5>(prm, maps, s);
+    case 5: return launch_decode_combine<6>(prm, maps, s);
+    case 6: return launch_decode_combine<7>(prm, maps, s);
+    case 7: return launch_decode_combine<8>(prm, maps, s);
+    default: return launch_decode_combine<9>(prm, maps, s);
   }
-  return cudaGetLastError() == cudaSuccess ? GDLA_OK : GDLA_ERR_CUDA;
 }
 
 int gdla_latent_rmsnorm(const void *c_kv, const void *rms_w, float eps, void *out,
