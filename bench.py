@@ -590,12 +590,15 @@ def _strip_comments(src):
 # The sources each kernel is built from (its launch code included): a
 # profiled counter applies to a kernel only while these are unchanged.
 KERNEL_SOURCES = {
-    "gdla_attn_fwd_kernel": ("gdla_api.cu", "attn_fwd.cuh", "sm100.cuh"),
-    "gdla_attn_win_kernel": ("gdla_api.cu", "attn_win.cuh", "attn_fwd.cuh", "sm100.cuh"),
-    "gdla_attn_rope_kernel": ("gdla_api.cu", "attn_rope.cuh", "attn_win.cuh", "attn_fwd.cuh",
-                              "sm100.cuh"),
-    "gdla_kv_expand_kernel": ("gdla_api.cu", "kv_expand.cuh", "sm100.cuh"),
-    "gdla_decode_attn_kernel": ("gdla_api.cu", "decode.cuh", "sm100.cuh"),
+    "gdla_attn_fwd_kernel": ("gdla_api.cu", "host_util.cuh", "attn_fwd.cuh", "sm100.cuh"),
+    "gdla_attn_win_kernel": ("gdla_api.cu", "host_util.cuh", "attn_win.cuh", "attn_fwd.cuh",
+                             "sm100.cuh"),
+    "gdla_attn_rope_kernel": ("gdla_api.cu", "host_util.cuh", "attn_rope.cuh", "attn_win.cuh",
+                              "attn_fwd.cuh", "sm100.cuh"),
+    "gdla_kv_expand_kernel": ("gdla_api.cu", "host_util.cuh", "kv_expand.cuh", "sm100.cuh"),
+    "gdla_decode_attn_kernel": ("gdla_api.cu", "host_util.cuh", "decode.cuh", "sm100.cuh"),
+    "gdla_attn_bwd": ("gdla_bwd.cu", "host_util.cuh", "bwd.cuh", "attn_rope.cuh", "attn_win.cuh",
+                      "attn_fwd.cuh", "sm100.cuh"),
 }
 
 

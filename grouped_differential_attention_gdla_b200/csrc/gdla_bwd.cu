@@ -2,7 +2,6 @@
 // include/gdla.h): argument validation, workspace layout, tensor maps and
 // the four launches of bwd.cuh on the caller's stream.  Like the forward
 // entry points, nothing here allocates, frees or synchronises.
-#include <atomic>
 #include <cmath>
 #include <cstdint>
 
@@ -10,65 +9,18 @@
 #include <cuda_runtime.h>
 
 #include "gdla.h"
+#include "host_util.cuh"
 #include "bwd.cuh"
 
 namespace {
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = []() -> EncodeTiledFn {
-    void *p = nullptr;
-    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
-            cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return nullptr;
-    return reinterpret_cast<EncodeTiledFn>(p);
-  }();
-  return fn;
-}
-
-bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+using namespace gdla_host;
 
 // 3-D row-major bf16 tensor [d2][d1][d0] with [1][128][64] boxes, 128B swizzle.
 bool map3(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1, uint64_t d2) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t gdim[3] = {d0, d1, d2};
-  const cuuint64_t gstride[2] = {d0 * 2, d0 * d1 * 2};
-  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(gdla::kBM), 1};
-  const cuuint32_t estride[3] = {1, 1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), gdim, gstride,
-            box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-         CUDA_SUCCESS;
-}
-
-// One-time dynamic shared-memory limit of kernel Kern per device.
-template <auto Kern>
-int prepare(uint32_t smem) {
-  static std::atomic<uint64_t> ready{0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return GDLA_ERR_CUDA;
-  const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
-  if (bit && (ready.load(std::memory_order_acquire) & bit)) return GDLA_OK;
-  if (cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
-    return GDLA_ERR_CUDA;
-  if (bit) ready.fetch_or(bit, std::memory_order_release);
-  return GDLA_OK;
-}
-
-int sms_of_device(int *sms) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return GDLA_ERR_CUDA;
-  return cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess
-             ? GDLA_OK
-             : GDLA_ERR_CUDA;
+  const uint64_t dims[3] = {d0, d1, d2};
+  const uint32_t box[3] = {64, static_cast<uint32_t>(gdla::kBM), 1};
+  return make_map(map, base, 3, dims, box);
 }
 
 // Workspace: H (fp32) of every head, its log-sum-exp and Delta (fp32,
@@ -107,13 +59,13 @@ int launch_bwd(const void *q_sig, const void *q_noise, const void *k, const void
       !map3(&tm_dox, bp.dox, H80 * D, T, B))
     return GDLA_ERR_CUDA;
   int sms = 0;
-  if (sms_of_device(&sms) != GDLA_OK) return GDLA_ERR_CUDA;
+  if (sm_count(&sms) != GDLA_OK) return GDLA_ERR_CUDA;
 
   // 1. the forward in save mode: H and the log-sum-exp of every head
   {
     using L = gdla::RopeSmemLayout<D, 0>;
     constexpr auto kern = gdla::gdla_attn_rope_kernel<D, 0, true, gdla::AttnSaveParams>;
-    const int rc = prepare<kern>(L::kBytes);
+    const int rc = prepare_kernel<kern>(L::kBytes, 0);
     if (rc != GDLA_OK) return rc;
     const uint64_t items = static_cast<uint64_t>(sp.n_qblk) * B * static_cast<uint64_t>(bp.Hn);
     if (items > 0x7fffffffull) return GDLA_ERR_UNSUPPORTED;
@@ -134,7 +86,7 @@ int launch_bwd(const void *q_sig, const void *q_noise, const void *k, const void
   {
     using L = gdla::DqSmemLayout<D>;
     constexpr auto kern = gdla::gdla_bwd_dq_kernel<D>;
-    const int rc = prepare<kern>(L::kBytes);
+    const int rc = prepare_kernel<kern>(L::kBytes, 0);
     if (rc != GDLA_OK) return rc;
     const uint64_t items = static_cast<uint64_t>(bp.n_qblk) * B * H80;
     if (items > 0x7fffffffull) return GDLA_ERR_UNSUPPORTED;
@@ -146,7 +98,7 @@ int launch_bwd(const void *q_sig, const void *q_noise, const void *k, const void
   {
     using L = gdla::DkdvSmemLayout<D>;
     constexpr auto kern = gdla::gdla_bwd_dkdv_kernel<D>;
-    const int rc = prepare<kern>(L::kBytes);
+    const int rc = prepare_kernel<kern>(L::kBytes, 0);
     if (rc != GDLA_OK) return rc;
     const uint64_t items = static_cast<uint64_t>(bp.n_kblk) * B * static_cast<uint64_t>(bp.Hn);
     if (items > 0x7fffffffull) return GDLA_ERR_UNSUPPORTED;
@@ -189,7 +141,7 @@ int gdla_attn_bwd(const void *q_sig, const void *q_noise, const void *k, const v
   const void *ptrs[] = {q_sig, q_noise, k, v, lambda, gate, d_out, dq_sig, dq_noise,
                         dk,    dv,      dlambda, dgate, workspace};
   for (const void *p : ptrs)
-    if (!al16(p)) return GDLA_ERR_ALIGNMENT;
+    if (!aligned16(p)) return GDLA_ERR_ALIGNMENT;
   if (d_status && (reinterpret_cast<uintptr_t>(d_status) & 3u) != 0) return GDLA_ERR_ALIGNMENT;
 
   uint8_t *wsb = static_cast<uint8_t *>(workspace);
