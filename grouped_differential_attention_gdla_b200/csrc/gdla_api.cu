@@ -456,7 +456,7 @@ int gdla_decode_fwd(const void *q_sig, const void *q_noise, const void *c_hat,
   if (B > 65535 || L_max > 0x7fffffffll - gdla::kDecTok) return GDLA_ERR_UNSUPPORTED;
   DecodePlan pl;
   if (!decode_plan(B, L_max, Hs, Hn, d_latent, window, &pl)) return GDLA_ERR_UNSUPPORTED;
-  if (pl.Np != 16 && pl.Np != 80) return GDLA_ERR_UNSUPPORTED;
+  if (pl.Np > 80) return GDLA_ERR_UNSUPPORTED;  // head rows: 16, 32, 48, 64 or 80
   if (workspace_bytes < pl.qt_bytes + pl.part_bytes) return GDLA_ERR_INVALID_ARG;
   if (!aligned16(q_sig) || !aligned16(q_noise) || !aligned16(c_hat) || !aligned16(w_kvb) ||
       !aligned16(lambda) || !aligned16(gate) || !aligned16(out) || !aligned16(workspace) ||
@@ -491,8 +491,14 @@ int gdla_decode_fwd(const void *q_sig, const void *q_noise, const void *c_hat,
   const int arc =
       d == 128 ? launch_decode_absorb<128>(prm, maps, s) : launch_decode_absorb<64>(prm, maps, s);
   if (arc != GDLA_OK) return arc;
-  const int rc = pl.Np == 80 ? launch_decode_attn<80>(prm, maps, s)
-                             : launch_decode_attn<16>(prm, maps, s);
+  int rc;
+  switch (pl.Np) {  // head rows of the attention tiles
+    case 16: rc = launch_decode_attn<16>(prm, maps, s); break;
+    case 32: rc = launch_decode_attn<32>(prm, maps, s); break;
+    case 48: rc = launch_decode_attn<48>(prm, maps, s); break;
+    case 64: rc = launch_decode_attn<64>(prm, maps, s); break;
+    default: rc = launch_decode_attn<80>(prm, maps, s); break;
+  }
   if (rc != GDLA_OK) return rc;
   switch (Hs / Hn) {  // the combine is specialised for the heads of a group
     case 1: return launch_decode_combine<2>(prm, maps, s);

@@ -234,8 +234,9 @@ size_t gdla_decode_workspace_bytes(int B, int64_t L_max, int Hs, int Hn,
  * scale      softmax scale on q.k; <= 0 selects 1/sqrt(d)
  * Cache rows the query does not keep (past cache_len, before the window)
  * are read and multiplied by zero weights: they must hold finite values.
- * Supported: Hn == Hkv, Hs / Hn <= 8, Hs + Hn rounded up to 16 equal to 16
- * or 80, d in {64, 128}, d_latent in {128, 256, 384, 512}, B <= 65535.
+ * Supported: Hn == Hkv, Hs / Hn <= 8, Hs + Hn <= 80 (the head rows are
+ * padded to a multiple of 16), d in {64, 128}, d_latent in {128, 256, 384,
+ * 512}, B <= 65535.
  */
 int gdla_decode_fwd(const void *q_sig, const void *q_noise, const void *c_hat,
                     const int32_t *cache_len, const void *w_kvb,

@@ -212,7 +212,7 @@ def _dec(lib, q=A, qn=A, c=A, cl=A, w=A, lam=A, gate=A, out=A, B=2, L=300, Hs=8,
     (dict(ws_bytes=1000), INVALID),
     (dict(Hn=2, Hkv=4), UNSUPPORTED), (dict(Hs=6, Hn=4, Hkv=4), UNSUPPORTED),
     (dict(Hs=18, Hn=2, Hkv=2), UNSUPPORTED),   # 10 signal heads per group
-    (dict(Hs=32, Hn=8, Hkv=8), UNSUPPORTED),   # 40 head rows: neither 16 nor 80
+    (dict(Hs=72, Hn=9, Hkv=9), UNSUPPORTED),   # 81 head rows: more than 80
     (dict(d=96), UNSUPPORTED), (dict(dl=448), UNSUPPORTED), (dict(dl=640), UNSUPPORTED),
     (dict(B=70000), UNSUPPORTED),
     (dict(c=M), ALIGN), (dict(ws=M), ALIGN), (dict(out=M), ALIGN), (dict(cl=0x100002), ALIGN),
@@ -231,6 +231,8 @@ def test_decode_workspace_size_follows_the_shapes(lib):
     # a 128-token window touches at most 2 chunks: one split per sequence
     assert f(64, 32768, 64, 16, 512, 128) == 64 * 80 * 512 * 2 + 64 * 1 * 80 * 514 * 4
     assert f(1, 100, 8, 2, 512, 0) == 16 * 512 * 2 + 1 * 1 * 16 * 514 * 4
+    # 32 + 8 heads: 40 head rows padded to 48
+    assert f(1, 100, 32, 8, 512, 0) == 48 * 512 * 2 + 1 * 1 * 48 * 514 * 4
     assert f(0, 100, 8, 2, 512, 0) == 0 and f(1, 0, 8, 2, 512, 0) == 0
 
 

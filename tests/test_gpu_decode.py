@@ -63,6 +63,14 @@ def _oracle(x, lens, window):
     (4, 2000, 64, 16, 128, 512, [2000, 1, 777, 1024], 0, False),
     (4, 2000, 64, 16, 128, 512, [2000, 1, 777, 1024], 128, True),
     (2, 5000, 64, 16, 128, 512, [5000, 3000], 1, False),
+    # one signal head per group (2 head rows per group in the combine)
+    (5, 600, 4, 4, 128, 512, [600, 1, 250, 599, 128], 0, False),
+    # three signal heads per group, d = 64, a 256-d latent
+    (3, 400, 6, 2, 64, 256, [400, 17, 256], 0, True),
+    # eight signal heads per group (9 head rows per group, 80 padded rows)
+    (2, 300, 16, 2, 128, 512, [300, 77], 64, False),
+    # 37 sequences: several sequences per output-GEMM CTA, the last block ragged
+    (37, 300, 64, 16, 128, 512, [300 - 8 * i for i in range(37)], 0, False),
 ])
 def test_decode_matches_oracle(B, L_max, Hs, Hn, d, dl, lens, window, with_w):
     x = _case(B, L_max, Hs, Hn, d, dl, seed=L_max + window, with_w=with_w)
