@@ -144,13 +144,15 @@ template <int D>
 struct DqSmemLayout {
   static constexpr uint32_t kSub = kBM * 128;        // [128][64] bf16 swizzled
   static constexpr uint32_t kTile = (D / 64) * kSub;  // [128][D]
-  static constexpr uint32_t kStages = 4;              // K/V ring (K_t, V_t alternate)
+  // K/V ring (K_t, V_t alternate); K_t is held until dQ(t), so five stages
+  // let K_{t+2} load while K_t and both tiles of t+1 are resident
+  static constexpr uint32_t kStages = 5;
   static constexpr uint32_t kQOff = 0;
   static constexpr uint32_t kDoOff = kQOff + kTile;
   static constexpr uint32_t kRingOff = kDoOff + kTile;
   static constexpr uint32_t kBarOff = kRingOff + kStages * kTile;
-  // qd_full kv_full[S] kv_empty[S] s_full p_full dq_done
-  static constexpr uint32_t kNumBars = 1 + 2 * kStages + 3;
+  // qd_full kv_full[S] kv_empty[S] s_full p_full[2] dp_free dq_done
+  static constexpr uint32_t kNumBars = 1 + 2 * kStages + 5;
   static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;
   static constexpr uint32_t kBytes = kMiscOff + 16;
   static_assert(kBytes <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
@@ -159,7 +161,11 @@ struct DqSmemLayout {
 // One CTA per (batch b, head x of Hs + Hn, query block), heaviest blocks
 // first.  Warps 0-7: P and dS (warpgroup `half` takes key columns
 // [64 half, 64 half + 64)); 8-11: dQ epilogue; 12: TMA; 13: TMEM and MMA.
-// TMEM: S [0,128) (dS packed over it), dP [128,256), dQ [256, 256+D).
+// TMEM: S of even tiles [0,128) and of odd tiles [384,512) (dS packed over
+// each), dP [128,256), dQ [256, 256+D).  The MMA warp computes S(t+1) while
+// the elementwise warps work on tile t, and dP(t+1) as soon as they have
+// read dP(t) (half-way through the tile), so the tensor core is busy with
+// the next tile's scores while the current tile's dS is formed.
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     gdla_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qs,
@@ -179,8 +185,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   auto kv_full = [&](uint32_t s) { return bar0 + 8u * (1 + s); };
   auto kv_empty = [&](uint32_t s) { return bar0 + 8u * (1 + L::kStages + s); };
   const uint32_t s_full = bar0 + 8u * (1 + 2 * L::kStages);
-  const uint32_t p_full = s_full + 8u;
-  const uint32_t dq_done = s_full + 16u;
+  auto p_full = [&](int t) { return s_full + 8u * (1 + (t & 1)); };  // dS(t) packed
+  const uint32_t dp_free = s_full + 24u;  // dP(t) read out by every elementwise warp
+  const uint32_t dq_done = s_full + 32u;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
   const int warp = threadIdx.x >> 5;
@@ -213,7 +220,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(kv_empty(s), 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(p_full, 8);
+    mbar_init(p_full(0), 8);
+    mbar_init(p_full(1), 8);
+    mbar_init(dp_free, 8);
     mbar_init(dq_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -226,7 +235,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t t_s = tmem, t_dp = tmem + 128u, t_dq = tmem + 256u;
+  const uint32_t t_dp = tmem + 128u, t_dq = tmem + 256u;
+  auto t_s = [&](int t) { return tmem + ((t & 1) ? 384u : 0u); };
 
   if (warp == kBwdProducerWarp) {
     // =============================== TMA: Q_x and dH_x, then K_t, V_t per tile
@@ -267,55 +277,72 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_wait_for(qd_full, 0, 100000000ull);
     }
   } else if (warp == kBwdMmaWarp) {
-    // =============================== MMA: S(t), dP(t); then dQ += dS(t) K_t
+    // =============================== MMA: S(t+1) and dP(t+1) ahead of dQ += dS(t) K_t
+    // (the ring holds K_t, V_t at positions 2t, 2t+1)
     const bool leader = elect_one();
     constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBN, false, false);
     constexpr uint32_t kIdescQ = idesc_bf16_f32(kBM, D, false, true);
     const uint64_t qd = sdesc_sw128(sbase + L::kQOff, 16, 1024);
     const uint64_t dod = sdesc_sw128(sbase + L::kDoOff, 16, 1024);
-    bool ok = __all_sync(0xffffffffu, mbar_wait(qd_full, 0, abort_flag));
-    uint32_t c = 0;
-    uint32_t done = 0;
-    for (int t = 0; t < n && ok; ++t) {
-      // S = Q K_t^T, dP = dH V_t^T (K-major operands, D/16 K-steps each)
-      const uint32_t sk = c % L::kStages;
-      ok = __all_sync(0xffffffffu, mbar_wait(kv_full(sk), (c / L::kStages) & 1u, abort_flag));
-      ++c;
-      if (!ok) break;
-      const uint32_t sv = c % L::kStages;
-      ok = __all_sync(0xffffffffu, mbar_wait(kv_full(sv), (c / L::kStages) & 1u, abort_flag));
-      ++c;
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t kbase = sbase + L::kRingOff + sk * L::kTile;
-      const uint32_t vbase = sbase + L::kRingOff + sv * L::kTile;
-      if (leader) {
-        const uint64_t kd = sdesc_sw128(kbase, 16, 1024);
-        const uint64_t vd = sdesc_sw128(vbase, 16, 1024);
+    auto slot = [&](uint32_t pos) { return pos % L::kStages; };
+    auto wait_full = [&](uint32_t pos) {
+      return __all_sync(0xffffffffu,
+                        mbar_wait(kv_full(slot(pos)), (pos / L::kStages) & 1u, abort_flag));
+    };
+    auto tile = [&](uint32_t pos) { return sbase + L::kRingOff + slot(pos) * L::kTile; };
+    // S(t) = Q K_t^T into t's S buffer (K-major operands, D/16 K-steps)
+    auto issue_s = [&](int t) {
+      if (!leader) return;
+      const uint64_t kd = sdesc_sw128(tile(2u * t), 16, 1024);
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (k >> 2) * L::kSub + (k & 3) * 32;
-          umma_ss(t_s, qd + (off >> 4), kd + (off >> 4), kIdescS, k > 0 ? 1u : 0u);
-        }
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (k >> 2) * L::kSub + (k & 3) * 32;
-          umma_ss(t_dp, dod + (off >> 4), vd + (off >> 4), kIdescS, k > 0 ? 1u : 0u);
-        }
-        umma_commit(s_full);
-        umma_commit(kv_empty(sv));  // V_t is no longer needed
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t off = (k >> 2) * L::kSub + (k & 3) * 32;
+        umma_ss(t_s(t), qd + (off >> 4), kd + (off >> 4), kIdescS, k > 0 ? 1u : 0u);
       }
-      ok = __all_sync(0xffffffffu, mbar_wait(p_full, static_cast<uint32_t>(t) & 1u, abort_flag));
+    };
+    // dP(t) = dH V_t^T, then S(t) and dP(t) are announced and V_t released
+    auto issue_dp = [&](int t) {
+      if (!leader) return;
+      const uint64_t vd = sdesc_sw128(tile(2u * t + 1u), 16, 1024);
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t off = (k >> 2) * L::kSub + (k & 3) * 32;
+        umma_ss(t_dp, dod + (off >> 4), vd + (off >> 4), kIdescS, k > 0 ? 1u : 0u);
+      }
+      umma_commit(s_full);
+      umma_commit(kv_empty(slot(2u * t + 1u)));
+    };
+    bool ok = __all_sync(0xffffffffu, mbar_wait(qd_full, 0, abort_flag));
+    uint32_t done = 0;
+    if (ok && n > 0) ok = wait_full(0) && wait_full(1);
+    if (ok && n > 0) {
+      tc_fence_after();
+      issue_s(0);
+      issue_dp(0);
+    }
+    for (int t = 0; t < n && ok; ++t) {
+      if (t + 1 < n) {
+        ok = wait_full(2u * (t + 1)) && wait_full(2u * (t + 1) + 1u);
+        if (!ok) break;
+        tc_fence_after();
+        issue_s(t + 1);  // its buffer last held dS(t-1), read by the dQ MMA issued before
+        ok = __all_sync(0xffffffffu, mbar_wait(dp_free, static_cast<uint32_t>(t) & 1u, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        issue_dp(t + 1);
+      }
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(p_full(t), static_cast<uint32_t>(t >> 1) & 1u, abort_flag));
       if (!ok) break;
       tc_fence_after();
       // dQ += dS K_t: A = dS (TMEM, packed halves), B = K_t MN-major over d
       if (leader) {
-        const uint64_t kmn = sdesc_sw128(kbase, kBN * 128, 1024);
+        const uint64_t kmn = sdesc_sw128(tile(2u * t), kBN * 128, 1024);
 #pragma unroll
         for (int k = 0; k < kBN / 16; ++k)
-          umma_ts(t_dq, t_s + split_col(k), kmn + ((k * (16 * 128)) >> 4), kIdescQ,
+          umma_ts(t_dq, t_s(t) + split_col(k), kmn + ((k * (16 * 128)) >> 4), kIdescQ,
                   (t > 0 || k > 0) ? 1u : 0u);
-        umma_commit(kv_empty(sk));
+        umma_commit(kv_empty(slot(2u * t)));
         if (t == n - 1) umma_commit(dq_done);
       }
       if (t == n - 1) ++done;
@@ -367,6 +394,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(s_full, static_cast<uint32_t>(t) & 1u, abort_flag));
       if (!ok) break;
       tc_fence_after();
+      const uint32_t ts = t_s(t);
       const int kbase = (j_lo + t) * kBN;
       int c_lo, c_hi;  // kept key columns of this row in the tile
       if (p.causal) {
@@ -380,7 +408,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int u = 0; u < 2; ++u) {
         const int cc = 2 * half + u;  // 32-column chunk of the tile
         uint32_t sv[32], dpv[32];
-        tmem_ld32x2_sync(t_s + lane_off + 32 * cc, t_dp + lane_off + 32 * cc, sv, dpv);
+        tmem_ld32x2_sync(ts + lane_off + 32 * cc, t_dp + lane_off + 32 * cc, sv, dpv);
+        if (u == 1) {  // this warp has read its whole dP(t): dP(t+1) may overwrite it
+          tc_fence_before();
+          warp_arrive(dp_free);
+        }
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
@@ -393,11 +425,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                               p1 * (__uint_as_float(dpv[2 * e + 1]) - dl));
         }
         // dS of this chunk, packed into this half's own S columns
-        tmem_st16(t_s + lane_off + 64 * half + 16 * u, pk);
+        tmem_st16(ts + lane_off + 64 * half + 16 * u, pk);
       }
       tmem_wait_st();
       tc_fence_before();
-      warp_arrive(p_full);
+      warp_arrive(p_full(t));
     }
   }
 
