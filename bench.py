@@ -215,8 +215,9 @@ class Layer:
                                                                    wl.d_latent, wl.window),
                                   dtype=torch.uint8, device=dev)
             self.out = torch.empty((wl.B, wl.Hs * wl.d), dtype=torch.bfloat16, device=dev)
+            # four kernels per call: absorb, attention, split merge, output GEMM
             self.launches.append(("%s/decode" % wl.name, "gdla_decode_attn_kernel",
-                                  wl.attn_flops(), wl.decode_bytes(), 3))
+                                  wl.attn_flops(), wl.decode_bytes(), 4))
             return
         if wl.bwd:
             # the six gradients in one buffer (the step's output), the scratch
