@@ -722,18 +722,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         uint32_t sv[32], dpv[32];
         tmem_ld32x2_sync(t_s + lane_off + 32 * cc, t_dp + lane_off + 32 * cc, sv, dpv);
         uint32_t pk[16], dk[16];
+        // the chunk's lse and Delta values, four columns per shared-memory read
+        const float4 *lse4 = reinterpret_cast<const float4 *>(lse + 32 * cc);
+        const float4 *dlt4 = reinterpret_cast<const float4 *>(dlt + 32 * cc);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int c0 = 32 * cc + 2 * e;
-          const bool a0 = c0 >= c_lo && c0 <= c_hi;
-          const bool a1 = c0 + 1 >= c_lo && c0 + 1 <= c_hi;
-          const float p0 = a0 ? ex2_approx(__uint_as_float(sv[2 * e]) * sl2 - lse[c0]) : 0.f;
-          const float p1 = a1 ? ex2_approx(__uint_as_float(sv[2 * e + 1]) * sl2 - lse[c0 + 1]) : 0.f;
-          pk[e] = pack_bf16x2(p0, p1);
-          // selected, not multiplied: a masked column's lse and Delta may be
-          // the unwritten padding past T
-          dk[e] = pack_bf16x2(a0 ? p0 * (__uint_as_float(dpv[2 * e]) - dlt[c0]) : 0.f,
-                              a1 ? p1 * (__uint_as_float(dpv[2 * e + 1]) - dlt[c0 + 1]) : 0.f);
+        for (int e2 = 0; e2 < 8; ++e2) {
+          const float4 l4 = lse4[e2], d4 = dlt4[e2];
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+          const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int e = 2 * e2 + h2;
+            const int c0 = 32 * cc + 2 * e;
+            const bool a0 = c0 >= c_lo && c0 <= c_hi;
+            const bool a1 = c0 + 1 >= c_lo && c0 + 1 <= c_hi;
+            const float p0 = a0 ? ex2_approx(__uint_as_float(sv[2 * e]) * sl2 - lv[2 * h2]) : 0.f;
+            const float p1 =
+                a1 ? ex2_approx(__uint_as_float(sv[2 * e + 1]) * sl2 - lv[2 * h2 + 1]) : 0.f;
+            pk[e] = pack_bf16x2(p0, p1);
+            // selected, not multiplied: a masked column's lse and Delta may be
+            // the unwritten padding past T
+            dk[e] = pack_bf16x2(a0 ? p0 * (__uint_as_float(dpv[2 * e]) - dv[2 * h2]) : 0.f,
+                                a1 ? p1 * (__uint_as_float(dpv[2 * e + 1]) - dv[2 * h2 + 1]) : 0.f);
+          }
         }
         tmem_st16(t_s + lane_off + 64 * half + 16 * u, pk);
         tmem_st16(t_dp + lane_off + 64 * half + 16 * u, dk);
