@@ -447,15 +447,17 @@ template <int D>
 struct DkdvSmemLayout {
   static constexpr uint32_t kSub = kBM * 128;
   static constexpr uint32_t kTile = (D / 64) * kSub;
-  static constexpr uint32_t kStages = 2;  // (Q_x, dH_x, lse, Delta) of one query block
+  static constexpr uint32_t kQStages = 2;   // Q_x of a query block, then its lse[128], Delta[128]
+  static constexpr uint32_t kDhStages = 3;  // dH_x of a query block
   static constexpr uint32_t kStatBytes = 2 * kBM * 4;
-  static constexpr uint32_t kEntry = 2 * kTile + 1024;  // tiles, then lse[128], Delta[128]
+  static constexpr uint32_t kQEntry = kTile + 1024;
   static constexpr uint32_t kKOff = 0;
   static constexpr uint32_t kVOff = kKOff + kTile;
-  static constexpr uint32_t kRingOff = kVOff + kTile;
-  static constexpr uint32_t kBarOff = kRingOff + kStages * kEntry;
-  // kv_full ring_full[S] ring_empty[S] s_full p_full acc_done
-  static constexpr uint32_t kNumBars = 1 + 2 * kStages + 3;
+  static constexpr uint32_t kQOff = kVOff + kTile;
+  static constexpr uint32_t kDhOff = kQOff + kQStages * kQEntry;
+  static constexpr uint32_t kBarOff = kDhOff + kDhStages * kTile;
+  // kv_full q_full[2] q_empty[2] dh_full[3] dh_empty[3] s_full p_full dp_free acc_done
+  static constexpr uint32_t kNumBars = 1 + 2 * kQStages + 2 * kDhStages + 4;
   static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;
   static constexpr uint32_t kBytes = kMiscOff + 16;
   static_assert(kBytes <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
@@ -481,8 +483,13 @@ __device__ __forceinline__ void dkdv_qrange(const BwdParams &p, int kb, int &qlo
 // One CTA per (batch b, KV group k, key block kb), heaviest (earliest) key
 // blocks first.  Warps 0-7: P^T and dS^T (warpgroup `half` takes query
 // columns [64 half, 64 half + 64)); 8-11: dK, dV epilogue; 12: TMA;
-// 13: TMEM and MMA.  TMEM: S^T [0,128) (P^T packed over it), dP^T [128,256)
-// (dS^T packed over it), dV [256, 256+D), dK [256+D, 256+2D).
+// 13: TMEM and MMA.  TMEM: S^T [0,128), dP^T [128,256), dV [256, 256+D),
+// dK [256+D, 256+2D).  Each 32-column chunk of S^T is overwritten by its own
+// P^T (16 columns of bf16 pairs) and dS^T (the next 16), so dP^T is free as
+// soon as the elementwise warps have read it and the MMA warp computes the
+// next tile's dP^T while they work.  K and V stay in shared memory; Q (with
+// the block's lse and Delta rows) and dH stream through rings of two and
+// three entries.
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     gdla_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qs,
@@ -499,11 +506,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + L::kBarOff;
   const uint32_t kv_full = bar0;
-  auto ring_full = [&](uint32_t s) { return bar0 + 8u * (1 + s); };
-  auto ring_empty = [&](uint32_t s) { return bar0 + 8u * (1 + L::kStages + s); };
-  const uint32_t s_full = bar0 + 8u * (1 + 2 * L::kStages);
+  auto q_full = [&](uint32_t s) { return bar0 + 8u * (1 + s); };
+  auto q_empty = [&](uint32_t s) { return bar0 + 8u * (1 + L::kQStages + s); };
+  auto dh_full = [&](uint32_t s) { return bar0 + 8u * (1 + 2 * L::kQStages + s); };
+  auto dh_empty = [&](uint32_t s) { return bar0 + 8u * (1 + 2 * L::kQStages + L::kDhStages + s); };
+  const uint32_t s_full = bar0 + 8u * (1 + 2 * L::kQStages + 2 * L::kDhStages);
   const uint32_t p_full = s_full + 8u;
-  const uint32_t acc_done = s_full + 16u;
+  const uint32_t dp_free = s_full + 16u;
+  const uint32_t acc_done = s_full + 24u;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
   const int warp = threadIdx.x >> 5;
@@ -524,15 +534,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int hh = tt / nq;
     return hh == 0 ? p.Hs + kvh : p.g * kvh + (hh - 1);
   };
+  auto q_slot = [](int tt) { return static_cast<uint32_t>(tt) % L::kQStages; };
+  auto q_par = [](int tt) { return (static_cast<uint32_t>(tt) / L::kQStages) & 1u; };
+  auto dh_slot = [](int tt) { return static_cast<uint32_t>(tt) % L::kDhStages; };
+  auto dh_par = [](int tt) { return (static_cast<uint32_t>(tt) / L::kDhStages) & 1u; };
+  auto q_base = [&](int tt) { return sbase + L::kQOff + q_slot(tt) * L::kQEntry; };
+  auto dh_base = [&](int tt) { return sbase + L::kDhOff + dh_slot(tt) * L::kTile; };
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
-    for (uint32_t s = 0; s < L::kStages; ++s) {
-      mbar_init(ring_full(s), 1);
-      mbar_init(ring_empty(s), 1);
+    for (uint32_t s = 0; s < L::kQStages; ++s) {
+      mbar_init(q_full(s), 1);
+      mbar_init(q_empty(s), 1);
+    }
+    for (uint32_t s = 0; s < L::kDhStages; ++s) {
+      mbar_init(dh_full(s), 1);
+      mbar_init(dh_empty(s), 1);
     }
     mbar_init(s_full, 1);
     mbar_init(p_full, 8);
+    mbar_init(dp_free, 8);
     mbar_init(acc_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -547,10 +568,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t t_s = tmem, t_dp = tmem + 128u;
   const uint32_t t_dv = tmem + 256u, t_dk = tmem + 256u + D;
+  // TMEM column (from t_s) of the bf16 pairs of query K-step k (16 queries):
+  // chunk 32 * (k / 2) of S^T, P^T in its first 16 columns, dS^T in the next
+  auto pt_col = [](int k) -> uint32_t { return 32u * (k >> 1) + 8u * (k & 1); };
 
   if (warp == kBwdProducerWarp) {
     // =============================== TMA: K, V once; then per tile the
-    // head's query block: Q_x, dH_x, its lse and Delta rows
+    // head's dH block, and its Q block with the lse and Delta rows
     const bool leader = elect_one();
     if (leader) {
       mbar_arrive_expect_tx(kv_full, 2 * L::kTile);
@@ -561,89 +585,125 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
     }
     bool ok = true;
-    uint32_t issued = 0;
+    uint32_t q_issued = 0, dh_issued = 0;
     for (int tt = 0; tt < n_tiles && ok; ++tt) {
-      const uint32_t s = tt % L::kStages;
-      ok = __all_sync(0xffffffffu,
-                      mbar_wait(ring_empty(s), ((tt / L::kStages) & 1u) ^ 1u, abort_flag));
-      if (!ok) break;
       const int xh = tile_head(tt);
       const int q0 = (qlo + tt % nq) * kBM;
-      const uint32_t dst = sbase + L::kRingOff + s * L::kEntry;
+      // dH first: its slot frees one tile earlier than Q's
+      ok = __all_sync(0xffffffffu, mbar_wait(dh_empty(dh_slot(tt)), dh_par(tt) ^ 1u, abort_flag));
+      if (!ok) break;
       if (leader) {
-        mbar_arrive_expect_tx(ring_full(s), 2 * L::kTile + L::kStatBytes);
+        mbar_arrive_expect_tx(dh_full(dh_slot(tt)), L::kTile);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(dh_base(tt) + c * L::kSub, &tm_dox, dh_full(dh_slot(tt)), xh * D + c * 64,
+                      q0, b);
+      }
+      ++dh_issued;
+      ok = __all_sync(0xffffffffu, mbar_wait(q_empty(q_slot(tt)), q_par(tt) ^ 1u, abort_flag));
+      if (!ok) break;
+      if (leader) {
+        const uint32_t dst = q_base(tt);
+        mbar_arrive_expect_tx(q_full(q_slot(tt)), L::kTile + L::kStatBytes);
         const bool noise = xh >= p.Hs;
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d(dst + c * L::kSub, noise ? &tm_qn : &tm_qs, ring_full(s),
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(dst + c * L::kSub, noise ? &tm_qn : &tm_qs, q_full(q_slot(tt)),
                       (noise ? xh - p.Hs : xh) * D + c * 64, q0, b);
-          tma_load_3d(dst + L::kTile + c * L::kSub, &tm_dox, ring_full(s), xh * D + c * 64, q0,
-                      b);
-        }
         const int64_t so = (static_cast<int64_t>(b) * H80 + xh) * p.tp + q0;
-        bulk_load(dst + 2 * L::kTile, p.lse + so, kBM * 4, ring_full(s));
-        bulk_load(dst + 2 * L::kTile + kBM * 4, p.delta + so, kBM * 4, ring_full(s));
+        bulk_load(dst + L::kTile, p.lse + so, kBM * 4, q_full(q_slot(tt)));
+        bulk_load(dst + L::kTile + kBM * 4, p.delta + so, kBM * 4, q_full(q_slot(tt)));
       }
-      ++issued;
+      ++q_issued;
     }
     if (!ok && leader) {
-      for (uint32_t s = 0; s < L::kStages; ++s) {
-        const uint32_t n_s = issued > s ? (issued - 1 - s) / L::kStages + 1 : 0;
-        if (n_s) mbar_wait_for(ring_full(s), (n_s - 1) & 1u, 100000000ull);
+      for (uint32_t s = 0; s < L::kQStages; ++s) {
+        const uint32_t n_s = q_issued > s ? (q_issued - 1 - s) / L::kQStages + 1 : 0;
+        if (n_s) mbar_wait_for(q_full(s), (n_s - 1) & 1u, 100000000ull);
+      }
+      for (uint32_t s = 0; s < L::kDhStages; ++s) {
+        const uint32_t n_s = dh_issued > s ? (dh_issued - 1 - s) / L::kDhStages + 1 : 0;
+        if (n_s) mbar_wait_for(dh_full(s), (n_s - 1) & 1u, 100000000ull);
       }
       mbar_wait_for(kv_full, 0, 100000000ull);
     }
   } else if (warp == kBwdMmaWarp) {
-    // =============================== MMA: S^T, dP^T; then dV += P^T dH,
-    // dK += dS^T Q
+    // =============================== MMA: S^T(t), dP^T(t); dP^T(t+1) once
+    // dP^T(t) is read; dV += P^T dH, dK += dS^T Q; then S^T(t+1)
     const bool leader = elect_one();
     constexpr uint32_t kIdescS = idesc_bf16_f32(kBN, kBM, false, false);
     constexpr uint32_t kIdescA = idesc_bf16_f32(kBN, D, false, true);
     const uint64_t kd = sdesc_sw128(sbase + L::kKOff, 16, 1024);
     const uint64_t vd = sdesc_sw128(sbase + L::kVOff, 16, 1024);
+    auto issue_st = [&](int tt) {  // S^T = K Q^T
+      if (!leader) return;
+      const uint64_t qdk = sdesc_sw128(q_base(tt), 16, 1024);
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t off = (k >> 2) * L::kSub + (k & 3) * 32;
+        umma_ss(t_s, kd + (off >> 4), qdk + (off >> 4), kIdescS, k > 0 ? 1u : 0u);
+      }
+    };
+    auto issue_dpt = [&](int tt) {  // dP^T = V dH^T
+      if (!leader) return;
+      const uint64_t dodk = sdesc_sw128(dh_base(tt), 16, 1024);
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t off = (k >> 2) * L::kSub + (k & 3) * 32;
+        umma_ss(t_dp, vd + (off >> 4), dodk + (off >> 4), kIdescS, k > 0 ? 1u : 0u);
+      }
+    };
+    auto wait_q = [&](int tt) {
+      return __all_sync(0xffffffffu, mbar_wait(q_full(q_slot(tt)), q_par(tt), abort_flag));
+    };
+    auto wait_dh = [&](int tt) {
+      return __all_sync(0xffffffffu, mbar_wait(dh_full(dh_slot(tt)), dh_par(tt), abort_flag));
+    };
     bool ok = __all_sync(0xffffffffu, mbar_wait(kv_full, 0, abort_flag));
     bool done = false;
-    for (int tt = 0; tt < n_tiles && ok; ++tt) {
-      const uint32_t s = tt % L::kStages;
-      ok = __all_sync(0xffffffffu, mbar_wait(ring_full(s), (tt / L::kStages) & 1u, abort_flag));
-      if (!ok) break;
+    if (ok && n_tiles > 0) ok = wait_q(0) && wait_dh(0);
+    if (ok && n_tiles > 0) {
       tc_fence_after();
-      const uint32_t qbase = sbase + L::kRingOff + s * L::kEntry;
-      const uint32_t dobase = qbase + L::kTile;
-      if (leader) {
-        const uint64_t qdk = sdesc_sw128(qbase, 16, 1024);
-        const uint64_t dodk = sdesc_sw128(dobase, 16, 1024);
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (k >> 2) * L::kSub + (k & 3) * 32;
-          umma_ss(t_s, kd + (off >> 4), qdk + (off >> 4), kIdescS, k > 0 ? 1u : 0u);
-        }
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (k >> 2) * L::kSub + (k & 3) * 32;
-          umma_ss(t_dp, vd + (off >> 4), dodk + (off >> 4), kIdescS, k > 0 ? 1u : 0u);
-        }
-        umma_commit(s_full);
+      issue_st(0);
+      issue_dpt(0);
+      if (leader) umma_commit(s_full);
+    }
+    for (int tt = 0; tt < n_tiles && ok; ++tt) {
+      if (tt + 1 < n_tiles) {
+        ok = wait_dh(tt + 1);
+        if (!ok) break;
+        ok = __all_sync(0xffffffffu, mbar_wait(dp_free, static_cast<uint32_t>(tt) & 1u, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        issue_dpt(tt + 1);
       }
       ok = __all_sync(0xffffffffu, mbar_wait(p_full, static_cast<uint32_t>(tt) & 1u, abort_flag));
       if (!ok) break;
       tc_fence_after();
       if (leader) {
         // B operands MN-major over d: dH_x and Q_x, 16 query rows per K-step
-        const uint64_t domn = sdesc_sw128(dobase, kBM * 128, 1024);
-        const uint64_t qmn = sdesc_sw128(qbase, kBM * 128, 1024);
+        const uint64_t domn = sdesc_sw128(dh_base(tt), kBM * 128, 1024);
+        const uint64_t qmn = sdesc_sw128(q_base(tt), kBM * 128, 1024);
 #pragma unroll
         for (int k = 0; k < kBM / 16; ++k)
-          umma_ts(t_dv, t_s + split_col(k), domn + ((k * (16 * 128)) >> 4), kIdescA,
+          umma_ts(t_dv, t_s + pt_col(k), domn + ((k * (16 * 128)) >> 4), kIdescA,
                   (tt > 0 || k > 0) ? 1u : 0u);
+        umma_commit(dh_empty(dh_slot(tt)));
 #pragma unroll
         for (int k = 0; k < kBM / 16; ++k)
-          umma_ts(t_dk, t_dp + split_col(k), qmn + ((k * (16 * 128)) >> 4), kIdescA,
+          umma_ts(t_dk, t_s + pt_col(k) + 16u, qmn + ((k * (16 * 128)) >> 4), kIdescA,
                   (tt > 0 || k > 0) ? 1u : 0u);
-        umma_commit(ring_empty(s));
+        umma_commit(q_empty(q_slot(tt)));
         if (tt == n_tiles - 1) umma_commit(acc_done);
       }
       if (tt == n_tiles - 1) done = true;
+      if (tt + 1 < n_tiles) {
+        ok = wait_q(tt + 1);
+        if (!ok) break;
+        tc_fence_after();
+        issue_st(tt + 1);  // over the P^T, dS^T columns the MMAs above read (issue order)
+        if (leader) umma_commit(s_full);
+      }
     }
     if (leader && done) mbar_wait_for(acc_done, 0, 100000000ull);
   } else if (warp >= 8 && warp < 12) {
@@ -690,19 +750,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const float sl2 = p.scale_log2;
     bool ok = true;
     for (int tt = 0; tt < n_tiles && ok; ++tt) {
-      const uint32_t s = tt % L::kStages;
       ok = __all_sync(0xffffffffu, mbar_wait(s_full, static_cast<uint32_t>(tt) & 1u, abort_flag));
-      // the entry's lse and Delta rows came by bulk copy: observe their barrier
-      // too (complete already; the stage is not reloaded before this tile's
-      // dV and dK MMAs, which wait for these warps)
-      if (ok)
-        ok = __all_sync(0xffffffffu,
-                        mbar_wait(ring_full(s), (static_cast<uint32_t>(tt) / L::kStages) & 1u,
-                                  abort_flag));
+      // the block's lse and Delta rows came by bulk copy with Q: observe that
+      // barrier too (complete already; the entry is not reloaded before this
+      // tile's dK MMA, which waits for these warps)
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(q_full(q_slot(tt)), q_par(tt), abort_flag));
       if (!ok) break;
       tc_fence_after();
-      const float *lse = reinterpret_cast<const float *>(smem + L::kRingOff + s * L::kEntry +
-                                                         2 * L::kTile);
+      const float *lse = reinterpret_cast<const float *>(smem + L::kQOff + q_slot(tt) * L::kQEntry +
+                                                         L::kTile);
       const float *dlt = lse + kBM;
       const int q0 = (qlo + tt % nq) * kBM;
       // query columns c of this tile that keep key j
@@ -721,6 +777,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int cc = 2 * half + u;
         uint32_t sv[32], dpv[32];
         tmem_ld32x2_sync(t_s + lane_off + 32 * cc, t_dp + lane_off + 32 * cc, sv, dpv);
+        if (u == 1) {  // this warp has read its whole dP^T: the next tile's may land
+          tc_fence_before();
+          warp_arrive(dp_free);
+        }
         uint32_t pk[16], dk[16];
         // the chunk's lse and Delta values, four columns per shared-memory read
         const float4 *lse4 = reinterpret_cast<const float4 *>(lse + 32 * cc);
@@ -746,8 +806,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                                 a1 ? p1 * (__uint_as_float(dpv[2 * e + 1]) - dv[2 * h2 + 1]) : 0.f);
           }
         }
-        tmem_st16(t_s + lane_off + 64 * half + 16 * u, pk);
-        tmem_st16(t_dp + lane_off + 64 * half + 16 * u, dk);
+        // P^T and dS^T over this chunk's own S^T columns (already read)
+        tmem_st16(t_s + lane_off + 32 * cc, pk);
+        tmem_st16(t_s + lane_off + 32 * cc + 16, dk);
       }
       tmem_wait_st();
       tc_fence_before();
