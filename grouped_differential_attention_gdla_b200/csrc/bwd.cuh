@@ -75,68 +75,103 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_
 __device__ __forceinline__ uint32_t split_col(int k) { return 8u * k + (k >= 4 ? 32u : 0u); }
 
 // ---------------------------------------------------------------- prep
-// One CTA per (token row, KV group k); thread c owns column c.  Per signal
-// head h of the group: dG, dD (bf16, the dQ/dK/dV operand), dlambda and
-// Delta_h = dD . H_S; then dH_N = -sum lambda dD and Delta_N = dH_N . H_N.
-// Delta uses the bf16-rounded dH the MMAs will read, so that sum_j dS_ij
-// stays zero for the gradients the kernels form.
+// One warp per (token row, KV group k), four per CTA; lane l owns columns
+// [CPL l, CPL l + CPL) with CPL = D / 32.  Per signal head h of the group:
+// dG, dD (bf16, the dQ/dK/dV operand), dlambda and Delta_h = dD . H_S; then
+// dH_N = -sum lambda dD and Delta_N = dH_N . H_N.  Delta uses the
+// bf16-rounded dH the MMAs will read, so that sum_j dS_ij stays zero for the
+// gradients the kernels form.
 template <int D>
-__global__ void __launch_bounds__(128) gdla_bwd_prep_kernel(const BwdParams p) {
-  const int64_t row = blockIdx.x;
-  const int k = blockIdx.y;
-  const int c = threadIdx.x;
+__device__ __forceinline__ void load_f32(const float *src, float (&v)[D / 32]) {
+  if constexpr (D / 32 == 4) {
+    const float4 t = *reinterpret_cast<const float4 *>(src);
+    v[0] = t.x, v[1] = t.y, v[2] = t.z, v[3] = t.w;
+  } else {
+    const float2 t = *reinterpret_cast<const float2 *>(src);
+    v[0] = t.x, v[1] = t.y;
+  }
+}
+template <int D>
+__device__ __forceinline__ void load_bf16(const __nv_bfloat16 *src, float (&v)[D / 32]) {
+  if constexpr (D / 32 == 4) {
+    const uint2 t = *reinterpret_cast<const uint2 *>(src);
+    v[0] = bf16lo_to_f32(t.x), v[1] = bf16hi_to_f32(t.x);
+    v[2] = bf16lo_to_f32(t.y), v[3] = bf16hi_to_f32(t.y);
+  } else {
+    const uint32_t t = *reinterpret_cast<const uint32_t *>(src);
+    v[0] = bf16lo_to_f32(t), v[1] = bf16hi_to_f32(t);
+  }
+}
+// Rounds v to bf16, stores it, and returns the rounded values in v.
+template <int D>
+__device__ __forceinline__ void store_bf16(__nv_bfloat16 *dst, float (&v)[D / 32]) {
+  if constexpr (D / 32 == 4) {
+    const uint2 t = make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
+    *reinterpret_cast<uint2 *>(dst) = t;
+    v[0] = bf16lo_to_f32(t.x), v[1] = bf16hi_to_f32(t.x);
+    v[2] = bf16lo_to_f32(t.y), v[3] = bf16hi_to_f32(t.y);
+  } else {
+    const uint32_t t = pack_bf16x2(v[0], v[1]);
+    *reinterpret_cast<uint32_t *>(dst) = t;
+    v[0] = bf16lo_to_f32(t), v[1] = bf16hi_to_f32(t);
+  }
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+constexpr int kPrepWarps = 4;  // (token, group) pairs per CTA of the prep kernel
+
+template <int D>
+__global__ void __launch_bounds__(32 * kPrepWarps) gdla_bwd_prep_kernel(const BwdParams p) {
+  constexpr int CPL = D / 32;
+  const int64_t pair = static_cast<int64_t>(blockIdx.x) * kPrepWarps + (threadIdx.x >> 5);
+  if (pair >= static_cast<int64_t>(p.B) * p.T * p.Hn) return;
+  const int64_t row = pair / p.Hn;
+  const int k = static_cast<int>(pair % p.Hn);
+  const int lane = threadIdx.x & 31, c = CPL * lane;
   const int g = p.g, H80 = p.Hs + p.Hn;
   const int64_t b = row / p.T, i = row % p.T;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  __shared__ float red[4][2 * kBwdMaxGroup + 1];
-  float part[2 * kBwdMaxGroup + 1];
+  float hn[CPL], dhn[CPL];
+  load_f32<D>(p.h + (row * H80 + p.Hs + k) * D + c, hn);
 #pragma unroll
-  for (int q = 0; q < 2 * kBwdMaxGroup + 1; ++q) part[q] = 0.f;
-  if (c < D) {
-    const float hn = p.h[(row * H80 + p.Hs + k) * D + c];
-    float dhn = 0.f;
+  for (int e = 0; e < CPL; ++e) dhn[e] = 0.f;
+  for (int j = 0; j < g; ++j) {
+    const int h = g * k + j;
+    const int64_t oc = (row * p.Hs + h) * D + c;
+    const float lam = __bfloat162float(p.lam[row * p.Hs + h]);
+    float hs[CPL], go[CPL], gt[CPL], dg[CPL], dd[CPL];
+    load_f32<D>(p.h + (row * H80 + h) * D + c, hs);
+    load_bf16<D>(p.dout + oc, go);
+    load_bf16<D>(p.gate + oc, gt);
+    float dlam = 0.f;
 #pragma unroll
-    for (int j = 0; j < kBwdMaxGroup; ++j) {
-      if (j < g) {
-        const int h = g * k + j;
-        const int64_t oc = (row * p.Hs + h) * D + c;
-        const float lam = __bfloat162float(p.lam[row * p.Hs + h]);
-        const float hs = p.h[(row * H80 + h) * D + c];
-        const float go = __bfloat162float(p.dout[oc]);
-        const float dd = go * __bfloat162float(p.gate[oc]);
-        const __nv_bfloat16 ddb = __float2bfloat16(dd);
-        p.dgate[oc] = __float2bfloat16(go * (hs - lam * hn));
-        p.dox[(row * H80 + h) * D + c] = ddb;
-        dhn -= lam * dd;
-        part[2 * j] = -dd * hn;                              // dlambda
-        part[2 * j + 1] = __bfloat162float(ddb) * hs;        // Delta of the signal head
-      }
+    for (int e = 0; e < CPL; ++e) {
+      dd[e] = go[e] * gt[e];
+      dg[e] = go[e] * (hs[e] - lam * hn[e]);
+      dhn[e] -= lam * dd[e];
+      dlam -= dd[e] * hn[e];
     }
-    const __nv_bfloat16 dhnb = __float2bfloat16(dhn);
-    p.dox[(row * H80 + p.Hs + k) * D + c] = dhnb;
-    part[2 * kBwdMaxGroup] = __bfloat162float(dhnb) * hn;  // Delta of the noise head
-  }
+    store_bf16<D>(p.dgate + oc, dg);
+    store_bf16<D>(p.dox + (row * H80 + h) * D + c, dd);  // dd now holds the rounded dD
+    float delta = 0.f;
 #pragma unroll
-  for (int q = 0; q < 2 * kBwdMaxGroup + 1; ++q) {
-    float v = part[q];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (lane == 0) red[warp][q] = v;
-  }
-  __syncthreads();
-  if (threadIdx.x < 2 * kBwdMaxGroup + 1) {
-    const int q = threadIdx.x;
-    const float v = red[0][q] + red[1][q] + red[2][q] + red[3][q];
-    if (q == 2 * kBwdMaxGroup) {
-      p.delta[(b * H80 + p.Hs + k) * p.tp + i] = v;
-    } else if (q / 2 < g) {
-      const int h = g * k + q / 2;
-      if (q & 1)
-        p.delta[(b * H80 + h) * p.tp + i] = v;
-      else
-        p.dlam[row * p.Hs + h] = __float2bfloat16(v);
+    for (int e = 0; e < CPL; ++e) delta += dd[e] * hs[e];
+    dlam = warp_sum(dlam);
+    delta = warp_sum(delta);
+    if (lane == 0) {
+      p.dlam[row * p.Hs + h] = __float2bfloat16(dlam);
+      p.delta[(b * H80 + h) * p.tp + i] = delta;
     }
   }
+  store_bf16<D>(p.dox + (row * H80 + p.Hs + k) * D + c, dhn);
+  float dn = 0.f;
+#pragma unroll
+  for (int e = 0; e < CPL; ++e) dn += dhn[e] * hn[e];
+  dn = warp_sum(dn);
+  if (lane == 0) p.delta[(b * H80 + p.Hs + k) * p.tp + i] = dn;
 }
 
 // ---------------------------------------------------------------- dQ

@@ -77,10 +77,12 @@ int launch_bwd(const void *q_sig, const void *q_noise, const void *k, const void
     if (cudaGetLastError() != cudaSuccess) return GDLA_ERR_CUDA;
   }
   // 2. dG, dlambda, dH of every head and Delta
-  if (B * T > 0x7fffffffull) return GDLA_ERR_UNSUPPORTED;
-  gdla::gdla_bwd_prep_kernel<D><<<dim3(static_cast<unsigned>(B * T),
-                                       static_cast<unsigned>(bp.Hn)),
-                                  128, 0, s>>>(bp);
+  const uint64_t pairs = static_cast<uint64_t>(B) * static_cast<uint64_t>(T) * bp.Hn;
+  if (B * T > 0x7fffffffull || (pairs + gdla::kPrepWarps - 1) / gdla::kPrepWarps > 0x7fffffffull)
+    return GDLA_ERR_UNSUPPORTED;
+  gdla::gdla_bwd_prep_kernel<D>
+      <<<static_cast<unsigned>((pairs + gdla::kPrepWarps - 1) / gdla::kPrepWarps),
+         32 * gdla::kPrepWarps, 0, s>>>(bp);
   if (cudaGetLastError() != cudaSuccess) return GDLA_ERR_CUDA;
   // 3. dQ of every head, heaviest query blocks first
   {
