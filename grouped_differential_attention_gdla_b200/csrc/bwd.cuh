@@ -186,21 +186,56 @@ struct DqSmemLayout {
   static constexpr uint32_t kDoOff = kQOff + kTile;
   static constexpr uint32_t kRingOff = kDoOff + kTile;
   static constexpr uint32_t kBarOff = kRingOff + kStages * kTile;
-  // qd_full kv_full[S] kv_empty[S] s_full p_full[2] dp_free dq_done
-  static constexpr uint32_t kNumBars = 1 + 2 * kStages + 5;
+  // qd_full kv_full[S] kv_empty[S] s_full p_full[2] dp_free dq_done qd_free dq_free
+  static constexpr uint32_t kNumBars = 1 + 2 * kStages + 7;
   static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;
   static constexpr uint32_t kBytes = kMiscOff + 16;
   static_assert(kBytes <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
 };
 
-// One CTA per (batch b, head x of Hs + Hn, query block), heaviest blocks
-// first.  Warps 0-7: P and dS (warpgroup `half` takes key columns
-// [64 half, 64 half + 64)); 8-11: dQ epilogue; 12: TMA; 13: TMEM and MMA.
+// A dQ item: (batch b, head x of Hs + Hn, query block), heaviest blocks
+// first in item order; its key tiles j_lo .. j_lo + n - 1.
+struct DqItem {
+  int b, x, kvh, q0, j_lo, n;
+  bool noise;
+};
+
+__device__ __forceinline__ DqItem dq_item(const BwdParams &p, int item) {
+  const int H80 = p.Hs + p.Hn;
+  DqItem it;
+  const int qb = p.n_qblk - 1 - item / (p.B * H80);
+  const int rest = item % (p.B * H80);
+  it.b = rest / H80;
+  it.x = rest % H80;
+  it.noise = it.x >= p.Hs;
+  it.kvh = it.noise ? it.x - p.Hs : it.x / p.g;
+  it.q0 = qb * kBM;
+  int j_hi;
+  it.j_lo = 0;
+  if (p.causal) {
+    j_hi = min(it.q0 + kBM - 1, p.T - 1) / kBN;
+    if (p.window > 0) {
+      const int64_t first = static_cast<int64_t>(it.q0) - p.window + 1;
+      it.j_lo = first > 0 ? static_cast<int>(first / kBN) : 0;
+    }
+  } else {
+    j_hi = (p.T - 1) / kBN;
+  }
+  it.n = j_hi - it.j_lo + 1;
+  return it;
+}
+
+// Persistent: CTA c takes items c, c + gridDim.x, ...; the tile pipeline
+// (ring positions, S buffers, barrier phases) runs on across items.
+// Warps 0-7: P and dS (warpgroup `half` takes key columns [64 half,
+// 64 half + 64)); 8-11: dQ epilogue; 12: TMA; 13: TMEM and MMA.
 // TMEM: S of even tiles [0,128) and of odd tiles [384,512) (dS packed over
 // each), dP [128,256), dQ [256, 256+D).  The MMA warp computes S(t+1) while
 // the elementwise warps work on tile t, and dP(t+1) as soon as they have
-// read dP(t) (half-way through the tile), so the tensor core is busy with
-// the next tile's scores while the current tile's dS is formed.
+// read dP(t) (half-way through the tile); the next tile may be the first of
+// the next item, whose Q and dH load as soon as the last S and dP MMAs of
+// the current item have read theirs.  An item's first dQ MMA waits for the
+// epilogue to have read the previous item's dQ.
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     gdla_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qs,
@@ -220,33 +255,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   auto kv_full = [&](uint32_t s) { return bar0 + 8u * (1 + s); };
   auto kv_empty = [&](uint32_t s) { return bar0 + 8u * (1 + L::kStages + s); };
   const uint32_t s_full = bar0 + 8u * (1 + 2 * L::kStages);
-  auto p_full = [&](int t) { return s_full + 8u * (1 + (t & 1)); };  // dS(t) packed
+  auto p_full = [&](uint32_t t) { return s_full + 8u * (1 + (t & 1u)); };  // dS(t) packed
   const uint32_t dp_free = s_full + 24u;  // dP(t) read out by every elementwise warp
-  const uint32_t dq_done = s_full + 32u;
+  const uint32_t dq_done = s_full + 32u;  // an item's dQ complete
+  const uint32_t qd_free = s_full + 40u;  // an item's last S and dP have read Q and dH
+  const uint32_t dq_free = s_full + 48u;  // the epilogue has read an item's dQ
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
   const int warp = threadIdx.x >> 5;
   const int H80 = p.Hs + p.Hn;
-
-  // the item: heaviest query blocks first
-  const int item = blockIdx.x;
-  const int qb = p.n_qblk - 1 - item / (p.B * H80);
-  const int rest = item % (p.B * H80);
-  const int b = rest / H80, x = rest % H80;
-  const bool noise = x >= p.Hs;
-  const int kvh = noise ? x - p.Hs : x / p.g;
-  const int q0 = qb * kBM;
-  int j_lo = 0, j_hi;
-  if (p.causal) {
-    j_hi = min(q0 + kBM - 1, p.T - 1) / kBN;
-    if (p.window > 0) {
-      const int64_t first = static_cast<int64_t>(q0) - p.window + 1;
-      j_lo = first > 0 ? static_cast<int>(first / kBN) : 0;
-    }
-  } else {
-    j_hi = (p.T - 1) / kBN;
-  }
-  const int n = j_hi - j_lo + 1;
+  const int n_items = p.n_qblk * p.B * H80;
+  const int G = static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
     mbar_init(qd_full, 1);
@@ -259,6 +278,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(p_full(1), 8);
     mbar_init(dp_free, 8);
     mbar_init(dq_done, 1);
+    mbar_init(qd_free, 1);
+    mbar_init(dq_free, 4);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -271,37 +292,49 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t t_dp = tmem + 128u, t_dq = tmem + 256u;
-  auto t_s = [&](int t) { return tmem + ((t & 1) ? 384u : 0u); };
+  auto t_s = [&](uint32_t t) { return tmem + ((t & 1u) ? 384u : 0u); };
 
   if (warp == kBwdProducerWarp) {
-    // =============================== TMA: Q_x and dH_x, then K_t, V_t per tile
+    // =============================== TMA: per item Q_x and dH_x, then K_t, V_t per tile
     const bool leader = elect_one();
     if (leader) {
-      mbar_arrive_expect_tx(qd_full, 2 * L::kTile);
-#pragma unroll
-      for (int kb = 0; kb < D / 64; ++kb) {
-        const int head = noise ? kvh : x;
-        tma_load_3d(sbase + L::kQOff + kb * L::kSub, noise ? &tm_qn : &tm_qs, qd_full,
-                    head * D + kb * 64, q0, b);
-        tma_load_3d(sbase + L::kDoOff + kb * L::kSub, &tm_dox, qd_full, x * D + kb * 64, q0, b);
-      }
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
     }
-    uint32_t c = 0;
+    uint32_t c = 0, ik = 0;
     bool ok = true;
-    for (int t = 0; t < n && ok; ++t) {
-      for (int kv = 0; kv < 2 && ok; ++kv) {
-        const uint32_t s = c % L::kStages;
-        ok = __all_sync(0xffffffffu,
-                        mbar_wait(kv_empty(s), ((c / L::kStages) & 1u) ^ 1u, abort_flag));
+    for (int item = blockIdx.x; item < n_items && ok; item += G, ++ik) {
+      const DqItem it = dq_item(p, item);
+      if (ik > 0) {  // the previous item's last S and dP have read Q and dH
+        ok = __all_sync(0xffffffffu, mbar_wait(qd_free, (ik - 1) & 1u, abort_flag));
         if (!ok) break;
-        if (leader) {
-          mbar_arrive_expect_tx(kv_full(s), L::kTile);
+      }
+      if (leader) {
+        mbar_arrive_expect_tx(qd_full, 2 * L::kTile);
 #pragma unroll
-          for (int kb = 0; kb < D / 64; ++kb)
-            tma_load_3d(sbase + L::kRingOff + s * L::kTile + kb * L::kSub, kv ? &tm_v : &tm_k,
-                        kv_full(s), kvh * D + kb * 64, (j_lo + t) * kBN, b);
+        for (int kb = 0; kb < D / 64; ++kb) {
+          const int head = it.noise ? it.kvh : it.x;
+          tma_load_3d(sbase + L::kQOff + kb * L::kSub, it.noise ? &tm_qn : &tm_qs, qd_full,
+                      head * D + kb * 64, it.q0, it.b);
+          tma_load_3d(sbase + L::kDoOff + kb * L::kSub, &tm_dox, qd_full, it.x * D + kb * 64,
+                      it.q0, it.b);
         }
-        ++c;
+      }
+      for (int t = 0; t < it.n && ok; ++t) {
+        for (int kv = 0; kv < 2 && ok; ++kv) {
+          const uint32_t s = c % L::kStages;
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait(kv_empty(s), ((c / L::kStages) & 1u) ^ 1u, abort_flag));
+          if (!ok) break;
+          if (leader) {
+            mbar_arrive_expect_tx(kv_full(s), L::kTile);
+#pragma unroll
+            for (int kb = 0; kb < D / 64; ++kb)
+              tma_load_3d(sbase + L::kRingOff + s * L::kTile + kb * L::kSub, kv ? &tm_v : &tm_k,
+                          kv_full(s), it.kvh * D + kb * 64, (it.j_lo + t) * kBN, it.b);
+          }
+          ++c;
+        }
       }
     }
     if (!ok && leader) {
@@ -309,11 +342,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t issued = c > s ? (c - 1 - s) / L::kStages + 1 : 0;
         if (issued) mbar_wait_for(kv_full(s), (issued - 1) & 1u, 100000000ull);
       }
-      mbar_wait_for(qd_full, 0, 100000000ull);
+      // the Q and dH of the last item this warp armed
+      if (ik > 0 || blockIdx.x < static_cast<unsigned>(n_items))
+        mbar_wait_for(qd_full, ik & 1u, 100000000ull);
     }
   } else if (warp == kBwdMmaWarp) {
-    // =============================== MMA: S(t+1) and dP(t+1) ahead of dQ += dS(t) K_t
-    // (the ring holds K_t, V_t at positions 2t, 2t+1)
+    // =============================== MMA: S(T+1) and dP(T+1) ahead of dQ += dS(T) K_T
+    // (T counts this CTA's tiles; the ring holds K_T, V_T at positions 2T, 2T+1)
     const bool leader = elect_one();
     constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBN, false, false);
     constexpr uint32_t kIdescQ = idesc_bf16_f32(kBM, D, false, true);
@@ -325,75 +360,115 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         mbar_wait(kv_full(slot(pos)), (pos / L::kStages) & 1u, abort_flag));
     };
     auto tile = [&](uint32_t pos) { return sbase + L::kRingOff + slot(pos) * L::kTile; };
-    // S(t) = Q K_t^T into t's S buffer (K-major operands, D/16 K-steps)
-    auto issue_s = [&](int t) {
+    // S(T) = Q K_T^T into T's S buffer (K-major operands, D/16 K-steps)
+    auto issue_s = [&](uint32_t T) {
       if (!leader) return;
-      const uint64_t kd = sdesc_sw128(tile(2u * t), 16, 1024);
+      const uint64_t kd = sdesc_sw128(tile(2u * T), 16, 1024);
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
         const uint32_t off = (k >> 2) * L::kSub + (k & 3) * 32;
-        umma_ss(t_s(t), qd + (off >> 4), kd + (off >> 4), kIdescS, k > 0 ? 1u : 0u);
+        umma_ss(t_s(T), qd + (off >> 4), kd + (off >> 4), kIdescS, k > 0 ? 1u : 0u);
       }
     };
-    // dP(t) = dH V_t^T, then S(t) and dP(t) are announced and V_t released
-    auto issue_dp = [&](int t) {
+    // dP(T) = dH V_T^T, then S(T) and dP(T) are announced and V_T released;
+    // after an item's last tile its Q and dH are released too
+    auto issue_dp = [&](uint32_t T, bool last_of_item) {
       if (!leader) return;
-      const uint64_t vd = sdesc_sw128(tile(2u * t + 1u), 16, 1024);
+      const uint64_t vd = sdesc_sw128(tile(2u * T + 1u), 16, 1024);
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
         const uint32_t off = (k >> 2) * L::kSub + (k & 3) * 32;
         umma_ss(t_dp, dod + (off >> 4), vd + (off >> 4), kIdescS, k > 0 ? 1u : 0u);
       }
       umma_commit(s_full);
-      umma_commit(kv_empty(slot(2u * t + 1u)));
+      umma_commit(kv_empty(slot(2u * T + 1u)));
+      if (last_of_item) umma_commit(qd_free);
     };
-    bool ok = __all_sync(0xffffffffu, mbar_wait(qd_full, 0, abort_flag));
-    uint32_t done = 0;
-    if (ok && n > 0) ok = wait_full(0) && wait_full(1);
-    if (ok && n > 0) {
-      tc_fence_after();
-      issue_s(0);
-      issue_dp(0);
-    }
-    for (int t = 0; t < n && ok; ++t) {
-      if (t + 1 < n) {
-        ok = wait_full(2u * (t + 1)) && wait_full(2u * (t + 1) + 1u);
-        if (!ok) break;
+    bool ok = true;
+    uint32_t T = 0, dq_commits = 0;
+    int item = blockIdx.x, t = 0;
+    uint32_t ik = 0;
+    DqItem it{};
+    if (item < n_items) {
+      it = dq_item(p, item);
+      ok = __all_sync(0xffffffffu, mbar_wait(qd_full, 0, abort_flag)) && wait_full(0) &&
+           wait_full(1);
+      if (ok) {
         tc_fence_after();
-        issue_s(t + 1);  // its buffer last held dS(t-1), read by the dQ MMA issued before
-        ok = __all_sync(0xffffffffu, mbar_wait(dp_free, static_cast<uint32_t>(t) & 1u, abort_flag));
-        if (!ok) break;
-        tc_fence_after();
-        issue_dp(t + 1);
+        issue_s(0);
+        issue_dp(0, it.n == 1);
       }
-      ok = __all_sync(0xffffffffu,
-                      mbar_wait(p_full(t), static_cast<uint32_t>(t >> 1) & 1u, abort_flag));
+    } else {
+      ok = false;
+    }
+    while (ok) {
+      // the next tile: t + 1 of this item, or the first of the next item
+      int n_item = item, n_t = t + 1;
+      uint32_t n_ik = ik;
+      DqItem nit = it;
+      if (n_t >= it.n) {
+        n_item = item + G;
+        n_t = 0;
+        n_ik = ik + 1;
+        if (n_item < n_items) nit = dq_item(p, n_item);
+      }
+      const bool has_next = n_item < n_items;
+      if (has_next) {
+        if (n_t == 0) {
+          ok = __all_sync(0xffffffffu, mbar_wait(qd_full, n_ik & 1u, abort_flag));
+          if (!ok) break;
+        }
+        ok = wait_full(2u * (T + 1)) && wait_full(2u * (T + 1) + 1u);
+        if (!ok) break;
+        tc_fence_after();
+        issue_s(T + 1);  // its buffer last held dS(T-1), read by the dQ MMA issued before
+        ok = __all_sync(0xffffffffu, mbar_wait(dp_free, T & 1u, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        issue_dp(T + 1, n_t == nit.n - 1);
+      }
+      ok = __all_sync(0xffffffffu, mbar_wait(p_full(T), (T >> 1) & 1u, abort_flag));
       if (!ok) break;
+      if (t == 0 && ik > 0) {  // the epilogue has read the previous item's dQ
+        ok = __all_sync(0xffffffffu, mbar_wait(dq_free, (ik - 1) & 1u, abort_flag));
+        if (!ok) break;
+      }
       tc_fence_after();
-      // dQ += dS K_t: A = dS (TMEM, packed halves), B = K_t MN-major over d
+      // dQ += dS K_T: A = dS (TMEM, packed halves), B = K_T MN-major over d
       if (leader) {
-        const uint64_t kmn = sdesc_sw128(tile(2u * t), kBN * 128, 1024);
+        const uint64_t kmn = sdesc_sw128(tile(2u * T), kBN * 128, 1024);
 #pragma unroll
         for (int k = 0; k < kBN / 16; ++k)
-          umma_ts(t_dq, t_s(t) + split_col(k), kmn + ((k * (16 * 128)) >> 4), kIdescQ,
+          umma_ts(t_dq, t_s(T) + split_col(k), kmn + ((k * (16 * 128)) >> 4), kIdescQ,
                   (t > 0 || k > 0) ? 1u : 0u);
-        umma_commit(kv_empty(slot(2u * t)));
-        if (t == n - 1) umma_commit(dq_done);
+        umma_commit(kv_empty(slot(2u * T)));
+        if (t == it.n - 1) umma_commit(dq_done);
       }
-      if (t == n - 1) ++done;
+      if (t == it.n - 1) ++dq_commits;
+      if (!has_next) break;
+      item = n_item;
+      t = n_t;
+      ik = n_ik;
+      it = nit;
+      ++T;
     }
-    if (leader && done) mbar_wait_for(dq_done, 0, 100000000ull);
+    if (leader && dq_commits) mbar_wait_for(dq_done, (dq_commits - 1) & 1u, 100000000ull);
   } else if (warp >= 8 && warp < 12) {
-    // =============================== epilogue: dQ_x = scale * (dS K), bf16 rows
+    // =============================== epilogue: dQ_x = scale * (dS K), bf16 rows, per item
     const int wq = warp & 3;
     const int r = threadIdx.x & 127;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const int i = q0 + r;
-    bool ok = __all_sync(0xffffffffu, mbar_wait(dq_done, 0, abort_flag));
-    if (ok) {
+    bool ok = true;
+    uint32_t ik = 0;
+    for (int item = blockIdx.x; item < n_items && ok; item += G, ++ik) {
+      const DqItem it = dq_item(p, item);
+      ok = __all_sync(0xffffffffu, mbar_wait(dq_done, ik & 1u, abort_flag));
+      if (!ok) break;
       tc_fence_after();
-      __nv_bfloat16 *dst = noise ? p.dq_noise + ((static_cast<int64_t>(b) * p.T + i) * p.Hn + kvh) * D
-                                 : p.dq_sig + ((static_cast<int64_t>(b) * p.T + i) * p.Hs + x) * D;
+      const int i = it.q0 + r;
+      __nv_bfloat16 *dst =
+          it.noise ? p.dq_noise + ((static_cast<int64_t>(it.b) * p.T + i) * p.Hn + it.kvh) * D
+                   : p.dq_sig + ((static_cast<int64_t>(it.b) * p.T + i) * p.Hs + it.x) * D;
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t v[32];
@@ -412,59 +487,66 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                                            __uint_as_float(v[8 * q + 7]) * p.scale));
         }
       }
+      tc_fence_before();
+      warp_arrive(dq_free);
     }
   } else if (warp < 8) {
     // =============================== P and dS, half a row per warpgroup
     const int half = warp >> 2, wq = warp & 3;
     const int r = threadIdx.x & 127;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const int i = q0 + r;
-    const bool row_ok = i < p.T;
-    const int64_t srow = (static_cast<int64_t>(b) * H80 + x) * p.tp + i;
-    const float lse = row_ok ? p.lse[srow] : 0.f;
-    const float dl = row_ok ? p.delta[srow] : 0.f;
     const float sl2 = p.scale_log2;
     bool ok = true;
-    for (int t = 0; t < n && ok; ++t) {
-      ok = __all_sync(0xffffffffu, mbar_wait(s_full, static_cast<uint32_t>(t) & 1u, abort_flag));
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t ts = t_s(t);
-      const int kbase = (j_lo + t) * kBN;
-      int c_lo, c_hi;  // kept key columns of this row in the tile
-      if (p.causal) {
-        c_hi = i - kbase;
-        c_lo = p.window > 0 ? static_cast<int>(static_cast<int64_t>(i) - p.window + 1 - kbase) : -1;
-      } else {
-        c_hi = p.T - 1 - kbase;
-        c_lo = -1;
-      }
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int cc = 2 * half + u;  // 32-column chunk of the tile
-        uint32_t sv[32], dpv[32];
-        tmem_ld32x2_sync(ts + lane_off + 32 * cc, t_dp + lane_off + 32 * cc, sv, dpv);
-        if (u == 1) {  // this warp has read its whole dP(t): dP(t+1) may overwrite it
-          tc_fence_before();
-          warp_arrive(dp_free);
+    uint32_t T = 0;
+    for (int item = blockIdx.x; item < n_items && ok; item += G) {
+      const DqItem it = dq_item(p, item);
+      const int i = it.q0 + r;
+      const bool row_ok = i < p.T;
+      const int64_t srow = (static_cast<int64_t>(it.b) * H80 + it.x) * p.tp + i;
+      const float lse = row_ok ? p.lse[srow] : 0.f;
+      const float dl = row_ok ? p.delta[srow] : 0.f;
+      for (int t = 0; t < it.n && ok; ++t, ++T) {
+        ok = __all_sync(0xffffffffu, mbar_wait(s_full, T & 1u, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t ts = t_s(T);
+        const int kbase = (it.j_lo + t) * kBN;
+        int c_lo, c_hi;  // kept key columns of this row in the tile
+        if (p.causal) {
+          c_hi = i - kbase;
+          c_lo = p.window > 0 ? static_cast<int>(static_cast<int64_t>(i) - p.window + 1 - kbase)
+                              : -1;
+        } else {
+          c_hi = p.T - 1 - kbase;
+          c_lo = -1;
         }
-        uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int c0 = 32 * cc + 2 * e;
-          const bool k0 = row_ok && c0 >= c_lo && c0 <= c_hi;
-          const bool k1 = row_ok && c0 + 1 >= c_lo && c0 + 1 <= c_hi;
-          const float p0 = k0 ? ex2_approx(__uint_as_float(sv[2 * e]) * sl2 - lse) : 0.f;
-          const float p1 = k1 ? ex2_approx(__uint_as_float(sv[2 * e + 1]) * sl2 - lse) : 0.f;
-          pk[e] = pack_bf16x2(p0 * (__uint_as_float(dpv[2 * e]) - dl),
-                              p1 * (__uint_as_float(dpv[2 * e + 1]) - dl));
+        for (int u = 0; u < 2; ++u) {
+          const int cc = 2 * half + u;  // 32-column chunk of the tile
+          uint32_t sv[32], dpv[32];
+          tmem_ld32x2_sync(ts + lane_off + 32 * cc, t_dp + lane_off + 32 * cc, sv, dpv);
+          if (u == 1) {  // this warp has read its whole dP(T): dP(T+1) may overwrite it
+            tc_fence_before();
+            warp_arrive(dp_free);
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int c0 = 32 * cc + 2 * e;
+            const bool k0 = row_ok && c0 >= c_lo && c0 <= c_hi;
+            const bool k1 = row_ok && c0 + 1 >= c_lo && c0 + 1 <= c_hi;
+            const float p0 = k0 ? ex2_approx(__uint_as_float(sv[2 * e]) * sl2 - lse) : 0.f;
+            const float p1 = k1 ? ex2_approx(__uint_as_float(sv[2 * e + 1]) * sl2 - lse) : 0.f;
+            pk[e] = pack_bf16x2(p0 * (__uint_as_float(dpv[2 * e]) - dl),
+                                p1 * (__uint_as_float(dpv[2 * e + 1]) - dl));
+          }
+          // dS of this chunk, packed into this half's own S columns
+          tmem_st16(ts + lane_off + 64 * half + 16 * u, pk);
         }
-        // dS of this chunk, packed into this half's own S columns
-        tmem_st16(ts + lane_off + 64 * half + 16 * u, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        warp_arrive(p_full(T));
       }
-      tmem_wait_st();
-      tc_fence_before();
-      warp_arrive(p_full(t));
     }
   }
 

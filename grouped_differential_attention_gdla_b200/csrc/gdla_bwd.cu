@@ -92,7 +92,9 @@ int launch_bwd(const void *q_sig, const void *q_noise, const void *k, const void
     if (rc != GDLA_OK) return rc;
     const uint64_t items = static_cast<uint64_t>(bp.n_qblk) * B * H80;
     if (items > 0x7fffffffull) return GDLA_ERR_UNSUPPORTED;
-    kern<<<static_cast<unsigned>(items), gdla::kBwdThreads, L::kBytes, s>>>(
+    // persistent: one CTA per SM walks the items
+    const uint64_t grid = items < static_cast<uint64_t>(sms) ? items : static_cast<uint64_t>(sms);
+    kern<<<static_cast<unsigned>(grid), gdla::kBwdThreads, L::kBytes, s>>>(
         tm_qs, tm_qn, tm_dox, tm_k, tm_v, bp);
     if (cudaGetLastError() != cudaSuccess) return GDLA_ERR_CUDA;
   }
