@@ -10,15 +10,17 @@
 //   s_j = q_h . (c_hat_j W_K) = (W_K q_h) . c_hat_j      absorbed query q~_h
 //   H_h = sum_j p_j (c_hat_j W_V) = (sum_j p_j c_hat_j) W_V
 // so attention runs in the latent space and reads 1 KB per cached token for
-// all 80 heads at once.  Three kernels:
-//   absorb   q~ = (scale log2 e) W_K q for every head, bf16, into workspace;
+// all 80 heads at once.  Four kernels:
+//   absorb   q~ = (scale log2 e) W_K q for every head, bf16, into workspace
+//            (tcgen05 GEMM tiles);
 //   attn     split-KV attention over the cache (tcgen05): per chunk of 128
 //            cached tokens, S^T = c_hat q~^T (M = 128 tokens, N = heads,
 //            K = latent), a per-head online softmax across tokens, and
 //            z^T += c_hat^T P (M = latent, N = heads, K = tokens); each CTA
 //            leaves (max, sum, z) of its chunks in workspace;
-//   combine  merges the splits per head, H = z W_V, then
-//            out = G (.) (H_S - lambda Repeat_g(H_N)).
+//   merge    folds the splits per head into z / l (bf16);
+//   out      H = z W_V (tcgen05 GEMM per KV group and block of sequences),
+//            then out = G (.) (H_S - lambda Repeat_g(H_N)).
 #pragma once
 
 #include "sm100.cuh"
@@ -601,7 +603,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   }
 }
 
-// ---------------------------------------------------------------- combine
+// ---------------------------------------------------------------- merge and output
 // Two kernels.  merge: one CTA per (KV group k, sequence b, head j of the
 // group; j < g: signal head g k + j, j = g: noise head k), thread = 4 latent
 // columns: over the splits, M = max_s m_s, l = sum_s 2^(m_s - M) l_s and

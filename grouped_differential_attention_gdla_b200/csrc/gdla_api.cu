@@ -263,7 +263,7 @@ int launch_decode_attn(const gdla::DecodeParams &prm, const DecodeMaps &m, cudaS
 
 // merge of the splits into Z, then the output GEMM and gate
 template <int NH>
-int launch_decode_combine(const gdla::DecodeParams &prm, const DecodeMaps &m,
+int launch_decode_merge_out(const gdla::DecodeParams &prm, const DecodeMaps &m,
                           cudaStream_t stream) {
   constexpr auto kout = gdla::gdla_decode_out_kernel<NH>;
   const int rc = prepare_kernel<kout>(gdla::CombSmem::kBytes, 0);
@@ -500,15 +500,15 @@ int gdla_decode_fwd(const void *q_sig, const void *q_noise, const void *c_hat,
     default: rc = launch_decode_attn<80>(prm, maps, s); break;
   }
   if (rc != GDLA_OK) return rc;
-  switch (Hs / Hn) {  // the combine is specialised for the heads of a group
-    case 1: return launch_decode_combine<2>(prm, maps, s);
-    case 2: return launch_decode_combine<3>(prm, maps, s);
-    case 3: return launch_decode_combine<4>(prm, maps, s);
-    case 4: return launch_decode_combine<5>(prm, maps, s);
-    case 5: return launch_decode_combine<6>(prm, maps, s);
-    case 6: return launch_decode_combine<7>(prm, maps, s);
-    case 7: return launch_decode_combine<8>(prm, maps, s);
-    default: return launch_decode_combine<9>(prm, maps, s);
+  switch (Hs / Hn) {  // merge and output are specialised for the heads of a group
+    case 1: return launch_decode_merge_out<2>(prm, maps, s);
+    case 2: return launch_decode_merge_out<3>(prm, maps, s);
+    case 3: return launch_decode_merge_out<4>(prm, maps, s);
+    case 4: return launch_decode_merge_out<5>(prm, maps, s);
+    case 5: return launch_decode_merge_out<6>(prm, maps, s);
+    case 6: return launch_decode_merge_out<7>(prm, maps, s);
+    case 7: return launch_decode_merge_out<8>(prm, maps, s);
+    default: return launch_decode_merge_out<9>(prm, maps, s);
   }
 }
 

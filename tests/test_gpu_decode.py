@@ -63,7 +63,7 @@ def _oracle(x, lens, window):
     (4, 2000, 64, 16, 128, 512, [2000, 1, 777, 1024], 0, False),
     (4, 2000, 64, 16, 128, 512, [2000, 1, 777, 1024], 128, True),
     (2, 5000, 64, 16, 128, 512, [5000, 3000], 1, False),
-    # one signal head per group (2 head rows per group in the combine)
+    # one signal head per group (2 head rows per group in the merge and output)
     (5, 600, 4, 4, 128, 512, [600, 1, 250, 599, 128], 0, False),
     # three signal heads per group, d = 64, a 256-d latent
     (3, 400, 6, 2, 64, 256, [400, 17, 256], 0, True),
