@@ -136,3 +136,45 @@ def test_decode_cache_len_out_of_range_sets_status():
     _decode(x, [0, 300], 0, status=status)
     torch.cuda.synchronize()
     assert int(status.item()) == gdla._binding.GDLA_ERR_INVALID_ARG
+
+
+def test_decode_graph_replay_matches_eager():
+    """A decode step captured once in a CUDA graph (as a serving loop, and the
+    benchmark, replay it) gives, for new queries copied into the captured
+    buffers, bit for bit the output of an eager call on those queries."""
+    B, L_max = 6, 1000
+    lens = [1000, 1, 517, 128, 129, 900]
+    x = _case(B, L_max, 64, 16, 128, 512, seed=21)
+    c_hat = gdla.gdla_latent_rmsnorm(x["c_kv"], None, 1e-6)
+    cl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    ws = torch.empty(gdla.gdla_decode_workspace_bytes(B, L_max, 64, 16, 512, 0),
+                     dtype=torch.uint8, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    q_sig, q_noise = x["q_sig"].clone(), x["q_noise"].clone()
+    out = torch.empty(B, 64 * 128, dtype=torch.bfloat16, device="cuda")
+
+    def call(o, qs, qn):
+        gdla.gdla_decode_fwd(qs, qn, c_hat, cl, x["w_kvb"], x["lam"], x["gate"], out=o,
+                             workspace=ws, d_status=status,
+                             stream=torch.cuda.current_stream())
+
+    call(out, q_sig, q_noise)  # one-time kernel set-up outside the capture
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call(out, q_sig, q_noise)
+    g = torch.Generator(device="cuda").manual_seed(5)
+    for _ in range(2):
+        new_s = torch.randn(q_sig.shape, generator=g, device="cuda").to(torch.bfloat16)
+        new_n = torch.randn(q_noise.shape, generator=g, device="cuda").to(torch.bfloat16)
+        q_sig.copy_(new_s)
+        q_noise.copy_(new_n)
+        graph.replay()
+        torch.cuda.synchronize()
+        replayed = out.clone()
+        eager = torch.empty_like(out)
+        call(eager, new_s, new_n)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        assert torch.equal(replayed, eager)
+    del graph
