@@ -16,17 +16,19 @@
 //      its log-sum-exp (log2 units of the scaled scores);
 //   2. gdla_bwd_prep_kernel (CUDA cores): dG, dlambda, dH of every head
 //      (bf16, the MMA operand) and Delta;
-//   3. gdla_bwd_dq_kernel (tcgen05): per (head, query block), over the key
-//      tiles: S = Q K^T and dP = dH V^T in TMEM, P and dS by two warpgroups
-//      (half the key columns each), dQ += dS K with dS read from TMEM;
+//   3. gdla_bwd_dq_kernel (tcgen05, persistent): per (head, query block),
+//      over the key tiles: S = Q K^T and dP = dH V^T in TMEM, P and dS by two
+//      warpgroups (half the key columns each), dQ += dS K with dS read from
+//      TMEM; the next tile's S and dP overlap the current tile's dS;
 //   4. gdla_bwd_dkdv_kernel (tcgen05): per (KV group, key block), over the
 //      group's g+1 heads and their query blocks: S^T = K Q^T and
 //      dP^T = V dH^T in TMEM, P^T and dS^T per key row, dV += P^T dH and
-//      dK += dS^T Q with both A operands read from TMEM.
+//      dK += dS^T Q with both A operands read from TMEM; the next tile's
+//      dP^T overlaps the current tile's P^T and dS^T.
 // The softmax statistics come from step 1, so neither kernel needs a running
 // maximum, and the two warpgroups that share a row never wait on each other:
-// each writes its packed bf16 operand into TMEM columns of its own half of the
-// tile (the MMA's A address skips to the second half for K-steps 4..7).
+// each writes its packed bf16 operands into TMEM columns of its own half of
+// the tile, over columns it has already read.
 #pragma once
 
 #include "attn_rope.cuh"
